@@ -1,0 +1,418 @@
+"""Pins of the fp64 CPU oracle against facts fixed by the pages and by mathematics.
+
+None of these tests touches a GPU.  Each pin is independent of the oracle's own
+code: printed values of the pages' worked example, brute-force selection, dense
+attention and its autograd gradients from torch (fp64), an explicit dense-mask
+formulation of the gated attention differentiated by torch autograd, central
+finite differences, the inner-gate gradient identity (Eq. 5 of the pages),
+and invariants (shift invariance of s, ds summing to zero, sparse == full scope
+when the budget covers the history).
+"""
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            vals[key] = [float(x) for x in rest]
+    return vals
+
+
+def _rand_train(rng, B, n, Hq, Hkv, d, bs, s_std=1.0, qk_std=0.5):
+    Cq = n // bs
+    q = rng.standard_normal((B, n, Hq, d)) * qk_std
+    k = rng.standard_normal((B, n, Hkv, d)) * qk_std
+    v = rng.standard_normal((B, n, Hkv, d))
+    s = rng.standard_normal((B, Hkv, Cq, Cq)) * s_std
+    dO = rng.standard_normal((B, n, Hq, d))
+    return q, k, v, s, dO
+
+
+def _brute_select(row, c, K):
+    if K >= c:
+        return list(range(c))
+    order = sorted(range(c), key=lambda m: (-row[m], m))
+    return sorted(order[:K])
+
+
+# --------------------------------------------------------------------------
+# worked example (jaehun.me review, walkthrough Steps 1-4)
+# --------------------------------------------------------------------------
+
+def test_worked_example_gate_and_topk():
+    g = _golden("worked_example.txt")
+    s_row = np.array(g["scores"])
+    C, K = len(s_row), int(g["top_k"][0])
+    assert int(g["n"][0]) // int(g["block_size"][0]) == C
+    # query in block C (0-based) sees history blocks 0..C-1 with the printed scores
+    s = np.zeros((1, 1, C + 1, C + 1))
+    s[0, 0, C, :C] = s_row
+    idx, lse = oracle.train_select(s, K)
+    assert sorted(idx[0, 0, C].tolist()) == sorted(int(x) for x in g["topk_0based"])
+    assert idx[0, 0, C].tolist() == sorted(idx[0, 0, C].tolist())  # ascending
+    L = lse[0, 0, C]
+    assert abs(np.exp(L) - g["exp_sum"][0]) <= g["exp_sum_tol"][0]
+    np.testing.assert_allclose(np.exp(s_row), g["exp_scores"], atol=g["exp_scores_tol"][0])
+    np.testing.assert_allclose(s_row - L, g["log_gate"], atol=g["log_gate_tol"][0])
+    # gates are a distribution over the history blocks
+    assert abs(np.exp(s_row - L).sum() - 1.0) < 1e-12
+
+
+def test_worked_example_attention_mass_closed_form():
+    """With q = 0 every logit equals its bias, so the attention mass of a selected
+    block is bs*g_m / (sum over selected bs*g + number of current-block keys):
+    the current block carries gate 1 and unselected blocks get nothing (Eq. 9)."""
+    g = _golden("worked_example.txt")
+    s_row = np.array(g["scores"])
+    C, K, bs = len(s_row), int(g["top_k"][0]), int(g["block_size"][0])
+    n = (C + 1) * bs
+    d = C + 1
+    q = np.zeros((1, n, 1, d))
+    k = np.random.default_rng(0).standard_normal((1, n, 1, d))
+    v = np.zeros((1, n, 1, d))
+    for j in range(n):
+        v[0, j, 0, j // bs] = 1.0  # one-hot block indicator
+    s = np.zeros((1, 1, C + 1, C + 1))
+    s[0, 0, C, :C] = s_row
+    o, lse = oracle.attn_fwd(q, k, v, s, bs, K)
+    gate = np.exp(s_row - scipy.special.logsumexp(s_row))
+    sel = _brute_select(s_row, C, K)
+    for i in (C * bs, C * bs + 17, n - 1):
+        cur = i - C * bs + 1
+        denom = bs * gate[sel].sum() + cur
+        for m in range(C):
+            want = bs * gate[m] / denom if m in sel else 0.0
+            assert abs(o[0, i, 0, m] - want) < 1e-13
+        assert abs(o[0, i, 0, C] - cur / denom) < 1e-13
+        assert abs(lse[0, 0, i] - np.log(denom)) < 1e-13
+
+
+# --------------------------------------------------------------------------
+# selection: brute force, ties, signed zeros, degenerate budgets
+# --------------------------------------------------------------------------
+
+def test_select_brute_force_with_ties():
+    rng = np.random.default_rng(1)
+    rows, L = 300, 70
+    s = rng.standard_normal((rows, L)).astype(np.float32)
+    s[::3] = np.round(s[::3] * 2) / 2  # many exact ties
+    s[5, :] = 0.0
+    s[6, ::2] = -0.0  # signed zeros compare equal
+    s[7, :] = np.float32(1.25)
+    ncand = rng.integers(0, L + 1, size=rows).astype(np.int32)
+    ncand[:4] = [0, 1, L, 2]
+    for K in (0, 1, 4, 16, 69, 70, 100):
+        idx, lse = oracle.select(s, ncand, K, idx_cols=max(K, 1))
+        for r in range(rows):
+            c = int(ncand[r])
+            want = _brute_select([float(x) for x in s[r]], c, K)
+            got = [x for x in idx[r].tolist() if x >= 0][: max(K, 0)]
+            assert got == want, (r, K)
+            assert all(x == -1 for x in idx[r].tolist()[len(want):])
+            if c == 0:
+                assert lse[r] == -np.inf
+            else:
+                assert abs(lse[r] - scipy.special.logsumexp(s[r, :c].astype(np.float64))) < 1e-12
+
+
+def test_select_full_scope_keeps_all_history():
+    s = np.random.default_rng(2).standard_normal((1, 2, 9, 9))
+    idx, _ = oracle.select(s, np.arange(9)[None, None, :], 2, full_scope=True, idx_cols=9)
+    for c in range(9):
+        assert idx[0, 1, c].tolist() == list(range(c)) + [-1] * (9 - c)
+
+
+# --------------------------------------------------------------------------
+# forward / backward against torch (fp64) library routines
+# --------------------------------------------------------------------------
+
+def _dense_masked_torch(q, k, v, s, bs, K, sigma, full_scope=False, gate=True):
+    """Explicit dense formulation of Eq. 9 with torch: an n x n bias matrix holding
+    log_softmax(s) on the selected history blocks, 0 on the causal current block and
+    -inf elsewhere; softmax / matmul from torch.  Selection by brute force."""
+    B, n, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    Cq = n // bs
+    outs = []
+    for b in range(B):
+        heads = []
+        for hq in range(Hq):
+            h = hq // G
+            rows = []
+            for c in range(Cq):
+                bias = torch.full((bs, n), float("-inf"), dtype=torch.float64)
+                if c > 0:
+                    logg = torch.log_softmax(s[b, h, c, :c], dim=0)
+                    row = s[b, h, c, :c].detach().tolist()
+                    sel = list(range(c)) if full_scope else _brute_select(row, c, K)
+                    for m in sel:
+                        bias[:, m * bs:(m + 1) * bs] = (logg[m] if gate else 0.0)
+                causal = torch.full((bs, bs), float("-inf"), dtype=torch.float64).triu(1)
+                bias[:, c * bs:(c + 1) * bs] = causal
+                rows.append(bias)
+            bias = torch.cat(rows, 0)
+            z = sigma * q[b, :, hq] @ k[b, :, h].T + bias
+            p = torch.softmax(z, dim=-1)
+            heads.append((p @ v[b, :, h], torch.logsumexp(z, dim=-1)))
+        outs.append(heads)
+    o = torch.stack([torch.stack([hd[0] for hd in bh], 1) for bh in outs], 0)
+    lse = torch.stack([torch.stack([hd[1] for hd in bh], 0) for bh in outs], 0)
+    return o, lse
+
+
+@pytest.mark.parametrize("full_scope", [False, True])
+def test_gated_fwd_bwd_vs_torch_dense_mask(full_scope):
+    rng = np.random.default_rng(3)
+    B, n, Hq, Hkv, d, bs, K = 2, 64, 4, 2, 16, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    sigma = 1 / np.sqrt(d)
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K, full_scope=full_scope, sigma=sigma)
+    o_fwd, lse_fwd = oracle.attn_fwd(q, k, v, s, bs, K, full_scope=full_scope, sigma=sigma)
+    T = [torch.tensor(x, requires_grad=True) for x in (q, k, v, s)]
+    o_t, lse_t = _dense_masked_torch(*T, bs, K, sigma, full_scope=full_scope)
+    (o_t * torch.tensor(dO)).sum().backward()
+    np.testing.assert_allclose(o_fwd, o_t.detach().numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(out["o"], o_fwd, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse_fwd, lse_t.detach().numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(out["lse"], lse_fwd, atol=1e-12, rtol=0)
+    for name, t in zip(("dq", "dk", "dv", "ds"), T):
+        ref = t.grad.numpy()
+        np.testing.assert_allclose(out[name], ref, atol=1e-11, rtol=0, err_msg=name)
+
+
+def test_gate_off_budget_covering_history_is_dense_causal_attention():
+    rng = np.random.default_rng(4)
+    B, n, Hq, Hkv, d, bs = 1, 48, 6, 2, 8, 8
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    K = n // bs
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K, gate=False)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    G = Hq // Hkv
+    o_ref = torch.nn.functional.scaled_dot_product_attention(
+        tq.transpose(1, 2), tk.repeat_interleave(G, 2).transpose(1, 2), tv.repeat_interleave(G, 2).transpose(1, 2),
+        is_causal=True).transpose(1, 2)
+    (o_ref * torch.tensor(dO)).sum().backward()
+    np.testing.assert_allclose(out["o"], o_ref.detach().numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(out["dq"], tq.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(out["dk"], tk.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(out["dv"], tv.grad.numpy(), atol=1e-11, rtol=0)
+    assert np.all(out["ds"] == 0.0)
+
+
+def test_zero_budget_is_block_local_causal_attention():
+    rng = np.random.default_rng(5)
+    B, n, Hq, Hkv, d, bs = 1, 40, 2, 1, 8, 8
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    o, lse = oracle.attn_fwd(q, k, v, s, bs, 0)
+    blk = np.arange(n) // bs
+    mask = (blk[:, None] == blk[None, :]) & (np.arange(n)[:, None] >= np.arange(n)[None, :])
+    am = torch.where(torch.tensor(mask), 0.0, float("-inf")).double()
+    o_ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q).transpose(1, 2), torch.tensor(k).repeat_interleave(2, 2).transpose(1, 2),
+        torch.tensor(v).repeat_interleave(2, 2).transpose(1, 2), attn_mask=am).transpose(1, 2)
+    np.testing.assert_allclose(o, o_ref.numpy(), atol=1e-12, rtol=0)
+
+
+def test_sparse_scope_equals_full_scope_when_budget_covers_history():
+    rng = np.random.default_rng(6)
+    B, n, Hq, Hkv, d, bs = 1, 48, 4, 2, 8, 8
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    a = oracle.attn_bwd(q, k, v, dO, s, bs, n // bs, full_scope=False)
+    b = oracle.attn_bwd(q, k, v, dO, s, bs, 0, full_scope=True)
+    for key in ("o", "lse", "dq", "dk", "dv", "ds"):
+        np.testing.assert_array_equal(a[key], b[key])
+
+
+def test_score_shift_invariance():
+    """o depends on s only through log g = s - LSE(s): s -> s + c changes nothing."""
+    rng = np.random.default_rng(7)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 2, 1, 8, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    a = oracle.attn_bwd(q, k, v, dO, s, bs, K)
+    b = oracle.attn_bwd(q, k, v, dO, s + 3.75, bs, K)
+    for key in ("o", "lse", "dq", "dk", "dv", "ds"):
+        np.testing.assert_allclose(a[key], b[key], atol=1e-12, rtol=0, err_msg=key)
+
+
+# --------------------------------------------------------------------------
+# gradients: finite differences, Eq. 5, ds invariants
+# --------------------------------------------------------------------------
+
+def test_central_finite_differences():
+    rng = np.random.default_rng(8)
+    B, n, Hq, Hkv, d, bs, K = 1, 32, 2, 1, 4, 8, 2
+    q, k, v, _, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    Cq = n // bs
+    # scores with gaps of >= 0.05 so that a 1e-6 step never changes the selection
+    s = (rng.permutation(Cq * Cq).reshape(1, 1, Cq, Cq) * 0.05 + rng.uniform(0, 0.01, (1, 1, Cq, Cq)))
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K)
+    eps = 1e-6
+
+    def loss(q_, k_, v_, s_):
+        o, _ = oracle.attn_fwd(q_, k_, v_, s_, bs, K)
+        return float((o * dO).sum())
+
+    for name, arr, pos in (("dq", q, 0), ("dk", k, 1), ("dv", v, 2), ("ds", s, 3)):
+        grad = out[name]
+        flat_idx = rng.choice(arr.size, size=min(arr.size, 40), replace=False)
+        for fi in flat_idx:
+            ix = np.unravel_index(fi, arr.shape)
+            args_p = [q, k, v, s]
+            args_m = [q, k, v, s]
+            ap, am = arr.copy(), arr.copy()
+            ap[ix] += eps
+            am[ix] -= eps
+            args_p[pos], args_m[pos] = ap, am
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad[ix]) <= 1e-6 * max(1.0, abs(grad[ix])), (name, ix, fd, grad[ix])
+
+
+def test_inner_gate_gradient_identity_eq5():
+    """Eq. 5 of the pages (inner gate): dg_m = sum_{i in B_m} (p_i/g_m) do.(v_i - o),
+    i.e. d(log g)_m = sum_{i in B_m} p_i do.(v_i - o), summed over the query rows
+    sharing the score row.  Evaluated here from the forward outputs only."""
+    rng = np.random.default_rng(9)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 4, 2, 8, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    sigma = 1 / np.sqrt(d)
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K, sigma=sigma)
+    o, lse = oracle.attn_fwd(q, k, v, s, bs, K, sigma=sigma)
+    G, Cq = Hq // Hkv, n // bs
+    for h in range(Hkv):
+        for c in range(1, Cq):
+            row = s[0, h, c, :c]
+            logg = row - scipy.special.logsumexp(row)
+            sel = _brute_select(row.tolist(), c, K)
+            for m in range(c):
+                want = 0.0
+                if m in sel:
+                    for hq in range(h * G, (h + 1) * G):
+                        for i in range(c * bs, (c + 1) * bs):
+                            for j in range(m * bs, (m + 1) * bs):
+                                p = np.exp(sigma * q[0, i, hq] @ k[0, j, h] + logg[m] - lse[0, hq, i])
+                                want += p * dO[0, i, hq] @ (v[0, j, h] - o[0, i, hq])
+                assert abs(out["dlogg"][0, h, c, m] - want) < 1e-11
+
+
+def test_ds_rows_sum_to_zero_and_unselected_share_one_ratio():
+    """ds is the softmax VJP, so each row sums to zero; in sparse scope an
+    unselected block m gets ds_m = -g_m * sum(dlogg), one common sign and a
+    ratio ds_m/g_m shared by all unselected blocks (shibing624 review, Fig. 4)."""
+    rng = np.random.default_rng(10)
+    B, n, Hq, Hkv, d, bs, K = 1, 96, 2, 1, 8, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K)
+    ds = out["ds"][0, 0]
+    Cq = n // bs
+    for c in range(Cq):
+        assert abs(ds[c].sum()) < 1e-12
+        assert np.all(ds[c, c:] == 0.0)
+        if c > K:
+            row = s[0, 0, c, :c]
+            g = np.exp(row - scipy.special.logsumexp(row))
+            sel = set(_brute_select(row.tolist(), c, K))
+            ratios = [ds[c, m] / g[m] for m in range(c) if m not in sel]
+            np.testing.assert_allclose(ratios, ratios[0], rtol=1e-10, atol=0)
+
+
+def test_sampled_masks_match_full_run():
+    rng = np.random.default_rng(11)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 2, 2, 8, 8, 2
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    full = oracle.attn_bwd(q, k, v, dO, s, bs, K)
+    Cq = n // bs
+    idx, _ = oracle.train_select(s, K)
+    h, m = 1, 5
+    qmask = np.zeros((B, Hkv, Cq), dtype=bool)
+    kvmask = np.zeros((B, Hkv, Cq), dtype=bool)
+    kvmask[0, h, m] = True
+    qmask[0, h, m] = True
+    for c in range(m + 1, Cq):
+        if m in idx[0, h, c].tolist():
+            qmask[0, h, c] = True
+    part = oracle.attn_bwd(q, k, v, dO, s, bs, K, qmask=qmask, kvmask=kvmask)
+    sl = slice(m * bs, (m + 1) * bs)
+    np.testing.assert_array_equal(part["dk"][0, sl, h], full["dk"][0, sl, h])
+    np.testing.assert_array_equal(part["dv"][0, sl, h], full["dv"][0, sl, h])
+    np.testing.assert_array_equal(part["ds"][0, h, m], full["ds"][0, h, m])
+    bad = qmask.copy()
+    bad[0, h, m] = False
+    with pytest.raises(RuntimeError):
+        oracle.attn_bwd(q, k, v, dO, s, bs, K, qmask=bad, kvmask=kvmask)
+
+
+def test_bf16_and_f32_inputs_are_widened_exactly():
+    rng = np.random.default_rng(12)
+    B, n, Hq, Hkv, d, bs, K = 1, 32, 2, 1, 8, 8, 2
+    q, k, v, s, dO = (torch.tensor(x).to(torch.bfloat16) for x in _rand_train(rng, B, n, Hq, Hkv, d, bs))
+    bits = [x.view(torch.int16).numpy().view(np.uint16) for x in (q, k, v)]
+    wide = [x.double().numpy() for x in (q, k, v)]
+    s32 = s.float().numpy()
+    a = oracle.attn_fwd(*bits, s32, bs, K)
+    b = oracle.attn_fwd(*wide, s32.astype(np.float64), bs, K)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+# --------------------------------------------------------------------------
+# decode (jaehun.me review, walkthrough Step 6: Top-K without the gate)
+# --------------------------------------------------------------------------
+
+def _decode_torch(q, kc, vc, T, keys, sigma):
+    G = q.shape[1] // kc.shape[1]
+    B = q.shape[0]
+    outs = []
+    for b in range(B):
+        heads = []
+        for hq in range(q.shape[1]):
+            h = hq // G
+            kk = torch.tensor(kc[b, h, keys[b][h]])
+            vv = torch.tensor(vc[b, h, keys[b][h]])
+            p = torch.softmax(sigma * (kk @ torch.tensor(q[b, hq])), 0)
+            heads.append(p @ vv)
+        outs.append(torch.stack(heads))
+    return torch.stack(outs).numpy()
+
+
+def test_decode_sparse_and_dense():
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, d, bs, K, Tmax = 3, 4, 2, 16, 8, 3, 100
+    q = rng.standard_normal((B, Hq, d))
+    kc = rng.standard_normal((B, Hkv, Tmax, d)) * 0.5
+    vc = rng.standard_normal((B, Hkv, Tmax, d))
+    ctx = np.array([100, 41, 8], dtype=np.int32)  # current block of 4 tokens, 1 token, 8 tokens
+    s = rng.standard_normal((B, Hkv, Tmax // bs)).astype(np.float32)
+    sigma = 1 / np.sqrt(d)
+    o, idx = oracle.decode(q, kc, vc, ctx, s, bs, K)
+    keys = []
+    for b in range(B):
+        t = ctx[b] - 1
+        Cb = t // bs
+        kb = []
+        for h in range(Hkv):
+            sel = _brute_select(s[b, h, :Cb].tolist(), Cb, K)
+            assert [x for x in idx[b, h].tolist() if x >= 0] == sel
+            kb.append([j for m in sel for j in range(m * bs, (m + 1) * bs)] + list(range(Cb * bs, t + 1)))
+        keys.append(kb)
+    np.testing.assert_allclose(o, _decode_torch(q, kc, vc, ctx, keys, sigma), atol=1e-12, rtol=0)
+    od, _ = oracle.decode(q, kc, vc, ctx, None, bs, K, dense=True)
+    dense_keys = [[list(range(ctx[b])) for _ in range(Hkv)] for b in range(B)]
+    np.testing.assert_allclose(od, _decode_torch(q, kc, vc, ctx, dense_keys, sigma), atol=1e-12, rtol=0)
+    # a budget covering the whole history is dense attention
+    ob, _ = oracle.decode(q, kc, vc, ctx, s, bs, Tmax)
+    np.testing.assert_allclose(ob, od, atol=1e-12, rtol=0)

@@ -1,0 +1,20 @@
+"""SAS gated block-sparse attention for B200 (sm_100a).
+
+The compute lives in ``libsas.so`` (hand-written CUDA behind a C ABI declared in
+``include/sas.h``).  ``trainable_block_sparse_sas_b200.api`` is the thin ctypes
+binding with the same entry-point names; importing it loads the library and
+raises if it has not been built.  ``synthetic`` draws the seeded inputs.
+"""
+__all__ = ["api", "synthetic"]
+
+
+def __getattr__(name):
+    if name == "api":
+        from . import api
+
+        return api
+    if name == "synthetic":
+        from . import synthetic
+
+        return synthetic
+    raise AttributeError(name)
