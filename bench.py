@@ -1,0 +1,521 @@
+#!/usr/bin/env python
+"""Benchmark of the SAS gated block-sparse attention hot path on B200.
+
+One step = the whole training hot path over one batch of the 32K workload
+(B=1, Hq=32, Hkv=8, d=128, n=32768, block 64, Top-K 32, bf16): score LSE and
+Top-K selection, the gated forward, and the backward with dq/dk/dv and ds.
+The metric counts tensor-core FLOPs on selected blocks only (4d per attended
+(query, key) pair forward, 10d backward; the current block counts its causal
+b(b+1)/2 pairs).  Extras (single GPU): full-scope 16K training, and the two
+decode workloads (selection included) in GB/s of algorithmic bytes.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 the driver launches one rank per GPU with torchrun; every rank
+processes its own independent batch (no collective on the data path), the
+timing is the max over ranks, and `value` is the aggregate over all ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "gated sparse attn fwd+bwd TFLOP/s & decode selected-KV GB/s, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------
+# workload arithmetic (algorithmic work, independent of any implementation)
+# ----------------------------------------------------------------------------
+
+def train_pairs(w) -> int:
+    """Attended (query row, key) pairs of a training workload, over all heads."""
+    hist = sum((c if w.full_scope else min(c, w.top_k)) for c in range(w.Cq))
+    per_head = hist * w.bs * w.bs + w.Cq * w.bs * (w.bs + 1) // 2
+    return w.B * w.Hq * per_head
+
+
+def train_flops(w) -> dict:
+    pairs = train_pairs(w)
+    return {"pairs": pairs, "fwd": 4 * w.d * pairs, "bwd": 10 * w.d * pairs, "total": 14 * w.d * pairs}
+
+
+def decode_bytes(w, dense: bool = False) -> int:
+    """Algorithmic HBM bytes of one decode step: attended K and V rows, the score
+    rows (sparse only), q and o."""
+    t = w.T - 1
+    cur = t - (t // w.bs) * w.bs + 1
+    toks = (t + 1) if dense else (min(w.top_k, w.C) * w.bs + cur)
+    kv = w.B * w.Hkv * toks * w.d * 2 * 2
+    s = 0 if dense else w.B * w.Hkv * w.C * 4
+    qo = 2 * w.B * w.Hq * w.d * 2
+    return kv + s + qo
+
+
+def load_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sources_sha(names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "trainable_block_sparse_sas_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(call: str):
+    """DRAM bytes per launch of an ABI call from a committed ncu summary, if the
+    kernel sources it was taken on are unchanged (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(call)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    if kernel_sources_sha(rec["sources"]) != rec["sources_sha"]:
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [ln.strip().split(",") for ln in self.out.read().splitlines() if ln.strip()]
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def visible_gpu_id(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ----------------------------------------------------------------------------
+# oracle on the host cores (CPU baseline and the reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(w, inp_host: dict, tokens: int):
+    """The oracle's fwd + bwd on the first `tokens` tokens of KV head 0 (its
+    query-head group): a complete sub-problem of the workload, since attention is
+    causal and KV heads are independent.  Returns (seconds, FLOPs, threads)."""
+    import oracle
+
+    G = w.Hq // w.Hkv
+    sub = dataclasses.replace(w, B=1, Hq=G, Hkv=1, n=tokens)
+    q = inp_host["q"][:1, :tokens, :G]
+    k = inp_host["k"][:1, :tokens, :1]
+    v = inp_host["v"][:1, :tokens, :1]
+    dO = inp_host["dO"][:1, :tokens, :G]
+    Cq = tokens // w.bs
+    s = inp_host["s"][:1, :1, :Cq, :Cq]
+    import numpy as np
+
+    q, k, v, dO, s = (np.ascontiguousarray(x) for x in (q, k, v, dO, s))
+    t0 = time.perf_counter()
+    oracle.train_select(s, w.top_k, full_scope=w.full_scope)
+    oracle.attn_fwd(q, k, v, s, w.bs, w.top_k, full_scope=w.full_scope)
+    oracle.attn_bwd(q, k, v, dO, s, w.bs, w.top_k, full_scope=w.full_scope)
+    dt = time.perf_counter() - t0
+    return dt, train_flops(sub)["total"], oracle.num_threads()
+
+
+def host_bits(t):
+    import numpy as np
+    import torch
+
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def run_reference(args, rank: int):
+    """The reference arm: the fp64 oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return
+    import torch
+
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    w = syn.WORKLOADS[args.workload]
+    import oracle
+
+    oracle.build()
+    tokens = args.reference_tokens
+    inp = syn.train_inputs(dataclasses.replace(w, n=tokens, B=1), device="cpu", seed=1000)
+    host = {k: host_bits(v) for k, v in inp.items()}
+    times = []
+    flops = 0
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        dt, flops, threads = oracle_sample(w, host, tokens)
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    sample = (f"first {tokens} tokens of KV head 0 ({w.Hq // w.Hkv} query heads) of {w.name}: "
+              f"select + fwd + bwd per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    del torch
+
+
+def workload_config(w, n_gpus: int) -> dict:
+    return {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d, "seq_len": w.n,
+            "block_size": w.bs, "top_k": w.top_k, "scope": "full" if w.full_scope else "sparse",
+            "parallelism": f"replicas x{n_gpus} (independent batches, no collective)",
+            "l2": "inputs larger than L2 (q and dO 268 MB each, k and v 67 MB each)"}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+class TrainRunner:
+    """Preallocated buffers and the three ABI calls of one training step."""
+
+    def __init__(self, api, w, inp):
+        import torch
+
+        self.api, self.w = api, w
+        self.inp = inp
+        q, k = inp["q"], inp["k"]
+        dev = q.device
+        self.desc = api.attn_desc(q, k, w.bs, w.top_k, w.full_scope)
+        self.lse_s = torch.empty((w.B, w.Hkv, w.Cq), dtype=torch.float32, device=dev)
+        self.idx = None if (w.full_scope or w.top_k == 0) else torch.empty(
+            (w.B, w.Hkv, w.Cq, w.top_k), dtype=torch.int32, device=dev)
+        self.o = torch.empty_like(q)
+        self.lse = torch.empty((w.B, w.Hq, w.n), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(inp["v"])
+        self.ds = torch.empty_like(inp["s"])
+        self.ws = api.workspace(api.sas_gated_attn_bwd_workspace_size(self.desc), dev)
+
+    def step(self, ev=None):
+        api, i = self.api, self.inp
+        if ev:
+            ev[0].record()
+        api.sas_topk_select(i["s"], self.w.Cq, self.w.Cq, self.w.top_k, idx=self.idx, lse_s=self.lse_s)
+        if ev:
+            ev[1].record()
+        api.sas_gated_attn_fwd(self.desc, i["q"], i["k"], i["v"], i["s"], self.lse_s, self.idx, self.o, self.lse)
+        if ev:
+            ev[2].record()
+        api.sas_gated_attn_bwd(self.desc, i["q"], i["k"], i["v"], self.o, self.lse, i["dO"], i["s"], self.lse_s,
+                               self.idx, self.dq, self.dk, self.dv, self.ds, self.ws)
+        if ev:
+            ev[3].record()
+
+    def outputs(self):
+        return {"o": self.o, "dq": self.dq, "dk": self.dk, "dv": self.dv, "ds": self.ds}
+
+
+def time_decode(api, w, steps: int, dense: bool = False):
+    """Median device time of select + decode (or the dense decode) with L2
+    flushed before every repetition."""
+    import torch
+
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    inp = syn.decode_inputs(w, device="cuda", seed=3000)
+    q, kc, vc, ctx, s = (inp[x] for x in ("q", "k_cache", "v_cache", "ctx_len", "s"))
+    desc = api.decode_desc(q, kc, w.bs, w.top_k)
+    idx = torch.empty((w.B, w.Hkv, w.top_k), dtype=torch.int32, device="cuda")
+    o = torch.empty_like(q)
+    ws = api.workspace(api.sas_sparse_decode_workspace_size(desc), q.device)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    s4 = s.view(w.B, w.Hkv, 1, -1)
+
+    def run():
+        if not dense:
+            api.sas_topk_select(s4, 1, s.shape[-1], w.top_k, idx=idx, ctx_len=ctx, block_size=w.bs)
+        api.sas_sparse_decode(desc, q, kc, vc, ctx, None if dense else idx, o, ws)
+
+    for _ in range(3):
+        run()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        run()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    del inp, kc, vc, flush
+    torch.cuda.empty_cache()
+    return statistics.median(times)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from trainable_block_sparse_sas_b200 import api
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = syn.WORKLOADS[args.workload]
+    inp = syn.train_inputs(w, device=dev, seed=1000 + rank)
+    runner = TrainRunner(api, w, inp)
+    fl = train_flops(w)
+    peaks, peak_kind = load_peaks()
+
+    def barrier():
+        if world > 1:
+            t = torch.ones(1, device=dev)
+            dist.all_reduce(t)
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        runner.step()
+    barrier()
+    clocks = ClockSampler(visible_gpu_id(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = api.sas_launch_count()
+    barrier()
+    start.record()
+    for i in range(args.steps):
+        runner.step(evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    launches = api.sas_launch_count() - launches0
+    barrier()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    per_call = {
+        "sas_topk_select": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+        "sas_gated_attn_fwd": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
+        "sas_gated_attn_bwd": statistics.mean(e[2].elapsed_time(e[3]) for e in evs),
+    }
+    value = world * fl["total"] * args.steps / (ms_max * 1e-3) / 1e12
+
+    # end to end through host buffers: pinned inputs copied in, outputs copied out
+    e2e_steps = max(1, min(args.steps, 5))
+    host_in = {k: v.cpu().pin_memory() for k, v in inp.items()}
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in runner.outputs().items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        for k_, v_ in host_in.items():
+            inp[k_].copy_(v_, non_blocking=True)
+        runner.step()
+        for k_, v_ in runner.outputs().items():
+            host_out[k_].copy_(v_, non_blocking=True)
+    b.record()
+    torch.cuda.synchronize()
+    t = torch.tensor([a.elapsed_time(b)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = world * fl["total"] * e2e_steps / (float(t.item()) * 1e-3) / 1e12
+    del host_in, host_out
+
+    if rank != 0:
+        barrier()
+        return
+    dom = max(per_call, key=per_call.get)
+    dom_flops = {"sas_topk_select": 0, "sas_gated_attn_fwd": fl["fwd"], "sas_gated_attn_bwd": fl["bwd"]}[dom]
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    achieved = dom_flops / (per_call[dom] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w, world),
+        "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(dom),
+                     "peak_source": f"{peak_kind} bf16 sustained", "per_call_ms": per_call,
+                     "flops_per_step": fl},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        host = {k: host_bits(v) for k, v in inp.items()}
+        dt, flops, threads = oracle_sample(w, host, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                "sample": f"first {args.cpu_tokens} tokens of KV head 0 (4 query heads): select + "
+                                          f"fwd + bwd, {dt:.1f} s"}
+    del runner, inp
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extra:
+        line["extra"] = extras(api, args, peaks, peak_kind)
+    print(json.dumps(line), flush=True)
+    barrier()
+
+
+def extras(api, args, peaks, peak_kind) -> dict:
+    import torch
+
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    out = {}
+    # full-scope training
+    w = syn.TRAIN_FULL_16K
+    inp = syn.train_inputs(w, device="cuda", seed=1500)
+    r = TrainRunner(api, w, inp)
+    for _ in range(2):
+        r.step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(2, min(args.steps, 5))
+    a.record()
+    for _ in range(n):
+        r.step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    fl = train_flops(w)
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    out[w.name] = {"ms_per_step": ms, "tflops": fl["total"] / (ms * 1e-3) / 1e12,
+                   "frac_of_bf16_peak": fl["total"] / (ms * 1e-3) / 1e12 / peak}
+    del r, inp
+    torch.cuda.empty_cache()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    for w in (syn.DECODE_128K, syn.DECODE_512K):
+        ms = time_decode(api, w, steps=20)
+        by = decode_bytes(w)
+        gbs = by / (ms * 1e-3) / 1e9
+        rec = {"ms": ms, "bytes": by, "gbs": gbs, "frac_of_hbm": gbs / hbm, "hbm_peak_gbs": hbm,
+               "peak_source": f"{peak_kind} copy", "l2": "flushed (512 MB write) before every repetition",
+               "includes": "Top-K selection + sparse decode"}
+        if w is syn.DECODE_512K:
+            msd = time_decode(api, w, steps=5, dense=True)
+            byd = decode_bytes(w, dense=True)
+            rec["dense_ms"] = msd
+            rec["dense_gbs"] = byd / (msd * 1e-3) / 1e9
+            rec["sparse_over_dense_speedup"] = msd / ms
+        out[w.name] = rec
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="train_sparse_32k")
+    ap.add_argument("--no-extra", action="store_true", help="skip the full-scope and decode extras")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=4096, help="tokens of the oracle's CPU-baseline sample")
+    ap.add_argument("--reference-tokens", type=int, default=1024, help="tokens of the reference arm's sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,197 @@
+/*
+ * sas.h -- C ABI of libsas, SAS gated block-sparse attention on B200 (sm_100a).
+ *
+ * The method ("SAS: Simple Attention Sparsification via End-to-End Optimization of
+ * Context Ranking"): a selector scores the b-token history blocks of each query
+ * block; g = softmax(s) over those history blocks; the hard Top-K of s plus the
+ * current block B_0 (gate 1, causal) is attended with the log-gate added to the
+ * logits, o = softmax(q K_S^T + log g_S) V_S.  Training carries the gradient back
+ * to s through log g = s - LSE(s); inference drops the gate and attends the Top-K
+ * blocks only.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates or frees memory.  Scratch ("workspace") is caller-owned, sized by
+ *     the matching *_workspace_size query and must be 256-byte aligned.
+ *   - Every call is asynchronous on the caller's stream; no implicit
+ *     synchronisation.  Calls are thread-safe and re-entrant.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns an error code and has no side effect.  Launch failures
+ *     return SAS_ERR_CUDA.  Nothing aborts, traps or throws across the ABI.
+ *   - Layouts are row-major with the last index contiguous:
+ *       training  q, o, dO, dq : [B, n, Hq, d]     k, v, dk, dv : [B, n, Hkv, d]
+ *                 s, ds        : [B, Hkv, Cq, Cq]  (Cq = n / b; row c scores the
+ *                                                   history blocks m < c)
+ *                 idx          : [B, Hkv, Cq, K]   int32, ascending, -1 padded
+ *                 lse_s        : [B, Hkv, Cq]      fp32, LSE of row c over m < c
+ *                 lse          : [B, Hq, n]        fp32, natural log, incl. gate
+ *       decode    q, o         : [B, Hq, d]        caches : [B, Hkv, Tmax, d]
+ *                 s            : [B, Hkv, s_cols]  idx    : [B, Hkv, K]
+ *   - Query head hq reads KV head hq / (Hq / Hkv) (grouped-query attention); the
+ *     heads of one group share one score row and one selection.
+ *   - The softmax scale is softmax_scale if > 0, else 1/sqrt(d).
+ *   - Preconditions the library cannot check cheaply (undefined results, never a
+ *     memory fault): scores are finite; idx rows were produced by
+ *     sas_topk_select (ascending, in range, -1 padded).
+ */
+#ifndef SAS_H_
+#define SAS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* sas_stream_t;
+
+typedef enum {
+    SAS_OK = 0,
+    SAS_ERR_INVALID_VALUE = 1,       /* null pointer, bad shape, inconsistent sizes */
+    SAS_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. head_dim) */
+    SAS_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_size query */
+    SAS_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
+    SAS_ERR_DEVICE_TIMEOUT = 5       /* a bounded device-side wait gave up */
+} sas_status;
+
+typedef enum { SAS_F32 = 0, SAS_BF16 = 1 } sas_dtype;
+typedef enum { SAS_SCOPE_SPARSE = 0, SAS_SCOPE_FULL = 1 } sas_scope;
+
+/* Training-shape problem.  Sparse scope attends the Top-K history blocks of each
+ * query block plus the current block; full scope attends every history block,
+ * all gated (the "training scope" design choice of the pages, shibing624 review
+ * Fig. 2(d); jaehun.me review, "Why the Four Design Choices Matter"). */
+typedef struct {
+    int32_t batch, n_q_heads, n_kv_heads, head_dim;
+    int32_t seq_len;    /* n, a multiple of block_size */
+    int32_t block_size; /* b */
+    int32_t top_k;      /* K (ignored in full scope) */
+    int32_t scope;      /* sas_scope */
+    int32_t dtype;      /* sas_dtype of q, k, v, o, dO, dq, dk, dv */
+    float softmax_scale;
+} sas_attn_desc;
+
+/* Decode-shape problem: one new token per sequence; ctx_len[b] counts the cached
+ * tokens including the new one, so the query sits at t = ctx_len[b] - 1, its
+ * current (partial) block is [C_b * b, t] and C_b = floor(t / b) full history
+ * blocks precede it. */
+typedef struct {
+    int32_t batch, n_q_heads, n_kv_heads, head_dim;
+    int32_t block_size;
+    int32_t top_k;
+    int32_t max_ctx; /* Tmax, the cache's token capacity per (sequence, kv head) */
+    int32_t dtype;   /* sas_dtype of q, caches and o */
+    float softmax_scale;
+} sas_decode_desc;
+
+/*
+ * sas_topk_select -- the gate normaliser and the hard Top-K of the scores.
+ *   Pages: log g_m = s_m - LSE(s) (jaehun.me review, section 4.2.2, "Gate
+ *   activation"); S = Top-K(s, K) over the history blocks (jaehun.me review,
+ *   Background Eq. 3; walkthrough Step 3), with the threshold selection of the
+ *   training kernel (shibing624 review, method section, last paragraph).
+ *   Ties go to the lower block index; -0.0 and +0.0 are equal.
+ * s        [batch, n_kv_heads, n_rows, row_len] fp32.
+ * ctx_len  NULL: training rows, row r has min(r, row_len) candidates (blocks
+ *          0..r-1).  Non-NULL (device int32 [batch]): decode rows, n_rows must
+ *          be 1 and row (b, h) has min(floor((ctx_len[b]-1)/block_size), row_len)
+ *          candidates.
+ * idx      [batch, n_kv_heads, n_rows, top_k] int32 out: the min(K, candidates)
+ *          chosen blocks ascending, then -1.  May be NULL (only lse_s wanted, as
+ *          in full scope); top_k must then still be >= 0.
+ * lse_s    [batch, n_kv_heads, n_rows] fp32 out, LSE over the candidates (-inf
+ *          for a row without candidates).  May be NULL.
+ * Errors: SAS_ERR_INVALID_VALUE for non-positive sizes, top_k < 0, s == NULL,
+ *         both outputs NULL, n_rows != 1 with ctx_len, block_size <= 0 with
+ *         ctx_len.
+ */
+sas_status sas_topk_select(const float* s, int32_t batch, int32_t n_kv_heads, int32_t n_rows, int32_t row_len,
+                           const int32_t* ctx_len, int32_t block_size, int32_t top_k, int32_t* idx, float* lse_s,
+                           sas_stream_t stream);
+
+/*
+ * sas_gated_attn_fwd -- o = softmax(sigma q K_S^T + log g_S) V_S for every query
+ *   row (shibing624 review, SAS equation; jaehun.me review, Eq. 9 and the
+ *   Kernel implementation paragraph).  Selected history block m of query block c
+ *   adds log g_m = s[b,h,c,m] - lse_s[b,h,c] to the logits of its b tokens; the
+ *   current block adds 0 and is causally masked; unselected blocks are skipped.
+ * q, k, v  bf16 or fp32 per desc->dtype; s [B,Hkv,Cq,Cq] fp32; lse_s [B,Hkv,Cq]
+ *          fp32 (from sas_topk_select); idx [B,Hkv,Cq,K] (sparse scope; NULL in
+ *          full scope).
+ * o        out, same dtype and layout as q.   lse out [B,Hq,n] fp32.
+ * Errors: SAS_ERR_INVALID_VALUE (null pointers, seq_len % block_size != 0,
+ *         n_q_heads % n_kv_heads != 0, sizes <= 0, top_k < 0, idx NULL in
+ *         sparse scope with top_k > 0); SAS_ERR_UNSUPPORTED (head_dim not 64 or
+ *         128, block_size not in {16, 32, 64}).
+ */
+sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
+                              const float* s, const float* lse_s, const int32_t* idx, void* o, float* lse,
+                              sas_stream_t stream);
+
+/* Bytes of workspace sas_gated_attn_bwd needs for this problem (0 on bad desc). */
+size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc);
+
+/*
+ * sas_gated_attn_bwd -- gradients of a loss L through the forward above, given
+ *   dO = dL/do: dq, dk, dv and the selector-score gradient ds.  The log-gate
+ *   gradient of a selected block is the sum of the logit gradients of its tokens
+ *   over the query rows and heads sharing the score row (jaehun.me review,
+ *   Kernel implementation paragraph; inner-gate gradient, section 4.2.2 Eq. 5),
+ *   carried to s through log g = s - LSE(s):
+ *     ds[b,h,c,m] = dlogg_m - g_m * sum_{m'<c} dlogg_{m'}  (m < c), 0 (m >= c),
+ *   so unselected blocks receive gradient only through the normaliser (jaehun.me
+ *   review, "Training scope"; shibing624 review, Fig. 4).
+ * o, lse   the forward's outputs.   dq, dk, dv out (dtype of q), ds out fp32.
+ * workspace, ws_bytes  caller scratch of at least the queried size.
+ * Errors: as sas_gated_attn_fwd, plus SAS_ERR_WORKSPACE_TOO_SMALL.
+ */
+sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
+                              const void* o, const float* lse, const void* dO, const float* s, const float* lse_s,
+                              const int32_t* idx, void* dq, void* dk, void* dv, float* ds, void* workspace,
+                              size_t ws_bytes, sas_stream_t stream);
+
+/* Bytes of workspace sas_sparse_decode needs for this problem (0 on bad desc). */
+size_t sas_sparse_decode_workspace_size(const sas_decode_desc* desc);
+
+/*
+ * sas_sparse_decode -- inference attention of one new token per sequence over
+ *   its Top-K history blocks plus its current partial block, with no gate
+ *   (jaehun.me review, walkthrough Step 6; shibing624 review, method section:
+ *   at inference the gate is dropped and plain hard Top-K remains).
+ *   o = softmax(sigma q K_S^T) V_S.
+ * q        [B,Hq,d]; k_cache, v_cache [B,Hkv,max_ctx,d]; ctx_len device int32 [B]
+ *          (1 <= ctx_len[b] <= max_ctx); idx [B,Hkv,top_k] from sas_topk_select in
+ *          decode mode, or NULL for dense attention over all ctx_len[b] tokens
+ *          (the full-attention comparator).
+ * o        out [B,Hq,d], dtype of q.
+ * Errors: SAS_ERR_INVALID_VALUE (null pointers, sizes <= 0, heads not divisible,
+ *         top_k < 0); SAS_ERR_UNSUPPORTED (head_dim != 128 for bf16 / not 64 or
+ *         128 for fp32, block_size not a multiple of 16 up to 256);
+ *         SAS_ERR_WORKSPACE_TOO_SMALL.
+ */
+sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* ctx_len, const int32_t* idx, void* o, void* workspace, size_t ws_bytes,
+                             sas_stream_t stream);
+
+/* Synchronises `stream`, then reports and clears the device-side status word that
+ * bounded waits inside the kernels set when they give up: SAS_OK or
+ * SAS_ERR_DEVICE_TIMEOUT (SAS_ERR_CUDA if the synchronisation itself fails). */
+sas_status sas_device_status(sas_stream_t stream);
+
+/* Number of kernels this library has launched in this process (all devices),
+ * counted on the host at each successful launch. */
+uint64_t sas_launch_count(void);
+
+/* Static English text for a status code. */
+const char* sas_status_string(sas_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t sas_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAS_H_ */

@@ -1,0 +1,135 @@
+"""Host-only checks of the C ABI: the library builds, loads and exports every
+symbol include/sas.h declares; arguments are rejected with the documented
+status before any device work; the CUDA library and the oracle are independent.
+No test here launches a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sas.h")
+PKG = os.path.join(ROOT, "trainable_block_sparse_sas_b200")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:sas_status|size_t|const char\s*\*|int32_t|uint64_t)\s+(sas_\w+)\s*\(", text,
+                                 flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def api():
+    from trainable_block_sparse_sas_b200 import build
+
+    build.build()
+    from trainable_block_sparse_sas_b200 import api as a
+
+    return a
+
+
+def test_header_declares_the_hot_path_entry_points():
+    names = _declared()
+    for want in ("sas_topk_select", "sas_gated_attn_fwd", "sas_gated_attn_bwd", "sas_sparse_decode"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(api):
+    lib = ctypes.CDLL(api._LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", api._LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (sas_\w+)$", out, flags=re.M))
+    assert set(_declared()) <= exported
+
+
+def test_status_strings(api):
+    for st in range(6):
+        assert api.lib.sas_status_string(st)
+    assert api.lib.sas_version() >= 100
+
+
+def _desc(api, **kw):
+    base = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, seq_len=256, block_size=64, top_k=2, scope=0,
+                dtype=1, softmax_scale=0.0)
+    base.update(kw)
+    return api.AttnDesc(**base)
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every case below fails validation first
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(batch=0), 1), (dict(n_q_heads=3), 1), (dict(seq_len=100), 1), (dict(top_k=-1), 1),
+    (dict(scope=7), 1), (dict(dtype=5), 1), (dict(head_dim=96), 2), (dict(block_size=48, seq_len=96), 2), (dict(block_size=128), 2),
+])
+def test_fwd_rejects_bad_descriptors(api, kw, status):
+    d = _desc(api, **kw)
+    st = api.lib.sas_gated_attn_fwd(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None)
+    assert st == status
+
+
+def test_fwd_rejects_null_pointers(api):
+    d = _desc(api)
+    args = [FAKE] * 8
+    for i in range(8):
+        a = list(args)
+        a[i] = None
+        if i == 5:  # idx
+            continue
+        assert api.lib.sas_gated_attn_fwd(ctypes.byref(d), *a, None) == 1, i
+    a = list(args)
+    a[5] = None  # idx missing in sparse scope with top_k > 0
+    assert api.lib.sas_gated_attn_fwd(ctypes.byref(d), *a, None) == 1
+
+
+def test_bwd_checks_workspace(api):
+    d = _desc(api)
+    need = api.lib.sas_gated_attn_bwd_workspace_size(ctypes.byref(d))
+    assert need > 0 and need % 256 == 0
+    args = [FAKE] * 13
+    st = api.lib.sas_gated_attn_bwd(ctypes.byref(d), *args, FAKE, need - 1, None)
+    assert st == 3
+    assert api.lib.sas_gated_attn_bwd_workspace_size(None) == 0
+    bad = _desc(api, seq_len=100)
+    assert api.lib.sas_gated_attn_bwd_workspace_size(ctypes.byref(bad)) == 0
+
+
+def test_decode_checks(api):
+    d = api.DecodeDesc(2, 8, 2, 128, 64, 4, 1000, 1, 0.0)
+    need = api.lib.sas_sparse_decode_workspace_size(ctypes.byref(d))
+    assert need > 0 and need % 256 == 0
+    st = api.lib.sas_sparse_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None)
+    assert st == 3
+    st = api.lib.sas_sparse_decode(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None)
+    assert st == 1
+    bad = api.DecodeDesc(2, 8, 3, 128, 64, 4, 1000, 1, 0.0)
+    assert api.lib.sas_sparse_decode(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 1
+    uns = api.DecodeDesc(2, 8, 2, 96, 64, 4, 1000, 1, 0.0)
+    assert api.lib.sas_sparse_decode(ctypes.byref(uns), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 2
+
+
+def test_select_checks(api):
+    L = api.lib
+    assert L.sas_topk_select(None, 1, 1, 4, 4, None, 0, 2, FAKE, FAKE, None) == 1
+    assert L.sas_topk_select(FAKE, 1, 1, 4, 4, None, 0, -1, FAKE, FAKE, None) == 1
+    assert L.sas_topk_select(FAKE, 1, 1, 4, 4, None, 0, 2, None, None, None) == 1
+    assert L.sas_topk_select(FAKE, 1, 1, 2, 4, FAKE, 64, 2, FAKE, None, None) == 1  # decode rows need n_rows 1
+    assert L.sas_topk_select(FAKE, 1, 1, 1, 4, FAKE, 0, 2, FAKE, None, None) == 1   # decode rows need block_size
+
+
+def test_cuda_library_and_oracle_share_nothing(api):
+    """The product path never imports, loads or links the oracle, and the oracle
+    never includes the library's headers or sources."""
+    for dirpath, _, files in os.walk(PKG):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
+                assert "sas_oracle" not in text and "liboracle" not in text, f
+    oracle_src = open(os.path.join(ROOT, "oracle", "sas_oracle.c")).read()
+    assert "#include \"" not in oracle_src and "sas.h" not in oracle_src
+    deps = subprocess.run(["ldd", api._LIB_PATH], capture_output=True, text=True).stdout
+    assert "oracle" not in deps

@@ -1,0 +1,303 @@
+"""GPU parity of the CUDA path (called through the C ABI) against the fp64 oracle.
+
+Selection is compared bit for bit; floating-point outputs within the stated
+tolerances (bf16: relative L2 <= 1e-2 and max |err| <= 3e-2; fp32: both <= 1e-4).
+Full-size workloads run exactly as the benchmark runs them; the oracle then
+checks sampled query blocks / key blocks of chosen KV heads (KV heads are
+independent, so a head slice is an exact sub-problem)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import BF16_TOL, F32_TOL, bits, compare, host, run_train
+from trainable_block_sparse_sas_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api(cuda_ok):
+    from trainable_block_sparse_sas_b200 import api as a
+
+    return a
+
+
+def _seeded(shape, std, dtype, seed, device="cuda"):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return (torch.randn(shape, generator=g) * std).to(dtype).to(device)
+
+
+# --------------------------------------------------------------------------
+# selection
+# --------------------------------------------------------------------------
+
+def _check_select(api, s, top_k, ctx_len=None, bs=0):
+    B, Hkv, R, L = s.shape
+    idx = torch.empty((B, Hkv, R, top_k), dtype=torch.int32, device="cuda")
+    lse = torch.empty((B, Hkv, R), dtype=torch.float32, device="cuda")
+    api.sas_topk_select(s, R, L, top_k, idx=idx, lse_s=lse, ctx_len=ctx_len, block_size=bs)
+    torch.cuda.synchronize()
+    if ctx_len is None:
+        ncand = np.broadcast_to(np.minimum(np.arange(R), L)[None, None, :], (B, Hkv, R))
+    else:
+        c = np.minimum((ctx_len.cpu().numpy() - 1) // bs, L)
+        ncand = np.broadcast_to(c[:, None, None], (B, Hkv, R))
+    want_idx, want_lse = oracle.select(bits(s), ncand, top_k, idx_cols=top_k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    got = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(want_lse)
+    assert np.array_equal(np.isfinite(got), fin)
+    compare("lse_s", got[fin], want_lse[fin], **F32_TOL)
+
+
+def test_select_training_rows_bit_exact(api):
+    s = _seeded((1, 8, 512, 512), 2.0, torch.float32, 11)
+    _check_select(api, s, 32)
+
+
+def test_select_ties_and_signed_zeros(api):
+    s = _seeded((2, 3, 300, 300), 1.0, torch.float32, 12)
+    s = torch.round(s * 2) / 2  # many exact ties
+    s[0, 0] = 0.0
+    s[0, 1, :, ::2] = -0.0
+    s[1, 2] = 0.75
+    for k in (1, 7, 64, 299, 300, 400):
+        _check_select(api, s.contiguous(), k)
+
+
+def test_select_decode_rows_bit_exact(api):
+    for B, Hkv, C, K, T in ((16, 8, 2048, 16, 131073), (4, 8, 8192, 32, 524289)):
+        s = _seeded((B, Hkv, 1, C), 1.0, torch.float32, 13)
+        ctx = torch.full((B,), T, dtype=torch.int32, device="cuda")
+        _check_select(api, s, K, ctx_len=ctx, bs=64)
+    s = _seeded((5, 2, 1, 40), 1.0, torch.float32, 14)
+    ctx = torch.tensor([1, 64, 65, 200, 2560], dtype=torch.int32, device="cuda")  # 0, 0, 1, 3, 39 history blocks
+    _check_select(api, s, 4, ctx_len=ctx, bs=64)
+
+
+# --------------------------------------------------------------------------
+# training-shape forward + backward, whole problems
+# --------------------------------------------------------------------------
+
+def _oracle_train(inp, bs, top_k, full_scope):
+    return oracle.attn_bwd(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]), bits(inp["dO"]), bits(inp["s"]), bs,
+                           top_k, full_scope=full_scope)
+
+
+def _compare_train(got, want, tol, idx_want=None):
+    if idx_want is not None and got["idx"] is not None:
+        np.testing.assert_array_equal(got["idx"].cpu().numpy(), idx_want)
+    b16 = got["o"].dtype == torch.bfloat16
+    compare("o", host(got["o"]), want["o"], **tol, bf16_out=b16)
+    compare("lse", host(got["lse"]), want["lse"], **tol)
+    for key in ("dq", "dk", "dv"):
+        compare(key, host(got[key]), want[key], **tol, bf16_out=b16)
+    compare("ds", host(got["ds"]), want["ds"], **tol)
+
+
+def test_tiny_fp32_workload(api):
+    """The 1-KV-head fp32 workload (d=64, n=512, b=16, Top-K 4): every output at 1e-4."""
+    w = syn.TINY_FP32
+    inp = syn.train_inputs(w, device="cuda", seed=1000)
+    got = run_train(api, inp, w.bs, w.top_k, w.full_scope)
+    want = _oracle_train(inp, w.bs, w.top_k, w.full_scope)
+    idx_want, _ = oracle.train_select(bits(inp["s"]), w.top_k)
+    _compare_train(got, want, F32_TOL, idx_want)
+
+
+@pytest.mark.parametrize("B,n,Hq,Hkv,d,bs,K,full", [
+    (2, 512, 4, 1, 128, 64, 3, False),   # GQA 4, rows with c < K
+    (1, 384, 5, 1, 64, 32, 4, False),    # GQA 5
+    (1, 256, 2, 2, 128, 16, 5, False),   # no GQA, small blocks
+    (1, 512, 8, 2, 128, 32, 6, False),   # GQA 4 over 2 KV heads, 32-token blocks
+    (1, 512, 4, 2, 128, 64, 0, True),    # full scope
+    (1, 256, 4, 2, 64, 64, 0, False),    # K = 0: current block only
+    (1, 1024, 4, 1, 128, 64, 40, False), # K >= C: sparse == full
+])
+def test_bf16_shapes(api, B, n, Hq, Hkv, d, bs, K, full):
+    Cq = n // bs
+    inp = {
+        "q": _seeded((B, n, Hq, d), 1.0, torch.bfloat16, 21),
+        "k": _seeded((B, n, Hkv, d), 1.0, torch.bfloat16, 22),
+        "v": _seeded((B, n, Hkv, d), 1.0, torch.bfloat16, 23),
+        "s": _seeded((B, Hkv, Cq, Cq), 2.0, torch.float32, 24),
+        "dO": _seeded((B, n, Hq, d), 1.0, torch.bfloat16, 25),
+    }
+    got = run_train(api, inp, bs, K, full)
+    want = _oracle_train(inp, bs, K, full)
+    idx_want = None if (full or K == 0) else oracle.train_select(bits(inp["s"]), K)[0]
+    _compare_train(got, want, BF16_TOL, idx_want)
+
+
+def test_unsupported_block_size_is_refused(api):
+    q = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((1, 256, 1, 128), dtype=torch.bfloat16, device="cuda")
+    s = torch.zeros((1, 1, 2, 2), dtype=torch.float32, device="cuda")
+    desc = api.attn_desc(q, k, 128, 1)
+    lse_s = torch.zeros((1, 1, 2), device="cuda")
+    idx = torch.zeros((1, 1, 2, 1), dtype=torch.int32, device="cuda")
+    o, lse = torch.empty_like(q), torch.empty((1, 2, 256), device="cuda")
+    with pytest.raises(api.SasError) as e:
+        api.sas_gated_attn_fwd(desc, q, k, k, s, lse_s, idx, o, lse)
+    assert e.value.status == api.SAS_ERR_UNSUPPORTED
+
+
+def test_fp32_shape_with_gqa(api):
+    B, n, Hq, Hkv, d, bs, K = 1, 256, 4, 2, 128, 32, 3
+    Cq = n // bs
+    inp = {
+        "q": _seeded((B, n, Hq, d), 0.3, torch.float32, 31),
+        "k": _seeded((B, n, Hkv, d), 0.3, torch.float32, 32),
+        "v": _seeded((B, n, Hkv, d), 1.0, torch.float32, 33),
+        "s": _seeded((B, Hkv, Cq, Cq), 1.0, torch.float32, 34),
+        "dO": _seeded((B, n, Hq, d), 1.0, torch.float32, 35),
+    }
+    got = run_train(api, inp, bs, K, False)
+    want = _oracle_train(inp, bs, K, False)
+    _compare_train(got, want, F32_TOL)
+
+
+def test_autograd_wrapper_matches_entry_points(api):
+    w = syn.TINY_FP32
+    inp = syn.train_inputs(w, device="cuda", seed=1001)
+    direct = run_train(api, inp, w.bs, w.top_k, w.full_scope)
+    q, k, v, s = (inp[x].clone().requires_grad_(True) for x in ("q", "k", "v", "s"))
+    o = api.sas_attention(q, k, v, s, w.bs, w.top_k)
+    o.backward(inp["dO"])
+    torch.cuda.synchronize()
+    for a, b in ((o, direct["o"]), (q.grad, direct["dq"]), (k.grad, direct["dk"]), (v.grad, direct["dv"]),
+                 (s.grad, direct["ds"])):
+        assert torch.equal(a, b)
+
+
+# --------------------------------------------------------------------------
+# full-size training workloads, sampled
+# --------------------------------------------------------------------------
+
+def _slice_inputs(inp, h, G):
+    sl = slice(h * G, (h + 1) * G)
+    return {
+        "q": bits(inp["q"][:, :, sl]), "k": bits(inp["k"][:, :, h:h + 1]), "v": bits(inp["v"][:, :, h:h + 1]),
+        "dO": bits(inp["dO"][:, :, sl]), "s": bits(inp["s"][:, h:h + 1]),
+    }
+
+
+def _sampled_full_size(api, w, q_blocks, kv_blocks, heads):
+    inp = syn.train_inputs(w, device="cuda", seed=2000)
+    got = run_train(api, inp, w.bs, w.top_k, w.full_scope)
+    G, Cq, bs = w.Hq // w.Hkv, w.Cq, w.bs
+    for h in heads:
+        si = _slice_inputs(inp, h, G)
+        sel = None
+        if not w.full_scope:
+            sel, _ = oracle.train_select(si["s"], w.top_k)
+            np.testing.assert_array_equal(got["idx"][:, h:h + 1].cpu().numpy(), sel)
+        qmask = np.zeros((1, 1, Cq), dtype=bool)
+        kvmask = np.zeros((1, 1, Cq), dtype=bool)
+        qmask[0, 0, list(q_blocks)] = True
+        for m in kv_blocks:
+            kvmask[0, 0, m] = True
+            qmask[0, 0, m] = True
+            for c in range(m + 1, Cq):
+                if w.full_scope or m in sel[0, 0, c].tolist():
+                    qmask[0, 0, c] = True
+        want = oracle.attn_bwd(si["q"], si["k"], si["v"], si["dO"], si["s"], bs, w.top_k, full_scope=w.full_scope,
+                               qmask=qmask, kvmask=kvmask)
+        rows = np.concatenate([np.arange(c * bs, (c + 1) * bs) for c in q_blocks])
+        hs = slice(h * G, (h + 1) * G)
+        compare(f"o[h{h}]", host(got["o"][:, rows, hs]), want["o"][:, rows], **BF16_TOL, bf16_out=True)
+        compare(f"lse[h{h}]", host(got["lse"][:, hs][:, :, rows]), want["lse"][:, :, rows], **BF16_TOL)
+        compare(f"dq[h{h}]", host(got["dq"][:, rows, hs]), want["dq"][:, rows], **BF16_TOL, bf16_out=True)
+        compare(f"ds[h{h}]", host(got["ds"][:, h, list(q_blocks)]), want["ds"][:, 0, list(q_blocks)], **BF16_TOL)
+        krows = np.concatenate([np.arange(m * bs, (m + 1) * bs) for m in kv_blocks])
+        compare(f"dk[h{h}]", host(got["dk"][:, krows, h]), want["dk"][:, krows, 0], **BF16_TOL, bf16_out=True)
+        compare(f"dv[h{h}]", host(got["dv"][:, krows, h]), want["dv"][:, krows, 0], **BF16_TOL, bf16_out=True)
+
+
+def test_train_sparse_32k_sampled(api):
+    w = syn.TRAIN_SPARSE_32K
+    _sampled_full_size(api, w, q_blocks=(0, 1, 31, 32, 33, 257, 511), kv_blocks=(511, 480, 350), heads=(0, 5))
+
+
+def test_train_full_16k_sampled(api):
+    w = syn.TRAIN_FULL_16K
+    _sampled_full_size(api, w, q_blocks=(0, 1, 100, 255), kv_blocks=(255, 250), heads=(3,))
+
+
+# --------------------------------------------------------------------------
+# decode
+# --------------------------------------------------------------------------
+
+def _run_decode(api, inp, bs, top_k, dense=False):
+    q, kc, vc, ctx, s = (inp[x] for x in ("q", "k_cache", "v_cache", "ctx_len", "s"))
+    B, Hkv = kc.shape[0], kc.shape[1]
+    desc = api.decode_desc(q, kc, bs, top_k)
+    idx = None
+    if not dense:
+        idx = torch.empty((B, Hkv, top_k), dtype=torch.int32, device="cuda")
+        api.sas_topk_select(s.view(B, Hkv, 1, -1), 1, s.shape[-1], top_k, idx=idx, ctx_len=ctx, block_size=bs)
+    o = torch.empty_like(q)
+    ws = api.workspace(api.sas_sparse_decode_workspace_size(desc), q.device)
+    api.sas_sparse_decode(desc, q, kc, vc, ctx, idx, o, ws)
+    torch.cuda.synchronize()
+    return o, idx
+
+
+def _oracle_decode_rows(inp, rows, bs, top_k, dense):
+    """Oracle on (b, h) rows one at a time (caches sliced on the device first)."""
+    G = inp["q"].shape[1] // inp["k_cache"].shape[1]
+    outs = {}
+    for b, h in rows:
+        T = int(inp["ctx_len"][b])
+        q = bits(inp["q"][b:b + 1, h * G:(h + 1) * G])
+        kc = bits(inp["k_cache"][b:b + 1, h:h + 1, :T])
+        vc = bits(inp["v_cache"][b:b + 1, h:h + 1, :T])
+        s = bits(inp["s"][b:b + 1, h:h + 1])
+        o, idx = oracle.decode(q, kc, vc, np.array([T], np.int32), s, bs, top_k, dense=dense)
+        outs[(b, h)] = (o[0], idx[0, 0])
+    return outs
+
+
+@pytest.mark.parametrize("w", [syn.DECODE_128K, syn.DECODE_512K], ids=lambda w: w.name)
+def test_decode_full_size_sampled(api, w):
+    inp = syn.decode_inputs(w, device="cuda", seed=3000)
+    o, idx = _run_decode(api, inp, w.bs, w.top_k)
+    ncand = np.full((w.B, w.Hkv), w.C, dtype=np.int32)
+    want_idx, _ = oracle.select(bits(inp["s"]), ncand, w.top_k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    G = w.Hq // w.Hkv
+    rows = [(0, 0), (w.B - 1, w.Hkv - 1), (w.B // 2, 3)]
+    ref = _oracle_decode_rows(inp, rows, w.bs, w.top_k, dense=False)
+    for (b, h), (ro, _) in ref.items():
+        compare(f"decode o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+    if w is syn.DECODE_512K:
+        od, _ = _run_decode(api, inp, w.bs, w.top_k, dense=True)
+        refd = _oracle_decode_rows(inp, rows[:2], w.bs, w.top_k, dense=True)
+        for (b, h), (ro, _) in refd.items():
+            compare(f"dense o[{b},{h}]", host(od[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64), (torch.float32, 128)])
+def test_decode_edge_cases(api, dtype, d):
+    B, Hq, Hkv, bs, K, Tmax = 7, 10, 2, 64, 3, 1100
+    ctx = torch.tensor([1, 2, 64, 65, 129, 300, 1100], dtype=torch.int32, device="cuda")
+    inp = {
+        "q": _seeded((B, Hq, d), 1.0, dtype, 41),
+        "k_cache": _seeded((B, Hkv, Tmax, d), 1.0, dtype, 42),
+        "v_cache": _seeded((B, Hkv, Tmax, d), 1.0, dtype, 43),
+        "ctx_len": ctx,
+        "s": _seeded((B, Hkv, Tmax // bs), 1.0, torch.float32, 44),
+    }
+    tol = BF16_TOL if dtype == torch.bfloat16 else F32_TOL
+    G = Hq // Hkv
+    rows = [(b, h) for b in range(B) for h in range(Hkv)]
+    for dense in (False, True):
+        o, idx = _run_decode(api, inp, bs, K, dense=dense)
+        ref = _oracle_decode_rows(inp, rows, bs, K, dense)
+        for (b, h), (ro, ridx) in ref.items():
+            if not dense:
+                np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx)
+            compare(f"o[{b},{h}] dense={dense}", host(o[b, h * G:(h + 1) * G]), ro, **tol,
+                    bf16_out=dtype == torch.bfloat16)

@@ -416,3 +416,16 @@ def test_decode_sparse_and_dense():
     # a budget covering the whole history is dense attention
     ob, _ = oracle.decode(q, kc, vc, ctx, s, bs, Tmax)
     np.testing.assert_allclose(ob, od, atol=1e-12, rtol=0)
+
+
+def test_bf16_half_ulp_allowance():
+    """The comparison allowance is exactly the worst-case rounding of x to bf16."""
+    import torch
+    from parity import bf16_half_ulp
+
+    x = (np.random.default_rng(14).standard_normal(100000)
+         * np.exp2(np.random.default_rng(15).integers(-10, 10, 100000))).astype(np.float32)
+    r = torch.tensor(x).to(torch.bfloat16).double().numpy()  # one rounding, fp32 -> bf16
+    x = x.astype(np.float64)
+    assert np.all(np.abs(r - x) <= bf16_half_ulp(x) * (1 + 1e-12))
+    assert np.max(np.abs(r - x) / bf16_half_ulp(x)) > 0.99

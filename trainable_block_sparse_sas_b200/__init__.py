@@ -5,16 +5,12 @@ The compute lives in ``libsas.so`` (hand-written CUDA behind a C ABI declared in
 binding with the same entry-point names; importing it loads the library and
 raises if it has not been built.  ``synthetic`` draws the seeded inputs.
 """
+import importlib
+
 __all__ = ["api", "synthetic"]
 
 
 def __getattr__(name):
-    if name == "api":
-        from . import api
-
-        return api
-    if name == "synthetic":
-        from . import synthetic
-
-        return synthetic
+    if name in __all__:
+        return importlib.import_module(f"{__name__}.{name}")
     raise AttributeError(name)

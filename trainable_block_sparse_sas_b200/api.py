@@ -1,0 +1,201 @@
+"""Thin Python binding of libsas (include/sas.h).
+
+Argument marshalling only: each function passes torch tensors' device pointers
+and the current CUDA stream to the C entry point of the same name, and raises
+``SasError`` on a non-zero status.  Every step of the computation runs in the
+library's CUDA kernels; there is no fallback.  Importing this module loads
+``libsas.so`` and fails loudly if it has not been built
+(``python -m trainable_block_sparse_sas_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libsas.so not built at {_LIB_PATH}: run python -m trainable_block_sparse_sas_b200.build")
+lib = ctypes.CDLL(_LIB_PATH)
+
+SAS_OK, SAS_ERR_INVALID_VALUE, SAS_ERR_UNSUPPORTED, SAS_ERR_WORKSPACE_TOO_SMALL, SAS_ERR_CUDA, \
+    SAS_ERR_DEVICE_TIMEOUT = range(6)
+SAS_F32, SAS_BF16 = 0, 1
+SAS_SCOPE_SPARSE, SAS_SCOPE_FULL = 0, 1
+
+
+class SasError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lib.sas_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+        self.status = status
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("scope", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+class DecodeDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("max_ctx", ctypes.c_int32), ("dtype", ctypes.c_int32), ("softmax_scale", ctypes.c_float)]
+
+
+_vp, _i32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+lib.sas_status_string.restype = ctypes.c_char_p
+lib.sas_status_string.argtypes = [ctypes.c_int]
+lib.sas_version.restype = ctypes.c_int32
+lib.sas_topk_select.restype = ctypes.c_int
+lib.sas_topk_select.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _vp, _vp]
+lib.sas_gated_attn_fwd.restype = ctypes.c_int
+lib.sas_gated_attn_fwd.argtypes = [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.sas_gated_attn_bwd_workspace_size.restype = _sz
+lib.sas_gated_attn_bwd_workspace_size.argtypes = [ctypes.POINTER(AttnDesc)]
+lib.sas_gated_attn_bwd.restype = ctypes.c_int
+lib.sas_gated_attn_bwd.argtypes = [ctypes.POINTER(AttnDesc)] + [_vp] * 14 + [_sz, _vp]
+lib.sas_sparse_decode_workspace_size.restype = _sz
+lib.sas_sparse_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeDesc)]
+lib.sas_sparse_decode.restype = ctypes.c_int
+lib.sas_sparse_decode.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7 + [_sz, _vp]
+lib.sas_launch_count.restype = ctypes.c_uint64
+lib.sas_launch_count.argtypes = []
+lib.sas_device_status.restype = ctypes.c_int
+lib.sas_device_status.argtypes = [_vp]
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != SAS_OK:
+        raise SasError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SAS_BF16
+    if t.dtype == torch.float32:
+        return SAS_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def attn_desc(q, k, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0) -> AttnDesc:
+    B, n, Hq, d = q.shape
+    return AttnDesc(B, Hq, k.shape[2], d, n, block_size, top_k, SAS_SCOPE_FULL if full_scope else SAS_SCOPE_SPARSE,
+                    _dtype_code(q), softmax_scale)
+
+
+def decode_desc(q, k_cache, block_size: int, top_k: int, softmax_scale: float = 0.0) -> DecodeDesc:
+    B, Hq, d = q.shape
+    return DecodeDesc(B, Hq, k_cache.shape[1], d, block_size, top_k, k_cache.shape[2], _dtype_code(q), softmax_scale)
+
+
+def sas_topk_select(s, n_rows, row_len, top_k, idx=None, lse_s=None, ctx_len=None, block_size=0, stream=None):
+    """s [B, Hkv, n_rows, row_len] fp32 -> writes idx [B,Hkv,n_rows,top_k] int32 and/or lse_s."""
+    B, Hkv = s.shape[0], s.shape[1]
+    st = lib.sas_topk_select(_p(s), B, Hkv, n_rows, row_len, _p(ctx_len), block_size, top_k, _p(idx), _p(lse_s),
+                             _stream(stream))
+    _check(st, "sas_topk_select")
+
+
+def sas_gated_attn_fwd(desc, q, k, v, s, lse_s, idx, o, lse, stream=None):
+    _check(lib.sas_gated_attn_fwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(s), _p(lse_s), _p(idx), _p(o), _p(lse),
+                                  _stream(stream)), "sas_gated_attn_fwd")
+
+
+def sas_gated_attn_bwd_workspace_size(desc) -> int:
+    return int(lib.sas_gated_attn_bwd_workspace_size(ctypes.byref(desc)))
+
+
+def sas_gated_attn_bwd(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, workspace, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.sas_gated_attn_bwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dO), _p(s), _p(lse_s),
+                                  _p(idx), _p(dq), _p(dk), _p(dv), _p(ds), _p(workspace), ws_bytes, _stream(stream)),
+           "sas_gated_attn_bwd")
+
+
+def sas_sparse_decode_workspace_size(desc) -> int:
+    return int(lib.sas_sparse_decode_workspace_size(ctypes.byref(desc)))
+
+
+def sas_sparse_decode(desc, q, k_cache, v_cache, ctx_len, idx, o, workspace, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.sas_sparse_decode(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx), _p(o),
+                                 _p(workspace), ws_bytes, _stream(stream)), "sas_sparse_decode")
+
+
+def sas_device_status(stream=None):
+    _check(lib.sas_device_status(_stream(stream)), "sas_device_status")
+
+
+def sas_launch_count() -> int:
+    """Kernels launched by libsas so far in this process."""
+    return int(lib.sas_launch_count())
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """Caller-owned scratch from torch's allocator (256-byte aligned)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------
+# convenience: one training-shape call sequence, and an autograd Function
+# ---------------------------------------------------------------------------
+
+def select_train(s, block_size: int, top_k: int, full_scope: bool = False, stream=None):
+    """Score rows of a training problem -> (idx or None, lse_s)."""
+    B, Hkv, Cq, _ = s.shape
+    lse_s = torch.empty((B, Hkv, Cq), dtype=torch.float32, device=s.device)
+    idx = None
+    if not full_scope and top_k > 0:
+        idx = torch.empty((B, Hkv, Cq, top_k), dtype=torch.int32, device=s.device)
+    sas_topk_select(s, Cq, Cq, top_k, idx=idx, lse_s=lse_s, stream=stream)
+    return idx, lse_s
+
+
+class _SASAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, s, block_size, top_k, full_scope, softmax_scale):
+        q, k, v, s = (t.contiguous() for t in (q, k, v, s))
+        desc = attn_desc(q, k, block_size, top_k, full_scope, softmax_scale)
+        idx, lse_s = select_train(s, block_size, top_k, full_scope)
+        o = torch.empty_like(q)
+        lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=q.device)
+        sas_gated_attn_fwd(desc, q, k, v, s, lse_s, idx, o, lse)
+        ctx.save_for_backward(q, k, v, s, o, lse, lse_s, idx if idx is not None else torch.empty(0))
+        ctx.desc = desc
+        ctx.has_idx = idx is not None
+        return o
+
+    @staticmethod
+    def backward(ctx, dO):
+        q, k, v, s, o, lse, lse_s, idx = ctx.saved_tensors
+        idx = idx if ctx.has_idx else None
+        dO = dO.contiguous()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ds = torch.empty_like(s)
+        ws = workspace(sas_gated_attn_bwd_workspace_size(ctx.desc), q.device)
+        sas_gated_attn_bwd(ctx.desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, ws)
+        return dq, dk, dv, ds, None, None, None, None
+
+
+def sas_attention(q, k, v, s, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0):
+    """Differentiable SAS gated attention: o = softmax(sigma q K_S^T + log g_S) V_S.
+
+    q [B,n,Hq,d], k/v [B,n,Hkv,d] (bf16 or fp32), s [B,Hkv,n/b,n/b] fp32."""
+    return _SASAttention.apply(q, k, v, s, block_size, top_k, full_scope, softmax_scale)
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

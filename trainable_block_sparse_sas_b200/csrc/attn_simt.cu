@@ -1,0 +1,581 @@
+// attn_simt.cu -- CUDA-core (FFMA) gated block-sparse attention, forward and
+// backward, for fp32 problems (where tensor cores cannot meet fp32 accuracy) and
+// for any shape the tensor-core kernels do not cover.
+//
+// Forward (jaehun.me review of SAS, Eq. 9 and the Kernel implementation
+// paragraph): one CTA per (batch, query head, query block c) streams the
+// attended key blocks -- the selected history blocks of c, ascending, each with
+// the log-gate bias log g_m = s[c,m] - lse_s[c], then the current block c with
+// bias 0 and a causal mask -- through shared memory with an online softmax.
+//
+// Backward, without atomics and therefore deterministic:
+//   bwd_rowdot   D_i = dO_i . o_i
+//   bwd_dq       one CTA per (batch, kv head, query block c), looping over the
+//                group's query heads: recomputes P from the saved lse, dS =
+//                P (dP - D), dq = sigma dS K, and the block-wise log-gate gradient
+//                dlogg[c,m] = sum of dS over the tile (jaehun.me review, Kernel
+//                implementation paragraph), then ds[c,:] = dlogg - g sum(dlogg).
+//   bwd_dkdv     one CTA per (batch, kv head, key block m), looping over the query
+//                blocks that attend m (m itself, and every c > m whose selection
+//                holds m) and the group's heads: dv = P^T dO, dk = sigma dS^T Q.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sas {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <int D, int BS>
+struct Cfg {
+    static constexpr int RG = BS / 4;         // 4-row groups of an S tile
+    static constexpr int NT_S = RG * RG;      // 4x4 micro-tiles of an S tile
+    static constexpr int CG = kThreads / RG;  // column groups of an O-like tile
+    static constexpr int COLS = D / CG;       // columns per thread of an O-like tile
+    static constexpr int LD = D + 1;          // padded row stride of [BS][D] tiles
+    static constexpr int LDS = BS + 1;        // padded row stride of [BS][BS] tiles
+    static_assert(BS % 4 == 0 && kThreads % RG == 0 && D % CG == 0, "tile mapping");
+};
+
+template <typename T>
+__device__ __forceinline__ float ldg(const void* p, long i) {
+    return to_f32<T>(static_cast<const T*>(p)[i]);
+}
+
+template <typename T>
+__device__ __forceinline__ void stg(void* p, long i, float v) {
+    static_cast<T*>(p)[i] = from_f32<T>(v);
+}
+
+// rows [BS] of head `head` (of `H` heads) starting at token t0 -> smem [BS][LD]
+template <typename T, int D, int BS>
+__device__ __forceinline__ void load_rows(float* dst, const void* src, int b, int n, int H, int head, int t0) {
+    using C = Cfg<D, BS>;
+    for (int i = threadIdx.x; i < BS * D; i += kThreads) {
+        const int r = i / D, e = i % D;
+        dst[r * C::LD + e] = ldg<T>(src, (((long)b * n + t0 + r) * H + head) * D + e);
+    }
+}
+
+// The attended history blocks of query block c, ascending, into blocks[]; the
+// current block is appended at blocks[count].  Entries of idx outside [0, c) are
+// dropped so that a malformed list cannot send a load out of range.
+__device__ __forceinline__ int build_list(const TrainParams& p, long unit, int c, int* blocks) {
+    __shared__ int cnt_sh;
+    if (p.full_scope) {
+        for (int i = threadIdx.x; i < c; i += kThreads) blocks[i] = i;
+        if (threadIdx.x == 0) {
+            blocks[c] = c;
+            cnt_sh = c;
+        }
+    } else if (threadIdx.x == 0) {
+        const int kk = min(p.top_k, c);
+        const int32_t* row = p.idx + unit * p.top_k;
+        int cnt = 0;
+        for (int i = 0; i < kk; ++i) {
+            const int v = row[i];
+            if (v >= 0 && v < c) blocks[cnt++] = v;
+        }
+        blocks[cnt] = c;
+        cnt_sh = cnt;
+    }
+    __syncthreads();
+    return cnt_sh;
+}
+
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
+    using C = Cfg<D, BS>;
+    extern __shared__ float smem[];
+    float* Qs = smem;
+    float* Ks = Qs + BS * C::LD;
+    float* Vs = Ks + BS * C::LD;
+    float* Ss = Vs + BS * C::LD;
+    float* row_m = Ss + BS * C::LDS;
+    float* row_l = row_m + BS;
+    float* row_a = row_l + BS;
+    int* blocks = reinterpret_cast<int*>(row_a + BS);
+
+    const int tid = threadIdx.x;
+    const int c = p.Cq - 1 - (int)(blockIdx.x % p.Cq);  // late (long) query blocks first
+    const int hq = (int)((blockIdx.x / p.Cq) % p.Hq);
+    const int b = (int)(blockIdx.x / ((long)p.Cq * p.Hq));
+    const int G = p.Hq / p.Hkv, h = hq / G;
+    const long unit = ((long)b * p.Hkv + h) * p.Cq + c;
+    const int nsel = build_list(p, unit, c, blocks);
+    const float* srow = p.s + unit * p.Cq;
+    const float lse_c = p.lse_s[unit];
+
+    load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
+    if (tid < BS) {
+        row_m[tid] = -INFINITY;
+        row_l[tid] = 0.f;
+    }
+    const int tr = tid / C::CG, tc = tid % C::CG;
+    float acc[4][C::COLS];
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int ee = 0; ee < C::COLS; ++ee) acc[ii][ee] = 0.f;
+
+    for (int t = 0; t <= nsel; ++t) {
+        const int blk = blocks[t];
+        const bool cur = (t == nsel);
+        const float bias = cur ? 0.f : (srow[blk] - lse_c);
+        __syncthreads();
+        load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
+        load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
+        __syncthreads();
+        for (int tile = tid; tile < C::NT_S; tile += kThreads) {
+            const int ttr = tile / C::RG, ttc = tile % C::RG;
+            float sacc[4][4] = {};
+            for (int e = 0; e < D; ++e) {
+                float qv[4], kv[4];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) qv[ii] = Qs[(ttr + C::RG * ii) * C::LD + e];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) kv[jj] = Ks[(ttc + C::RG * jj) * C::LD + e];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) sacc[ii][jj] = fmaf(qv[ii], kv[jj], sacc[ii][jj]);
+            }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int r = ttr + C::RG * ii, j = ttc + C::RG * jj;
+                    float z = fmaf(p.scale, sacc[ii][jj], bias);
+                    if (cur && j > r) z = -INFINITY;
+                    Ss[r * C::LDS + j] = z;
+                }
+        }
+        __syncthreads();
+        if (tid < BS) {
+            float* srow_s = Ss + tid * C::LDS;
+            float mx = row_m[tid];
+            for (int j = 0; j < BS; ++j) mx = fmaxf(mx, srow_s[j]);
+            const float alpha = expf(row_m[tid] - mx);
+            float sum = 0.f;
+            for (int j = 0; j < BS; ++j) {
+                const float pv = expf(srow_s[j] - mx);
+                srow_s[j] = pv;
+                sum += pv;
+            }
+            row_l[tid] = row_l[tid] * alpha + sum;
+            row_m[tid] = mx;
+            row_a[tid] = alpha;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            const float a = row_a[tr + C::RG * ii];
+#pragma unroll
+            for (int ee = 0; ee < C::COLS; ++ee) acc[ii][ee] *= a;
+        }
+        for (int j = 0; j < BS; ++j) {
+            float pv[4];
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) pv[ii] = Ss[(tr + C::RG * ii) * C::LDS + j];
+#pragma unroll
+            for (int ee = 0; ee < C::COLS; ++ee) {
+                const float vv = Vs[j * C::LD + tc + C::CG * ee];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) acc[ii][ee] = fmaf(pv[ii], vv, acc[ii][ee]);
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii) {
+        const int r = tr + C::RG * ii;
+        const float inv = 1.f / row_l[r];
+        const long base = (((long)b * p.n + c * BS + r) * p.Hq + hq) * D;
+#pragma unroll
+        for (int ee = 0; ee < C::COLS; ++ee) stg<T>(p.o, base + tc + C::CG * ee, acc[ii][ee] * inv);
+    }
+    if (tid < BS) p.lse[((long)b * p.Hq + hq) * p.n + c * BS + tid] = row_m[tid] + logf(row_l[tid]);
+}
+
+// D_i = dO_i . o_i, one warp per row.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) bwd_rowdot_kernel(TrainParams p) {
+    const long rows = (long)p.B * p.n * p.Hq;
+    const long row = (long)blockIdx.x * (kThreads / 32) + threadIdx.x / 32;
+    if (row >= rows) return;
+    const int lane = threadIdx.x & 31;
+    float acc = 0.f;
+    for (int e = lane; e < p.d; e += 32) acc += ldg<T>(p.dO, row * p.d + e) * ldg<T>(p.o_in, row * p.d + e);
+    acc = warp_sum(acc);
+    if (lane == 0) {
+        const int hq = (int)(row % p.Hq);
+        const long bi = row / p.Hq;  // b * n + i
+        const int b = (int)(bi / p.n), i = (int)(bi % p.n);
+        p.Dbuf[((long)b * p.Hq + hq) * p.n + i] = acc;
+    }
+}
+
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
+    using C = Cfg<D, BS>;
+    extern __shared__ float smem[];
+    float* Qs = smem;
+    float* dOs = Qs + BS * C::LD;
+    float* Ks = dOs + BS * C::LD;
+    float* Vs = Ks + BS * C::LD;
+    float* Ss = Vs + BS * C::LD;  // dS tile
+    float* rowL = Ss + BS * C::LDS;
+    float* rowD = rowL + BS;
+    float* red = rowD + BS;  // 33
+    float* dlg = red + 33;   // [Cq]
+    int* blocks = reinterpret_cast<int*>(dlg + p.Cq);
+
+    const int tid = threadIdx.x;
+    const int c = p.Cq - 1 - (int)(blockIdx.x % p.Cq);
+    const int h = (int)((blockIdx.x / p.Cq) % p.Hkv);
+    const int b = (int)(blockIdx.x / ((long)p.Cq * p.Hkv));
+    const int G = p.Hq / p.Hkv;
+    const long unit = ((long)b * p.Hkv + h) * p.Cq + c;
+    const int nsel = build_list(p, unit, c, blocks);
+    const float* srow = p.s + unit * p.Cq;
+    const float lse_c = p.lse_s[unit];
+    for (int i = tid; i < nsel; i += kThreads) dlg[i] = 0.f;
+    const int tr = tid / C::CG, tc = tid % C::CG;
+
+    for (int g = 0; g < G; ++g) {
+        const int hq = h * G + g;
+        __syncthreads();
+        load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
+        load_rows<T, D, BS>(dOs, p.dO, b, p.n, p.Hq, hq, c * BS);
+        if (tid < BS) {
+            const long ri = ((long)b * p.Hq + hq) * p.n + c * BS + tid;
+            rowL[tid] = p.lse_in[ri];
+            rowD[tid] = p.Dbuf[ri];
+        }
+        float acc[4][C::COLS];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int ee = 0; ee < C::COLS; ++ee) acc[ii][ee] = 0.f;
+
+        for (int t = 0; t <= nsel; ++t) {
+            const int blk = blocks[t];
+            const bool cur = (t == nsel);
+            const float bias = cur ? 0.f : (srow[blk] - lse_c);
+            __syncthreads();
+            load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
+            load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
+            __syncthreads();
+            float local = 0.f;
+            for (int tile = tid; tile < C::NT_S; tile += kThreads) {
+                const int ttr = tile / C::RG, ttc = tile % C::RG;
+                float sacc[4][4] = {}, pacc[4][4] = {};
+                for (int e = 0; e < D; ++e) {
+                    float qv[4], gv[4], kv[4], vv[4];
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii) {
+                        qv[ii] = Qs[(ttr + C::RG * ii) * C::LD + e];
+                        gv[ii] = dOs[(ttr + C::RG * ii) * C::LD + e];
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        kv[jj] = Ks[(ttc + C::RG * jj) * C::LD + e];
+                        vv[jj] = Vs[(ttc + C::RG * jj) * C::LD + e];
+                    }
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            sacc[ii][jj] = fmaf(qv[ii], kv[jj], sacc[ii][jj]);
+                            pacc[ii][jj] = fmaf(gv[ii], vv[jj], pacc[ii][jj]);
+                        }
+                }
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int r = ttr + C::RG * ii, j = ttc + C::RG * jj;
+                        const float z = fmaf(p.scale, sacc[ii][jj], bias);
+                        const float pr = (cur && j > r) ? 0.f : expf(z - rowL[r]);
+                        const float dS = pr * (pacc[ii][jj] - rowD[r]);
+                        Ss[r * C::LDS + j] = dS;
+                        local += dS;
+                    }
+            }
+            if (!cur) {
+                const float tot = block_sum(local, red);
+                if (tid == 0) dlg[t] += tot;
+            }
+            __syncthreads();
+            for (int j = 0; j < BS; ++j) {
+                float sv[4];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) sv[ii] = Ss[(tr + C::RG * ii) * C::LDS + j];
+#pragma unroll
+                for (int ee = 0; ee < C::COLS; ++ee) {
+                    const float kv = Ks[j * C::LD + tc + C::CG * ee];
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii) acc[ii][ee] = fmaf(sv[ii], kv, acc[ii][ee]);
+                }
+            }
+        }
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            const int r = tr + C::RG * ii;
+            const long base = (((long)b * p.n + c * BS + r) * p.Hq + hq) * D;
+#pragma unroll
+            for (int ee = 0; ee < C::COLS; ++ee) stg<T>(p.dq, base + tc + C::CG * ee, p.scale * acc[ii][ee]);
+        }
+    }
+    __syncthreads();
+    // ds[c, m] = dlogg_m - g_m * sum(dlogg) for m < c, 0 for m >= c
+    float part = 0.f;
+    for (int i = tid; i < nsel; i += kThreads) part += dlg[i];
+    const float tot = block_sum(part, red);
+    float* dsrow = p.ds + unit * p.Cq;
+    for (int m = tid; m < p.Cq; m += kThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
+    __syncthreads();
+    for (int i = tid; i < nsel; i += kThreads) dsrow[blocks[i]] += dlg[i];
+}
+
+// is history block m in the (ascending) selection of query block c?
+__device__ __forceinline__ bool selected(const TrainParams& p, long unit_c, int c, int m) {
+    if (p.full_scope) return m < c;
+    int lo = 0, hi = min(p.top_k, c) - 1;
+    const int32_t* row = p.idx + unit_c * p.top_k;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int v = row[mid];
+        if (v == m) return true;
+        if (v >= 0 && v < m) lo = mid + 1;
+        else hi = mid - 1;
+    }
+    return false;
+}
+
+template <typename T, int D, int BS>
+__global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
+    using C = Cfg<D, BS>;
+    extern __shared__ float smem[];
+    float* Ks = smem;
+    float* Vs = Ks + BS * C::LD;
+    float* Qs = Vs + BS * C::LD;
+    float* dOs = Qs + BS * C::LD;
+    float* Ps = dOs + BS * C::LD;
+    float* dSs = Ps + BS * C::LDS;
+    float* rowL = dSs + BS * C::LDS;
+    float* rowD = rowL + BS;
+    int* clist = reinterpret_cast<int*>(rowD + BS);  // [kThreads]
+    int* scan = clist + kThreads;                    // [33]
+
+    const int tid = threadIdx.x;
+    const int m = (int)(blockIdx.x % p.Cq);  // early (heavily selected) key blocks first
+    const int h = (int)((blockIdx.x / p.Cq) % p.Hkv);
+    const int b = (int)(blockIdx.x / ((long)p.Cq * p.Hkv));
+    const int G = p.Hq / p.Hkv;
+    const long ubase = ((long)b * p.Hkv + h) * p.Cq;
+    load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, m * BS);
+    load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, m * BS);
+    const int tr = tid / C::CG, tc = tid % C::CG;  // rows here are keys j
+    float dk[4][C::COLS], dv[4][C::COLS];
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int ee = 0; ee < C::COLS; ++ee) dk[ii][ee] = dv[ii][ee] = 0.f;
+
+    for (int c0 = m; c0 < p.Cq; c0 += kThreads) {
+        const int cc = c0 + tid;
+        const int att = (cc < p.Cq && (cc == m || selected(p, ubase + cc, cc, m))) ? 1 : 0;
+        int cnt;
+        const int pos = block_exclusive_scan(att, scan, &cnt);
+        if (att) clist[pos] = cc;
+        __syncthreads();
+        for (int li = 0; li < cnt; ++li) {
+            const int c = clist[li];
+            const bool diag = (c == m);
+            const float bias = diag ? 0.f : (p.s[(ubase + c) * p.Cq + m] - p.lse_s[ubase + c]);
+            for (int g = 0; g < G; ++g) {
+                const int hq = h * G + g;
+                __syncthreads();
+                load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
+                load_rows<T, D, BS>(dOs, p.dO, b, p.n, p.Hq, hq, c * BS);
+                if (tid < BS) {
+                    const long ri = ((long)b * p.Hq + hq) * p.n + c * BS + tid;
+                    rowL[tid] = p.lse_in[ri];
+                    rowD[tid] = p.Dbuf[ri];
+                }
+                __syncthreads();
+                for (int tile = tid; tile < C::NT_S; tile += kThreads) {
+                    const int ttr = tile / C::RG, ttc = tile % C::RG;  // query rows, keys
+                    float sacc[4][4] = {}, pacc[4][4] = {};
+                    for (int e = 0; e < D; ++e) {
+                        float qv[4], gv[4], kv[4], vv[4];
+#pragma unroll
+                        for (int ii = 0; ii < 4; ++ii) {
+                            qv[ii] = Qs[(ttr + C::RG * ii) * C::LD + e];
+                            gv[ii] = dOs[(ttr + C::RG * ii) * C::LD + e];
+                        }
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            kv[jj] = Ks[(ttc + C::RG * jj) * C::LD + e];
+                            vv[jj] = Vs[(ttc + C::RG * jj) * C::LD + e];
+                        }
+#pragma unroll
+                        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                sacc[ii][jj] = fmaf(qv[ii], kv[jj], sacc[ii][jj]);
+                                pacc[ii][jj] = fmaf(gv[ii], vv[jj], pacc[ii][jj]);
+                            }
+                    }
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int r = ttr + C::RG * ii, j = ttc + C::RG * jj;
+                            const float z = fmaf(p.scale, sacc[ii][jj], bias);
+                            const float pr = (diag && j > r) ? 0.f : expf(z - rowL[r]);
+                            Ps[r * C::LDS + j] = pr;
+                            dSs[r * C::LDS + j] = pr * (pacc[ii][jj] - rowD[r]);
+                        }
+                }
+                __syncthreads();
+                for (int r = 0; r < BS; ++r) {
+                    float pv[4], sv[4];
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii) {
+                        pv[ii] = Ps[r * C::LDS + tr + C::RG * ii];
+                        sv[ii] = dSs[r * C::LDS + tr + C::RG * ii];
+                    }
+#pragma unroll
+                    for (int ee = 0; ee < C::COLS; ++ee) {
+                        const float gv = dOs[r * C::LD + tc + C::CG * ee];
+                        const float qv = Qs[r * C::LD + tc + C::CG * ee];
+#pragma unroll
+                        for (int ii = 0; ii < 4; ++ii) {
+                            dv[ii][ee] = fmaf(pv[ii], gv, dv[ii][ee]);
+                            dk[ii][ee] = fmaf(sv[ii], qv, dk[ii][ee]);
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii) {
+        const int j = tr + C::RG * ii;
+        const long base = (((long)b * p.n + m * BS + j) * p.Hkv + h) * D;
+#pragma unroll
+        for (int ee = 0; ee < C::COLS; ++ee) {
+            stg<T>(p.dk, base + tc + C::CG * ee, p.scale * dk[ii][ee]);
+            stg<T>(p.dv, base + tc + C::CG * ee, dv[ii][ee]);
+        }
+    }
+}
+
+size_t fwd_smem(int D, int BS, int Cq) {
+    return sizeof(float) * (3 * BS * (D + 1) + BS * (BS + 1) + 3 * BS) + sizeof(int) * (Cq + 1);
+}
+size_t dq_smem(int D, int BS, int Cq) {
+    return sizeof(float) * (4 * BS * (D + 1) + BS * (BS + 1) + 2 * BS + 33 + Cq) + sizeof(int) * (Cq + 1);
+}
+size_t dkdv_smem(int D, int BS) {
+    return sizeof(float) * (4 * BS * (D + 1) + 2 * BS * (BS + 1) + 2 * BS) + sizeof(int) * (kThreads + 33);
+}
+
+template <typename Kern>
+cudaError_t launch(Kern kern, long grid, size_t smem, const TrainParams& p, cudaStream_t stream) {
+    if (grid <= 0) return cudaSuccess;
+    if (grid > 0x7fffffffL) return cudaErrorInvalidValue;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
+    err = cudaGetLastError();
+    if (err == cudaSuccess) count_launch();
+    return err;
+}
+
+#define SAS_DISPATCH_SIMT(KERNEL, GRID, SMEM)                                                         \
+    do {                                                                                              \
+        if (p.is_bf16) {                                                                              \
+            if (p.d == 128) {                                                                         \
+                switch (p.bs) {                                                                       \
+                    case 16: return launch(KERNEL<__nv_bfloat16, 128, 16>, GRID, SMEM, p, stream);    \
+                    case 32: return launch(KERNEL<__nv_bfloat16, 128, 32>, GRID, SMEM, p, stream);    \
+                    case 64: return launch(KERNEL<__nv_bfloat16, 128, 64>, GRID, SMEM, p, stream);    \
+                }                                                                                     \
+            } else if (p.d == 64) {                                                                   \
+                switch (p.bs) {                                                                       \
+                    case 16: return launch(KERNEL<__nv_bfloat16, 64, 16>, GRID, SMEM, p, stream);     \
+                    case 32: return launch(KERNEL<__nv_bfloat16, 64, 32>, GRID, SMEM, p, stream);     \
+                    case 64: return launch(KERNEL<__nv_bfloat16, 64, 64>, GRID, SMEM, p, stream);     \
+                }                                                                                     \
+            }                                                                                         \
+        } else {                                                                                      \
+            if (p.d == 128) {                                                                         \
+                switch (p.bs) {                                                                       \
+                    case 16: return launch(KERNEL<float, 128, 16>, GRID, SMEM, p, stream);            \
+                    case 32: return launch(KERNEL<float, 128, 32>, GRID, SMEM, p, stream);            \
+                    case 64: return launch(KERNEL<float, 128, 64>, GRID, SMEM, p, stream);            \
+                }                                                                                     \
+            } else if (p.d == 64) {                                                                   \
+                switch (p.bs) {                                                                       \
+                    case 16: return launch(KERNEL<float, 64, 16>, GRID, SMEM, p, stream);             \
+                    case 32: return launch(KERNEL<float, 64, 32>, GRID, SMEM, p, stream);             \
+                    case 64: return launch(KERNEL<float, 64, 64>, GRID, SMEM, p, stream);             \
+                }                                                                                     \
+            }                                                                                         \
+        }                                                                                             \
+        return cudaErrorNotSupported;                                                                 \
+    } while (0)
+
+cudaError_t launch_fwd_impl(const TrainParams& p, cudaStream_t stream) {
+    const long grid = (long)p.B * p.Hq * p.Cq;
+    const size_t smem = fwd_smem(p.d, p.bs, p.Cq);
+    SAS_DISPATCH_SIMT(fwd_simt_kernel, grid, smem);
+}
+
+cudaError_t launch_dq_impl(const TrainParams& p, cudaStream_t stream) {
+    const long grid = (long)p.B * p.Hkv * p.Cq;
+    const size_t smem = dq_smem(p.d, p.bs, p.Cq);
+    SAS_DISPATCH_SIMT(bwd_dq_kernel, grid, smem);
+}
+
+cudaError_t launch_dkdv_impl(const TrainParams& p, cudaStream_t stream) {
+    const long grid = (long)p.B * p.Hkv * p.Cq;
+    const size_t smem = dkdv_smem(p.d, p.bs);
+    SAS_DISPATCH_SIMT(bwd_dkdv_kernel, grid, smem);
+}
+
+}  // namespace
+
+size_t simt_max_smem(int D, int BS, int Cq) {
+    size_t a = fwd_smem(D, BS, Cq), b = dq_smem(D, BS, Cq), c = dkdv_smem(D, BS);
+    return a > b ? (a > c ? a : c) : (b > c ? b : c);
+}
+
+cudaError_t launch_fwd_simt(const TrainParams& p, cudaStream_t stream) { return launch_fwd_impl(p, stream); }
+
+size_t bwd_simt_workspace(const TrainParams& p) {
+    return sizeof(float) * (size_t)p.B * p.Hq * p.n;  // D rows
+}
+
+cudaError_t launch_bwd_simt(const TrainParams& p, cudaStream_t stream) {
+    const long rows = (long)p.B * p.n * p.Hq;
+    const long grid = (rows + kThreads / 32 - 1) / (kThreads / 32);
+    if (grid > 0) {
+        if (p.is_bf16)
+            bwd_rowdot_kernel<__nv_bfloat16><<<(unsigned)grid, kThreads, 0, stream>>>(p);
+        else
+            bwd_rowdot_kernel<float><<<(unsigned)grid, kThreads, 0, stream>>>(p);
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+        count_launch();
+    }
+    cudaError_t err = launch_dq_impl(p, stream);
+    if (err != cudaSuccess) return err;
+    return launch_dkdv_impl(p, stream);
+}
+
+}  // namespace sas

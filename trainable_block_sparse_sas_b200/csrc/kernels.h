@@ -1,0 +1,61 @@
+// kernels.h -- launchers of the libsas kernels (host side, internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sas {
+
+// Host-side count of successful kernel launches (reported by sas_launch_count).
+void count_launch(int n = 1);
+
+struct TrainParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* s;
+    const float* lse_s;
+    const int32_t* idx;
+    void* o;
+    float* lse;
+    // backward
+    const void* o_in;
+    const float* lse_in;
+    const void* dO;
+    float* Dbuf;  // [B, Hq, n] row dot(dO, o)
+    void* dq;
+    void* dk;
+    void* dv;
+    float* ds;
+    int* status;  // device status word (bounded waits)
+    int B, Hq, Hkv, d, n, bs, Cq, top_k, full_scope, is_bf16;
+    float scale;
+};
+
+struct DecodeParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    const int32_t* ctx_len;
+    const int32_t* idx;  // nullptr: dense
+    void* o;
+    float* part;  // [B*Hkv, nsplit, G, d + 2] partial (o, m, l)
+    int B, Hq, Hkv, d, bs, top_k, Tmax, is_bf16, nsplit, per_split, list_max;
+    float scale;
+};
+
+cudaError_t launch_topk_select(const float* s, int batch, int n_kv_heads, int n_rows, int row_len,
+                               const int32_t* ctx_len, int block_size, int top_k, int32_t* idx, float* lse_s,
+                               cudaStream_t stream);
+
+cudaError_t launch_fwd_simt(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_bwd_simt(const TrainParams& p, cudaStream_t stream);
+size_t bwd_simt_workspace(const TrainParams& p);
+size_t simt_max_smem(int D, int BS, int Cq);
+
+void decode_plan(DecodeParams& p);
+size_t decode_workspace(const DecodeParams& p);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+
+}  // namespace sas

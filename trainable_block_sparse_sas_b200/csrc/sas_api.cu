@@ -1,0 +1,284 @@
+// sas_api.cu -- the C ABI declared in include/sas.h: argument checks (before any
+// launch, no side effects on failure), kernel dispatch, and the device status
+// word that bounded device-side waits set when they give up.
+#include <math.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "kernels.h"
+#include "sas.h"
+
+namespace sas {
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Per-device status word: kernels with bounded waits write a non-zero code here.
+__device__ int g_status_word;
+
+struct DeviceInfo {
+    bool init = false;
+    int n_sm = 0;
+    int max_smem_optin = 0;
+    int* status = nullptr;  // device address of g_status_word
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+// Set-up once per device, with that device current: SM count, shared-memory
+// limit and the device address of the status word.
+cudaError_t device_info(DeviceInfo* out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.init) {
+        err = cudaDeviceGetAttribute(&di.n_sm, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess) return err;
+        err = cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (err != cudaSuccess) return err;
+        void* addr = nullptr;
+        err = cudaGetSymbolAddress(&addr, g_status_word);
+        if (err != cudaSuccess) return err;
+        di.status = static_cast<int*>(addr);
+        di.init = true;
+    }
+    *out = di;
+    return cudaSuccess;
+}
+
+sas_status from_cuda(cudaError_t err) {
+    if (err == cudaSuccess) return SAS_OK;
+    if (err == cudaErrorNotSupported) return SAS_ERR_UNSUPPORTED;
+    return SAS_ERR_CUDA;
+}
+
+bool check_train(const sas_attn_desc* d) {
+    if (!d) return false;
+    if (d->batch <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0) return false;
+    if (d->seq_len <= 0 || d->block_size <= 0 || d->top_k < 0) return false;
+    if (d->n_q_heads % d->n_kv_heads != 0 || d->seq_len % d->block_size != 0) return false;
+    if (d->scope != SAS_SCOPE_SPARSE && d->scope != SAS_SCOPE_FULL) return false;
+    if (d->dtype != SAS_F32 && d->dtype != SAS_BF16) return false;
+    if (!isfinite(d->softmax_scale)) return false;
+    return true;
+}
+
+bool supported_train(const sas_attn_desc* d) {
+    if (d->head_dim != 64 && d->head_dim != 128) return false;
+    if (d->block_size != 16 && d->block_size != 32 && d->block_size != 64) return false;
+    return true;
+}
+
+TrainParams make_train(const sas_attn_desc* d) {
+    TrainParams p = {};
+    p.B = d->batch;
+    p.Hq = d->n_q_heads;
+    p.Hkv = d->n_kv_heads;
+    p.d = d->head_dim;
+    p.n = d->seq_len;
+    p.bs = d->block_size;
+    p.Cq = d->seq_len / d->block_size;
+    p.top_k = d->top_k;
+    p.full_scope = d->scope == SAS_SCOPE_FULL ? 1 : 0;
+    p.is_bf16 = d->dtype == SAS_BF16 ? 1 : 0;
+    p.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->head_dim);
+    return p;
+}
+
+bool check_decode(const sas_decode_desc* d) {
+    if (!d) return false;
+    if (d->batch <= 0 || d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0) return false;
+    if (d->block_size <= 0 || d->top_k < 0 || d->max_ctx <= 0) return false;
+    if (d->n_q_heads % d->n_kv_heads != 0) return false;
+    if (d->dtype != SAS_F32 && d->dtype != SAS_BF16) return false;
+    if (!isfinite(d->softmax_scale)) return false;
+    return true;
+}
+
+bool supported_decode(const sas_decode_desc* d) {
+    if (d->head_dim != 64 && d->head_dim != 128) return false;
+    if (d->block_size % 16 != 0 || d->block_size > 256) return false;
+    if (d->n_q_heads / d->n_kv_heads > 16) return false;
+    return true;
+}
+
+DecodeParams make_decode(const sas_decode_desc* d) {
+    DecodeParams p = {};
+    p.B = d->batch;
+    p.Hq = d->n_q_heads;
+    p.Hkv = d->n_kv_heads;
+    p.d = d->head_dim;
+    p.bs = d->block_size;
+    p.top_k = d->top_k;
+    p.Tmax = d->max_ctx;
+    p.is_bf16 = d->dtype == SAS_BF16 ? 1 : 0;
+    p.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->head_dim);
+    return p;
+}
+
+// Workspace of a decode call: the larger of the sparse and the dense plans, so
+// that one query covers both kinds of call.
+size_t decode_ws_bytes(const DecodeParams& base) {
+    DecodeParams sp = base, dn = base;
+    sp.idx = reinterpret_cast<const int32_t*>(1);  // plan only, never dereferenced
+    dn.idx = nullptr;
+    decode_plan(sp);
+    decode_plan(dn);
+    const size_t a = decode_workspace(sp), b = decode_workspace(dn);
+    return ((a > b ? a : b) + 255) & ~(size_t)255;
+}
+
+}  // namespace
+}  // namespace sas
+
+using namespace sas;
+
+extern "C" {
+
+sas_status sas_topk_select(const float* s, int32_t batch, int32_t n_kv_heads, int32_t n_rows, int32_t row_len,
+                           const int32_t* ctx_len, int32_t block_size, int32_t top_k, int32_t* idx, float* lse_s,
+                           sas_stream_t stream) {
+    if (!s || batch <= 0 || n_kv_heads <= 0 || n_rows <= 0 || row_len <= 0 || top_k < 0) return SAS_ERR_INVALID_VALUE;
+    if (!idx && !lse_s) return SAS_ERR_INVALID_VALUE;
+    if (ctx_len && (n_rows != 1 || block_size <= 0)) return SAS_ERR_INVALID_VALUE;
+    return from_cuda(launch_topk_select(s, batch, n_kv_heads, n_rows, row_len, ctx_len, block_size, top_k, idx,
+                                        lse_s, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
+                              const float* s, const float* lse_s, const int32_t* idx, void* o, float* lse,
+                              sas_stream_t stream) {
+    if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !s || !lse_s || !o || !lse) return SAS_ERR_INVALID_VALUE;
+    if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
+    if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    cudaError_t err = device_info(&di);
+    if (err != cudaSuccess) return SAS_ERR_CUDA;
+    TrainParams p = make_train(desc);
+    if (simt_max_smem(p.d, p.bs, p.Cq) > (size_t)di.max_smem_optin) return SAS_ERR_UNSUPPORTED;
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.s = s;
+    p.lse_s = lse_s;
+    p.idx = desc->scope == SAS_SCOPE_SPARSE ? idx : nullptr;
+    if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k == 0) p.idx = nullptr;
+    p.o = o;
+    p.lse = lse;
+    p.status = di.status;
+    return from_cuda(launch_fwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc) {
+    if (!check_train(desc)) return 0;
+    TrainParams p = make_train(desc);
+    return (bwd_simt_workspace(p) + 255) & ~(size_t)255;
+}
+
+sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
+                              const void* o, const float* lse, const void* dO, const float* s, const float* lse_s,
+                              const int32_t* idx, void* dq, void* dk, void* dv, float* ds, void* workspace,
+                              size_t ws_bytes, sas_stream_t stream) {
+    if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !o || !lse || !dO || !s || !lse_s || !dq || !dk || !dv || !ds) return SAS_ERR_INVALID_VALUE;
+    if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
+    if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
+    const size_t need = sas_gated_attn_bwd_workspace_size(desc);
+    if (ws_bytes < need) return SAS_ERR_WORKSPACE_TOO_SMALL;
+    if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))) return SAS_ERR_INVALID_VALUE;
+    DeviceInfo di;
+    cudaError_t err = device_info(&di);
+    if (err != cudaSuccess) return SAS_ERR_CUDA;
+    TrainParams p = make_train(desc);
+    if (simt_max_smem(p.d, p.bs, p.Cq) > (size_t)di.max_smem_optin) return SAS_ERR_UNSUPPORTED;
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.s = s;
+    p.lse_s = lse_s;
+    p.idx = desc->scope == SAS_SCOPE_SPARSE ? idx : nullptr;
+    if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k == 0) p.idx = nullptr;
+    p.o_in = o;
+    p.lse_in = lse;
+    p.dO = dO;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.ds = ds;
+    p.Dbuf = static_cast<float*>(workspace);
+    p.status = di.status;
+    return from_cuda(launch_bwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t sas_sparse_decode_workspace_size(const sas_decode_desc* desc) {
+    if (!check_decode(desc)) return 0;
+    return decode_ws_bytes(make_decode(desc));
+}
+
+sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* ctx_len, const int32_t* idx, void* o, void* workspace, size_t ws_bytes,
+                             sas_stream_t stream) {
+    if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_cache || !v_cache || !ctx_len || !o) return SAS_ERR_INVALID_VALUE;
+    if (!supported_decode(desc)) return SAS_ERR_UNSUPPORTED;
+    DecodeParams p = make_decode(desc);
+    const size_t need = decode_ws_bytes(p);
+    if (ws_bytes < need) return SAS_ERR_WORKSPACE_TOO_SMALL;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SAS_ERR_INVALID_VALUE;
+    DeviceInfo di;
+    cudaError_t err = device_info(&di);
+    if (err != cudaSuccess) return SAS_ERR_CUDA;
+    p.q = q;
+    p.k = k_cache;
+    p.v = v_cache;
+    p.ctx_len = ctx_len;
+    p.idx = desc->top_k > 0 ? idx : nullptr;
+    if (!idx) p.idx = nullptr;
+    p.o = o;
+    p.part = static_cast<float*>(workspace);
+    decode_plan(p);
+    return from_cuda(launch_decode(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_device_status(sas_stream_t stream) {
+    DeviceInfo di;
+    cudaError_t err = device_info(&di);
+    if (err != cudaSuccess) return SAS_ERR_CUDA;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SAS_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, di.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SAS_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(di.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SAS_ERR_CUDA;
+        return SAS_ERR_DEVICE_TIMEOUT;
+    }
+    return SAS_OK;
+}
+
+const char* sas_status_string(sas_status status) {
+    switch (status) {
+        case SAS_OK: return "success";
+        case SAS_ERR_INVALID_VALUE: return "invalid argument";
+        case SAS_ERR_UNSUPPORTED: return "unsupported problem shape or type";
+        case SAS_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case SAS_ERR_CUDA: return "CUDA error";
+        case SAS_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t sas_version(void) { return 100; }
+
+uint64_t sas_launch_count(void) { return (uint64_t)g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"
