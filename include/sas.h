@@ -175,6 +175,32 @@ sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const v
                              const int32_t* ctx_len, const int32_t* idx, void* o, void* workspace, size_t ws_bytes,
                              sas_stream_t stream);
 
+/*
+ * sas_sparse_decode_noalloc -- the same decode as sas_sparse_decode (same
+ *   arguments, layouts and results) for callers that cannot allocate device
+ *   memory: a plugin whose host program owns all device memory, or a serving
+ *   loop that may not call cudaMalloc (which synchronises the device) between
+ *   steps.  It takes no workspace.  The paper has no counterpart to this entry
+ *   point; it exists for those callers only.
+ * Scratch: the split-K partials live in a fixed 4 MiB array inside the library
+ *   (every GPU that loads the library holds it until the process exits).
+ *   Problems whose partials need more than 4 MiB return
+ *   SAS_ERR_WORKSPACE_TOO_SMALL before any launch; sparse calls of the Qwen3
+ *   decode shapes need about 1.4 MiB, long dense calls may exceed the limit.
+ * The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  It allocates nothing (no cudaMalloc or cudaFree, no allocating
+ *   library routine).
+ * All calls share the one array: each call writes every partial it later reads,
+ *   so nothing has to start at zero, but calls that overlap on the GPU (other
+ *   streams, other host threads) race on it and must be serialised by the caller.
+ * Errors: as sas_sparse_decode, with SAS_ERR_WORKSPACE_TOO_SMALL meaning the
+ *   built-in array is too small for this problem.
+ */
+sas_status sas_sparse_decode_noalloc(const sas_decode_desc* desc, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* ctx_len, const int32_t* idx, void* o,
+                                     sas_stream_t stream);
+
 /* Synchronises `stream`, then reports and clears the device-side status word that
  * bounded waits inside the kernels set when they give up: SAS_OK or
  * SAS_ERR_DEVICE_TIMEOUT (SAS_ERR_CUDA if the synchronisation itself fails). */

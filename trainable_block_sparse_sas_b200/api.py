@@ -62,6 +62,8 @@ lib.sas_sparse_decode_workspace_size.restype = _sz
 lib.sas_sparse_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeDesc)]
 lib.sas_sparse_decode.restype = ctypes.c_int
 lib.sas_sparse_decode.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7 + [_sz, _vp]
+lib.sas_sparse_decode_noalloc.restype = ctypes.c_int
+lib.sas_sparse_decode_noalloc.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7
 lib.sas_launch_count.restype = ctypes.c_uint64
 lib.sas_launch_count.argtypes = []
 lib.sas_device_status.restype = ctypes.c_int
@@ -133,6 +135,14 @@ def sas_sparse_decode(desc, q, k_cache, v_cache, ctx_len, idx, o, workspace, str
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.sas_sparse_decode(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx), _p(o),
                                  _p(workspace), ws_bytes, _stream(stream)), "sas_sparse_decode")
+
+
+def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream=None):
+    """sas_sparse_decode without a workspace, for callers that cannot allocate
+    device memory: the partials use a fixed 4 MiB array inside the library.
+    Overlapping calls race on that array."""
+    _check(lib.sas_sparse_decode_noalloc(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx),
+                                         _p(o), _stream(stream)), "sas_sparse_decode_noalloc")
 
 
 def sas_device_status(stream=None):
