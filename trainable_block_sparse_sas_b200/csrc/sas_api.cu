@@ -176,6 +176,7 @@ sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const vo
     p.o = o;
     p.lse = lse;
     p.status = di.status;
+    if (fwd_sm100_supported(p)) return from_cuda(launch_fwd_sm100(p, reinterpret_cast<cudaStream_t>(stream)));
     return from_cuda(launch_fwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
