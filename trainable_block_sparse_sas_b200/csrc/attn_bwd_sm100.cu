@@ -1,0 +1,682 @@
+// attn_bwd_sm100.cu -- tensor-core (tcgen05 / TMEM / TMA) backward of SAS gated
+// block-sparse attention for bf16, head_dim 128, block size 64, 2 or 4 query
+// heads per KV head.  Two kernels, no atomics (results are deterministic):
+//
+// bwd_dq_sm100: one CTA per (batch, kv head, query block c), the group's query
+//   heads stacked into 128-row M-tiles as in the forward.  For each attended key
+//   block (selected history blocks, then the current block):
+//     S_i = Q_i K^T and dP_i = dO_i V^T             (SS MMAs into TMEM)
+//     softmax warps: P = exp(S sigma + log g_m - lse), dS = P (dP - D),
+//       dS written back to TMEM as bf16, and the tile sum of dS kept per warp
+//       -- the block-wise log-gate gradient dlogg[c,m] (jaehun.me review of SAS,
+//       Kernel implementation paragraph; inner-gate gradient, section 4.2.2)
+//     dQ_i += dS_i K                                  (TS MMA, dS read from TMEM)
+//   Epilogue: dq = sigma dQ, and ds[c,m] = dlogg_m - g_m sum(dlogg) for m < c.
+//
+// bwd_dkdv_sm100: one CTA per (batch, kv head, key block m).  It walks the query
+//   blocks that attend m (m itself with the causal mask, and every later block
+//   whose selection holds m), one 128-row M-tile at a time:
+//     S = Q K_m^T and dP = dO V_m^T                   (SS MMAs, double-buffered TMEM)
+//     softmax warps: P and dS as above, written as bf16 rows into swizzled smem
+//     dV^T += dO^T P and dK^T += Q^T dS               (SS MMAs, M = head_dim = 128)
+//   Epilogue: dk = sigma dK, dv = dV.
+//
+// D_i = dO_i . o_i comes from a small row-dot kernel run first (workspace).
+// Every wait is time-bounded and reports through the device status word.
+#include <cstring>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace sas {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kBS = 64;
+constexpr int kStages = 2;
+constexpr uint32_t kSlab64 = 64 * 128;    // 64 rows x 128 B: one block, one 64-wide d slab
+constexpr uint32_t kSlab128 = 128 * 128;  // 128 rows x 128 B
+
+struct BwdArgs {
+    CUtensorMap tq, tdo, tk, tv;
+    const float* s;
+    const float* lse_s;
+    const int32_t* idx;
+    const float* lse;
+    const float* Dbuf;
+    __nv_bfloat16* dq;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* ds;
+    int* status;
+    int B, Hq, Hkv, n, Cq, top_k, full_scope;
+    float scale, scale_log2;
+};
+
+__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
+    tmem_ld32(taddr, r);
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// ============================================================================
+// dq / ds kernel
+// ============================================================================
+constexpr int kDqThreads = 320;
+
+template <int MT>
+struct DqLayout {
+    static constexpr int G = 2 * MT;
+    static constexpr uint32_t kHalf = MT * kSlab128;  // all query rows, one d slab
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kDO = kQ + 2 * kHalf;
+    static constexpr uint32_t kK = kDO + 2 * kHalf;
+    static constexpr uint32_t kV = kK + kStages * 2 * kSlab64;
+    static constexpr uint32_t kBars = kV + kStages * 2 * kSlab64;
+    // q_full, kv_full[S], kv_empty[S], s_full[2], ds_ready[2], dq_done, drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
+    static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
+    static constexpr uint32_t kList = kMisc + 16;
+    __host__ __device__ static uint32_t part_off(int Cq) { return (kList + 4 * (uint32_t)(Cq + 1) + 15) & ~15u; }
+    static size_t bytes(int Cq) { return 1024 + part_off(Cq) + 32 * (size_t)(Cq + 1); }
+};
+
+template <int MT>
+__global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __grid_constant__ BwdArgs a) {
+    using L = DqLayout<MT>;
+    constexpr int G = L::G;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO, sK = sbase + L::kK, sV = sbase + L::kV;
+    const uint32_t bar0 = sbase + L::kBars;
+    const uint32_t q_full = bar0;
+    auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto kv_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
+    auto s_full = [&](int i) { return bar0 + 8u * (1 + 2 * kStages + i); };
+    auto ds_ready = [&](int i) { return bar0 + 8u * (3 + 2 * kStages + i); };
+    const uint32_t dq_done = bar0 + 8u * (5 + 2 * kStages);
+    const uint32_t drain = bar0 + 8u * (6 + 2 * kStages);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
+    int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
+    float* tot_sh = reinterpret_cast<float*>(base + L::kMisc + 12);
+    int* list = reinterpret_cast<int*>(base + L::kList);
+    float* part = reinterpret_cast<float*>(base + L::part_off(a.Cq));  // [slot][8 softmax warps]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = a.B * a.Hkv;
+    const int c = a.Cq - 1 - (int)(blockIdx.x / BH);
+    const int bh = (int)(blockIdx.x % BH);
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const long unit = (long)bh * a.Cq + c;
+
+    for (int i = threadIdx.x; i < 8 * (a.Cq + 1); i += kDqThreads) part[i] = 0.f;
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(kv_full(s), 1);
+            mbar_init(kv_empty(s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(s_full(i), 1);
+            mbar_init(ds_ready(i), 128);
+        }
+        mbar_init(dq_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        int cnt = 0;
+        if (a.full_scope) {
+            for (int m = 0; m < c; ++m) list[cnt++] = m;
+        } else {
+            const int kk = min(a.top_k, c);
+            const int32_t* row = a.idx + unit * a.top_k;
+            for (int i = 0; i < kk; ++i) {
+                const int v = row[i];
+                if (v >= 0 && v < c) list[cnt++] = v;
+            }
+        }
+        list[cnt] = c;
+        *list_count = cnt + 1;
+        fence_barrier_init();
+        prefetch_tmap(&a.tq);
+        prefetch_tmap(&a.tdo);
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nlist = *list_count;  // history blocks + the current block
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int q_row = b * a.n + c * kBS;
+            mbar_arrive_expect_tx(q_full, 4 * L::kHalf);
+            for (int kh = 0; kh < 2; ++kh) {
+                tma_load_3d(sQ + kh * L::kHalf, &a.tq, q_full, kh * 64, h * G, q_row);
+                tma_load_3d(sDO + kh * L::kHalf, &a.tdo, q_full, kh * 64, h * G, q_row);
+            }
+            for (int t = 0; t < nlist; ++t) {
+                const int s = t % kStages;
+                if (t >= kStages && !mbar_wait(kv_empty(s), (t / kStages - 1) & 1, abort_flag, a.status)) break;
+                mbar_arrive_expect_tx(kv_full(s), 4 * kSlab64);
+                const int row0 = b * a.n + list[t] * kBS;
+                for (int kh = 0; kh < 2; ++kh) {
+                    tma_load_3d(sK + s * 2 * kSlab64 + kh * kSlab64, &a.tk, kv_full(s), kh * 64, h, row0);
+                    tma_load_3d(sV + s * 2 * kSlab64 + kh * kSlab64, &a.tv, kv_full(s), kh * 64, h, row0);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+            constexpr uint32_t idesc_dq = idesc_bf16_f32(128, 128, false, true);
+            bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
+            for (int t = 0; ok && t < nlist; ++t) {
+                const int s = t % kStages;
+                if (!mbar_wait(kv_full(s), (t / kStages) & 1, abort_flag, a.status)) break;
+                tc_fence_after();
+                const uint32_t kst = sK + s * 2 * kSlab64, vst = sV + s * 2 * kSlab64;
+                for (int i = 0; i < MT; ++i) {
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const int kh = ks >> 2, kk = ks & 3;
+                        const uint64_t bd = sdesc_sw128(kst + kh * kSlab64 + kk * 32, 16, 1024);
+                        const uint64_t ad = sdesc_sw128(sQ + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
+                        mma_ss(tmem + i * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const int kh = ks >> 2, kk = ks & 3;
+                        const uint64_t bd = sdesc_sw128(vst + kh * kSlab64 + kk * 32, 16, 1024);
+                        const uint64_t ad = sdesc_sw128(sDO + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
+                        mma_ss(tmem + i * 128 + 64, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(s_full(i));
+                }
+                for (int i = 0; i < MT; ++i) {
+                    if (!mbar_wait(ds_ready(i), t & 1, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kBS / 16; ++ks) {
+                        const uint64_t bd = sdesc_sw128(kst + ks * 2048, kSlab64, 1024);
+                        mma_ts(tmem + 256 + i * 128, tmem + i * 128 + ks * 8, bd, idesc_dq,
+                               (t > 0 || ks > 0) ? 1u : 0u);
+                    }
+                }
+                if (ok && t + kStages < nlist) mma_commit(kv_empty(s));
+            }
+            mma_commit(dq_done);
+            mma_commit(drain);
+            mbar_wait_drain(drain, 0, a.status);
+        }
+    } else {
+        const int wi = warp - 2;  // 0..7
+        const int grp = wi >> 2;
+        const int quad = warp & 3;
+        if (grp < MT) {
+            const int row = 32 * quad + lane;
+            const int r_unit = 128 * grp + row;
+            const int tok = r_unit / G, g = r_unit % G;
+            const int hq = h * G + g;
+            const long ri = ((long)b * a.Hq + hq) * a.n + c * kBS + tok;
+            const float lse2 = a.lse[ri] * kLog2e;
+            const float Drow = a.Dbuf[ri];
+            const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+            const uint32_t tS = tmem + lane_off + grp * 128, tP = tS + 64;
+            const uint32_t tQ = tmem + lane_off + 256 + grp * 128;
+            const float* srow = a.s + unit * a.Cq;
+            const float lse_c = a.lse_s[unit];
+            bool ok = true;
+            for (int t = 0; t < nlist; ++t) {
+                if (!mbar_wait(s_full(grp), t & 1, abort_flag, a.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int blk = list[t];
+                const bool cur = (blk == c);
+                const float off = (cur ? 0.f : (srow[blk] - lse_c) * kLog2e) - lse2;
+                float rs = 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t sr[32], dr[32];
+                    tmem_ld32_sync(tS + ch * 32, sr);
+                    tmem_ld32_sync(tP + ch * 32, dr);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        float dsv[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * jj + e, key = ch * 32 + j;
+                            float p = ex2(fmaf(__uint_as_float(sr[j]), a.scale_log2, off));
+                            if (cur && key > tok) p = 0.f;
+                            dsv[e] = p * (__uint_as_float(dr[j]) - Drow);
+                            rs += dsv[e];
+                        }
+                        pk[ch * 16 + jj] = pack_bf16x2(dsv[0], dsv[1]);
+                    }
+                }
+                tmem_st32(tS, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(ds_ready(grp));
+                if (!cur) {
+                    rs = warp_sum(rs);
+                    if (lane == 0) part[t * 8 + wi] = rs;
+                }
+            }
+            if (ok && mbar_wait(dq_done, 0, abort_flag, a.status)) {
+                tc_fence_after();
+                __nv_bfloat16* drow = a.dq + (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(tQ + ch * 32, r);
+                    uint32_t o[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        o[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * a.scale, __uint_as_float(r[2 * j + 1]) * a.scale);
+                    uint4* dst = reinterpret_cast<uint4*>(drow + ch * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    // ds row: dlogg over the group's warps, then ds = dlogg - g * sum(dlogg)
+    const int nsel = nlist - 1;
+    for (int t = threadIdx.x; t < nsel; t += kDqThreads) {
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc += part[t * 8 + w];
+        part[t * 8] = acc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float tot = 0.f;
+        for (int t = 0; t < nsel; ++t) tot += part[t * 8];
+        *tot_sh = tot;
+    }
+    __syncthreads();
+    if (*abort_flag) return;
+    const float tot = *tot_sh;
+    const float* srow = a.s + unit * a.Cq;
+    const float lse_c = a.lse_s[unit];
+    float* dsrow = a.ds + unit * a.Cq;
+    for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
+    __syncthreads();
+    for (int t = threadIdx.x; t < nsel; t += kDqThreads) dsrow[list[t]] += part[t * 8];
+}
+
+// ============================================================================
+// dk / dv kernel
+// ============================================================================
+constexpr int kKvThreads = 192;
+
+struct DkvLayout {
+    static constexpr uint32_t kK = 0;                     // 2 slabs x 64 rows
+    static constexpr uint32_t kV = kK + 2 * kSlab64;
+    static constexpr uint32_t kQ = kV + 2 * kSlab64;      // [stage][slab] 128 rows
+    static constexpr uint32_t kDO = kQ + kStages * 2 * kSlab128;
+    static constexpr uint32_t kP = kDO + kStages * 2 * kSlab128;  // 128 rows x 64 keys bf16
+    static constexpr uint32_t kDS = kP + kSlab128;
+    static constexpr uint32_t kBars = kDS + kSlab128;
+    // kv_full, qd_full[S], qd_empty[S], s_full[2], p_ready, item_done, final, drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4;
+    static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
+    static constexpr uint32_t kList = kMisc + 16;
+    static constexpr uint32_t kScan = kList;  // scan scratch precedes the list
+    static size_t bytes(int Cq) { return 1024 + kList + 4 * 40 + 4 * (size_t)(Cq + 1); }
+};
+
+// is history block m in the ascending selection of query block c (unit uc)?
+__device__ __forceinline__ bool holds(const BwdArgs& a, long uc, int c, int m) {
+    int lo = 0, hi = min(a.top_k, c) - 1;
+    const int32_t* row = a.idx + uc * a.top_k;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int v = row[mid];
+        if (v == m) return true;
+        if (v >= 0 && v < m) lo = mid + 1;
+        else hi = mid - 1;
+    }
+    return false;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __grid_constant__ BwdArgs a) {
+    using L = DkvLayout;
+    constexpr int G = 2 * MT;
+    constexpr int kRowsTok = 128 / G;  // tokens per 128-row item
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t sK = sbase + L::kK, sV = sbase + L::kV, sQ = sbase + L::kQ, sDO = sbase + L::kDO;
+    const uint32_t sP = sbase + L::kP, sDS = sbase + L::kDS;
+    const uint32_t bar0 = sbase + L::kBars;
+    const uint32_t kv_full = bar0;
+    auto qd_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto qd_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
+    auto s_full = [&](int i) { return bar0 + 8u * (1 + 2 * kStages + i); };
+    const uint32_t p_ready = bar0 + 8u * (3 + 2 * kStages);
+    const uint32_t item_done = bar0 + 8u * (4 + 2 * kStages);
+    const uint32_t final_bar = bar0 + 8u * (5 + 2 * kStages);
+    const uint32_t drain = bar0 + 8u * (6 + 2 * kStages);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
+    int* scan = reinterpret_cast<int*>(base + L::kScan);  // 33 ints
+    int* list = scan + 40;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = a.B * a.Hkv;
+    const int m = (int)(blockIdx.x / BH);  // early (widely selected) key blocks first
+    const int bh = (int)(blockIdx.x % BH);
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const long ubase = (long)bh * a.Cq;
+
+    // query blocks attending key block m: m itself, then every c > m holding m
+    list[0] = m;
+    int nlist = 1;
+    for (int c0 = m + 1; c0 < a.Cq; c0 += kKvThreads) {
+        const int cc = c0 + (int)threadIdx.x;
+        const int att = (cc < a.Cq && (a.full_scope || holds(a, ubase + cc, cc, m))) ? 1 : 0;
+        int cnt;
+        const int pos = block_exclusive_scan(att, scan, &cnt);
+        if (att) list[nlist + pos] = cc;
+        nlist += cnt;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(qd_full(s), 1);
+            mbar_init(qd_empty(s), 1);
+        }
+        mbar_init(s_full(0), 1);
+        mbar_init(s_full(1), 1);
+        mbar_init(p_ready, 128);
+        mbar_init(item_done, 1);
+        mbar_init(final_bar, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tmap(&a.tq);
+        prefetch_tmap(&a.tdo);
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nitems = nlist * MT;
+    // TMEM: S/dP buffers at 0 and 128 (S | dP), dV^T at 256, dK^T at 320
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(kv_full, 4 * kSlab64);
+            const int krow = b * a.n + m * kBS;
+            for (int kh = 0; kh < 2; ++kh) {
+                tma_load_3d(sK + kh * kSlab64, &a.tk, kv_full, kh * 64, h, krow);
+                tma_load_3d(sV + kh * kSlab64, &a.tv, kv_full, kh * 64, h, krow);
+            }
+            for (int j = 0; j < nitems; ++j) {
+                const int st = j % kStages;
+                if (j >= kStages && !mbar_wait(qd_empty(st), (j / kStages - 1) & 1, abort_flag, a.status)) break;
+                const int c = list[j / MT], i = j % MT;
+                const int qrow = b * a.n + c * kBS + i * kRowsTok;
+                mbar_arrive_expect_tx(qd_full(st), 4 * kSlab128);
+                for (int kh = 0; kh < 2; ++kh) {
+                    tma_load_3d(sQ + (st * 2 + kh) * kSlab128, &a.tq, qd_full(st), kh * 64, h * G, qrow);
+                    tma_load_3d(sDO + (st * 2 + kh) * kSlab128, &a.tdo, qd_full(st), kh * 64, h * G, qrow);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+            constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, true, true);
+            auto issue_s = [&](int j) {
+                const int st = j % kStages, buf = j & 1;
+                const uint32_t q = sQ + st * 2 * kSlab128, o = sDO + st * 2 * kSlab128;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const int kh = ks >> 2, kk = ks & 3;
+                    mma_ss(tmem + buf * 128, sdesc_sw128(q + kh * kSlab128 + kk * 32, 16, 1024),
+                           sdesc_sw128(sK + kh * kSlab64 + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const int kh = ks >> 2, kk = ks & 3;
+                    mma_ss(tmem + buf * 128 + 64, sdesc_sw128(o + kh * kSlab128 + kk * 32, 16, 1024),
+                           sdesc_sw128(sV + kh * kSlab64 + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full(buf));
+            };
+            bool ok = mbar_wait(kv_full, 0, abort_flag, a.status);
+            if (ok && nitems > 0) {
+                ok = mbar_wait(qd_full(0), 0, abort_flag, a.status);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0);
+                }
+            }
+            for (int j = 0; ok && j < nitems; ++j) {
+                if (j + 1 < nitems) {
+                    if (!mbar_wait(qd_full((j + 1) % kStages), ((j + 1) / kStages) & 1, abort_flag, a.status)) break;
+                    tc_fence_after();
+                    issue_s(j + 1);
+                }
+                if (!mbar_wait(p_ready, j & 1, abort_flag, a.status)) break;
+                tc_fence_after();
+                const int st = j % kStages;
+                const uint32_t q = sQ + st * 2 * kSlab128, o = sDO + st * 2 * kSlab128;
+#pragma unroll
+                for (int ks = 0; ks < 128 / 16; ++ks) {
+                    mma_ss(tmem + 256, sdesc_sw128(o + ks * 2048, kSlab128, 1024),
+                           sdesc_sw128(sP + ks * 2048, kSlab128, 1024), idesc_g, (j > 0 || ks > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < 128 / 16; ++ks) {
+                    mma_ss(tmem + 320, sdesc_sw128(q + ks * 2048, kSlab128, 1024),
+                           sdesc_sw128(sDS + ks * 2048, kSlab128, 1024), idesc_g, (j > 0 || ks > 0) ? 1u : 0u);
+                }
+                mma_commit(item_done);
+                if (j + kStages < nitems) mma_commit(qd_empty(st));
+            }
+            mma_commit(final_bar);
+            mma_commit(drain);
+            mbar_wait_drain(drain, 0, a.status);
+        }
+    } else {
+        const int quad = warp & 3;
+        const int row = 32 * quad + lane;  // row of the 128-row item
+        const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+        bool ok = true;
+        for (int j = 0; j < nitems; ++j) {
+            const int buf = j & 1;
+            const int c = list[j / MT], i = j % MT;
+            const int r_unit = 128 * i + row;
+            const int tok = r_unit / G, g = r_unit % G;
+            const long ri = ((long)b * a.Hq + h * G + g) * a.n + c * kBS + tok;
+            const float lse2 = a.lse[ri] * kLog2e;
+            const float Drow = a.Dbuf[ri];
+            const bool diag = (c == m);
+            const float off = (diag ? 0.f : (a.s[(ubase + c) * a.Cq + m] - a.lse_s[ubase + c]) * kLog2e) - lse2;
+            if (!mbar_wait(s_full(buf), (j >> 1) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t pp[32], dd[32];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32_sync(tmem + lane_off + buf * 128 + ch * 32, sr);
+                tmem_ld32_sync(tmem + lane_off + buf * 128 + 64 + ch * 32, dr);
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    float pv[2], dv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int jx = 2 * jj + e, key = ch * 32 + jx;
+                        float p = ex2(fmaf(__uint_as_float(sr[jx]), a.scale_log2, off));
+                        if (diag && key > tok) p = 0.f;
+                        pv[e] = p;
+                        dv[e] = p * (__uint_as_float(dr[jx]) - Drow);
+                    }
+                    pp[ch * 16 + jj] = pack_bf16x2(pv[0], pv[1]);
+                    dd[ch * 16 + jj] = pack_bf16x2(dv[0], dv[1]);
+                }
+            }
+            tc_fence_before();
+            // P / dS smem buffers are free once the MMAs of item j-1 completed
+            if (j > 0 && !mbar_wait(item_done, (j - 1) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+            }
+            const uint32_t rbase = (uint32_t)row * 128u;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint32_t sw = (uint32_t)((ch ^ (row & 7)) * 16);
+                st_shared_v4(sP + rbase + sw, pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
+                st_shared_v4(sDS + rbase + sw, dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(p_ready);
+        }
+        if (ok && mbar_wait(final_bar, 0, abort_flag, a.status)) {
+            tc_fence_after();
+            const int d = 32 * quad + lane;  // dV^T / dK^T: TMEM lane = head-dim index
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16* dst = which == 0 ? a.dv : a.dk;
+                const float mul = which == 0 ? 1.f : a.scale;
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32_sync(tmem + lane_off + 256 + which * 64 + ch * 32, r);
+#pragma unroll
+                    for (int jx = 0; jx < 32; ++jx) {
+                        const int key = ch * 32 + jx;
+                        dst[(((long)b * a.n + m * kBS + key) * a.Hkv + h) * kD + d] =
+                            __float2bfloat16_rn(__uint_as_float(r[jx]) * mul);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <typename Kern>
+cudaError_t launch_kernel(Kern kern, long grid, int threads, size_t smem, const BwdArgs& a, cudaStream_t stream) {
+    if (grid <= 0) return cudaSuccess;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    kern<<<(unsigned)grid, threads, smem, stream>>>(a);
+    err = cudaGetLastError();
+    if (err == cudaSuccess) count_launch();
+    return err;
+}
+
+template <int MT>
+cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
+    constexpr int G = 2 * MT;
+    BwdArgs a;
+    memset(&a, 0, sizeof(a));
+    const long rows = (long)p.B * p.n;
+    const long grid = (long)p.B * p.Hkv * p.Cq;
+    a.s = p.s;
+    a.lse_s = p.lse_s;
+    a.idx = p.idx;
+    a.lse = p.lse_in;
+    a.Dbuf = p.Dbuf;
+    a.dq = static_cast<__nv_bfloat16*>(p.dq);
+    a.dk = static_cast<__nv_bfloat16*>(p.dk);
+    a.dv = static_cast<__nv_bfloat16*>(p.dv);
+    a.ds = p.ds;
+    a.status = p.status;
+    a.B = p.B;
+    a.Hq = p.Hq;
+    a.Hkv = p.Hkv;
+    a.n = p.n;
+    a.Cq = p.Cq;
+    a.top_k = p.top_k;
+    a.full_scope = p.full_scope;
+    a.scale = p.scale;
+    a.scale_log2 = p.scale * kLog2e;
+    // query-major kernel: the whole query block (64 tokens x G heads) per box
+    if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, kBS) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, kBS) ||
+        !encode_tma_rows(&a.tk, p.k, p.Hkv, rows, 1, kBS) || !encode_tma_rows(&a.tv, p.v, p.Hkv, rows, 1, kBS))
+        return cudaErrorInvalidValue;
+    cudaError_t err = launch_kernel(bwd_dq_sm100_kernel<MT>, grid, kDqThreads, DqLayout<MT>::bytes(p.Cq), a, stream);
+    if (err != cudaSuccess) return err;
+    // key-major kernel: 128-row items (128/G tokens x G heads) per box
+    if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, 128 / G) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, 128 / G))
+        return cudaErrorInvalidValue;
+    return launch_kernel(bwd_dkdv_sm100_kernel<MT>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream);
+}
+
+}  // namespace
+
+bool bwd_sm100_supported(const TrainParams& p) {
+    if (!p.is_bf16 || p.d != kD || p.bs != kBS) return false;
+    const int G = p.Hq / p.Hkv;
+    if (G != 2 && G != 4) return false;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
+                         reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.dO) |
+                         reinterpret_cast<uintptr_t>(p.dq) | reinterpret_cast<uintptr_t>(p.dk) |
+                         reinterpret_cast<uintptr_t>(p.dv);
+    if (al & 15u) return false;
+    if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq > 0x7fffffffL) return false;
+    return DqLayout<2>::bytes(p.Cq) <= 227 * 1024 && DkvLayout::bytes(p.Cq) <= 227 * 1024;
+}
+
+cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream) {
+    cudaError_t err = launch_rowdot(p, stream);
+    if (err != cudaSuccess) return err;
+    const int G = p.Hq / p.Hkv;
+    return G == 4 ? launch_mt<2>(p, stream) : launch_mt<1>(p, stream);
+}
+
+}  // namespace sas

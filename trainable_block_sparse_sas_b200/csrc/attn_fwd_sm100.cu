@@ -335,6 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     }
 }
 
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -347,26 +349,29 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [rows, heads, 128] bf16 viewed as a 3-D tensor {d, heads, rows}; box {64, box_heads, 64}
-bool encode_rows(CUtensorMap* map, const void* ptr, int heads, long rows, int box_heads) {
+// [rows, heads, 128] bf16 viewed as a 3-D tensor {d, heads, rows};
+// box {64, box_heads, box_rows} with 128-byte swizzle
+bool encode_tma_rows(CUtensorMap* map, const void* ptr, int heads, long rows, int box_heads, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)heads, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)heads * kD * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)box_heads, 64};
+    cuuint64_t dims[3] = {(cuuint64_t)128, (cuuint64_t)heads, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)128 * 2, (cuuint64_t)heads * 128 * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <int MT>
 cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     FwdArgs a;
     memset(&a, 0, sizeof(a));
     const long rows = (long)p.B * p.n;
-    if (!encode_rows(&a.tq, p.q, p.Hq, rows, 2 * MT) || !encode_rows(&a.tk, p.k, p.Hkv, rows, 1) ||
-        !encode_rows(&a.tv, p.v, p.Hkv, rows, 1))
+    if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, 2 * MT, kBS) || !encode_tma_rows(&a.tk, p.k, p.Hkv, rows, 1, kBS) ||
+        !encode_tma_rows(&a.tv, p.v, p.Hkv, rows, 1, kBS))
         return cudaErrorInvalidValue;
     a.s = p.s;
     a.lse_s = p.lse_s;

@@ -561,19 +561,24 @@ size_t bwd_simt_workspace(const TrainParams& p) {
     return sizeof(float) * (size_t)p.B * p.Hq * p.n;  // D rows
 }
 
-cudaError_t launch_bwd_simt(const TrainParams& p, cudaStream_t stream) {
+cudaError_t launch_rowdot(const TrainParams& p, cudaStream_t stream) {
     const long rows = (long)p.B * p.n * p.Hq;
     const long grid = (rows + kThreads / 32 - 1) / (kThreads / 32);
-    if (grid > 0) {
-        if (p.is_bf16)
-            bwd_rowdot_kernel<__nv_bfloat16><<<(unsigned)grid, kThreads, 0, stream>>>(p);
-        else
-            bwd_rowdot_kernel<float><<<(unsigned)grid, kThreads, 0, stream>>>(p);
-        cudaError_t err = cudaGetLastError();
-        if (err != cudaSuccess) return err;
-        count_launch();
-    }
-    cudaError_t err = launch_dq_impl(p, stream);
+    if (grid <= 0) return cudaSuccess;
+    if (grid > 0x7fffffffL) return cudaErrorInvalidValue;
+    if (p.is_bf16)
+        bwd_rowdot_kernel<__nv_bfloat16><<<(unsigned)grid, kThreads, 0, stream>>>(p);
+    else
+        bwd_rowdot_kernel<float><<<(unsigned)grid, kThreads, 0, stream>>>(p);
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) count_launch();
+    return err;
+}
+
+cudaError_t launch_bwd_simt(const TrainParams& p, cudaStream_t stream) {
+    cudaError_t err = launch_rowdot(p, stream);
+    if (err != cudaSuccess) return err;
+    err = launch_dq_impl(p, stream);
     if (err != cudaSuccess) return err;
     return launch_dkdv_impl(p, stream);
 }

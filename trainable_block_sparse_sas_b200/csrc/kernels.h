@@ -51,6 +51,9 @@ cudaError_t launch_topk_select(const float* s, int batch, int n_kv_heads, int n_
 
 cudaError_t launch_fwd_simt(const TrainParams& p, cudaStream_t stream);
 bool fwd_sm100_supported(const TrainParams& p);
+bool bwd_sm100_supported(const TrainParams& p);
+cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream);
+cudaError_t launch_rowdot(const TrainParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_sm100(const TrainParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_simt(const TrainParams& p, cudaStream_t stream);
 size_t bwd_simt_workspace(const TrainParams& p);

@@ -218,6 +218,7 @@ sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const vo
     p.ds = ds;
     p.Dbuf = static_cast<float*>(workspace);
     p.status = di.status;
+    if (bwd_sm100_supported(p)) return from_cuda(launch_bwd_sm100(p, reinterpret_cast<cudaStream_t>(stream)));
     return from_cuda(launch_bwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -211,4 +211,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 }  // namespace sm100
+
+// Host: tensor map of a [rows, heads, 128] bf16 tensor viewed as {d, heads,
+// rows}, box {64, box_heads, box_rows}, 128-byte swizzle.
+bool encode_tma_rows(CUtensorMap* map, const void* ptr, int heads, long rows, int box_heads, int box_rows);
+
 }  // namespace sas
