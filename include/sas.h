@@ -176,6 +176,25 @@ sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const v
                              sas_stream_t stream);
 
 /*
+ * sas_sparse_decode_select -- the decode step with its selection fused: the
+ *   Top-K of the block scores (as sas_topk_select in decode mode: ties to the
+ *   lower index) and the gate-free attention of sas_sparse_decode, in one launch
+ *   and without workspace (one thread-block cluster per (sequence, kv head)).
+ *   The selection stage is the decode bottleneck the pages report at long
+ *   context (shibing624 review, Fig. 7c; jaehun.me review, Decoding Efficiency).
+ * s        [B, Hkv, s_cols] fp32 block scores; row (b, h) scores blocks
+ *          0 .. floor((ctx_len[b]-1)/block_size) - 1, which must be <= s_cols.
+ * idx_out  [B, Hkv, top_k] int32 out (nullable): the chosen blocks, ascending,
+ *          -1 padded.
+ * Other arguments as sas_sparse_decode.
+ * Errors: as sas_sparse_decode; SAS_ERR_UNSUPPORTED unless dtype is bf16,
+ *         head_dim 128, block_size 64 and at most 16 query heads per kv head.
+ */
+sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* ctx_len, const float* s, int32_t s_cols,
+                                    void* o, int32_t* idx_out, sas_stream_t stream);
+
+/*
  * sas_sparse_decode_noalloc -- the same decode as sas_sparse_decode (same
  *   arguments, layouts and results) for callers that cannot allocate device
  *   memory: a plugin whose host program owns all device memory, or a serving

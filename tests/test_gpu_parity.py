@@ -230,10 +230,16 @@ def test_train_full_16k_sampled(api):
 # decode
 # --------------------------------------------------------------------------
 
-def _run_decode(api, inp, bs, top_k, dense=False):
+def _run_decode(api, inp, bs, top_k, dense=False, fused=False):
     q, kc, vc, ctx, s = (inp[x] for x in ("q", "k_cache", "v_cache", "ctx_len", "s"))
     B, Hkv = kc.shape[0], kc.shape[1]
     desc = api.decode_desc(q, kc, bs, top_k)
+    if fused:
+        idx = torch.full((B, Hkv, top_k), -7, dtype=torch.int32, device="cuda")
+        o = torch.empty_like(q)
+        api.sas_sparse_decode_select(desc, q, kc, vc, ctx, s, o, idx)
+        torch.cuda.synchronize()
+        return o, idx
     idx = None
     if not dense:
         idx = torch.empty((B, Hkv, top_k), dtype=torch.int32, device="cuda")
@@ -272,6 +278,10 @@ def test_decode_full_size_sampled(api, w):
     ref = _oracle_decode_rows(inp, rows, w.bs, w.top_k, dense=False)
     for (b, h), (ro, _) in ref.items():
         compare(f"decode o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+    of, idxf = _run_decode(api, inp, w.bs, w.top_k, fused=True)
+    np.testing.assert_array_equal(idxf.cpu().numpy(), want_idx)
+    for (b, h), (ro, _) in ref.items():
+        compare(f"fused decode o[{b},{h}]", host(of[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
     if w is syn.DECODE_512K:
         od, _ = _run_decode(api, inp, w.bs, w.top_k, dense=True)
         refd = _oracle_decode_rows(inp, rows[:2], w.bs, w.top_k, dense=True)
@@ -293,11 +303,39 @@ def test_decode_edge_cases(api, dtype, d):
     tol = BF16_TOL if dtype == torch.bfloat16 else F32_TOL
     G = Hq // Hkv
     rows = [(b, h) for b in range(B) for h in range(Hkv)]
-    for dense in (False, True):
-        o, idx = _run_decode(api, inp, bs, K, dense=dense)
+    modes = [("sparse", False, False), ("dense", True, False)]
+    if dtype == torch.bfloat16:
+        modes.append(("fused", False, True))
+    for name, dense, fused in modes:
+        o, idx = _run_decode(api, inp, bs, K, dense=dense, fused=fused)
         ref = _oracle_decode_rows(inp, rows, bs, K, dense)
         for (b, h), (ro, ridx) in ref.items():
             if not dense:
                 np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx)
-            compare(f"o[{b},{h}] dense={dense}", host(o[b, h * G:(h + 1) * G]), ro, **tol,
+            compare(f"o[{b},{h}] {name}", host(o[b, h * G:(h + 1) * G]), ro, **tol,
                     bf16_out=dtype == torch.bfloat16)
+
+
+def test_decode_cluster_sizes_and_ties(api):
+    """Row counts that pick every cluster size (1..8 CTAs per row), tie-heavy scores
+    (the selection splits equal keys across CTAs lowest index first), G = 1 and 8."""
+    bs = 64
+    # rows (B*Hkv) 1, 4, 16 -> 8 CTAs per row; 64 -> 4; 128 -> 2; 320 -> 1
+    for B, Hq, Hkv, K, nblk in ((1, 8, 1, 40, 300), (2, 16, 2, 20, 300), (4, 8, 4, 9, 300), (8, 16, 8, 3, 60),
+                                (16, 32, 8, 5, 40), (40, 8, 8, 3, 20), (3, 3, 3, 300, 300)):
+        Tmax = 64 * nblk + 5
+        ctx = torch.tensor([Tmax - 64 * (i % 3) for i in range(B)], dtype=torch.int32, device="cuda")
+        s = torch.round(_seeded((B, Hkv, Tmax // bs), 1.0, torch.float32, 61) * 2) / 2
+        inp = {
+            "q": _seeded((B, Hq, 128), 1.0, torch.bfloat16, 62),
+            "k_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 63),
+            "v_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 64),
+            "ctx_len": ctx, "s": s.contiguous(),
+        }
+        G = Hq // Hkv
+        o, idx = _run_decode(api, inp, bs, K, fused=True)
+        rows = [(b, h) for b in range(min(B, 3)) for h in range(Hkv)]
+        ref = _oracle_decode_rows(inp, rows, bs, K, False)
+        for (b, h), (ro, ridx) in ref.items():
+            np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx)
+            compare(f"o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)

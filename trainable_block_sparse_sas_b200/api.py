@@ -62,6 +62,8 @@ lib.sas_sparse_decode_workspace_size.restype = _sz
 lib.sas_sparse_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeDesc)]
 lib.sas_sparse_decode.restype = ctypes.c_int
 lib.sas_sparse_decode.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7 + [_sz, _vp]
+lib.sas_sparse_decode_select.restype = ctypes.c_int
+lib.sas_sparse_decode_select.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 5 + [_i32, _vp, _vp, _vp]
 lib.sas_sparse_decode_noalloc.restype = ctypes.c_int
 lib.sas_sparse_decode_noalloc.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7
 lib.sas_launch_count.restype = ctypes.c_uint64
@@ -135,6 +137,12 @@ def sas_sparse_decode(desc, q, k_cache, v_cache, ctx_len, idx, o, workspace, str
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.sas_sparse_decode(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx), _p(o),
                                  _p(workspace), ws_bytes, _stream(stream)), "sas_sparse_decode")
+
+
+def sas_sparse_decode_select(desc, q, k_cache, v_cache, ctx_len, s, o, idx_out=None, stream=None):
+    """Fused decode step: Top-K of s [B, Hkv, s_cols] and the gate-free attention."""
+    _check(lib.sas_sparse_decode_select(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(s),
+                                        s.shape[-1], _p(o), _p(idx_out), _stream(stream)), "sas_sparse_decode_select")
 
 
 def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream=None):

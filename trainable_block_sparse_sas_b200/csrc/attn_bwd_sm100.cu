@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             const float lse_c = a.lse_s[unit];
             bool ok = true;
             for (int t = 0; t < nlist; ++t) {
-                if (!mbar_wait(s_full(grp), t & 1, abort_flag, a.status)) {
+                if (!warp_wait(s_full(grp), t & 1, abort_flag, a.status)) {
                     ok = false;
                     break;
                 }
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                     if (lane == 0) part[t * 8 + wi] = rs;
                 }
             }
-            if (ok && mbar_wait(dq_done, 0, abort_flag, a.status)) {
+            if (ok && warp_wait(dq_done, 0, abort_flag, a.status)) {
                 tc_fence_after();
                 __nv_bfloat16* drow = a.dq + (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
 #pragma unroll
@@ -312,6 +312,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();  // lane 0 ran the MMA loop alone: reconverge before the .aligned dealloc
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -537,7 +538,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             const float Drow = a.Dbuf[ri];
             const bool diag = (c == m);
             const float off = (diag ? 0.f : (a.s[(ubase + c) * a.Cq + m] - a.lse_s[ubase + c]) * kLog2e) - lse2;
-            if (!mbar_wait(s_full(buf), (j >> 1) & 1, abort_flag, a.status)) {
+            if (!warp_wait(s_full(buf), (j >> 1) & 1, abort_flag, a.status)) {
                 ok = false;
                 break;
             }
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             }
             tc_fence_before();
             // P / dS smem buffers are free once the MMAs of item j-1 completed
-            if (j > 0 && !mbar_wait(item_done, (j - 1) & 1, abort_flag, a.status)) {
+            if (j > 0 && !warp_wait(item_done, (j - 1) & 1, abort_flag, a.status)) {
                 ok = false;
                 break;
             }
@@ -579,7 +580,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             fence_proxy_async_smem();
             mbar_arrive(p_ready);
         }
-        if (ok && mbar_wait(final_bar, 0, abort_flag, a.status)) {
+        if (ok && warp_wait(final_bar, 0, abort_flag, a.status)) {
             tc_fence_after();
             const int d = 32 * quad + lane;  // dV^T / dK^T: TMEM lane = head-dim index
 #pragma unroll
@@ -603,6 +604,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();  // lane 0 ran the MMA loop alone: reconverge before the .aligned dealloc
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             float m_used = -INFINITY, l = 0.f;
             bool ok = true;
             for (int t = 0; t < nsteps; ++t) {
-                if (!mbar_wait(s_full(grp), t & 1, abort_flag, a.status)) {
+                if (!warp_wait(s_full(grp), t & 1, abort_flag, a.status)) {
                     ok = false;
                     break;
                 }
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                 tc_fence_before();
                 mbar_arrive(p_ready(grp));
             }
-            if (ok && mbar_wait(o_done(grp), (nsteps - 1) & 1, abort_flag, a.status)) {
+            if (ok && warp_wait(o_done(grp), (nsteps - 1) & 1, abort_flag, a.status)) {
                 tc_fence_after();
                 const float inv_l = 1.f / l;
                 const int hq = h * G + g;
@@ -330,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();  // lane 0 ran the MMA loop alone: reconverge before the .aligned dealloc
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -1,0 +1,529 @@
+// decode_sm100.cu -- gate-free hard-Top-K decode for bf16 caches, head_dim 128,
+// block size 64 (jaehun.me review of SAS, walkthrough Step 6: at inference the
+// gate is dropped and only the Top-K blocks plus the current block are attended).
+//
+// One thread-block cluster of CL CTAs per (sequence, kv head); one launch per
+// decode step, no workspace:
+//   1. selection (optional, fused): the cluster's CTAs split the row's block
+//      scores, run a 4-pass 8-bit radix select of the K-th largest order key with
+//      histograms summed over distributed shared memory, and write the chosen
+//      blocks (ties to the lower index, ascending) into every CTA's list;
+//   2. attention: the attended list (current partial block first, then the
+//      history blocks) is split over the CTAs; a TMA ring streams each block's K
+//      and V (2 x 16 KB, 128-byte swizzle); all 8 consumer warps take every block,
+//      each warp 16 tokens and one half of the head dimension: S = q K^T and
+//      O += P V on the tensor cores with mma.sync m16n8k16 (the G <= 16 query heads
+//      of the group padded to 16 rows), online softmax in registers;
+//   3. the CTA's 8 warp partials merge in shared memory, then CTA 0 merges the
+//      cluster's partials over distributed shared memory and writes o.
+#include <cstring>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace sas {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kBS = 64;
+constexpr int kThreads = 288;  // warp 0: TMA producer; warps 1..8: consumers
+constexpr int kStages = 3;
+constexpr uint32_t kHalf = 64 * 128;   // 64 rows x 128 B: one 64-wide d slab of a block
+constexpr uint32_t kTile = 2 * kHalf;  // a block of K (or V): 16 KB
+constexpr uint32_t kStage = 2 * kTile;  // K + V
+constexpr int kQLd = 136;              // padded row (bf16 elements) of the q tile in smem
+
+struct DecArgs {
+    CUtensorMap tk, tv;  // caches as {d, Tmax, B*Hkv}, box {64, 64, 1}
+    const __nv_bfloat16* q;
+    const int32_t* ctx_len;
+    const int32_t* idx;  // mode 0
+    const float* s;      // mode 1
+    int32_t* idx_out;    // mode 1, nullable
+    __nv_bfloat16* o;
+    int* status;
+    int B, Hq, Hkv, Tmax, top_k, s_cols, mode;  // mode 0: given idx, 1: fused selection, 2: dense
+    float scale_log2;
+};
+
+struct Layout {
+    static constexpr uint32_t kRing = 0;
+    static constexpr uint32_t kQ = kRing + kStages * kStage;  // 16 rows x kQLd bf16
+    static constexpr uint32_t kBars = kQ + 16 * kQLd * 2;
+    static constexpr uint32_t kMisc = kBars + 8 * 2 * kStages;  // abort, bin, above, count, scratch
+    static constexpr uint32_t kHist = kMisc + 64;              // 2 x 256 ints
+    static constexpr uint32_t kGsum = kHist + 2 * 256 * 4;     // 256 ints
+    static constexpr uint32_t kScan = kGsum + 256 * 4;         // 40 ints
+    static constexpr uint32_t kCnt = kScan + 40 * 4;           // 2 ints (gt, eq) of this CTA
+    static constexpr uint32_t kCpart = kCnt + 16;              // [G][d + 2] floats
+    __host__ __device__ static uint32_t list_off(int G) { return kCpart + 4 * (uint32_t)G * (kD + 2); }
+    static size_t bytes(int G, int list_cap) { return 1024 + list_off(G) + 4 * (size_t)list_cap; }
+};
+
+__device__ __forceinline__ int block_sum_int(int v, int* scan) {
+    int tot;
+    block_exclusive_scan(v, scan, &tot);
+    return tot;
+}
+
+// Fused Top-K over the row's Cb block scores, split across the cluster.
+// Fills list[1 .. K] (ascending) in every CTA; returns the number selected.
+template <int CL>
+__device__ int cluster_topk(const DecArgs& a, int bh, int Cb, uint32_t rank, uint8_t* base, int* list) {
+    const int tid = threadIdx.x;
+    const int K = a.top_k;
+    if (K >= Cb) {
+        for (int i = tid; i < Cb; i += kThreads) list[1 + i] = i;
+        __syncthreads();
+        return Cb;
+    }
+    int* hist = reinterpret_cast<int*>(base + Layout::kHist);
+    int* gsum = reinterpret_cast<int*>(base + Layout::kGsum);
+    int* scan = reinterpret_cast<int*>(base + Layout::kScan);
+    int* cnt = reinterpret_cast<int*>(base + Layout::kCnt);
+    int* misc = reinterpret_cast<int*>(base + Layout::kMisc);
+    const float* srow = a.s + (long)bh * a.s_cols;
+    const int lo = (int)((long)rank * Cb / CL), hi = (int)((long)(rank + 1) * Cb / CL);
+    uint32_t prefix = 0u, pmask = 0u;
+    int remaining = K;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        int* hst = hist + (pass & 1) * 256;
+        if (tid < 256) hst[tid] = 0;
+        __syncthreads();
+        for (int m = lo + tid; m < hi; m += kThreads) {
+            const uint32_t key = order_key(srow[m]);
+            if ((key & pmask) == prefix) atomicAdd(&hst[(key >> shift) & 255u], 1);
+        }
+        cluster_sync();
+        if (tid < 256) {
+            const uint32_t local = smem_u32(&hst[tid]);
+            int tot = 0;
+#pragma unroll
+            for (int r = 0; r < CL; ++r) tot += (int)ld_dsmem_u32(mapa(local, (uint32_t)r));
+            gsum[tid] = tot;
+        }
+        __syncthreads();
+        if (tid < 32) {
+            int c8[8], sum = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                c8[q] = gsum[255 - (tid * 8 + q)];
+                sum += c8[q];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid >= o) incl += y;
+            }
+            const int excl = incl - sum;
+            if (excl < remaining && remaining <= incl) {
+                int acc = excl;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    if (acc + c8[q] >= remaining) {
+                        misc[1] = 255 - (tid * 8 + q);
+                        misc[2] = acc;
+                        break;
+                    }
+                    acc += c8[q];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)misc[1] << shift;
+        pmask |= 0xFFu << shift;
+        remaining -= misc[2];
+        __syncthreads();
+    }
+    // counts above / equal to the threshold key in this CTA's slice
+    int gt = 0, eq = 0;
+    for (int m = lo + tid; m < hi; m += kThreads) {
+        const uint32_t key = order_key(srow[m]);
+        gt += key > prefix;
+        eq += key == prefix;
+    }
+    gt = block_sum_int(gt, scan);
+    eq = block_sum_int(eq, scan);
+    if (tid == 0) {
+        cnt[0] = gt;
+        cnt[1] = eq;
+    }
+    cluster_sync();
+    // this CTA's output base and its share of the threshold-equal keys (lowest indices first)
+    int base_pos = 0, eq_before = 0;
+    for (int r = 0; r < (int)rank; ++r) {
+        const int g_r = (int)ld_dsmem_u32(mapa(smem_u32(&cnt[0]), (uint32_t)r));
+        const int e_r = (int)ld_dsmem_u32(mapa(smem_u32(&cnt[1]), (uint32_t)r));
+        base_pos += g_r + max(0, min(e_r, remaining - eq_before));
+        eq_before += e_r;
+    }
+    const int eq_quota = max(0, min(eq, remaining - eq_before));
+    int out = base_pos, eq_seen = 0;
+    for (int m0 = lo; m0 < hi; m0 += kThreads) {
+        const int m = m0 + tid;
+        const uint32_t key = m < hi ? order_key(srow[m]) : 0u;
+        const int is_eq = (m < hi && key == prefix) ? 1 : 0;
+        int tot_eq;
+        const int eq_rank = block_exclusive_scan(is_eq, scan, &tot_eq) + eq_seen;
+        const int take = (m < hi && (key > prefix || (is_eq && eq_rank < eq_quota))) ? 1 : 0;
+        int tot_take;
+        const int pos = block_exclusive_scan(take, scan, &tot_take) + out;
+        if (take && pos < K) {
+            const uint32_t local = smem_u32(&list[1 + pos]);
+#pragma unroll
+            for (int r = 0; r < CL; ++r) st_dsmem_u32(mapa(local, (uint32_t)r), (uint32_t)m);
+        }
+        eq_seen += tot_eq;
+        out += tot_take;
+    }
+    cluster_sync();
+    return K;
+}
+
+template <int CL>
+__global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __grid_constant__ DecArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(base);
+    const uint32_t ring = sbase + Layout::kRing;
+    const uint32_t bar0 = sbase + Layout::kBars;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (kStages + s); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(base + Layout::kMisc);
+    const int G = a.Hq / a.Hkv;
+    float* cpart = reinterpret_cast<float*>(base + Layout::kCpart);
+    int* list = reinterpret_cast<int*>(base + Layout::list_off(G));
+    __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(base + Layout::kQ);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int bh = blockIdx.y;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    int T = a.ctx_len[b];
+    T = max(1, min(T, a.Tmax));
+    const int t = T - 1, Cb = t / kBS;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 8);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tmap(&a.tk);
+        prefetch_tmap(&a.tv);
+    }
+    // q of the group, padded to 16 rows
+    for (int i = tid; i < 16 * kD; i += kThreads) {
+        const int r = i / kD, e = i % kD;
+        qs[r * kQLd + e] = r < G ? a.q[((long)b * a.Hq + h * G + r) * kD + e] : __float2bfloat16_rn(0.f);
+    }
+    // attended list: entry 0 = current (partial) block, entries 1.. = history blocks ascending
+    int nsel;
+    if (a.mode == 2) {
+        nsel = Cb;
+        __syncthreads();
+    } else if (a.mode == 0) {
+        if (tid == 0) {
+            const int32_t* row = a.idx + (long)bh * a.top_k;
+            int c = 0;
+            while (c < a.top_k && row[c] >= 0 && row[c] < Cb) {
+                list[1 + c] = row[c];
+                ++c;
+            }
+            reinterpret_cast<int*>(base + Layout::kMisc)[3] = c;
+        }
+        __syncthreads();
+        nsel = reinterpret_cast<int*>(base + Layout::kMisc)[3];
+    } else {
+        __syncthreads();
+        nsel = cluster_topk<CL>(a, bh, min(Cb, a.s_cols), rank, base, list);
+        if (rank == 0 && a.idx_out)
+            for (int i = tid; i < a.top_k; i += kThreads) a.idx_out[(long)bh * a.top_k + i] = i < nsel ? list[1 + i] : -1;
+    }
+    const int L = nsel + 1;
+    const int e0 = (int)((long)rank * L / CL), e1 = (int)((long)(rank + 1) * L / CL);
+    auto block_of = [&](int e) { return e == 0 ? Cb : (a.mode == 2 ? e - 1 : list[e]); };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int i = 0; e0 + i < e1; ++i) {
+                const int st = i % kStages;
+                if (i >= kStages && !mbar_wait(empty(st), (i / kStages - 1) & 1, abort_flag, a.status)) break;
+                const int row0 = block_of(e0 + i) * kBS;
+                const uint32_t dst = ring + st * kStage;
+                mbar_arrive_expect_tx(full(st), kStage);
+                tma_load_3d(dst, &a.tk, full(st), 0, row0, bh);
+                tma_load_3d(dst + kHalf, &a.tk, full(st), 64, row0, bh);
+                tma_load_3d(dst + kTile, &a.tv, full(st), 0, row0, bh);
+                tma_load_3d(dst + kTile + kHalf, &a.tv, full(st), 64, row0, bh);
+            }
+        }
+    } else {
+        // Every consumer warp takes every block of this CTA (one in-order consumer
+        // sequence per ring stage, so parity waits are exact): warp cw covers
+        // tokens [16 wg, 16 wg + 16) of the block and head-dim half dh of O.
+        const int cw = warp - 1;   // 0..7
+        const int wg = cw & 3;     // 16-token slice of the block
+        const int dh = cw >> 2;    // 64-wide half of the head dimension for P V
+        const int r0 = lane >> 2;  // fragment rows r0 and r0 + 8 (query heads)
+        const int cq = lane & 3;
+        float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+        float O[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) O[nt][0] = O[nt][1] = O[nt][2] = O[nt][3] = 0.f;
+        const uint32_t qbase = smem_u32(qs);
+        for (int i = 0; e0 + i < e1; ++i) {
+            const int st = i % kStages;
+            if (!warp_wait(full(st), (i / kStages) & 1, abort_flag, a.status)) break;
+            const int blk = block_of(e0 + i);
+            const uint32_t kb = ring + st * kStage, vb = kb + kTile;
+            const int tok0 = blk * kBS + 16 * wg;  // absolute first token of this warp's slice
+            const bool partial = tok0 + 15 > t;
+            if (partial) {  // partial block: zero this warp's V rows past the query (their P is 0)
+                if (lane < 16 && tok0 + lane > t) {
+                    uint8_t* row = base + Layout::kRing + st * kStage + kTile + dh * kHalf + (16 * wg + lane) * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4*>(row)[c] = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+            float sacc[2][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                uint32_t qa[4];
+                {
+                    // A = q rows (16) x d (16kk .. 16kk+15)
+                    const int rr = (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int cc = 16 * kk + (lane >> 4) * 8;
+                    ldmatrix_x4(qbase + (uint32_t)(rr * kQLd + cc) * 2u, qa[0], qa[1], qa[2], qa[3]);
+                }
+                const int half = kk >> 2, ch = (kk & 3) * 2 + ((lane >> 3) & 1);
+                const int j = 16 * wg + ((lane >> 4) & 1) * 8 + (lane & 7);
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(kb + half * kHalf + j * 128 + ((ch ^ (j & 7)) << 4), b0, b1, b2, b3);
+                mma_16816(sacc[0], qa, b0, b1);
+                mma_16816(sacc[1], qa, b2, b3);
+            }
+            // scores in log2 units; mask tokens past the query
+            float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = tok0 + 8 * nt + 2 * cq + (e & 1);
+                    float v = sacc[nt][e] * a.scale_log2;
+                    if (tok > t) v = -INFINITY;
+                    sacc[nt][e] = v;
+                    mx[e >> 1] = fmaxf(mx[e >> 1], v);
+                }
+            float alpha[2], mref[2];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+                mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+                const float mnew = fmaxf(m_r[rr], mx[rr]);
+                mref[rr] = mnew == -INFINITY ? 0.f : mnew;
+                alpha[rr] = ex2(m_r[rr] - mref[rr]);
+                m_r[rr] = mnew;
+            }
+            float p[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) p[nt][e] = ex2(sacc[nt][e] - mref[e >> 1]);
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) l_r[rr] *= alpha[rr];
+            l_r[0] += p[0][0] + p[0][1] + p[1][0] + p[1][1];
+            l_r[1] += p[0][2] + p[0][3] + p[1][2] + p[1][3];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                O[nt][0] *= alpha[0];
+                O[nt][1] *= alpha[0];
+                O[nt][2] *= alpha[1];
+                O[nt][3] *= alpha[1];
+            }
+            uint32_t pa[4];
+            pa[0] = pack_bf16x2(p[0][0], p[0][1]);
+            pa[1] = pack_bf16x2(p[0][2], p[0][3]);
+            pa[2] = pack_bf16x2(p[1][0], p[1][1]);
+            pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                const int ch = 2 * np + (lane >> 4);
+                const int j = 16 * wg + ((lane >> 3) & 1) * 8 + (lane & 7);
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(vb + dh * kHalf + j * 128 + ((ch ^ (j & 7)) << 4), b0, b1, b2, b3);
+                mma_16816(O[2 * np], pa, b0, b1);
+                mma_16816(O[2 * np + 1], pa, b2, b3);
+            }
+            // generic-proxy writes (the zeroed rows) before the stage goes back to TMA
+            if (partial) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(st));
+        }
+        // row sums over the 4 lanes sharing a row
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            l_r[rr] += __shfl_xor_sync(0xffffffffu, l_r[rr], 1);
+            l_r[rr] += __shfl_xor_sync(0xffffffffu, l_r[rr], 2);
+        }
+        // warp partials into the (now idle) ring: [warp][G][d + 2], this warp's d half only
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        float* wpart = reinterpret_cast<float*>(base + Layout::kRing);
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int g = r0 + 8 * rr;
+            if (g < G) {
+                float* dst = wpart + ((long)cw * G + g) * (kD + 2);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) {
+                    dst[64 * dh + 8 * nt + 2 * cq] = O[nt][2 * rr];
+                    dst[64 * dh + 8 * nt + 2 * cq + 1] = O[nt][2 * rr + 1];
+                }
+                if (cq == 0) {
+                    dst[kD] = m_r[rr];
+                    dst[kD + 1] = l_r[rr];
+                }
+            }
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        // merge the 4 token slices -> this CTA's partial (d < 128: warps of that d half;
+        // the running sum: the warps of half 0, which saw the same scores)
+        for (int i = tid - 32; i < G * (kD + 1); i += 256) {
+            const int g = i / (kD + 1), d = i % (kD + 1);
+            const int wbase = d < kD ? 4 * (d >> 6) : 0;
+            float M = -INFINITY;
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, wpart[((long)(wbase + w) * G + g) * (kD + 2) + kD]);
+            float acc = 0.f;
+            if (M != -INFINITY) {
+                for (int w = 0; w < 4; ++w) {
+                    const float* src = wpart + ((long)(wbase + w) * G + g) * (kD + 2);
+                    const float f = ex2(src[kD] - M);
+                    acc += (d < kD ? src[d] : src[kD + 1]) * f;
+                }
+            }
+            if (d < kD) cpart[g * (kD + 2) + d] = acc;
+            else {
+                cpart[g * (kD + 2) + kD] = M;
+                cpart[g * (kD + 2) + kD + 1] = acc;
+            }
+        }
+    }
+    __syncwarp();
+    cluster_sync();
+    if (rank == 0) {
+        const uint32_t cp_local = smem_u32(cpart);
+        for (int i = tid; i < G * kD; i += kThreads) {
+            const int g = i / kD, d = i % kD;
+            float M = -INFINITY;
+            for (int r = 0; r < CL; ++r)
+                M = fmaxf(M, ld_dsmem_f32(mapa(cp_local + 4u * (g * (kD + 2) + kD), (uint32_t)r)));
+            float num = 0.f, den = 0.f;
+            for (int r = 0; r < CL; ++r) {
+                const uint32_t pr = mapa(cp_local, (uint32_t)r);
+                const float mr = ld_dsmem_f32(pr + 4u * (g * (kD + 2) + kD));
+                if (mr == -INFINITY) continue;
+                const float f = ex2(mr - M);
+                num += ld_dsmem_f32(pr + 4u * (g * (kD + 2) + d)) * f;
+                den += ld_dsmem_f32(pr + 4u * (g * (kD + 2) + kD + 1)) * f;
+            }
+            a.o[((long)b * a.Hq + h * G + g) * kD + d] = __float2bfloat16_rn(num / den);
+        }
+    }
+    cluster_sync();  // keep every CTA's shared memory alive until CTA 0 has read it
+}
+
+bool encode_cache(CUtensorMap* map, const void* ptr, int Tmax, long rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)Tmax, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)Tmax * kD * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int CL>
+cudaError_t launch_cl(const DecArgs& a, int list_cap, cudaStream_t stream) {
+    const int G = a.Hq / a.Hkv;
+    const size_t smem = Layout::bytes(G, list_cap);
+    cudaError_t err =
+        cudaFuncSetAttribute(decode_cluster_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL, a.B * a.Hkv, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, decode_cluster_kernel<CL>, a);
+    if (err == cudaSuccess) count_launch();
+    return err;
+}
+
+}  // namespace
+
+bool decode_sm100_supported(const DecodeParams& p) {
+    if (!p.is_bf16 || p.d != kD || p.bs != kBS) return false;
+    const int G = p.Hq / p.Hkv;
+    if (G < 1 || G > 16) return false;
+    if ((reinterpret_cast<uintptr_t>(p.k) | reinterpret_cast<uintptr_t>(p.v)) & 15u) return false;
+    if ((long)p.B * p.Hkv > 65535) return false;
+    return Layout::bytes(G, p.top_k + 1) <= 227 * 1024;
+}
+
+// Cluster size: about two CTAs per SM over all rows, at most 8, at most the
+// attended blocks of a row.
+static int pick_cluster(const DecodeParams& p, int max_entries) {
+    const long rows = (long)p.B * p.Hkv;
+    int cl = 1;
+    while (cl < 8 && rows * cl * 2 <= 2L * 148 && cl * 2 <= max_entries) cl *= 2;
+    return cl;
+}
+
+cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,
+                                cudaStream_t stream) {
+    DecArgs a;
+    memset(&a, 0, sizeof(a));
+    const long rows = (long)p.B * p.Hkv;
+    if (!encode_cache(&a.tk, p.k, p.Tmax, rows) || !encode_cache(&a.tv, p.v, p.Tmax, rows))
+        return cudaErrorInvalidValue;
+    a.q = static_cast<const __nv_bfloat16*>(p.q);
+    a.ctx_len = p.ctx_len;
+    a.idx = p.idx;
+    a.s = s;
+    a.idx_out = idx_out;
+    a.o = static_cast<__nv_bfloat16*>(p.o);
+    a.status = p.status;
+    a.B = p.B;
+    a.Hq = p.Hq;
+    a.Hkv = p.Hkv;
+    a.Tmax = p.Tmax;
+    a.top_k = p.top_k;
+    a.s_cols = s_cols;
+    a.mode = s ? 1 : (p.idx ? 0 : 2);
+    a.scale_log2 = p.scale * kLog2e;
+    const int max_entries = a.mode == 2 ? (p.Tmax + kBS - 1) / kBS : p.top_k + 1;
+    const int list_cap = a.mode == 2 ? 1 : p.top_k + 1;
+    switch (pick_cluster(p, max_entries)) {
+        case 1: return launch_cl<1>(a, list_cap, stream);
+        case 2: return launch_cl<2>(a, list_cap, stream);
+        case 4: return launch_cl<4>(a, list_cap, stream);
+        default: return launch_cl<8>(a, list_cap, stream);
+    }
+}
+
+}  // namespace sas

@@ -41,6 +41,7 @@ struct DecodeParams {
     const int32_t* idx;  // nullptr: dense
     void* o;
     float* part;  // [B*Hkv, nsplit, G, d + 2] partial (o, m, l)
+    int* status;  // device status word (bounded waits)
     int B, Hq, Hkv, d, bs, top_k, Tmax, is_bf16, nsplit, per_split, list_max;
     float scale;
 };
@@ -62,5 +63,9 @@ size_t simt_max_smem(int D, int BS, int Cq);
 void decode_plan(DecodeParams& p);
 size_t decode_workspace(const DecodeParams& p);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+bool decode_sm100_supported(const DecodeParams& p);
+// s != nullptr: fused Top-K selection from s [B, Hkv, s_cols] (idx_out nullable)
+cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,
+                                cudaStream_t stream);
 
 }  // namespace sas

@@ -248,8 +248,30 @@ sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const v
     if (!idx) p.idx = nullptr;
     p.o = o;
     p.part = static_cast<float*>(workspace);
+    p.status = di.status;
+    if (decode_sm100_supported(p))
+        return from_cuda(launch_decode_sm100(p, nullptr, 0, nullptr, reinterpret_cast<cudaStream_t>(stream)));
     decode_plan(p);
     return from_cuda(launch_decode(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* ctx_len, const float* s, int32_t s_cols,
+                                    void* o, int32_t* idx_out, sas_stream_t stream) {
+    if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_cache || !v_cache || !ctx_len || !s || !o || s_cols <= 0) return SAS_ERR_INVALID_VALUE;
+    DecodeParams p = make_decode(desc);
+    p.q = q;
+    p.k = k_cache;
+    p.v = v_cache;
+    p.ctx_len = ctx_len;
+    p.idx = nullptr;
+    p.o = o;
+    if (!supported_decode(desc) || !decode_sm100_supported(p)) return SAS_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    if (device_info(&di) != cudaSuccess) return SAS_ERR_CUDA;
+    p.status = di.status;
+    return from_cuda(launch_decode_sm100(p, s, s_cols, idx_out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_device_status(sas_stream_t stream) {
