@@ -291,9 +291,12 @@ class TrainRunner:
         return {"o": self.o, "dq": self.dq, "dk": self.dk, "dv": self.dv, "ds": self.ds}
 
 
-def time_decode(api, w, steps: int, dense: bool = False):
-    """Median device time of select + decode (or the dense decode) with L2
-    flushed before every repetition."""
+def time_decode(api, w, steps: int, mode: str = "fused"):
+    """Median device time of one decode step with L2 flushed (a 512 MB read, so
+    no dirty lines are written back inside the timed window) before every
+    repetition.  mode: "fused" (sas_sparse_decode_select: selection + attention
+    in one launch), "two_call" (sas_topk_select then sas_sparse_decode), or
+    "dense" (sas_sparse_decode over every cached token)."""
     import torch
 
     from trainable_block_sparse_sas_b200 import synthetic as syn
@@ -304,19 +307,22 @@ def time_decode(api, w, steps: int, dense: bool = False):
     idx = torch.empty((w.B, w.Hkv, w.top_k), dtype=torch.int32, device="cuda")
     o = torch.empty_like(q)
     ws = api.workspace(api.sas_sparse_decode_workspace_size(desc), q.device)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
     s4 = s.view(w.B, w.Hkv, 1, -1)
 
     def run():
-        if not dense:
+        if mode == "fused":
+            api.sas_sparse_decode_select(desc, q, kc, vc, ctx, s, o, idx)
+            return
+        if mode == "two_call":
             api.sas_topk_select(s4, 1, s.shape[-1], w.top_k, idx=idx, ctx_len=ctx, block_size=w.bs)
-        api.sas_sparse_decode(desc, q, kc, vc, ctx, None if dense else idx, o, ws)
+        api.sas_sparse_decode(desc, q, kc, vc, ctx, None if mode == "dense" else idx, o, ws)
 
     for _ in range(3):
         run()
     times = []
     for _ in range(steps):
-        flush.zero_()
+        flush.sum()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         run()
@@ -465,14 +471,15 @@ def extras(api, args, peaks, peak_kind) -> dict:
     torch.cuda.empty_cache()
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     for w in (syn.DECODE_128K, syn.DECODE_512K):
-        ms = time_decode(api, w, steps=20)
+        ms = time_decode(api, w, steps=20, mode="fused")
         by = decode_bytes(w)
         gbs = by / (ms * 1e-3) / 1e9
         rec = {"ms": ms, "bytes": by, "gbs": gbs, "frac_of_hbm": gbs / hbm, "hbm_peak_gbs": hbm,
-               "peak_source": f"{peak_kind} copy", "l2": "flushed (512 MB write) before every repetition",
-               "includes": "Top-K selection + sparse decode"}
+               "peak_source": f"{peak_kind} copy", "l2": "flushed (512 MB read) before every repetition",
+               "includes": "Top-K selection + sparse decode in one launch (sas_sparse_decode_select)",
+               "two_call_ms": time_decode(api, w, steps=10, mode="two_call")}
         if w is syn.DECODE_512K:
-            msd = time_decode(api, w, steps=5, dense=True)
+            msd = time_decode(api, w, steps=5, mode="dense")
             byd = decode_bytes(w, dense=True)
             rec["dense_ms"] = msd
             rec["dense_gbs"] = byd / (msd * 1e-3) / 1e9
@@ -492,6 +499,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4096, help="tokens of the oracle's CPU-baseline sample")
     ap.add_argument("--reference-tokens", type=int, default=1024, help="tokens of the reference arm's sample")
+    ap.add_argument("--profile-decode", type=int, default=0, metavar="T",
+                    help="only run the fused decode of the 128K workload's geometry with a T-token cache "
+                         "(a small case for profiler captures) and print its timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -500,6 +510,14 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.profile_decode:
+        from trainable_block_sparse_sas_b200 import api
+        from trainable_block_sparse_sas_b200 import synthetic as syn
+
+        w = dataclasses.replace(syn.DECODE_128K, name="decode_128k_geometry", T=args.profile_decode)
+        ms = time_decode(api, w, steps=args.steps, mode="fused")
+        print(json.dumps({"workload": w.name, "T": w.T, "ms": ms, "gbs": decode_bytes(w) / (ms * 1e-3) / 1e9}))
         return
     if world > 1:
         import torch

@@ -14,8 +14,9 @@
 //      each warp 16 tokens and one half of the head dimension: S = q K^T and
 //      O += P V on the tensor cores with mma.sync m16n8k16 (the G <= 16 query heads
 //      of the group padded to 16 rows), online softmax in registers;
-//   3. the CTA's 8 warp partials merge in shared memory, then CTA 0 merges the
-//      cluster's partials over distributed shared memory and writes o.
+//   3. the CTA's 8 warp partials merge in shared memory, then every CTA merges a
+//      slice of the outputs from the cluster's partials over distributed shared
+//      memory and writes it to o.
 #include <cstring>
 
 #include "kernels.h"
@@ -62,6 +63,14 @@ struct Layout {
     static size_t bytes(int G, int list_cap) { return 1024 + list_off(G) + 4 * (size_t)list_cap; }
 };
 
+// Histogram increment with one shared-memory atomic per distinct bin in the
+// warp (scores concentrate in few top-byte bins, so plain atomics serialise).
+// Called by whole warps; bin < 0 means "no increment" for this lane.
+__device__ __forceinline__ void hist_add_warp(int* hist, int bin) {
+    const unsigned same = __match_any_sync(0xffffffffu, bin);
+    if (bin >= 0 && (int)(threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+}
+
 __device__ __forceinline__ int block_sum_int(int v, int* scan) {
     int tot;
     block_exclusive_scan(v, scan, &tot);
@@ -93,9 +102,14 @@ __device__ int cluster_topk(const DecArgs& a, int bh, int Cb, uint32_t rank, uin
         int* hst = hist + (pass & 1) * 256;
         if (tid < 256) hst[tid] = 0;
         __syncthreads();
-        for (int m = lo + tid; m < hi; m += kThreads) {
-            const uint32_t key = order_key(srow[m]);
-            if ((key & pmask) == prefix) atomicAdd(&hst[(key >> shift) & 255u], 1);
+        for (int m0 = lo; m0 < hi; m0 += kThreads) {
+            const int m = m0 + tid;
+            int bin = -1;
+            if (m < hi) {
+                const uint32_t key = order_key(srow[m]);
+                if ((key & pmask) == prefix) bin = (int)((key >> shift) & 255u);
+            }
+            hist_add_warp(hst, bin);
         }
         cluster_sync();
         if (tid < 256) {
@@ -184,6 +198,215 @@ __device__ int cluster_topk(const DecArgs& a, int bh, int Cb, uint32_t rank, uin
     return K;
 }
 
+// Local exact Top-K of this CTA's slice of the score row (keys staged in ring
+// stage 1), candidates sent to CTA 0 (ring stage 2) over distributed shared
+// memory; CTA 0 ranks the <= CL*K candidates by (score desc, index asc) and
+// writes the chosen blocks, ascending, into every CTA's list[1 .. K].
+// Needs a slice of <= kStage/4 keys and CL*K <= kStage/8 candidates.
+template <int CL>
+__device__ int cluster_topk_fast(const DecArgs& a, int bh, int Cb, uint32_t rank, uint8_t* base, int* list) {
+    const int tid = threadIdx.x;
+    const int K = a.top_k;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(base + Layout::kRing + kStage);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(base + Layout::kRing + 2 * kStage);  // [CL*K][2] on CTA 0
+    int* hist = reinterpret_cast<int*>(base + Layout::kHist);
+    int* gsum = reinterpret_cast<int*>(base + Layout::kGsum);  // [0..CL) candidate counts on CTA 0
+    int* scan = reinterpret_cast<int*>(base + Layout::kScan);
+    int* misc = reinterpret_cast<int*>(base + Layout::kMisc);
+    const float* srow = a.s + (long)bh * a.s_cols;
+    const int lo = (int)((long)rank * Cb / CL), hi = (int)((long)(rank + 1) * Cb / CL), n = hi - lo;
+    for (int i = tid; i < n; i += kThreads) keys[i] = order_key(srow[lo + i]);
+    if (tid == 0) misc[4] = 0;
+    __syncthreads();
+    uint32_t thr = 0u;   // keys above thr are taken; `rem` keys equal to thr, lowest index first
+    int rem = 0, gt = n;
+    if (n > K) {
+        uint32_t prefix = 0u, pmask = 0u;
+        int remaining = K;
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            if (tid < 256) hist[tid] = 0;
+            __syncthreads();
+            for (int i0 = 0; i0 < n; i0 += kThreads) {
+                const int i = i0 + tid;
+                int bin = -1;
+                if (i < n) {
+                    const uint32_t key = keys[i];
+                    if ((key & pmask) == prefix) bin = (int)((key >> shift) & 255u);
+                }
+                hist_add_warp(hist, bin);
+            }
+            __syncthreads();
+            if (tid < 32) {
+                int c8[8], sum = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    c8[q] = hist[255 - (tid * 8 + q)];
+                    sum += c8[q];
+                }
+                int incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (tid >= o) incl += y;
+                }
+                const int excl = incl - sum;
+                if (excl < remaining && remaining <= incl) {
+                    int acc = excl;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (acc + c8[q] >= remaining) {
+                            misc[1] = 255 - (tid * 8 + q);
+                            misc[2] = acc;
+                            break;
+                        }
+                        acc += c8[q];
+                    }
+                }
+            }
+            __syncthreads();
+            prefix |= (uint32_t)misc[1] << shift;
+            pmask |= 0xFFu << shift;
+            remaining -= misc[2];
+            __syncthreads();
+        }
+        thr = prefix;
+        rem = remaining;
+        gt = K - remaining;
+    }
+    // every CTA of the cluster is running before its shared memory is written remotely
+    cluster_sync();
+    // send candidates (key, block index) to CTA 0: all keys above thr, and the
+    // `rem` lowest-index keys equal to thr (ordered scan only when that matters)
+    const uint32_t cand0 = smem_u32(cand), cnt0 = smem_u32(gsum);
+    auto send = [&](int slot, uint32_t key, int m) {
+        const uint32_t dst = mapa(cand0 + 8u * (uint32_t)(rank * K + slot), 0u);
+        st_dsmem_u32(dst, key);
+        st_dsmem_u32(dst + 4u, (uint32_t)m);
+    };
+    if (n <= K) {
+        for (int i = tid; i < n; i += kThreads) send(i, keys[i], lo + i);
+        if (tid == 0) st_dsmem_u32(mapa(cnt0 + 4u * rank, 0u), (uint32_t)n);
+    } else {
+        int eq = 0;
+        for (int i = tid; i < n; i += kThreads) eq += keys[i] == thr;
+        int eq_tot;
+        block_exclusive_scan(eq, scan, &eq_tot);
+        if (eq_tot <= rem) {
+            for (int i = tid; i < n; i += kThreads)
+                if (keys[i] >= thr) send(atomicAdd(&misc[4], 1), keys[i], lo + i);
+        } else {
+            int out = 0, eq_seen = 0;
+            for (int i0 = 0; i0 < n; i0 += kThreads) {
+                const int i = i0 + tid;
+                const uint32_t key = i < n ? keys[i] : 0u;
+                const int is_eq = (i < n && key == thr) ? 1 : 0;
+                int te;
+                const int er = block_exclusive_scan(is_eq, scan, &te) + eq_seen;
+                const int take = (i < n && (key > thr || (is_eq && er < rem))) ? 1 : 0;
+                int tt;
+                const int pos = block_exclusive_scan(take, scan, &tt) + out;
+                if (take) send(pos, key, lo + i);
+                eq_seen += te;
+                out += tt;
+            }
+        }
+        if (tid == 0) st_dsmem_u32(mapa(cnt0 + 4u * rank, 0u), (uint32_t)(gt + rem));
+    }
+    cluster_sync();
+    if (rank == 0 && K <= 32) {
+        // Each list (<= 32 candidates, one per lane) is sorted by warp `r` on the
+        // 64-bit key (order key, then the complement of the index: larger = better,
+        // equal scores resolve to the lower index).  A candidate's rank is its place in
+        // its own list plus, for every other list, how many entries beat it (binary
+        // search); ranks are unique, so the chosen K fill slots 0..K-1.
+        unsigned long long* sorted = reinterpret_cast<unsigned long long*>(keys);  // [CL][32]
+        unsigned long long* chosen = sorted + CL * 32;                              // [K]
+        const int w = tid >> 5, ln = tid & 31;
+        if (w < CL) {
+            const int c = gsum[w];
+            unsigned long long v = 0ull;
+            if (ln < c) {
+                const int s = w * K + ln;
+                v = ((unsigned long long)cand[2 * s] << 32) | (0xFFFFFFFFu - cand[2 * s + 1]);
+            }
+#pragma unroll
+            for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+                for (int j = k >> 1; j > 0; j >>= 1) {
+                    const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
+                    const bool desc = (ln & k) == 0;  // overall order: descending
+                    const bool lower = (ln & j) == 0;
+                    const bool keep_max = (lower == desc);
+                    v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+                }
+            }
+            sorted[w * 32 + ln] = v;
+        }
+        __syncthreads();
+        for (int s = tid; s < CL * 32; s += kThreads) {
+            const int r = s >> 5, pidx = s & 31;
+            if (pidx >= gsum[r]) continue;
+            const unsigned long long key = sorted[s];
+            int rk = pidx;
+            for (int r2 = 0; r2 < CL; ++r2) {
+                if (r2 == r) continue;
+                int lo2 = 0, hi2 = gsum[r2];  // count entries of list r2 greater than key
+                while (lo2 < hi2) {
+                    const int mid = (lo2 + hi2) >> 1;
+                    if (sorted[r2 * 32 + mid] > key) lo2 = mid + 1;
+                    else hi2 = mid;
+                }
+                rk += lo2;
+            }
+            if (rk < K) chosen[rk] = key;
+        }
+        __syncthreads();
+        for (int j = tid; j < K; j += kThreads) {
+            const uint32_t m = 0xFFFFFFFFu - (uint32_t)(chosen[j] & 0xFFFFFFFFull);
+            int pos = 0;
+            for (int j2 = 0; j2 < K; ++j2) pos += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m;
+            const uint32_t local = smem_u32(&list[1 + pos]);
+#pragma unroll
+            for (int r = 0; r < CL; ++r) st_dsmem_u32(mapa(local, (uint32_t)r), m);
+        }
+    } else if (rank == 0) {
+        // a candidate is chosen when fewer than K candidates beat it; its place in the
+        // ascending list is the number of chosen candidates with a lower index
+        const int N = CL * K;
+        int* chosen = reinterpret_cast<int*>(keys);  // reuse stage 1: [N] flags
+        for (int s = tid; s < N; s += kThreads) {
+            const int r = s / K;
+            int ok = 0;
+            if (s - r * K < gsum[r]) {
+                const uint32_t key = cand[2 * s], m = cand[2 * s + 1];
+                int beats = 0;
+                for (int r2 = 0; r2 < CL; ++r2)
+                    for (int s2 = r2 * K; s2 < r2 * K + gsum[r2]; ++s2) {
+                        const uint32_t k2 = cand[2 * s2], m2 = cand[2 * s2 + 1];
+                        beats += (k2 > key) || (k2 == key && m2 < m);
+                    }
+                ok = beats < K;
+            }
+            chosen[s] = ok;
+        }
+        __syncthreads();
+        for (int s = tid; s < N; s += kThreads) {
+            if (!chosen[s]) continue;
+            const uint32_t m = cand[2 * s + 1];
+            int pos = 0;
+            for (int s2 = 0; s2 < N; ++s2) pos += chosen[s2] && cand[2 * s2 + 1] < m;
+            const uint32_t local = smem_u32(&list[1 + pos]);
+#pragma unroll
+            for (int r = 0; r < CL; ++r) st_dsmem_u32(mapa(local, (uint32_t)r), m);
+        }
+    }
+    // generic-proxy writes to ring stages 1 and 2 before TMA reuses them
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    cluster_sync();
+    return K;
+}
+
 template <int CL>
 __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __grid_constant__ DecArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -228,30 +451,48 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         nsel = Cb;
         __syncthreads();
     } else if (a.mode == 0) {
-        if (tid == 0) {
-            const int32_t* row = a.idx + (long)bh * a.top_k;
-            int c = 0;
-            while (c < a.top_k && row[c] >= 0 && row[c] < Cb) {
-                list[1 + c] = row[c];
-                ++c;
-            }
-            reinterpret_cast<int*>(base + Layout::kMisc)[3] = c;
+        // the valid prefix of the ascending, -1 padded row: entries before the first
+        // one outside [0, Cb)
+        int* misc = reinterpret_cast<int*>(base + Layout::kMisc);
+        if (tid == 0) misc[3] = a.top_k;
+        __syncthreads();
+        const int32_t* row = a.idx + (long)bh * a.top_k;
+        for (int c = tid; c < a.top_k; c += kThreads) {
+            const int v = row[c];
+            list[1 + c] = v;
+            if (v < 0 || v >= Cb) atomicMin(&misc[3], c);
         }
         __syncthreads();
-        nsel = reinterpret_cast<int*>(base + Layout::kMisc)[3];
+        nsel = misc[3];
     } else {
         __syncthreads();
-        nsel = cluster_topk<CL>(a, bh, min(Cb, a.s_cols), rank, base, list);
+        // the current block (entry 0, on CTA 0) loads while the selection runs
+        if (rank == 0 && tid == 0) {
+            const int row0 = Cb * kBS;
+            mbar_arrive_expect_tx(full(0), kStage);
+            tma_load_3d(ring, &a.tk, full(0), 0, row0, bh);
+            tma_load_3d(ring + kHalf, &a.tk, full(0), 64, row0, bh);
+            tma_load_3d(ring + kTile, &a.tv, full(0), 0, row0, bh);
+            tma_load_3d(ring + kTile + kHalf, &a.tv, full(0), 64, row0, bh);
+        }
+        const int Csel = min(Cb, a.s_cols);
+        const int chunk = (Csel + CL - 1) / CL;
+        if (a.top_k < Csel && chunk <= (int)(kStage / 4) && CL * a.top_k <= (int)(kStage / 8))
+            nsel = cluster_topk_fast<CL>(a, bh, Csel, rank, base, list);
+        else
+            nsel = cluster_topk<CL>(a, bh, Csel, rank, base, list);
         if (rank == 0 && a.idx_out)
             for (int i = tid; i < a.top_k; i += kThreads) a.idx_out[(long)bh * a.top_k + i] = i < nsel ? list[1 + i] : -1;
     }
     const int L = nsel + 1;
-    const int e0 = (int)((long)rank * L / CL), e1 = (int)((long)(rank + 1) * L / CL);
+    // ceil split: CTA 0 always owns entry 0 (the current block, prefetched in mode 1)
+    const int e0 = (int)(((long)rank * L + CL - 1) / CL), e1 = (int)(((long)(rank + 1) * L + CL - 1) / CL);
     auto block_of = [&](int e) { return e == 0 ? Cb : (a.mode == 2 ? e - 1 : list[e]); };
 
     if (warp == 0) {
         if (lane == 0) {
-            for (int i = 0; e0 + i < e1; ++i) {
+            const int first = (a.mode == 1 && rank == 0) ? 1 : 0;  // entry 0 already in flight
+            for (int i = first; e0 + i < e1; ++i) {
                 const int st = i % kStages;
                 if (i >= kStages && !mbar_wait(empty(st), (i / kStages - 1) & 1, abort_flag, a.status)) break;
                 const int row0 = block_of(e0 + i) * kBS;
@@ -416,26 +657,37 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     }
     __syncwarp();
     cluster_sync();
-    if (rank == 0) {
+    {
+        // every CTA merges its slice of the G*128 outputs from the cluster's partials
         const uint32_t cp_local = smem_u32(cpart);
-        for (int i = tid; i < G * kD; i += kThreads) {
+        const int total = G * kD;
+        const int per = (total + CL - 1) / CL;
+        const int o0 = (int)rank * per, o1 = min(total, o0 + per);
+        for (int i = o0 + tid; i < o1; i += kThreads) {
             const int g = i / kD, d = i % kD;
-            float M = -INFINITY;
-            for (int r = 0; r < CL; ++r)
-                M = fmaxf(M, ld_dsmem_f32(mapa(cp_local + 4u * (g * (kD + 2) + kD), (uint32_t)r)));
-            float num = 0.f, den = 0.f;
+            float mr[CL], num[CL], den[CL];
+#pragma unroll
             for (int r = 0; r < CL; ++r) {
-                const uint32_t pr = mapa(cp_local, (uint32_t)r);
-                const float mr = ld_dsmem_f32(pr + 4u * (g * (kD + 2) + kD));
-                if (mr == -INFINITY) continue;
-                const float f = ex2(mr - M);
-                num += ld_dsmem_f32(pr + 4u * (g * (kD + 2) + d)) * f;
-                den += ld_dsmem_f32(pr + 4u * (g * (kD + 2) + kD + 1)) * f;
+                const uint32_t pr = mapa(cp_local, (uint32_t)r) + 4u * (uint32_t)(g * (kD + 2));
+                mr[r] = ld_dsmem_f32(pr + 4u * kD);
+                den[r] = ld_dsmem_f32(pr + 4u * (kD + 1));
+                num[r] = ld_dsmem_f32(pr + 4u * d);
             }
-            a.o[((long)b * a.Hq + h * G + g) * kD + d] = __float2bfloat16_rn(num / den);
+            float M = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < CL; ++r) M = fmaxf(M, mr[r]);
+            float n_ = 0.f, d_ = 0.f;
+#pragma unroll
+            for (int r = 0; r < CL; ++r) {
+                if (mr[r] == -INFINITY) continue;
+                const float f = ex2(mr[r] - M);
+                n_ += num[r] * f;
+                d_ += den[r] * f;
+            }
+            a.o[((long)b * a.Hq + h * G + g) * kD + d] = __float2bfloat16_rn(n_ / d_);
         }
     }
-    cluster_sync();  // keep every CTA's shared memory alive until CTA 0 has read it
+    cluster_sync();  // keep every CTA's shared memory alive until all remote reads are done
 }
 
 bool encode_cache(CUtensorMap* map, const void* ptr, int Tmax, long rows) {

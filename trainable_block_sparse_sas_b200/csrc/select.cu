@@ -65,9 +65,17 @@ __global__ void __launch_bounds__(kThreads)
         const int shift = 24 - 8 * pass;
         for (int i = tid; i < 256; i += nt) hist[i] = 0;
         __syncthreads();
-        for (int m = tid; m < c; m += nt) {
-            const uint32_t key = order_key(srow[m]);
-            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        for (int m0 = 0; m0 < c; m0 += nt) {
+            // one shared-memory atomic per distinct bin in the warp (scores crowd into
+            // few top-byte bins, so per-lane atomics would serialise)
+            const int m = m0 + tid;
+            int bin = -1;
+            if (m < c) {
+                const uint32_t key = order_key(srow[m]);
+                if ((key & pmask) == prefix) bin = (int)((key >> shift) & 255u);
+            }
+            const unsigned same = __match_any_sync(0xffffffffu, bin);
+            if (bin >= 0 && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
         }
         __syncthreads();
         if (tid < 32) {
