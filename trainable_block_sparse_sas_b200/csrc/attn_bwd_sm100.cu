@@ -93,7 +93,8 @@ struct DqLayout {
     static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
     static constexpr uint32_t kList = kMisc + 16;
-    __host__ __device__ static uint32_t part_off(int Cq) { return (kList + 4 * (uint32_t)(Cq + 1) + 15) & ~15u; }
+    // list [Cq + 1] ints, biases [Cq + 1] floats, then the per-warp dlogg partials
+    __host__ __device__ static uint32_t part_off(int Cq) { return (kList + 8 * (uint32_t)(Cq + 1) + 15) & ~15u; }
     static size_t bytes(int Cq) { return 1024 + part_off(Cq) + 32 * (size_t)(Cq + 1); }
 };
 
@@ -119,11 +120,12 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     float* tot_sh = reinterpret_cast<float*>(base + L::kMisc + 12);
     int* list = reinterpret_cast<int*>(base + L::kList);
     float* part = reinterpret_cast<float*>(base + L::part_off(a.Cq));  // [slot][8 softmax warps]
+    float* bias2 = reinterpret_cast<float*>(base + L::kList + 4 * (a.Cq + 1));  // log-gate, log2 units
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = a.B * a.Hkv;
-    const int c = a.Cq - 1 - (int)(blockIdx.x / BH);
-    const int bh = (int)(blockIdx.x % BH);
+    // head-major order (concurrent CTAs share one KV head in L2), long query blocks first
+    const int c = a.Cq - 1 - (int)(blockIdx.x % a.Cq);
+    const int bh = (int)(blockIdx.x / a.Cq);
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long unit = (long)bh * a.Cq + c;
 
@@ -141,24 +143,37 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         mbar_init(dq_done, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
-        int cnt = 0;
-        if (a.full_scope) {
-            for (int m = 0; m < c; ++m) list[cnt++] = m;
-        } else {
-            const int kk = min(a.top_k, c);
-            const int32_t* row = a.idx + unit * a.top_k;
-            for (int i = 0; i < kk; ++i) {
-                const int v = row[i];
-                if (v >= 0 && v < c) list[cnt++] = v;
-            }
-        }
-        list[cnt] = c;
-        *list_count = cnt + 1;
         fence_barrier_init();
         prefetch_tmap(&a.tq);
         prefetch_tmap(&a.tdo);
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
+    }
+    if (warp == 0) {
+        // attended history blocks (ascending) with their log-gate biases, then the
+        // current block (bias 0); lanes read the selection in parallel
+        const float* srow = a.s + unit * a.Cq;
+        const float lse_c = a.lse_s[unit];
+        int cnt = 0;
+        const int kk = a.full_scope ? c : min(a.top_k, c);
+        const int32_t* row = a.idx + unit * a.top_k;
+        for (int base_i = 0; base_i < kk; base_i += 32) {
+            const int i = base_i + lane;
+            const int v = i < kk ? (a.full_scope ? i : row[i]) : -1;
+            const bool ok = v >= 0 && v < c;
+            const unsigned bal = __ballot_sync(0xffffffffu, ok);
+            if (ok) {
+                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                list[pos] = v;
+                bias2[pos] = (srow[v] - lse_c) * kLog2e;
+            }
+            cnt += __popc(bal);
+        }
+        if (lane == 0) {
+            list[cnt] = c;
+            bias2[cnt] = 0.f;
+            *list_count = cnt + 1;
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -249,8 +264,6 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
             const uint32_t tS = tmem + lane_off + grp * 128, tP = tS + 64;
             const uint32_t tQ = tmem + lane_off + 256 + grp * 128;
-            const float* srow = a.s + unit * a.Cq;
-            const float lse_c = a.lse_s[unit];
             bool ok = true;
             for (int t = 0; t < nlist; ++t) {
                 if (!warp_wait(s_full(grp), t & 1, abort_flag, a.status)) {
@@ -258,30 +271,41 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                     break;
                 }
                 tc_fence_after();
-                const int blk = list[t];
-                const bool cur = (blk == c);
-                const float off = (cur ? 0.f : (srow[blk] - lse_c) * kLog2e) - lse2;
-                float rs = 0.f;
+                const bool cur = (t == nlist - 1);
+                const float off = bias2[t] - lse2;
+                const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
+                const uint64_t negD2 = f2_pack(-Drow, -Drow);
+                uint64_t rs2 = 0ull;
                 uint32_t pk[32];
+                {
+                    uint32_t s0r[32], s1r[32], d0r[32], d1r[32];
+                    tmem_ld64_sync(tS, s0r, s1r);
+                    tmem_ld64_sync(tP, d0r, d1r);
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    uint32_t sr[32], dr[32];
-                    tmem_ld32_sync(tS + ch * 32, sr);
-                    tmem_ld32_sync(tP + ch * 32, dr);
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        float dsv[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int j = 2 * jj + e, key = ch * 32 + j;
-                            float p = ex2(fmaf(__uint_as_float(sr[j]), a.scale_log2, off));
-                            if (cur && key > tok) p = 0.f;
-                            dsv[e] = p * (__uint_as_float(dr[j]) - Drow);
-                            rs += dsv[e];
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const uint32_t* sr = jj < 16 ? s0r : s1r;
+                        const uint32_t* dr = jj < 16 ? d0r : d1r;
+                        const int jl = (jj & 15) * 2;
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[jl]), __uint_as_float(sr[jl + 1])), sc2, off2), x0,
+                                  x1);
+                        float p0 = ex2(x0), p1 = ex2(x1);
+                        if (cur) {
+                            if (2 * jj > tok) p0 = 0.f;
+                            if (2 * jj + 1 > tok) p1 = 0.f;
                         }
-                        pk[ch * 16 + jj] = pack_bf16x2(dsv[0], dsv[1]);
+                        const uint64_t ds2 = f2_mul(
+                            f2_pack(p0, p1),
+                            f2_add(f2_pack(__uint_as_float(dr[jl]), __uint_as_float(dr[jl + 1])), negD2));
+                        rs2 = f2_add(rs2, ds2);
+                        float d0, d1;
+                        f2_unpack(ds2, d0, d1);
+                        pk[jj] = pack_bf16x2(d0, d1);
                     }
                 }
+                float rsa, rsb;
+                f2_unpack(rs2, rsa, rsb);
+                float rs = rsa + rsb;
                 tmem_st32(tS, pk);
                 tmem_wait_st();
                 tc_fence_before();
@@ -344,7 +368,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
 // ============================================================================
 // dk / dv kernel
 // ============================================================================
-constexpr int kKvThreads = 192;
+constexpr int kKvThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 two softmax groups (key halves)
 
 struct DkvLayout {
     static constexpr uint32_t kK = 0;                     // 2 slabs x 64 rows
@@ -401,9 +425,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     int* list = scan + 40;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = a.B * a.Hkv;
-    const int m = (int)(blockIdx.x / BH);  // early (widely selected) key blocks first
-    const int bh = (int)(blockIdx.x % BH);
+    // head-major order (concurrent CTAs share one KV head's Q/dO in L2); within a
+    // head, early (widely selected) key blocks first
+    const int m = (int)(blockIdx.x % a.Cq);
+    const int bh = (int)(blockIdx.x / a.Cq);
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long ubase = (long)bh * a.Cq;
 
@@ -426,7 +451,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         }
         mbar_init(s_full(0), 1);
         mbar_init(s_full(1), 1);
-        mbar_init(p_ready, 128);
+        mbar_init(p_ready, 256);
         mbar_init(item_done, 1);
         mbar_init(final_bar, 1);
         mbar_init(drain, 1);
@@ -496,11 +521,16 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                     issue_s(0);
                 }
             }
+            // S/dP of item j+1 goes ahead of dV/dK of item j only when its Q/dO tiles
+            // have already landed; otherwise dV/dK of item j is issued first, so that its
+            // stage is released (and the load of item j+2 starts) without waiting.
+            int next_s = 1;
             for (int j = 0; ok && j < nitems; ++j) {
-                if (j + 1 < nitems) {
-                    if (!mbar_wait(qd_full((j + 1) % kStages), ((j + 1) / kStages) & 1, abort_flag, a.status)) break;
+                if (next_s == j + 1 && next_s < nitems &&
+                    mbar_try_wait(qd_full(next_s % kStages), (next_s / kStages) & 1)) {
                     tc_fence_after();
-                    issue_s(j + 1);
+                    issue_s(next_s);
+                    ++next_s;
                 }
                 if (!mbar_wait(p_ready, j & 1, abort_flag, a.status)) break;
                 tc_fence_after();
@@ -518,6 +548,12 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                 }
                 mma_commit(item_done);
                 if (j + kStages < nitems) mma_commit(qd_empty(st));
+                if (next_s == j + 1 && next_s < nitems) {
+                    if (!mbar_wait(qd_full(next_s % kStages), (next_s / kStages) & 1, abort_flag, a.status)) break;
+                    tc_fence_after();
+                    issue_s(next_s);
+                    ++next_s;
+                }
             }
             mma_commit(final_bar);
             mma_commit(drain);
@@ -525,45 +561,67 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         }
     } else {
         const int quad = warp & 3;
-        const int row = 32 * quad + lane;  // row of the 128-row item
+        const int kw = (warp - 2) >> 2;       // key half of the block handled by this group
+        const int row = 32 * quad + lane;     // row of the 128-row item
         const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
         bool ok = true;
-        for (int j = 0; j < nitems; ++j) {
-            const int buf = j & 1;
+        // per-item row statistics, fetched one item ahead
+        auto fetch = [&](int j, float& off, float& dneg, int& tok, bool& diag) {
             const int c = list[j / MT], i = j % MT;
             const int r_unit = 128 * i + row;
-            const int tok = r_unit / G, g = r_unit % G;
+            tok = r_unit / G;
+            const int g = r_unit % G;
             const long ri = ((long)b * a.Hq + h * G + g) * a.n + c * kBS + tok;
-            const float lse2 = a.lse[ri] * kLog2e;
-            const float Drow = a.Dbuf[ri];
-            const bool diag = (c == m);
-            const float off = (diag ? 0.f : (a.s[(ubase + c) * a.Cq + m] - a.lse_s[ubase + c]) * kLog2e) - lse2;
+            diag = (c == m);
+            const float bias = diag ? 0.f : (a.s[(ubase + c) * a.Cq + m] - a.lse_s[ubase + c]) * kLog2e;
+            off = bias - a.lse[ri] * kLog2e;
+            dneg = -a.Dbuf[ri];
+        };
+        float off = 0.f, dneg = 0.f;
+        int tok = 0;
+        bool diag = false;
+        if (nitems > 0) fetch(0, off, dneg, tok, diag);
+        for (int j = 0; j < nitems; ++j) {
+            const int buf = j & 1;
+            float n_off = 0.f, n_dneg = 0.f;
+            int n_tok = 0;
+            bool n_diag = false;
+            if (j + 1 < nitems) fetch(j + 1, n_off, n_dneg, n_tok, n_diag);
             if (!warp_wait(s_full(buf), (j >> 1) & 1, abort_flag, a.status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t pp[32], dd[32];
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
+            const uint64_t dn2 = f2_pack(dneg, dneg);
+            uint32_t pp[16], dd[16];
+            {
                 uint32_t sr[32], dr[32];
-                tmem_ld32_sync(tmem + lane_off + buf * 128 + ch * 32, sr);
-                tmem_ld32_sync(tmem + lane_off + buf * 128 + 64 + ch * 32, dr);
+                tmem_ld32x2_sync(tmem + lane_off + buf * 128 + 32 * kw, tmem + lane_off + buf * 128 + 64 + 32 * kw,
+                                 sr, dr);
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
-                    float pv[2], dv[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int jx = 2 * jj + e, key = ch * 32 + jx;
-                        float p = ex2(fmaf(__uint_as_float(sr[jx]), a.scale_log2, off));
-                        if (diag && key > tok) p = 0.f;
-                        pv[e] = p;
-                        dv[e] = p * (__uint_as_float(dr[jx]) - Drow);
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * jj]), __uint_as_float(sr[2 * jj + 1])), sc2, off2),
+                              x0, x1);
+                    float p0 = ex2(x0), p1 = ex2(x1);
+                    if (diag) {
+                        const int key = 32 * kw + 2 * jj;
+                        if (key > tok) p0 = 0.f;
+                        if (key + 1 > tok) p1 = 0.f;
                     }
-                    pp[ch * 16 + jj] = pack_bf16x2(pv[0], pv[1]);
-                    dd[ch * 16 + jj] = pack_bf16x2(dv[0], dv[1]);
+                    float d0, d1;
+                    f2_unpack(f2_mul(f2_pack(p0, p1),
+                                     f2_add(f2_pack(__uint_as_float(dr[2 * jj]), __uint_as_float(dr[2 * jj + 1])), dn2)),
+                              d0, d1);
+                    pp[jj] = pack_bf16x2(p0, p1);
+                    dd[jj] = pack_bf16x2(d0, d1);
                 }
             }
+            off = n_off;
+            dneg = n_dneg;
+            tok = n_tok;
+            diag = n_diag;
             tc_fence_before();
             // P / dS smem buffers are free once the MMAs of item j-1 completed
             if (j > 0 && !warp_wait(item_done, (j - 1) & 1, abort_flag, a.status)) {
@@ -572,8 +630,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             }
             const uint32_t rbase = (uint32_t)row * 128u;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint32_t sw = (uint32_t)((ch ^ (row & 7)) * 16);
+            for (int ch = 0; ch < 4; ++ch) {
+                const int chunk = 4 * kw + ch;  // 16-byte chunk = 8 keys
+                const uint32_t sw = (uint32_t)((chunk ^ (row & 7)) * 16);
                 st_shared_v4(sP + rbase + sw, pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
                 st_shared_v4(sDS + rbase + sw, dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
             }
@@ -582,21 +641,19 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         }
         if (ok && warp_wait(final_bar, 0, abort_flag, a.status)) {
             tc_fence_after();
-            const int d = 32 * quad + lane;  // dV^T / dK^T: TMEM lane = head-dim index
+            // group 0 writes dv, group 1 dk; TMEM lane = head-dim index
+            const int d = 32 * quad + lane;
+            __nv_bfloat16* dst = kw == 0 ? a.dv : a.dk;
+            const float mul = kw == 0 ? 1.f : a.scale;
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16* dst = which == 0 ? a.dv : a.dk;
-                const float mul = which == 0 ? 1.f : a.scale;
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t r[32];
+                tmem_ld32_sync(tmem + lane_off + 256 + kw * 64 + ch * 32, r);
 #pragma unroll
-                for (int ch = 0; ch < 2; ++ch) {
-                    uint32_t r[32];
-                    tmem_ld32_sync(tmem + lane_off + 256 + which * 64 + ch * 32, r);
-#pragma unroll
-                    for (int jx = 0; jx < 32; ++jx) {
-                        const int key = ch * 32 + jx;
-                        dst[(((long)b * a.n + m * kBS + key) * a.Hkv + h) * kD + d] =
-                            __float2bfloat16_rn(__uint_as_float(r[jx]) * mul);
-                    }
+                for (int jx = 0; jx < 32; ++jx) {
+                    const int key = ch * 32 + jx;
+                    dst[(((long)b * a.n + m * kBS + key) * a.Hkv + h) * kD + d] =
+                        __float2bfloat16_rn(__uint_as_float(r[jx]) * mul);
                 }
             }
         }

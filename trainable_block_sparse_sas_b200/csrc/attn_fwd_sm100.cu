@@ -68,8 +68,8 @@ struct FwdLayout {
     // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], drain
     static constexpr int kNumBars = 1 + 2 * kStages + 6 + 1;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;  // tmem base, abort flag, list count
-    static constexpr uint32_t kList = kMisc + 16;
-    static size_t bytes(int Cq) { return 1024 + kList + 4 * (size_t)(Cq + 1); }
+    static constexpr uint32_t kList = kMisc + 16;  // [Cq + 1] ints, then [Cq + 1] biases
+    static size_t bytes(int Cq) { return 1024 + kList + 8 * (size_t)(Cq + 1); }
 };
 
 __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
@@ -104,11 +104,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
     int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
     int* list = reinterpret_cast<int*>(base + L::kList);
+    float* bias2 = reinterpret_cast<float*>(base + L::kList + 4 * (a.Cq + 1));  // log-gate, log2 units
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = a.B * a.Hkv;
-    const int c = a.Cq - 1 - (int)(blockIdx.x / BH);  // long (late) query blocks first
-    const int bh = (int)(blockIdx.x % BH);
+    // head-major order: concurrent CTAs share one KV head's K/V in L2; within a
+    // head, long (late) query blocks first
+    const int c = a.Cq - 1 - (int)(blockIdx.x % a.Cq);
+    const int bh = (int)(blockIdx.x / a.Cq);
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long unit = (long)bh * a.Cq + c;
 
@@ -125,24 +127,36 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        // attended history blocks (ascending), then the current block
-        int cnt = 0;
-        if (a.full_scope) {
-            for (int m = 0; m < c; ++m) list[cnt++] = m;
-        } else {
-            const int kk = min(a.top_k, c);
-            const int32_t* row = a.idx + unit * a.top_k;
-            for (int i = 0; i < kk; ++i) {
-                const int v = row[i];
-                if (v >= 0 && v < c) list[cnt++] = v;
-            }
-        }
-        list[cnt] = c;
-        *list_count = cnt + 1;
         fence_barrier_init();
         prefetch_tmap(&a.tq);
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
+    }
+    if (warp == 0) {
+        // attended history blocks (ascending) with their log-gate biases, then the
+        // current block (bias 0); lanes read the selection in parallel
+        const float* srow = a.s + unit * a.Cq;
+        const float lse_c = a.lse_s[unit];
+        int cnt = 0;
+        const int kk = a.full_scope ? c : min(a.top_k, c);
+        const int32_t* row = a.idx + unit * a.top_k;
+        for (int base_i = 0; base_i < kk; base_i += 32) {
+            const int i = base_i + lane;
+            const int v = i < kk ? (a.full_scope ? i : row[i]) : -1;
+            const bool ok = v >= 0 && v < c;
+            const unsigned bal = __ballot_sync(0xffffffffu, ok);
+            if (ok) {
+                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                list[pos] = v;
+                bias2[pos] = (srow[v] - lse_c) * kLog2e;
+            }
+            cnt += __popc(bal);
+        }
+        if (lane == 0) {
+            list[cnt] = c;
+            bias2[cnt] = 0.f;
+            *list_count = cnt + 1;
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -228,8 +242,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             const int tok = r_unit / G, g = r_unit % G;
             const uint32_t tS = tmem + ((uint32_t)(32 * quad) << 16) + grp * 128;
             const uint32_t tO = tmem + ((uint32_t)(32 * quad) << 16) + 256 + grp * 128;
-            const float* srow = a.s + unit * a.Cq;
-            const float lse_c = a.lse_s[unit];
             float m_used = -INFINITY, l = 0.f;
             bool ok = true;
             for (int t = 0; t < nsteps; ++t) {
@@ -239,34 +251,34 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                 }
                 tc_fence_after();
                 const int nb = min(2, nlist - 2 * t);
-                float bias[2];
-                bool cur[2];
+                // pass 1: row max over the raw logits (sigma > 0), causal mask on the
+                // current block only
+                float mb[2];
 #pragma unroll
                 for (int bi = 0; bi < 2; ++bi) {
-                    const int blk = bi < nb ? list[2 * t + bi] : c;
-                    cur[bi] = (blk == c);
-                    bias[bi] = cur[bi] ? 0.f : (srow[blk] - lse_c) * kLog2e;
-                }
-                float sv[128];
-                float mx = -INFINITY;
-#pragma unroll
-                for (int bi = 0; bi < 2; ++bi) {
+                    mb[bi] = -INFINITY;
                     if (bi < nb) {
-#pragma unroll
-                        for (int ch = 0; ch < 2; ++ch) {
-                            uint32_t r[32];
-                            tmem_ld32_sync(tS + bi * 64 + ch * 32, r);
+                        const bool cur = (2 * t + bi == nlist - 1);
+                        uint32_t r0[32], r1[32];
+                        tmem_ld64_sync(tS + bi * 64, r0, r1);
+                        float m0 = -INFINITY, m1 = -INFINITY;
+                        if (!cur) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j) {
-                                const int key = ch * 32 + j;
-                                float v = fmaf(__uint_as_float(r[j]), a.scale_log2, bias[bi]);
-                                if (cur[bi] && key > tok) v = -INFINITY;
-                                sv[bi * 64 + key] = v;
-                                mx = fmaxf(mx, v);
+                                m0 = fmaxf(m0, __uint_as_float(r0[j]));
+                                m1 = fmaxf(m1, __uint_as_float(r1[j]));
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                if (j <= tok) m0 = fmaxf(m0, __uint_as_float(r0[j]));
+                                if (32 + j <= tok) m1 = fmaxf(m1, __uint_as_float(r1[j]));
                             }
                         }
+                        mb[bi] = fmaf(fmaxf(m0, m1), a.scale_log2, bias2[2 * t + bi]);
                     }
                 }
+                const float mx = fmaxf(mb[0], mb[1]);
                 const float m_new = fmaxf(m_used, mx);
                 const bool need = m_new > m_used + kRescaleLog2;
                 if (__any_sync(0xffffffffu, need)) {
@@ -285,21 +297,39 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                     l *= alpha;
                     if (need) m_used = m_new;
                 }
-                float rs = 0.f;
+                // pass 2: p = 2^(S sigma log2e + bias - m) with packed fp32 pairs, written
+                // as bf16 pairs over the columns already read
+                uint64_t rs2 = 0ull;
 #pragma unroll
                 for (int bi = 0; bi < 2; ++bi) {
                     if (bi < nb) {
+                        const bool cur = (2 * t + bi == nlist - 1);
+                        const float off = bias2[2 * t + bi] - m_used;
+                        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
+                        uint32_t r0[32], r1[32];
+                        tmem_ld64_sync(tS + bi * 64, r0, r1);
                         uint32_t pk[32];
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) {
-                            const float p0 = ex2(sv[bi * 64 + 2 * jj] - m_used);
-                            const float p1 = ex2(sv[bi * 64 + 2 * jj + 1] - m_used);
-                            rs += p0 + p1;
+                            const uint32_t* rr = jj < 16 ? r0 : r1;
+                            const int jl = (jj & 15) * 2;
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(rr[jl]), __uint_as_float(rr[jl + 1])), sc2, off2),
+                                      x0, x1);
+                            float p0 = ex2(x0), p1 = ex2(x1);
+                            if (cur) {
+                                if (2 * jj > tok) p0 = 0.f;
+                                if (2 * jj + 1 > tok) p1 = 0.f;
+                            }
+                            rs2 = f2_add(rs2, f2_pack(p0, p1));
                             pk[jj] = pack_bf16x2(p0, p1);
                         }
                         tmem_st32(tS + bi * 32, pk);
                     }
                 }
+                float rsa, rsb;
+                f2_unpack(rs2, rsa, rsb);
+                const float rs = rsa + rsb;
                 tmem_wait_st();
                 l += rs;
                 tc_fence_before();
