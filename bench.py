@@ -67,6 +67,24 @@ def decode_bytes(w, dense: bool = False) -> int:
     return kv + s + qo
 
 
+def max_over_ranks(value: float, world: int, device="cpu") -> float:
+    """Max of a per-rank timing over all ranks (identity for one rank).  The
+    collective is plumbing for the measurement only, never on the data path."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, flops_per_step: float, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processes its own batch (weak scaling)."""
+    return world * flops_per_step * steps / (ms_max * 1e-3) / 1e12
+
+
 def load_peaks() -> tuple[dict, str]:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -373,17 +391,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     launches = api.sas_launch_count() - launches0
     barrier()
     clk = clocks.stop()
-    ms = start.elapsed_time(end)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(start.elapsed_time(end), world, dev)
     per_call = {
         "sas_topk_select": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
         "sas_gated_attn_fwd": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
         "sas_gated_attn_bwd": statistics.mean(e[2].elapsed_time(e[3]) for e in evs),
     }
-    value = world * fl["total"] * args.steps / (ms_max * 1e-3) / 1e12
+    value = aggregate_tflops(world, fl["total"], args.steps, ms_max)
 
     # end to end through host buffers: pinned inputs copied in, outputs copied out
     e2e_steps = max(1, min(args.steps, 5))
@@ -402,10 +416,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             host_out[k_].copy_(v_, non_blocking=True)
     b.record()
     torch.cuda.synchronize()
-    t = torch.tensor([a.elapsed_time(b)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * fl["total"] * e2e_steps / (float(t.item()) * 1e-3) / 1e12
+    e2e_value = aggregate_tflops(world, fl["total"], e2e_steps, max_over_ranks(a.elapsed_time(b), world, dev))
     del host_in, host_out
 
     if rank != 0:

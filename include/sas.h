@@ -225,6 +225,14 @@ sas_status sas_sparse_decode_noalloc(const sas_decode_desc* desc, const void* q,
  * SAS_ERR_DEVICE_TIMEOUT (SAS_ERR_CUDA if the synchronisation itself fails). */
 sas_status sas_device_status(sas_stream_t stream);
 
+/* Self-test of the failure path: launches one thread that waits on an mbarrier
+ * nothing ever arrives at, bounded by limit_ms (1..10000), exactly as the
+ * tensor-core kernels bound their waits.  The wait gives up, records a timeout
+ * in the device status word and returns: sas_device_status then reports
+ * SAS_ERR_DEVICE_TIMEOUT once, and the context stays usable.  No fault, trap or
+ * hang is involved.  Errors: SAS_ERR_INVALID_VALUE for a limit out of range. */
+sas_status sas_selftest_bounded_wait(int32_t limit_ms, sas_stream_t stream);
+
 /* Number of kernels this library has launched in this process (all devices),
  * counted on the host at each successful launch. */
 uint64_t sas_launch_count(void);

@@ -66,6 +66,8 @@ lib.sas_sparse_decode_select.restype = ctypes.c_int
 lib.sas_sparse_decode_select.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 5 + [_i32, _vp, _vp, _vp]
 lib.sas_sparse_decode_noalloc.restype = ctypes.c_int
 lib.sas_sparse_decode_noalloc.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7
+lib.sas_selftest_bounded_wait.restype = ctypes.c_int
+lib.sas_selftest_bounded_wait.argtypes = [_i32, _vp]
 lib.sas_launch_count.restype = ctypes.c_uint64
 lib.sas_launch_count.argtypes = []
 lib.sas_device_status.restype = ctypes.c_int
@@ -155,6 +157,10 @@ def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream
 
 def sas_device_status(stream=None):
     _check(lib.sas_device_status(_stream(stream)), "sas_device_status")
+
+
+def sas_selftest_bounded_wait(limit_ms: int, stream=None):
+    _check(lib.sas_selftest_bounded_wait(limit_ms, _stream(stream)), "sas_selftest_bounded_wait")
 
 
 def sas_launch_count() -> int:

@@ -207,29 +207,36 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
             constexpr uint32_t idesc_dq = idesc_bf16_f32(128, 128, false, true);
-            bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
+            // per-tile interleaving: S_i/dP_i of block t+1 are issued right after dQ_i of
+            // block t, so tile 0's next softmax overlaps tile 1's current one
+            auto issue_sdp = [&](int t, int i) {
+                const int s = t % kStages;
+                const uint32_t kst = sK + s * 2 * kSlab64, vst = sV + s * 2 * kSlab64;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const int kh = ks >> 2, kk = ks & 3;
+                    const uint64_t bd = sdesc_sw128(kst + kh * kSlab64 + kk * 32, 16, 1024);
+                    const uint64_t ad = sdesc_sw128(sQ + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
+                    mma_ss(tmem + i * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const int kh = ks >> 2, kk = ks & 3;
+                    const uint64_t bd = sdesc_sw128(vst + kh * kSlab64 + kk * 32, 16, 1024);
+                    const uint64_t ad = sdesc_sw128(sDO + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
+                    mma_ss(tmem + i * 128 + 64, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full(i));
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag, a.status) && mbar_wait(kv_full(0), 0, abort_flag, a.status);
+            if (ok) {
+                tc_fence_after();
+                for (int i = 0; i < MT; ++i) issue_sdp(0, i);
+            }
             for (int t = 0; ok && t < nlist; ++t) {
                 const int s = t % kStages;
-                if (!mbar_wait(kv_full(s), (t / kStages) & 1, abort_flag, a.status)) break;
-                tc_fence_after();
-                const uint32_t kst = sK + s * 2 * kSlab64, vst = sV + s * 2 * kSlab64;
-                for (int i = 0; i < MT; ++i) {
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const int kh = ks >> 2, kk = ks & 3;
-                        const uint64_t bd = sdesc_sw128(kst + kh * kSlab64 + kk * 32, 16, 1024);
-                        const uint64_t ad = sdesc_sw128(sQ + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
-                        mma_ss(tmem + i * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const int kh = ks >> 2, kk = ks & 3;
-                        const uint64_t bd = sdesc_sw128(vst + kh * kSlab64 + kk * 32, 16, 1024);
-                        const uint64_t ad = sdesc_sw128(sDO + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
-                        mma_ss(tmem + i * 128 + 64, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(s_full(i));
-                }
+                const uint32_t kst = sK + s * 2 * kSlab64;
+                bool next_ready = false;
                 for (int i = 0; i < MT; ++i) {
                     if (!mbar_wait(ds_ready(i), t & 1, abort_flag, a.status)) {
                         ok = false;
@@ -242,8 +249,19 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                         mma_ts(tmem + 256 + i * 128, tmem + i * 128 + ks * 8, bd, idesc_dq,
                                (t > 0 || ks > 0) ? 1u : 0u);
                     }
+                    if (i == MT - 1 && t + kStages < nlist) mma_commit(kv_empty(s));
+                    if (t + 1 < nlist) {
+                        if (!next_ready) {
+                            if (!mbar_wait(kv_full((t + 1) % kStages), ((t + 1) / kStages) & 1, abort_flag, a.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            next_ready = true;
+                        }
+                        issue_sdp(t + 1, i);
+                    }
                 }
-                if (ok && t + kStages < nlist) mma_commit(kv_empty(s));
             }
             mma_commit(dq_done);
             mma_commit(drain);

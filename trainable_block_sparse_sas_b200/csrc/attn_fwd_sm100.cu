@@ -196,23 +196,30 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             constexpr uint32_t idesc_s64 = idesc_bf16_f32(128, 64, false, false);
             constexpr uint32_t idesc_s128 = idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
-            bool ok = mbar_wait(q_full(), 0, abort_flag, a.status);
-            for (int t = 0; ok && t < nsteps; ++t) {
+            // per-tile interleaving: S_i(t+1) is issued right after PV_i(t), so tile 0's
+            // next softmax overlaps tile 1's current one
+            auto issue_s = [&](int t, int i) {
                 const int s = t % kStages;
-                if (!mbar_wait(kv_full(s), (t / kStages) & 1, abort_flag, a.status)) break;
-                tc_fence_after();
                 const int nb = min(2, nlist - 2 * t);
                 const uint32_t idesc_s = nb == 2 ? idesc_s128 : idesc_s64;
-                for (int i = 0; i < MT; ++i) {
 #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const int kh = ks >> 2, kk = ks & 3;
-                        const uint64_t ad = sdesc_sw128(sQ + kh * L::kQHalf + i * 128 * 128 + kk * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(sK + s * kKvStage + kh * kKvHalf + kk * 32, 16, 1024);
-                        mma_ss(tmem + i * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(s_full(i));
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const int kh = ks >> 2, kk = ks & 3;
+                    const uint64_t ad = sdesc_sw128(sQ + kh * L::kQHalf + i * 128 * 128 + kk * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sK + s * kKvStage + kh * kKvHalf + kk * 32, 16, 1024);
+                    mma_ss(tmem + i * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
                 }
+                mma_commit(s_full(i));
+            };
+            bool ok = mbar_wait(q_full(), 0, abort_flag, a.status) && mbar_wait(kv_full(0), 0, abort_flag, a.status);
+            if (ok) {
+                tc_fence_after();
+                for (int i = 0; i < MT; ++i) issue_s(0, i);
+            }
+            for (int t = 0; ok && t < nsteps; ++t) {
+                const int s = t % kStages;
+                const int nb = min(2, nlist - 2 * t);
+                bool next_ready = false;
                 for (int i = 0; i < MT; ++i) {
                     if (!mbar_wait(p_ready(i), t & 1, abort_flag, a.status)) {
                         ok = false;
@@ -225,8 +232,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                                (t > 0 || ks > 0) ? 1u : 0u);
                     }
                     mma_commit(o_done(i));
+                    if (i == MT - 1 && t + kStages < nsteps) mma_commit(kv_empty(s));
+                    if (t + 1 < nsteps) {
+                        if (!next_ready) {
+                            if (!mbar_wait(kv_full((t + 1) % kStages), ((t + 1) / kStages) & 1, abort_flag, a.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            next_ready = true;
+                        }
+                        issue_s(t + 1, i);
+                    }
                 }
-                if (ok && t + kStages < nsteps) mma_commit(kv_empty(s));
             }
             // all issued MMAs complete before TMEM is released
             mma_commit(drain);

@@ -63,6 +63,7 @@ size_t simt_max_smem(int D, int BS, int Cq);
 void decode_plan(DecodeParams& p);
 size_t decode_workspace(const DecodeParams& p);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);
 bool decode_sm100_supported(const DecodeParams& p);
 // s != nullptr: fused Top-K selection from s [B, Hkv, s_cols] (idx_out nullable)
 cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,

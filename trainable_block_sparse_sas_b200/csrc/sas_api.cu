@@ -289,6 +289,14 @@ sas_status sas_device_status(sas_stream_t stream) {
     return SAS_OK;
 }
 
+sas_status sas_selftest_bounded_wait(int32_t limit_ms, sas_stream_t stream) {
+    if (limit_ms <= 0 || limit_ms > 10000) return SAS_ERR_INVALID_VALUE;
+    DeviceInfo di;
+    if (device_info(&di) != cudaSuccess) return SAS_ERR_CUDA;
+    return from_cuda(launch_selftest_wait(di.status, (unsigned long long)limit_ms * 1000000ull,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char* sas_status_string(sas_status status) {
     switch (status) {
         case SAS_OK: return "success";
