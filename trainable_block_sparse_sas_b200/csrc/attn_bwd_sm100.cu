@@ -21,7 +21,8 @@
 //     dV^T += dO^T P and dK^T += Q^T dS               (SS MMAs, M = head_dim = 128)
 //   Epilogue: dk = sigma dK, dv = dV.
 //
-// D_i = dO_i . o_i comes from a small row-dot kernel run first (workspace).
+// D_i = dO_i . o_i is computed by the dq kernel's softmax threads (one row each)
+// and written to the workspace for the dk/dv kernel, which runs after it.
 // Every wait is time-bounded and reports through the device status word.
 #include <cstring>
 
@@ -45,7 +46,9 @@ struct BwdArgs {
     const float* lse_s;
     const int32_t* idx;
     const float* lse;
-    const float* Dbuf;
+    float* Dbuf;
+    const __nv_bfloat16* o;
+    const __nv_bfloat16* dO;
     __nv_bfloat16* dq;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
@@ -78,7 +81,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // ============================================================================
 // dq / ds kernel
 // ============================================================================
-constexpr int kDqThreads = 320;
+// warp 0 TMA; per M-tile i, warp 1 + 2i issues the S chain and warp 2 + 2i the
+// dQ and dP chain (a single thread's chain of small MMAs is latency-bound, so
+// each tile has two); warps 5..12 softmax, one group per M-tile.  The two tiles
+// take turns: tile 1 issues block t once tile 0 has issued it, tile 0 issues
+// block t+1 once tile 1 has issued block t, so one tile's MMAs run while the
+// other tile's softmax does.
+constexpr int kDqThreads = 416;
+constexpr int kDqSoftmaxWarp0 = 5;
 
 template <int MT>
 struct DqLayout {
@@ -89,8 +99,8 @@ struct DqLayout {
     static constexpr uint32_t kK = kDO + 2 * kHalf;
     static constexpr uint32_t kV = kK + kStages * 2 * kSlab64;
     static constexpr uint32_t kBars = kV + kStages * 2 * kSlab64;
-    // q_full, kv_full[S], kv_empty[S], s_full[2], ds_ready[2], dq_done, drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
+    // q_full, kv_full[S], kv_empty[S], s_full[2], ds_ready[2], dq_done, drain, issued[2]
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 2;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
     static constexpr uint32_t kList = kMisc + 16;
     // list [Cq + 1] ints, biases [Cq + 1] floats, then the per-warp dlogg partials
@@ -114,6 +124,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     auto ds_ready = [&](int i) { return bar0 + 8u * (3 + 2 * kStages + i); };
     const uint32_t dq_done = bar0 + 8u * (5 + 2 * kStages);
     const uint32_t drain = bar0 + 8u * (6 + 2 * kStages);
+    auto issued = [&](int i) { return bar0 + 8u * (7 + 2 * kStages + i); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
     int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
@@ -134,14 +145,15 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         mbar_init(q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(kv_full(s), 1);
-            mbar_init(kv_empty(s), 1);
+            mbar_init(kv_empty(s), MT);  // each tile's dQ/dP issuer, after its dQ of the stage
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(s_full(i), 1);
+            mbar_init(s_full(i), 2);  // S chain and dP chain
             mbar_init(ds_ready(i), 128);
+            mbar_init(issued(i), 2);  // both issuers of tile i have issued a block
         }
-        mbar_init(dq_done, 1);
-        mbar_init(drain, 1);
+        mbar_init(dq_done, MT);
+        mbar_init(drain, 2 * MT);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&a.tq);
@@ -203,72 +215,61 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 }
             }
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
+    } else if (warp < kDqSoftmaxWarp0) {
+        const int i = (warp - 1) >> 1;       // M-tile
+        const bool dp_chain = ((warp - 1) & 1) != 0;
+        if (lane == 0 && i < MT) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
             constexpr uint32_t idesc_dq = idesc_bf16_f32(128, 128, false, true);
-            // per-tile interleaving: S_i/dP_i of block t+1 are issued right after dQ_i of
-            // block t, so tile 0's next softmax overlaps tile 1's current one
-            auto issue_sdp = [&](int t, int i) {
-                const int s = t % kStages;
-                const uint32_t kst = sK + s * 2 * kSlab64, vst = sV + s * 2 * kSlab64;
+            // S_i = Q_i K^T (columns i*128) or dP_i = dO_i V^T (columns i*128 + 64); the
+            // softmax writes dS over dP, so dQ_i(t-1) = dS K precedes dP_i(t) in the
+            // dP thread's order
+            const uint32_t a_base = (dp_chain ? sDO : sQ) + i * kSlab128;
+            const uint32_t b_base = dp_chain ? sV : sK;
+            const uint32_t d_col = tmem + i * 128 + (dp_chain ? 64 : 0);
+            auto issue_dq = [&](int t) {
+                const uint32_t kst = sK + (t % kStages) * 2 * kSlab64;
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const int kh = ks >> 2, kk = ks & 3;
-                    const uint64_t bd = sdesc_sw128(kst + kh * kSlab64 + kk * 32, 16, 1024);
-                    const uint64_t ad = sdesc_sw128(sQ + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
-                    mma_ss(tmem + i * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < kBS / 16; ++ks) {
+                    const uint64_t bd = sdesc_sw128(kst + ks * 2048, kSlab64, 1024);
+                    mma_ts(tmem + 256 + i * 128, tmem + i * 128 + 64 + ks * 8, bd, idesc_dq, (t > 0 || ks > 0) ? 1u : 0u);
                 }
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const int kh = ks >> 2, kk = ks & 3;
-                    const uint64_t bd = sdesc_sw128(vst + kh * kSlab64 + kk * 32, 16, 1024);
-                    const uint64_t ad = sdesc_sw128(sDO + kh * L::kHalf + i * kSlab128 + kk * 32, 16, 1024);
-                    mma_ss(tmem + i * 128 + 64, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(s_full(i));
             };
-            bool ok = mbar_wait(q_full, 0, abort_flag, a.status) && mbar_wait(kv_full(0), 0, abort_flag, a.status);
-            if (ok) {
-                tc_fence_after();
-                for (int i = 0; i < MT; ++i) issue_sdp(0, i);
-            }
+            bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
             for (int t = 0; ok && t < nlist; ++t) {
                 const int s = t % kStages;
-                const uint32_t kst = sK + s * 2 * kSlab64;
-                bool next_ready = false;
-                for (int i = 0; i < MT; ++i) {
-                    if (!mbar_wait(ds_ready(i), t & 1, abort_flag, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < kBS / 16; ++ks) {
-                        const uint64_t bd = sdesc_sw128(kst + ks * 2048, kSlab64, 1024);
-                        mma_ts(tmem + 256 + i * 128, tmem + i * 128 + ks * 8, bd, idesc_dq,
-                               (t > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    if (i == MT - 1 && t + kStages < nlist) mma_commit(kv_empty(s));
-                    if (t + 1 < nlist) {
-                        if (!next_ready) {
-                            if (!mbar_wait(kv_full((t + 1) % kStages), ((t + 1) / kStages) & 1, abort_flag, a.status)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            next_ready = true;
-                        }
-                        issue_sdp(t + 1, i);
-                    }
+                if (!mbar_wait(kv_full(s), (t / kStages) & 1, abort_flag, a.status)) break;
+                // block t reuses the tile's S/dP columns once softmax(t-1) is done with them
+                if (t > 0 && !mbar_wait(ds_ready(i), (t - 1) & 1, abort_flag, a.status)) break;
+                if (MT == 2) {  // turn order between the two tiles
+                    if (i == 1 && !mbar_wait(issued(0), t & 1, abort_flag, a.status)) break;
+                    if (i == 0 && t > 0 && !mbar_wait(issued(1), (t - 1) & 1, abort_flag, a.status)) break;
                 }
+                tc_fence_after();
+                if (dp_chain && t > 0) {
+                    issue_dq(t - 1);
+                    if (t - 1 + kStages < nlist) mma_commit(kv_empty((t - 1) % kStages));
+                }
+                const uint32_t bst = b_base + s * 2 * kSlab64;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const int kh = ks >> 2, kk = ks & 3;
+                    mma_ss(d_col, sdesc_sw128(a_base + kh * L::kHalf + kk * 32, 16, 1024),
+                           sdesc_sw128(bst + kh * kSlab64 + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full(i));
+                if (MT == 2) mbar_arrive(issued(i));
             }
-            mma_commit(dq_done);
+            if (ok && dp_chain && nlist > 0 && mbar_wait(ds_ready(i), (nlist - 1) & 1, abort_flag, a.status)) {
+                tc_fence_after();
+                issue_dq(nlist - 1);
+            }
+            if (dp_chain) mma_commit(dq_done);
             mma_commit(drain);
             mbar_wait_drain(drain, 0, a.status);
         }
     } else {
-        const int wi = warp - 2;  // 0..7
+        const int wi = warp - kDqSoftmaxWarp0;  // 0..7
         const int grp = wi >> 2;
         const int quad = warp & 3;
         if (grp < MT) {
@@ -278,7 +279,30 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             const int hq = h * G + g;
             const long ri = ((long)b * a.Hq + hq) * a.n + c * kBS + tok;
             const float lse2 = a.lse[ri] * kLog2e;
-            const float Drow = a.Dbuf[ri];
+            // D = dO . o of this row (fp32 sum of the bf16 products), kept for the
+            // dk/dv kernel as well
+            float Drow;
+            {
+                const long e0 = (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
+                const uint4* po = reinterpret_cast<const uint4*>(a.o + e0);
+                const uint4* pd = reinterpret_cast<const uint4*>(a.dO + e0);
+                uint64_t acc2 = 0ull;
+#pragma unroll 4
+                for (int v4 = 0; v4 < kD / 8; ++v4) {
+                    const uint4 x = po[v4], y = pd[v4];
+                    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[u]));
+                        const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[u]));
+                        acc2 = f2_fma(f2_pack(xf.x, xf.y), f2_pack(yf.x, yf.y), acc2);
+                    }
+                }
+                float da, db;
+                f2_unpack(acc2, da, db);
+                Drow = da + db;
+                a.Dbuf[ri] = Drow;
+            }
             const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
             const uint32_t tS = tmem + lane_off + grp * 128, tP = tS + 64;
             const uint32_t tQ = tmem + lane_off + 256 + grp * 128;
@@ -295,18 +319,16 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 const uint64_t negD2 = f2_pack(-Drow, -Drow);
                 uint64_t rs2 = 0ull;
                 uint32_t pk[32];
-                {
-                    uint32_t s0r[32], s1r[32], d0r[32], d1r[32];
-                    tmem_ld64_sync(tS, s0r, s1r);
-                    tmem_ld64_sync(tP, d0r, d1r);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const uint32_t* sr = jj < 16 ? s0r : s1r;
-                        const uint32_t* dr = jj < 16 ? d0r : d1r;
-                        const int jl = (jj & 15) * 2;
+                for (int hh = 0; hh < 2; ++hh) {  // 32 keys at a time
+                    uint32_t sr[32], dr[32];
+                    tmem_ld32x2_sync(tS + 32 * hh, tP + 32 * hh, sr, dr);
+#pragma unroll
+                    for (int jq = 0; jq < 16; ++jq) {
+                        const int jj = 16 * hh + jq;
                         float x0, x1;
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[jl]), __uint_as_float(sr[jl + 1])), sc2, off2), x0,
-                                  x1);
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * jq]), __uint_as_float(sr[2 * jq + 1])), sc2, off2),
+                                  x0, x1);
                         float p0 = ex2(x0), p1 = ex2(x1);
                         if (cur) {
                             if (2 * jj > tok) p0 = 0.f;
@@ -314,7 +336,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                         }
                         const uint64_t ds2 = f2_mul(
                             f2_pack(p0, p1),
-                            f2_add(f2_pack(__uint_as_float(dr[jl]), __uint_as_float(dr[jl + 1])), negD2));
+                            f2_add(f2_pack(__uint_as_float(dr[2 * jq]), __uint_as_float(dr[2 * jq + 1])), negD2));
                         rs2 = f2_add(rs2, ds2);
                         float d0, d1;
                         f2_unpack(ds2, d0, d1);
@@ -324,7 +346,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 float rsa, rsb;
                 f2_unpack(rs2, rsa, rsb);
                 float rs = rsa + rsb;
-                tmem_st32(tS, pk);
+                tmem_st32(tP, pk);  // dS over dP, for dQ = dS K
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ds_ready(grp));
@@ -386,7 +408,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
 // ============================================================================
 // dk / dv kernel
 // ============================================================================
-constexpr int kKvThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 two softmax groups (key halves)
+// warp 0 TMA; warps 1 and 2 issue the S and dP MMA chains, warps 3 and 4 the dV
+// and dK chains with lanes 0 and 1 taking the two 64-row halves of each item
+// into separate accumulators (a single thread's chain of small MMAs is
+// latency-bound; several chains run concurrently); warps 5..12 two softmax
+// groups (key halves)
+constexpr int kKvThreads = 416;
+constexpr int kKvSoftmaxWarp0 = 5;
 
 struct DkvLayout {
     static constexpr uint32_t kK = 0;                     // 2 slabs x 64 rows
@@ -396,8 +424,8 @@ struct DkvLayout {
     static constexpr uint32_t kP = kDO + kStages * 2 * kSlab128;  // 128 rows x 64 keys bf16
     static constexpr uint32_t kDS = kP + kSlab128;
     static constexpr uint32_t kBars = kDS + kSlab128;
-    // kv_full, qd_full[S], qd_empty[S], s_full[2], p_ready, item_done, final, drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 4;
+    // kv_full, qd_full[S], qd_empty[S], s_full[2], s_free[2], p_ready, item_done, final, drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
     static constexpr uint32_t kList = kMisc + 16;
     static constexpr uint32_t kScan = kList;  // scan scratch precedes the list
@@ -433,10 +461,11 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     auto qd_full = [&](int s) { return bar0 + 8u * (1 + s); };
     auto qd_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
     auto s_full = [&](int i) { return bar0 + 8u * (1 + 2 * kStages + i); };
-    const uint32_t p_ready = bar0 + 8u * (3 + 2 * kStages);
-    const uint32_t item_done = bar0 + 8u * (4 + 2 * kStages);
-    const uint32_t final_bar = bar0 + 8u * (5 + 2 * kStages);
-    const uint32_t drain = bar0 + 8u * (6 + 2 * kStages);
+    auto s_free = [&](int i) { return bar0 + 8u * (3 + 2 * kStages + i); };
+    const uint32_t p_ready = bar0 + 8u * (5 + 2 * kStages);
+    const uint32_t item_done = bar0 + 8u * (6 + 2 * kStages);
+    const uint32_t final_bar = bar0 + 8u * (7 + 2 * kStages);
+    const uint32_t drain = bar0 + 8u * (8 + 2 * kStages);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
     int* scan = reinterpret_cast<int*>(base + L::kScan);  // 33 ints
@@ -462,17 +491,20 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         nlist += cnt;
     }
     if (threadIdx.x == 0) {
+        // arrival counts: commits of the chains that must all have completed
         mbar_init(kv_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(qd_full(s), 1);
-            mbar_init(qd_empty(s), 1);
+            mbar_init(qd_empty(s), 4);  // dV and dK chains (S/dP of the item completed earlier)
         }
-        mbar_init(s_full(0), 1);
-        mbar_init(s_full(1), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(s_full(i), 2);    // S and dP chains
+            mbar_init(s_free(i), 256);  // softmax threads have read the buffer
+        }
         mbar_init(p_ready, 256);
-        mbar_init(item_done, 1);
-        mbar_init(final_bar, 1);
-        mbar_init(drain, 1);
+        mbar_init(item_done, 4);
+        mbar_init(final_bar, 4);
+        mbar_init(drain, 6);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&a.tq);
@@ -488,7 +520,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int nitems = nlist * MT;
-    // TMEM: S/dP buffers at 0 and 128 (S | dP), dV^T at 256, dK^T at 320
+    // TMEM: S/dP buffers at 0 and 128 (S | dP), dV^T halves at 256 and 320, dK^T halves at 384 and 448
 
     if (warp == 0) {
         if (lane == 0) {
@@ -510,76 +542,61 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                 }
             }
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
-            constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, true, true);
-            auto issue_s = [&](int j) {
-                const int st = j % kStages, buf = j & 1;
-                const uint32_t q = sQ + st * 2 * kSlab128, o = sDO + st * 2 * kSlab128;
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const int kh = ks >> 2, kk = ks & 3;
-                    mma_ss(tmem + buf * 128, sdesc_sw128(q + kh * kSlab128 + kk * 32, 16, 1024),
-                           sdesc_sw128(sK + kh * kSlab64 + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const int kh = ks >> 2, kk = ks & 3;
-                    mma_ss(tmem + buf * 128 + 64, sdesc_sw128(o + kh * kSlab128 + kk * 32, 16, 1024),
-                           sdesc_sw128(sV + kh * kSlab64 + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(s_full(buf));
-            };
-            bool ok = mbar_wait(kv_full, 0, abort_flag, a.status);
-            if (ok && nitems > 0) {
-                ok = mbar_wait(qd_full(0), 0, abort_flag, a.status);
-                if (ok) {
+    } else if (warp < kKvSoftmaxWarp0) {
+        const int chain = warp - 1;  // 0 S, 1 dP, 2 dV, 3 dK
+        if (lane < (chain < 2 ? 1 : 2)) {
+            bool ok = true;
+            if (chain < 2) {
+                // S = Q K^T (chain 0) or dP = dO V^T (chain 1) of item j into TMEM buffer j & 1,
+                // once the softmax threads have read that buffer's previous item
+                constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+                const uint32_t a_base = chain == 0 ? sQ : sDO, b_base = chain == 0 ? sK : sV;
+                ok = mbar_wait(kv_full, 0, abort_flag, a.status);
+                for (int j = 0; ok && j < nitems; ++j) {
+                    const int st = j % kStages, buf = j & 1;
+                    if (j >= 2 && !mbar_wait(s_free(buf), ((j >> 1) - 1) & 1, abort_flag, a.status)) break;
+                    if (!mbar_wait(qd_full(st), (j / kStages) & 1, abort_flag, a.status)) break;
                     tc_fence_after();
-                    issue_s(0);
+                    const uint32_t at = a_base + st * 2 * kSlab128;
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const int kh = ks >> 2, kk = ks & 3;
+                        mma_ss(tmem + buf * 128 + chain * 64, sdesc_sw128(at + kh * kSlab128 + kk * 32, 16, 1024),
+                               sdesc_sw128(b_base + kh * kSlab64 + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(s_full(buf));
                 }
+            } else {
+                // dV^T += dO^T P (chain 2) or dK^T += Q^T dS (chain 3), accumulated over all
+                // items; lane 0 sums rows 0..63 of each item, lane 1 rows 64..127
+                constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, true, true);
+                const uint32_t a_base = chain == 2 ? sDO : sQ, b_base = chain == 2 ? sP : sDS;
+                const uint32_t acc = tmem + 256 + (chain - 2) * 128 + lane * 64;
+                for (int j = 0; j < nitems; ++j) {
+                    if (!mbar_wait(p_ready, j & 1, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t at = a_base + (j % kStages) * 2 * kSlab128 + lane * 4 * 2048;
+                    const uint32_t bt = b_base + lane * 4 * 2048;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        mma_ss(acc, sdesc_sw128(at + ks * 2048, kSlab128, 1024), sdesc_sw128(bt + ks * 2048, kSlab128, 1024),
+                               idesc_g, (j > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(item_done);
+                    if (j + kStages < nitems) mma_commit(qd_empty(j % kStages));
+                }
+                if (ok) mma_commit(final_bar);
             }
-            // S/dP of item j+1 goes ahead of dV/dK of item j only when its Q/dO tiles
-            // have already landed; otherwise dV/dK of item j is issued first, so that its
-            // stage is released (and the load of item j+2 starts) without waiting.
-            int next_s = 1;
-            for (int j = 0; ok && j < nitems; ++j) {
-                if (next_s == j + 1 && next_s < nitems &&
-                    mbar_try_wait(qd_full(next_s % kStages), (next_s / kStages) & 1)) {
-                    tc_fence_after();
-                    issue_s(next_s);
-                    ++next_s;
-                }
-                if (!mbar_wait(p_ready, j & 1, abort_flag, a.status)) break;
-                tc_fence_after();
-                const int st = j % kStages;
-                const uint32_t q = sQ + st * 2 * kSlab128, o = sDO + st * 2 * kSlab128;
-#pragma unroll
-                for (int ks = 0; ks < 128 / 16; ++ks) {
-                    mma_ss(tmem + 256, sdesc_sw128(o + ks * 2048, kSlab128, 1024),
-                           sdesc_sw128(sP + ks * 2048, kSlab128, 1024), idesc_g, (j > 0 || ks > 0) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int ks = 0; ks < 128 / 16; ++ks) {
-                    mma_ss(tmem + 320, sdesc_sw128(q + ks * 2048, kSlab128, 1024),
-                           sdesc_sw128(sDS + ks * 2048, kSlab128, 1024), idesc_g, (j > 0 || ks > 0) ? 1u : 0u);
-                }
-                mma_commit(item_done);
-                if (j + kStages < nitems) mma_commit(qd_empty(st));
-                if (next_s == j + 1 && next_s < nitems) {
-                    if (!mbar_wait(qd_full(next_s % kStages), (next_s / kStages) & 1, abort_flag, a.status)) break;
-                    tc_fence_after();
-                    issue_s(next_s);
-                    ++next_s;
-                }
-            }
-            mma_commit(final_bar);
+            // every chain's MMAs complete before TMEM is released
             mma_commit(drain);
             mbar_wait_drain(drain, 0, a.status);
         }
     } else {
         const int quad = warp & 3;
-        const int kw = (warp - 2) >> 2;       // key half of the block handled by this group
+        const int kw = (warp - kKvSoftmaxWarp0) >> 2;  // key half of the block handled by this group
         const int row = 32 * quad + lane;     // row of the 128-row item
         const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
         bool ok = true;
@@ -617,6 +634,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                 uint32_t sr[32], dr[32];
                 tmem_ld32x2_sync(tmem + lane_off + buf * 128 + 32 * kw, tmem + lane_off + buf * 128 + 64 + 32 * kw,
                                  sr, dr);
+                tc_fence_before();
+                mbar_arrive(s_free(buf));
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     float x0, x1;
@@ -659,19 +678,21 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         }
         if (ok && warp_wait(final_bar, 0, abort_flag, a.status)) {
             tc_fence_after();
-            // group 0 writes dv, group 1 dk; TMEM lane = head-dim index
+            // group 0 writes dv, group 1 dk, each the sum of its two row-half
+            // accumulators; TMEM lane = head-dim index
             const int d = 32 * quad + lane;
             __nv_bfloat16* dst = kw == 0 ? a.dv : a.dk;
             const float mul = kw == 0 ? 1.f : a.scale;
-#pragma unroll
+#pragma unroll 1
             for (int ch = 0; ch < 2; ++ch) {
-                uint32_t r[32];
-                tmem_ld32_sync(tmem + lane_off + 256 + kw * 64 + ch * 32, r);
+                uint32_t r0[32], r1[32];
+                tmem_ld32x2_sync(tmem + lane_off + 256 + kw * 128 + ch * 32, tmem + lane_off + 320 + kw * 128 + ch * 32,
+                                 r0, r1);
 #pragma unroll
                 for (int jx = 0; jx < 32; ++jx) {
                     const int key = ch * 32 + jx;
                     dst[(((long)b * a.n + m * kBS + key) * a.Hkv + h) * kD + d] =
-                        __float2bfloat16_rn(__uint_as_float(r[jx]) * mul);
+                        __float2bfloat16_rn((__uint_as_float(r0[jx]) + __uint_as_float(r1[jx])) * mul);
                 }
             }
         }
@@ -708,6 +729,8 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.idx = p.idx;
     a.lse = p.lse_in;
     a.Dbuf = p.Dbuf;
+    a.o = static_cast<const __nv_bfloat16*>(p.o_in);
+    a.dO = static_cast<const __nv_bfloat16*>(p.dO);
     a.dq = static_cast<__nv_bfloat16*>(p.dq);
     a.dk = static_cast<__nv_bfloat16*>(p.dk);
     a.dv = static_cast<__nv_bfloat16*>(p.dv);
@@ -743,15 +766,13 @@ bool bwd_sm100_supported(const TrainParams& p) {
     const uintptr_t al = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
                          reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.dO) |
                          reinterpret_cast<uintptr_t>(p.dq) | reinterpret_cast<uintptr_t>(p.dk) |
-                         reinterpret_cast<uintptr_t>(p.dv);
+                         reinterpret_cast<uintptr_t>(p.dv) | reinterpret_cast<uintptr_t>(p.o_in);
     if (al & 15u) return false;
     if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq > 0x7fffffffL) return false;
     return DqLayout<2>::bytes(p.Cq) <= 227 * 1024 && DkvLayout::bytes(p.Cq) <= 227 * 1024;
 }
 
 cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream) {
-    cudaError_t err = launch_rowdot(p, stream);
-    if (err != cudaSuccess) return err;
     const int G = p.Hq / p.Hkv;
     return G == 4 ? launch_mt<2>(p, stream) : launch_mt<1>(p, stream);
 }

@@ -338,6 +338,37 @@ __device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&r0)[32
                  : "memory");
 }
 
+// four TMEM chunks of 32 consecutive columns (128 columns) with a single wait
+__device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r0)[32], uint32_t (&r1)[32],
+                                                uint32_t (&r2)[32], uint32_t (&r3)[32]) {
+    tmem_ld32(taddr, r0);
+    tmem_ld32(taddr + 32, r1);
+    tmem_ld32(taddr + 64, r2);
+    tmem_ld32(taddr + 96, r3);
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r0[0]), "+r"(r0[1]), "+r"(r0[2]), "+r"(r0[3]), "+r"(r0[4]), "+r"(r0[5]), "+r"(r0[6]),
+                   "+r"(r0[7]), "+r"(r0[8]), "+r"(r0[9]), "+r"(r0[10]), "+r"(r0[11]), "+r"(r0[12]), "+r"(r0[13]),
+                   "+r"(r0[14]), "+r"(r0[15]), "+r"(r0[16]), "+r"(r0[17]), "+r"(r0[18]), "+r"(r0[19]), "+r"(r0[20]),
+                   "+r"(r0[21]), "+r"(r0[22]), "+r"(r0[23]), "+r"(r0[24]), "+r"(r0[25]), "+r"(r0[26]), "+r"(r0[27]),
+                   "+r"(r0[28]), "+r"(r0[29]), "+r"(r0[30]), "+r"(r0[31]), "+r"(r1[0]), "+r"(r1[1]), "+r"(r1[2]),
+                   "+r"(r1[3]), "+r"(r1[4]), "+r"(r1[5]), "+r"(r1[6]), "+r"(r1[7]), "+r"(r1[8]), "+r"(r1[9]),
+                   "+r"(r1[10]), "+r"(r1[11]), "+r"(r1[12]), "+r"(r1[13]), "+r"(r1[14]), "+r"(r1[15]), "+r"(r1[16]),
+                   "+r"(r1[17]), "+r"(r1[18]), "+r"(r1[19]), "+r"(r1[20]), "+r"(r1[21]), "+r"(r1[22]), "+r"(r1[23]),
+                   "+r"(r1[24]), "+r"(r1[25]), "+r"(r1[26]), "+r"(r1[27]), "+r"(r1[28]), "+r"(r1[29]), "+r"(r1[30]),
+                   "+r"(r1[31]), "+r"(r2[0]), "+r"(r2[1]), "+r"(r2[2]), "+r"(r2[3]), "+r"(r2[4]), "+r"(r2[5]),
+                   "+r"(r2[6]), "+r"(r2[7]), "+r"(r2[8]), "+r"(r2[9]), "+r"(r2[10]), "+r"(r2[11]), "+r"(r2[12]),
+                   "+r"(r2[13]), "+r"(r2[14]), "+r"(r2[15]), "+r"(r2[16]), "+r"(r2[17]), "+r"(r2[18]), "+r"(r2[19]),
+                   "+r"(r2[20]), "+r"(r2[21]), "+r"(r2[22]), "+r"(r2[23]), "+r"(r2[24]), "+r"(r2[25]), "+r"(r2[26]),
+                   "+r"(r2[27]), "+r"(r2[28]), "+r"(r2[29]), "+r"(r2[30]), "+r"(r2[31]), "+r"(r3[0]), "+r"(r3[1]),
+                   "+r"(r3[2]), "+r"(r3[3]), "+r"(r3[4]), "+r"(r3[5]), "+r"(r3[6]), "+r"(r3[7]), "+r"(r3[8]),
+                   "+r"(r3[9]), "+r"(r3[10]), "+r"(r3[11]), "+r"(r3[12]), "+r"(r3[13]), "+r"(r3[14]), "+r"(r3[15]),
+                   "+r"(r3[16]), "+r"(r3[17]), "+r"(r3[18]), "+r"(r3[19]), "+r"(r3[20]), "+r"(r3[21]), "+r"(r3[22]),
+                   "+r"(r3[23]), "+r"(r3[24]), "+r"(r3[25]), "+r"(r3[26]), "+r"(r3[27]), "+r"(r3[28]), "+r"(r3[29]),
+                   "+r"(r3[30]), "+r"(r3[31])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
