@@ -4,10 +4,12 @@
 //
 // One thread-block cluster of CL CTAs per (sequence, kv head); one launch per
 // decode step, no workspace:
-//   1. selection (optional, fused): the cluster's CTAs split the row's block
-//      scores, run a 4-pass 8-bit radix select of the K-th largest order key with
-//      histograms summed over distributed shared memory, and write the chosen
-//      blocks (ties to the lower index, ascending) into every CTA's list;
+//   1. selection (optional, fused): every CTA finds the row's Top-K blocks on its
+//      own (a threshold from the threads' maxima, then an exact rank of the few
+//      keys above it; ties to the lower index, list ascending); when too many
+//      scores tie at the threshold, the cluster's CTAs split the row and run a
+//      4-pass 8-bit radix select with candidates merged over distributed shared
+//      memory;
 //   2. attention: the attended list (current partial block first, then the
 //      history blocks) is split over the CTAs; a TMA ring streams each block's K
 //      and V (2 x 16 KB, 128-byte swizzle); all 8 consumer warps take every block,
@@ -75,6 +77,112 @@ __device__ __forceinline__ int block_sum_int(int v, int* scan) {
     int tot;
     block_exclusive_scan(v, scan, &tot);
     return tot;
+}
+
+// Exact Top-K of the row's first Cb block scores, computed by this CTA alone
+// (every CTA of the cluster derives the same list, so no exchange is needed).
+// Each score m becomes the unique 64-bit key (order key << 32) | (2^32 - 1 - m):
+// larger keys are better and equal scores prefer the lower block index.  The
+// K-th largest of the threads' maxima is a lower bound of the K-th largest key
+// (K maxima reach it), so every key at or above it is a candidate; the K
+// best candidates by rank are the selection.  Returns K, or -1 when more than
+// kCandCap keys reach the bound (the caller then runs the radix select).
+// Rows of up to kPer * kThreads blocks (9216: 589,824 tokens at block 64).
+constexpr int kCandCap = 512;
+constexpr int kPer = 32;  // scores per thread held in registers
+
+__device__ int row_topk_filter(const DecArgs& a, int bh, int Cb, uint8_t* base, int* list) {
+    constexpr int kWarps = kThreads / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = a.top_k;
+    const float* srow = a.s + (long)bh * a.s_cols;
+    // scratch in ring stage 1 (stage 0 may hold the prefetched current block)
+    unsigned long long* sorted = reinterpret_cast<unsigned long long*>(base + Layout::kRing + kStage);
+    unsigned long long* cand = sorted + kWarps * 32;
+    unsigned long long* chosen = cand + kCandCap;
+    unsigned long long* thr_sh = chosen + 64;
+    int* misc = reinterpret_cast<int*>(base + Layout::kMisc);
+    auto key_of = [&](float x, int m) -> unsigned long long {
+        return ((unsigned long long)order_key(x) << 32) | (0xFFFFFFFFu - (uint32_t)m);
+    };
+    // the row is read once, every load of a thread in flight together, and kept in
+    // registers for both passes (rows of up to kPer * kThreads blocks)
+    float x[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int m = tid + u * kThreads;
+        x[u] = m < Cb ? srow[m] : 0.f;
+    }
+    unsigned long long v = 0ull;  // 0: no score (every real key is larger)
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int m = tid + u * kThreads;
+        const unsigned long long k = m < Cb ? key_of(x[u], m) : 0ull;
+        v = k > v ? k : v;
+    }
+    if (tid == 0) {
+        misc[5] = 0;
+        *thr_sh = 0ull;
+    }
+    // each warp's 32 maxima, sorted descending
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
+            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+            v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+        }
+    }
+    sorted[warp * 32 + lane] = v;
+    __syncthreads();
+    if (v != 0ull) {
+        int rk = lane;  // keys are unique: `lane` entries of this warp's list are larger
+        for (int w2 = 0; w2 < kWarps; ++w2) {
+            if (w2 == warp) continue;
+            int lo = 0, hi = 32;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (sorted[w2 * 32 + mid] > v) lo = mid + 1;
+                else hi = mid;
+            }
+            rk += lo;
+        }
+        if (rk == K - 1) *thr_sh = v;
+    }
+    __syncthreads();
+    const unsigned long long thr = *thr_sh;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int m = tid + u * kThreads;
+        if (m < Cb) {
+            const unsigned long long k = key_of(x[u], m);
+            if (k >= thr) {
+                const int pos = atomicAdd(&misc[5], 1);
+                if (pos < kCandCap) cand[pos] = k;
+            }
+        }
+    }
+    __syncthreads();
+    const int C = misc[5];
+    if (C > kCandCap) return -1;
+    for (int c = tid; c < C; c += kThreads) {
+        const unsigned long long k = cand[c];
+        int rk = 0;
+        for (int j = 0; j < C; ++j) rk += cand[j] > k;
+        if (rk < K) chosen[rk] = k;
+    }
+    __syncthreads();
+    for (int j = tid; j < K; j += kThreads) {
+        const uint32_t m = 0xFFFFFFFFu - (uint32_t)(chosen[j] & 0xFFFFFFFFull);
+        int pos = 0;
+        for (int j2 = 0; j2 < K; ++j2) pos += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m;
+        list[1 + pos] = (int)m;
+    }
+    // generic-proxy writes to ring stage 1 before TMA reuses it
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    return K;
 }
 
 // Fused Top-K over the row's Cb block scores, split across the cluster.
@@ -440,10 +548,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
     }
-    // q of the group, padded to 16 rows
-    for (int i = tid; i < 16 * kD; i += kThreads) {
-        const int r = i / kD, e = i % kD;
-        qs[r * kQLd + e] = r < G ? a.q[((long)b * a.Hq + h * G + r) * kD + e] : __float2bfloat16_rn(0.f);
+    // q of the group, padded to 16 rows: one 16-byte load per thread
+    if (tid < 16 * kD / 8) {
+        const int r = tid / (kD / 8), e = (tid % (kD / 8)) * 8;
+        const uint4 val = r < G ? *reinterpret_cast<const uint4*>(a.q + ((long)b * a.Hq + h * G + r) * kD + e)
+                                : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(qs + r * kQLd + e) = val;
     }
     // attended list: entry 0 = current (partial) block, entries 1.. = history blocks ascending
     int nsel;
@@ -477,10 +587,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         }
         const int Csel = min(Cb, a.s_cols);
         const int chunk = (Csel + CL - 1) / CL;
-        if (a.top_k < Csel && chunk <= (int)(kStage / 4) && CL * a.top_k <= (int)(kStage / 8))
-            nsel = cluster_topk_fast<CL>(a, bh, Csel, rank, base, list);
-        else
-            nsel = cluster_topk<CL>(a, bh, Csel, rank, base, list);
+        nsel = (a.top_k < Csel && a.top_k <= 64 && Csel <= kPer * kThreads) ? row_topk_filter(a, bh, Csel, base, list)
+                                                                            : -1;
+        if (nsel < 0) {
+            if (a.top_k < Csel && chunk <= (int)(kStage / 4) && CL * a.top_k <= (int)(kStage / 8))
+                nsel = cluster_topk_fast<CL>(a, bh, Csel, rank, base, list);
+            else
+                nsel = cluster_topk<CL>(a, bh, Csel, rank, base, list);
+        }
         if (rank == 0 && a.idx_out)
             for (int i = tid; i < a.top_k; i += kThreads) a.idx_out[(long)bh * a.top_k + i] = i < nsel ? list[1 + i] : -1;
     }
@@ -732,7 +846,9 @@ bool decode_sm100_supported(const DecodeParams& p) {
     if (!p.is_bf16 || p.d != kD || p.bs != kBS) return false;
     const int G = p.Hq / p.Hkv;
     if (G < 1 || G > 16) return false;
-    if ((reinterpret_cast<uintptr_t>(p.k) | reinterpret_cast<uintptr_t>(p.v)) & 15u) return false;
+    if ((reinterpret_cast<uintptr_t>(p.k) | reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.q)) &
+        15u)
+        return false;
     if ((long)p.B * p.Hkv > 65535) return false;
     return Layout::bytes(G, p.top_k + 1) <= 227 * 1024;
 }
