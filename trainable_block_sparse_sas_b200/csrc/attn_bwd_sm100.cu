@@ -36,7 +36,8 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kBS = 64;
-constexpr int kStages = 2;
+constexpr int kStages = 2;                   // dk/dv Q/dO ring depth
+constexpr size_t kSmemLimit = 227 * 1024;     // dynamic shared memory per CTA
 constexpr uint32_t kSlab64 = 64 * 128;    // 64 rows x 128 B: one block, one 64-wide d slab
 constexpr uint32_t kSlab128 = 128 * 128;  // 128 rows x 128 B
 
@@ -90,27 +91,35 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 constexpr int kDqThreads = 416;
 constexpr int kDqSoftmaxWarp0 = 5;
 
-template <int MT>
+// ST: depth of the K/V ring (3 where the shared memory allows it: a block's
+// K/V is then requested two blocks ahead of its use).
+template <int MT, int ST>
 struct DqLayout {
     static constexpr int G = 2 * MT;
     static constexpr uint32_t kHalf = MT * kSlab128;  // all query rows, one d slab
     static constexpr uint32_t kQ = 0;
     static constexpr uint32_t kDO = kQ + 2 * kHalf;
     static constexpr uint32_t kK = kDO + 2 * kHalf;
-    static constexpr uint32_t kV = kK + kStages * 2 * kSlab64;
-    static constexpr uint32_t kBars = kV + kStages * 2 * kSlab64;
+    static constexpr uint32_t kV = kK + ST * 2 * kSlab64;
+    static constexpr uint32_t kBars = kV + ST * 2 * kSlab64;
     // q_full, kv_full[S], kv_empty[S], s_full[2], ds_ready[2], dq_done, drain, issued[2]
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 2;
+    static constexpr int kNumBars = 1 + 2 * ST + 2 + 2 + 1 + 1 + 2;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
     static constexpr uint32_t kList = kMisc + 16;
-    // list [Cq + 1] ints, biases [Cq + 1] floats, then the per-warp dlogg partials
-    __host__ __device__ static uint32_t part_off(int Cq) { return (kList + 8 * (uint32_t)(Cq + 1) + 15) & ~15u; }
-    static size_t bytes(int Cq) { return 1024 + part_off(Cq) + 32 * (size_t)(Cq + 1); }
+    // list [nl] ints, biases [nl] floats, then the per-warp dlogg partials [nl][8];
+    // nl = the longest list (attended history blocks + the current block)
+    __host__ __device__ static uint32_t part_off(int nl) { return (kList + 8 * (uint32_t)nl + 15) & ~15u; }
+    static size_t bytes(int nl) { return 1024 + part_off(nl) + 32 * (size_t)nl; }
 };
 
-template <int MT>
+__host__ __device__ inline int dq_list_max(int Cq, int top_k, int full_scope) {
+    return (full_scope ? Cq : min(top_k, Cq)) + 1;
+}
+
+template <int MT, int ST>
 __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __grid_constant__ BwdArgs a) {
-    using L = DqLayout<MT>;
+    using L = DqLayout<MT, ST>;
+    constexpr int kStages = ST;
     constexpr int G = L::G;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -130,8 +139,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
     float* tot_sh = reinterpret_cast<float*>(base + L::kMisc + 12);
     int* list = reinterpret_cast<int*>(base + L::kList);
-    float* part = reinterpret_cast<float*>(base + L::part_off(a.Cq));  // [slot][8 softmax warps]
-    float* bias2 = reinterpret_cast<float*>(base + L::kList + 4 * (a.Cq + 1));  // log-gate, log2 units
+    const int nl = dq_list_max(a.Cq, a.top_k, a.full_scope);
+    float* part = reinterpret_cast<float*>(base + L::part_off(nl));  // [slot][8 softmax warps]
+    float* bias2 = reinterpret_cast<float*>(base + L::kList + 4 * nl);  // log-gate, log2 units
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // head-major order (concurrent CTAs share one KV head in L2), long query blocks first
@@ -140,7 +150,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long unit = (long)bh * a.Cq + c;
 
-    for (int i = threadIdx.x; i < 8 * (a.Cq + 1); i += kDqThreads) part[i] = 0.f;
+    for (int i = threadIdx.x; i < 8 * nl; i += kDqThreads) part[i] = 0.f;
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int s = 0; s < kStages; ++s) {
@@ -749,7 +759,10 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, kBS) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, kBS) ||
         !encode_tma_rows(&a.tk, p.k, p.Hkv, rows, 1, kBS) || !encode_tma_rows(&a.tv, p.v, p.Hkv, rows, 1, kBS))
         return cudaErrorInvalidValue;
-    cudaError_t err = launch_kernel(bwd_dq_sm100_kernel<MT>, grid, kDqThreads, DqLayout<MT>::bytes(p.Cq), a, stream);
+    const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope);
+    cudaError_t err = DqLayout<MT, 3>::bytes(nl) <= kSmemLimit
+                          ? launch_kernel(bwd_dq_sm100_kernel<MT, 3>, grid, kDqThreads, DqLayout<MT, 3>::bytes(nl), a, stream)
+                          : launch_kernel(bwd_dq_sm100_kernel<MT, 2>, grid, kDqThreads, DqLayout<MT, 2>::bytes(nl), a, stream);
     if (err != cudaSuccess) return err;
     // key-major kernel: 128-row items (128/G tokens x G heads) per box
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, 128 / G) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, 128 / G))
@@ -769,7 +782,8 @@ bool bwd_sm100_supported(const TrainParams& p) {
                          reinterpret_cast<uintptr_t>(p.dv) | reinterpret_cast<uintptr_t>(p.o_in);
     if (al & 15u) return false;
     if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq > 0x7fffffffL) return false;
-    return DqLayout<2>::bytes(p.Cq) <= 227 * 1024 && DkvLayout::bytes(p.Cq) <= 227 * 1024;
+    const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope);
+    return DqLayout<2, 2>::bytes(nl) <= kSmemLimit && DkvLayout::bytes(p.Cq) <= kSmemLimit;
 }
 
 cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream) {
