@@ -339,3 +339,37 @@ def test_decode_cluster_sizes_and_ties(api):
         for (b, h), (ro, ridx) in ref.items():
             np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx)
             compare(f"o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+
+
+def test_decode_selection_paths(api):
+    """The fused selection's paths, each against the oracle: the per-CTA threshold
+    filter (random scores); its fall-back to the radix select when more than 512
+    keys reach the threshold (a score that depends only on the block index modulo
+    the CTA's thread count, so whole threads' strides tie above it); and Top-K above
+    the filter's limit of 64."""
+    bs = 64
+    nblk = 3000
+    Tmax = bs * nblk + 7
+    B, Hq, Hkv = 2, 4, 2
+    base = {
+        "q": _seeded((B, Hq, 128), 1.0, torch.bfloat16, 71),
+        "k_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 72),
+        "v_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 73),
+        "ctx_len": torch.tensor([Tmax, Tmax - 200], dtype=torch.int32, device="cuda"),
+    }
+    C = Tmax // bs
+    m = torch.arange(C, dtype=torch.float32, device="cuda")
+    strided = ((m % 288) * 0.01).expand(B, Hkv, C).contiguous()
+    strided[1, 1] += 0.003  # rows differ
+    cases = (("filter", _seeded((B, Hkv, C), 1.0, torch.float32, 74), 48),
+             ("radix fall-back", strided, 64),
+             ("K above the filter", _seeded((B, Hkv, C), 1.0, torch.float32, 75), 100))
+    G = Hq // Hkv
+    rows = [(b, h) for b in range(B) for h in range(Hkv)]
+    for name, s, K in cases:
+        inp = dict(base, s=s)
+        o, idx = _run_decode(api, inp, bs, K, fused=True)
+        ref = _oracle_decode_rows(inp, rows, bs, K, False)
+        for (b, h), (ro, ridx) in ref.items():
+            np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx, err_msg=f"{name} idx[{b},{h}]")
+            compare(f"{name} o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)

@@ -10,18 +10,22 @@
 // One CTA per (batch, kv head, query block).  The G query heads of the group
 // share the selection, so their 64 rows each are stacked into G*64 query rows
 // (row r = token * G + head, exactly the order of a TMA box over [token, head,
-// d]) and processed as G/2 M-tiles of 128 rows.  Attended key blocks go two at a
-// time (N = 128 keys) through a 2-stage shared-memory ring.
+// d]) and processed as G/2 M-tiles of 128 rows.  Attended key blocks go one at a
+// time (N = 64 keys) through a 4-stage shared-memory ring of K and V.
 //   warp 0      TMA producer: Q once, then K and V blocks by block index
-//   warp 1      TMEM allocation and the single MMA-issuing thread:
-//                 S_i = Q_i K^T        (SS MMA, S in TMEM, 128 lanes x N columns)
-//                 O_i += P_i V         (TS MMA, P read from TMEM where S was)
-//   warps 2..9  softmax, one warpgroup per M-tile, one thread per row: scale,
+//   warps 1..4  MMA issuers, two per M-tile (a single thread's chain of small
+//               MMAs is latency-bound; the chains run concurrently):
+//                 S_i = Q_i K^T   (SS MMA into TMEM buffer t mod 2 of tile i)
+//                 O_i += P_i V    (TS MMA, P read from the buffer it was written to)
+//               With two S buffers per tile, S of block t+1 is computed while the
+//               softmax of block t runs; S of block t+2 waits for PV of block t.
+//   warps 5..12 softmax, one warpgroup per M-tile, one thread per row: scale,
 //               add the block's log-gate bias (log2 units), mask the current
 //               block causally, online max with lazy rescale of O (only when the
 //               max grows by more than 2^8), exponentiate, write P as bf16 into
 //               TMEM, and finally normalise O and store o and lse.
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+// TMEM columns: tile i's S buffers [128 i, 128 i + 64) and [128 i + 64, 128 i + 128)
+// (P in the first 32 columns of its buffer), O_i [256 + 128 i, 384 + 128 i).
 // Every wait is time-bounded; on a timeout the kernel records the device status
 // word, drains its MMAs, frees TMEM and returns.
 #include <cudaTypedefs.h>
@@ -38,12 +42,13 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kBS = 64;
-constexpr int kStages = 2;
-constexpr int kThreads = 320;
+constexpr int kStages = 4;                 // K/V ring, one attended block per stage
+// warp 0 TMA; warps 1..4 MMA issuers (S and PV per M-tile); warps 5..12 softmax
+constexpr int kThreads = 416;
+constexpr int kSoftmaxWarp0 = 5;
 constexpr float kRescaleLog2 = 8.f;
-constexpr uint32_t kKvHalf = 128 * 128;     // 2 blocks x 64 rows x 128 B (one 64-wide d slab)
-constexpr uint32_t kKvStage = 2 * kKvHalf;  // both d slabs
-constexpr uint32_t kBlockSlab = 64 * 128;   // one block, one d slab
+constexpr uint32_t kSlab = 64 * 128;        // one block (64 rows x 128 B), one 64-wide d slab
+constexpr uint32_t kStage = 4 * kSlab;      // K (2 slabs) then V (2 slabs)
 
 struct FwdArgs {
     CUtensorMap tq, tk, tv;
@@ -62,11 +67,12 @@ struct FwdLayout {
     static constexpr int G = 2 * MT;
     static constexpr uint32_t kQHalf = MT * 128 * 128;  // all query rows, one d slab
     static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kK = kQ + 2 * kQHalf;
-    static constexpr uint32_t kV = kK + kStages * kKvStage;
-    static constexpr uint32_t kBars = kV + kStages * kKvStage;
-    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 6 + 1;
+    static constexpr uint32_t kKV = kQ + 2 * kQHalf;     // [stage] { K: 2 slabs, V: 2 slabs }
+    static constexpr uint32_t kBars = kKV + kStages * kStage;
+    // q_full, kv_full[S], kv_empty[S], s_full[tile][buf], p_ready[tile][buf], pv_done[tile][buf],
+    // drain.  Per-buffer barriers: a buffer's next phase needs this block's PV, so no
+    // waiter can fall two phases behind.
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4 + 4 + 1;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;  // tmem base, abort flag, list count
     static constexpr uint32_t kList = kMisc + 16;  // [Cq + 1] ints, then [Cq + 1] biases
     static size_t bytes(int Cq) { return 1024 + kList + 8 * (size_t)(Cq + 1); }
@@ -91,15 +97,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(base);
-    const uint32_t sQ = sbase + L::kQ, sK = sbase + L::kK, sV = sbase + L::kV;
+    const uint32_t sQ = sbase + L::kQ, sKV = sbase + L::kKV;
     const uint32_t bar0 = sbase + L::kBars;
-    auto q_full = [&]() { return bar0; };
+    const uint32_t q_full = bar0;
     auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
     auto kv_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
-    auto s_full = [&](int i) { return bar0 + 8u * (1 + 2 * kStages + i); };
-    auto p_ready = [&](int i) { return bar0 + 8u * (3 + 2 * kStages + i); };
-    auto o_done = [&](int i) { return bar0 + 8u * (5 + 2 * kStages + i); };
-    const uint32_t drain = bar0 + 8u * (7 + 2 * kStages);
+    auto s_full = [&](int i, int bf) { return bar0 + 8u * (1 + 2 * kStages + 2 * i + bf); };
+    auto p_ready = [&](int i, int bf) { return bar0 + 8u * (5 + 2 * kStages + 2 * i + bf); };
+    auto pv_done = [&](int i, int bf) { return bar0 + 8u * (9 + 2 * kStages + 2 * i + bf); };
+    const uint32_t drain = bar0 + 8u * (13 + 2 * kStages);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
     int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
@@ -115,17 +121,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     const long unit = (long)bh * a.Cq + c;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full(), 1);
+        mbar_init(q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(kv_full(s), 1);
-            mbar_init(kv_empty(s), 1);
+            mbar_init(kv_empty(s), MT);  // each tile's PV issuer, after its PV of the block
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(s_full(i), 1);
-            mbar_init(p_ready(i), 128);
-            mbar_init(o_done(i), 1);
+            for (int bf = 0; bf < 2; ++bf) {
+                mbar_init(s_full(i, bf), 1);
+                mbar_init(p_ready(i, bf), 128);
+                mbar_init(pv_done(i, bf), 1);
+            }
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2 * MT);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&a.tq);
@@ -165,85 +173,66 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int nlist = *list_count;
-    const int nsteps = (nlist + 1) / 2;
+    const int nlist = *list_count;  // one step per attended block
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const int q_row = b * a.n + c * kBS;
-            mbar_arrive_expect_tx(q_full(), 2 * L::kQHalf);
-            tma_load_3d(sQ, &a.tq, q_full(), 0, h * G, q_row);
-            tma_load_3d(sQ + L::kQHalf, &a.tq, q_full(), 64, h * G, q_row);
-            for (int t = 0; t < nsteps; ++t) {
-                const int s = t % kStages, use = t / kStages;
-                if (t >= kStages && !mbar_wait(kv_empty(s), (use - 1) & 1, abort_flag, a.status)) break;
-                const int nb = min(2, nlist - 2 * t);
-                mbar_arrive_expect_tx(kv_full(s), (uint32_t)nb * 4u * kBlockSlab);
-                for (int bi = 0; bi < nb; ++bi) {
-                    const int row0 = b * a.n + list[2 * t + bi] * kBS;
-                    for (int kh = 0; kh < 2; ++kh) {
-                        const uint32_t off = s * kKvStage + kh * kKvHalf + bi * kBlockSlab;
-                        tma_load_3d(sK + off, &a.tk, kv_full(s), kh * 64, h, row0);
-                        tma_load_3d(sV + off, &a.tv, kv_full(s), kh * 64, h, row0);
-                    }
+            mbar_arrive_expect_tx(q_full, 2 * L::kQHalf);
+            tma_load_3d(sQ, &a.tq, q_full, 0, h * G, q_row);
+            tma_load_3d(sQ + L::kQHalf, &a.tq, q_full, 64, h * G, q_row);
+            for (int t = 0; t < nlist; ++t) {
+                const int s = t % kStages;
+                if (t >= kStages && !mbar_wait(kv_empty(s), (t / kStages - 1) & 1, abort_flag, a.status)) break;
+                mbar_arrive_expect_tx(kv_full(s), kStage);
+                const int row0 = b * a.n + list[t] * kBS;
+                const uint32_t st = sKV + s * kStage;
+                for (int kh = 0; kh < 2; ++kh) {
+                    tma_load_3d(st + kh * kSlab, &a.tk, kv_full(s), kh * 64, h, row0);
+                    tma_load_3d(st + 2 * kSlab + kh * kSlab, &a.tv, kv_full(s), kh * 64, h, row0);
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s64 = idesc_bf16_f32(128, 64, false, false);
-            constexpr uint32_t idesc_s128 = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
-            // per-tile interleaving: S_i(t+1) is issued right after PV_i(t), so tile 0's
-            // next softmax overlaps tile 1's current one
-            auto issue_s = [&](int t, int i) {
-                const int s = t % kStages;
-                const int nb = min(2, nlist - 2 * t);
-                const uint32_t idesc_s = nb == 2 ? idesc_s128 : idesc_s64;
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const int kh = ks >> 2, kk = ks & 3;
-                    const uint64_t ad = sdesc_sw128(sQ + kh * L::kQHalf + i * 128 * 128 + kk * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(sK + s * kKvStage + kh * kKvHalf + kk * 32, 16, 1024);
-                    mma_ss(tmem + i * 128, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(s_full(i));
-            };
-            bool ok = mbar_wait(q_full(), 0, abort_flag, a.status) && mbar_wait(kv_full(0), 0, abort_flag, a.status);
-            if (ok) {
-                tc_fence_after();
-                for (int i = 0; i < MT; ++i) issue_s(0, i);
-            }
-            for (int t = 0; ok && t < nsteps; ++t) {
-                const int s = t % kStages;
-                const int nb = min(2, nlist - 2 * t);
-                bool next_ready = false;
-                for (int i = 0; i < MT; ++i) {
-                    if (!mbar_wait(p_ready(i), t & 1, abort_flag, a.status)) {
-                        ok = false;
-                        break;
-                    }
+    } else if (warp <= 4) {
+        // ------------------------------------------------------------ MMA issuers
+        // warps 1, 3: S_i = Q_i K^T for tile i = (warp - 1) / 2; warps 2, 4: O_i += P_i V
+        const int i = (warp - 1) >> 1;
+        const bool pv_chain = ((warp - 1) & 1) != 0;
+        if (lane == 0 && i < MT) {
+            bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
+            if (!pv_chain) {
+                constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+                for (int t = 0; ok && t < nlist; ++t) {
+                    const int s = t % kStages, bf = t & 1;
+                    if (!mbar_wait(kv_full(s), (t / kStages) & 1, abort_flag, a.status)) break;
+                    // buffer bf holds P of block t-2 until its PV has run
+                    if (t >= 2 && !mbar_wait(pv_done(i, bf), ((t >> 1) - 1) & 1, abort_flag, a.status)) break;
                     tc_fence_after();
-                    for (int ks = 0; ks < 4 * nb; ++ks) {
-                        const uint64_t bd = sdesc_sw128(sV + s * kKvStage + ks * 2048, kKvHalf, 1024);
-                        mma_ts(tmem + 256 + i * 128, tmem + i * 128 + ks * 8, bd, idesc_pv,
-                               (t > 0 || ks > 0) ? 1u : 0u);
+                    const uint32_t kst = sKV + s * kStage;
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const int kh = ks >> 2, kk = ks & 3;
+                        mma_ss(tmem + i * 128 + bf * 64, sdesc_sw128(sQ + kh * L::kQHalf + i * 128 * 128 + kk * 32, 16, 1024),
+                               sdesc_sw128(kst + kh * kSlab + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                     }
-                    mma_commit(o_done(i));
-                    if (i == MT - 1 && t + kStages < nsteps) mma_commit(kv_empty(s));
-                    if (t + 1 < nsteps) {
-                        if (!next_ready) {
-                            if (!mbar_wait(kv_full((t + 1) % kStages), ((t + 1) / kStages) & 1, abort_flag, a.status)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            next_ready = true;
-                        }
-                        issue_s(t + 1, i);
+                    mma_commit(s_full(i, bf));
+                }
+            } else {
+                constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+                for (int t = 0; ok && t < nlist; ++t) {
+                    const int s = t % kStages, bf = t & 1;
+                    if (!mbar_wait(kv_full(s), (t / kStages) & 1, abort_flag, a.status)) break;
+                    if (!mbar_wait(p_ready(i, bf), (t >> 1) & 1, abort_flag, a.status)) break;
+                    tc_fence_after();
+                    const uint32_t vst = sKV + s * kStage + 2 * kSlab;
+#pragma unroll
+                    for (int ks = 0; ks < kBS / 16; ++ks) {
+                        mma_ts(tmem + 256 + i * 128, tmem + i * 128 + bf * 64 + ks * 8,
+                               sdesc_sw128(vst + ks * 2048, kSlab, 1024), idesc_pv, (t > 0 || ks > 0) ? 1u : 0u);
                     }
+                    mma_commit(pv_done(i, bf));
+                    if (t + kStages < nlist) mma_commit(kv_empty(s));
                 }
             }
             // all issued MMAs complete before TMEM is released
@@ -252,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         }
     } else {
         // ------------------------------------------------------------ softmax
-        const int grp = (warp - 2) >> 2;
+        const int grp = (warp - kSoftmaxWarp0) >> 2;
         const int quad = warp & 3;  // TMEM lane quadrant this warp may access
         if (grp < MT) {
             const int row = 32 * quad + lane;
@@ -262,98 +251,86 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             const uint32_t tO = tmem + ((uint32_t)(32 * quad) << 16) + 256 + grp * 128;
             float m_used = -INFINITY, l = 0.f;
             bool ok = true;
-            for (int t = 0; t < nsteps; ++t) {
-                if (!warp_wait(s_full(grp), t & 1, abort_flag, a.status)) {
+            for (int t = 0; t < nlist; ++t) {
+                const int bf = t & 1;
+                if (!warp_wait(s_full(grp, bf), (t >> 1) & 1, abort_flag, a.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int nb = min(2, nlist - 2 * t);
-                // pass 1: row max over the raw logits (sigma > 0), causal mask on the
-                // current block only
-                float mb[2];
+                const bool cur = (t == nlist - 1);
+                uint32_t r0[32], r1[32];
+                tmem_ld64_sync(tS + bf * 64, r0, r1);
+                // row max over the raw logits (sigma > 0), causal mask on the current block
+                float m0 = -INFINITY, m1 = -INFINITY;
+                if (!cur) {
 #pragma unroll
-                for (int bi = 0; bi < 2; ++bi) {
-                    mb[bi] = -INFINITY;
-                    if (bi < nb) {
-                        const bool cur = (2 * t + bi == nlist - 1);
-                        uint32_t r0[32], r1[32];
-                        tmem_ld64_sync(tS + bi * 64, r0, r1);
-                        float m0 = -INFINITY, m1 = -INFINITY;
-                        if (!cur) {
+                    for (int j = 0; j < 32; ++j) {
+                        m0 = fmaxf(m0, __uint_as_float(r0[j]));
+                        m1 = fmaxf(m1, __uint_as_float(r1[j]));
+                    }
+                } else {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                m0 = fmaxf(m0, __uint_as_float(r0[j]));
-                                m1 = fmaxf(m1, __uint_as_float(r1[j]));
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                if (j <= tok) m0 = fmaxf(m0, __uint_as_float(r0[j]));
-                                if (32 + j <= tok) m1 = fmaxf(m1, __uint_as_float(r1[j]));
-                            }
-                        }
-                        mb[bi] = fmaf(fmaxf(m0, m1), a.scale_log2, bias2[2 * t + bi]);
+                    for (int j = 0; j < 32; ++j) {
+                        if (j <= tok) m0 = fmaxf(m0, __uint_as_float(r0[j]));
+                        if (32 + j <= tok) m1 = fmaxf(m1, __uint_as_float(r1[j]));
                     }
                 }
-                const float mx = fmaxf(mb[0], mb[1]);
+                const float mx = fmaf(fmaxf(m0, m1), a.scale_log2, bias2[t]);
                 const float m_new = fmaxf(m_used, mx);
                 const bool need = m_new > m_used + kRescaleLog2;
                 if (__any_sync(0xffffffffu, need)) {
                     const float alpha = need ? ex2(m_used - m_new) : 1.f;
-                    if (t > 0) {  // PV of step t-1 completed before S of step t did
-#pragma unroll
+                    if (t > 0) {
+                        // O is final for block t-1 once that block's PV has completed
+                        if (!warp_wait(pv_done(grp, (t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag, a.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll 1
                         for (int ch = 0; ch < 4; ++ch) {
-                            uint32_t r[32];
-                            tmem_ld32_sync(tO + ch * 32, r);
+                            uint32_t ro[32];
+                            tmem_ld32_sync(tO + ch * 32, ro);
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                            tmem_st32(tO + ch * 32, r);
+                            for (int j = 0; j < 32; ++j) ro[j] = __float_as_uint(__uint_as_float(ro[j]) * alpha);
+                            tmem_st32(tO + ch * 32, ro);
                         }
                         tmem_wait_st();
                     }
                     l *= alpha;
                     if (need) m_used = m_new;
                 }
-                // pass 2: p = 2^(S sigma log2e + bias - m) with packed fp32 pairs, written
-                // as bf16 pairs over the columns already read
+                // p = 2^(S sigma log2e + bias - m) with packed fp32 pairs, written as bf16
+                // pairs over the first 32 columns of this buffer
+                const float off = bias2[t] - m_used;
+                const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
                 uint64_t rs2 = 0ull;
+                uint32_t pk[32];
 #pragma unroll
-                for (int bi = 0; bi < 2; ++bi) {
-                    if (bi < nb) {
-                        const bool cur = (2 * t + bi == nlist - 1);
-                        const float off = bias2[2 * t + bi] - m_used;
-                        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
-                        uint32_t r0[32], r1[32];
-                        tmem_ld64_sync(tS + bi * 64, r0, r1);
-                        uint32_t pk[32];
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const uint32_t* rr = jj < 16 ? r0 : r1;
-                            const int jl = (jj & 15) * 2;
-                            float x0, x1;
-                            f2_unpack(f2_fma(f2_pack(__uint_as_float(rr[jl]), __uint_as_float(rr[jl + 1])), sc2, off2),
-                                      x0, x1);
-                            float p0 = ex2(x0), p1 = ex2(x1);
-                            if (cur) {
-                                if (2 * jj > tok) p0 = 0.f;
-                                if (2 * jj + 1 > tok) p1 = 0.f;
-                            }
-                            rs2 = f2_add(rs2, f2_pack(p0, p1));
-                            pk[jj] = pack_bf16x2(p0, p1);
-                        }
-                        tmem_st32(tS + bi * 32, pk);
+                for (int jj = 0; jj < 32; ++jj) {
+                    const uint32_t* rr = jj < 16 ? r0 : r1;
+                    const int jl = (jj & 15) * 2;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(rr[jl]), __uint_as_float(rr[jl + 1])), sc2, off2), x0, x1);
+                    float p0 = ex2(x0), p1 = ex2(x1);
+                    if (cur) {
+                        if (2 * jj > tok) p0 = 0.f;
+                        if (2 * jj + 1 > tok) p1 = 0.f;
                     }
+                    rs2 = f2_add(rs2, f2_pack(p0, p1));
+                    pk[jj] = pack_bf16x2(p0, p1);
                 }
+                tmem_st32(tS + bf * 64, pk);
                 float rsa, rsb;
                 f2_unpack(rs2, rsa, rsb);
-                const float rs = rsa + rsb;
                 tmem_wait_st();
-                l += rs;
+                l += rsa + rsb;
                 tc_fence_before();
-                mbar_arrive(p_ready(grp));
+                mbar_arrive(p_ready(grp, bf));
             }
-            if (ok && warp_wait(o_done(grp), (nsteps - 1) & 1, abort_flag, a.status)) {
+            const int tl = nlist - 1;
+            if (ok && warp_wait(pv_done(grp, tl & 1), (tl >> 1) & 1, abort_flag, a.status)) {
                 tc_fence_after();
                 const float inv_l = 1.f / l;
                 const int hq = h * G + g;
