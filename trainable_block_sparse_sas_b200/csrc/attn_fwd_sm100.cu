@@ -70,9 +70,9 @@ struct FwdLayout {
     static constexpr uint32_t kKV = kQ + 2 * kQHalf;     // [stage] { K: 2 slabs, V: 2 slabs }
     static constexpr uint32_t kBars = kKV + kStages * kStage;
     // q_full, kv_full[S], kv_empty[S], s_full[tile][buf], p_ready[tile][buf], pv_done[tile][buf],
-    // drain.  Per-buffer barriers: a buffer's next phase needs this block's PV, so no
-    // waiter can fall two phases behind.
-    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4 + 4 + 1;
+    // drain, stagger.  Per-buffer barriers: a buffer's next phase needs this block's
+    // PV, so no waiter can fall two phases behind.
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4 + 4 + 1 + 1;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;  // tmem base, abort flag, list count
     static constexpr uint32_t kList = kMisc + 16;  // [Cq + 1] ints, then [Cq + 1] biases
     static size_t bytes(int Cq) { return 1024 + kList + 8 * (size_t)(Cq + 1); }
@@ -106,6 +106,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     auto p_ready = [&](int i, int bf) { return bar0 + 8u * (5 + 2 * kStages + 2 * i + bf); };
     auto pv_done = [&](int i, int bf) { return bar0 + 8u * (9 + 2 * kStages + 2 * i + bf); };
     const uint32_t drain = bar0 + 8u * (13 + 2 * kStages);
+    // single phase: tile 0's softmax has begun; tile 1 starts then, so that the two
+    // tiles' softmax phases (exponentials) and latency-bound phases interleave
+    const uint32_t stagger = bar0 + 8u * (14 + 2 * kStages);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
     int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
@@ -134,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             }
         }
         mbar_init(drain, 2 * MT);
+        mbar_init(stagger, 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&a.tq);
@@ -208,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                     if (!mbar_wait(kv_full(s), (t / kStages) & 1, abort_flag, a.status)) break;
                     // buffer bf holds P of block t-2 until its PV has run
                     if (t >= 2 && !mbar_wait(pv_done(i, bf), ((t >> 1) - 1) & 1, abort_flag, a.status)) break;
+                    if (i == 1 && t == 0 && !mbar_wait(stagger, 0, abort_flag, a.status)) break;
                     tc_fence_after();
                     const uint32_t kst = sKV + s * kStage;
 #pragma unroll
@@ -257,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                     ok = false;
                     break;
                 }
+                if (t == 0 && grp == 0 && quad == 0 && lane == 0) mbar_arrive(stagger);
                 tc_fence_after();
                 const bool cur = (t == nlist - 1);
                 uint32_t r0[32], r1[32];
