@@ -87,32 +87,25 @@ __device__ __forceinline__ int block_sum_int(int v, int* scan) {
 // (K maxima reach it), so every key at or above it is a candidate; the K
 // best candidates by rank are the selection.  Returns K, or -1 when more than
 // kCandCap keys reach the bound (the caller then runs the radix select).
-// Rows of up to kPer * kThreads blocks (9216: 589,824 tokens at block 64).
+// Rows of up to kPer * kThreads blocks (9216: 589,824 tokens at block 64); the
+// caller loads the thread's scores x[u] = s[tid + u * kThreads] at kernel entry,
+// so their latency overlaps the prologue.
 constexpr int kCandCap = 512;
 constexpr int kPer = 32;  // scores per thread held in registers
 
-__device__ int row_topk_filter(const DecArgs& a, int bh, int Cb, uint8_t* base, int* list) {
+__device__ int row_topk_filter(const DecArgs& a, int Cb, const float (&x)[kPer], uint8_t* base, int* list) {
     constexpr int kWarps = kThreads / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int K = a.top_k;
-    const float* srow = a.s + (long)bh * a.s_cols;
     // scratch in ring stage 1 (stage 0 may hold the prefetched current block)
     unsigned long long* sorted = reinterpret_cast<unsigned long long*>(base + Layout::kRing + kStage);
     unsigned long long* cand = sorted + kWarps * 32;
     unsigned long long* chosen = cand + kCandCap;
     unsigned long long* thr_sh = chosen + 64;
     int* misc = reinterpret_cast<int*>(base + Layout::kMisc);
-    auto key_of = [&](float x, int m) -> unsigned long long {
-        return ((unsigned long long)order_key(x) << 32) | (0xFFFFFFFFu - (uint32_t)m);
+    auto key_of = [&](float s, int m) -> unsigned long long {
+        return ((unsigned long long)order_key(s) << 32) | (0xFFFFFFFFu - (uint32_t)m);
     };
-    // the row is read once, every load of a thread in flight together, and kept in
-    // registers for both passes (rows of up to kPer * kThreads blocks)
-    float x[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-        const int m = tid + u * kThreads;
-        x[u] = m < Cb ? srow[m] : 0.f;
-    }
     unsigned long long v = 0ull;  // 0: no score (every real key is larger)
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
@@ -136,31 +129,45 @@ __device__ int row_topk_filter(const DecArgs& a, int bh, int Cb, uint8_t* base, 
     }
     sorted[warp * 32 + lane] = v;
     __syncthreads();
-    if (v != 0ull) {
-        int rk = lane;  // keys are unique: `lane` entries of this warp's list are larger
-        for (int w2 = 0; w2 < kWarps; ++w2) {
-            if (w2 == warp) continue;
-            int lo = 0, hi = 32;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (sorted[w2 * 32 + mid] > v) lo = mid + 1;
-                else hi = mid;
+    // rank of this maximum among all: `lane` larger ones in its own list (keys are
+    // unique), plus a branch-free fixed-step search of every other list (the
+    // searches are independent, so their loads overlap)
+    {
+        int cnt[kWarps];
+#pragma unroll
+        for (int w2 = 0; w2 < kWarps; ++w2) cnt[w2] = 0;
+#pragma unroll
+        for (int step = 16; step > 0; step >>= 1) {
+#pragma unroll
+            for (int w2 = 0; w2 < kWarps; ++w2) {
+                const unsigned long long e = sorted[w2 * 32 + cnt[w2] + step - 1];
+                cnt[w2] += e > v ? step : 0;
             }
-            rk += lo;
         }
-        if (rk == K - 1) *thr_sh = v;
+        int rk = lane;
+#pragma unroll
+        for (int w2 = 0; w2 < kWarps; ++w2) {
+            // cnt counts up to 31 entries; the last entry is compared apart
+            const int c2 = cnt[w2] + (sorted[w2 * 32 + 31] > v ? 1 : 0) * (cnt[w2] == 31 ? 1 : 0);
+            rk += w2 == warp ? 0 : c2;
+        }
+        if (v != 0ull && rk == K - 1) *thr_sh = v;
     }
     __syncthreads();
     const unsigned long long thr = *thr_sh;
+    // candidates: every key at or above thr, one shared-memory atomic per warp and pass
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
         const int m = tid + u * kThreads;
-        if (m < Cb) {
-            const unsigned long long k = key_of(x[u], m);
-            if (k >= thr) {
-                const int pos = atomicAdd(&misc[5], 1);
-                if (pos < kCandCap) cand[pos] = k;
-            }
+        const unsigned long long k = m < Cb ? key_of(x[u], m) : 0ull;
+        const bool take = m < Cb && k >= thr;
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        if (bal) {
+            int base_pos = 0;
+            if (lane == 0) base_pos = atomicAdd(&misc[5], __popc(bal));
+            base_pos = __shfl_sync(0xffffffffu, base_pos, 0);
+            const int pos = base_pos + __popc(bal & ((1u << lane) - 1u));
+            if (take && pos < kCandCap) cand[pos] = k;
         }
     }
     __syncthreads();
@@ -168,14 +175,17 @@ __device__ int row_topk_filter(const DecArgs& a, int bh, int Cb, uint8_t* base, 
     if (C > kCandCap) return -1;
     for (int c = tid; c < C; c += kThreads) {
         const unsigned long long k = cand[c];
-        int rk = 0;
-        for (int j = 0; j < C; ++j) rk += cand[j] > k;
+        int rk = 0, j = 0;
+        for (; j + 4 <= C; j += 4)
+            rk += (cand[j] > k) + (cand[j + 1] > k) + (cand[j + 2] > k) + (cand[j + 3] > k);
+        for (; j < C; ++j) rk += cand[j] > k;
         if (rk < K) chosen[rk] = k;
     }
     __syncthreads();
     for (int j = tid; j < K; j += kThreads) {
         const uint32_t m = 0xFFFFFFFFu - (uint32_t)(chosen[j] & 0xFFFFFFFFull);
         int pos = 0;
+#pragma unroll 4
         for (int j2 = 0; j2 < K; ++j2) pos += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m;
         list[1 + pos] = (int)m;
     }
@@ -537,6 +547,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     int T = a.ctx_len[b];
     T = max(1, min(T, a.Tmax));
     const int t = T - 1, Cb = t / kBS;
+    // fused selection by the per-CTA filter: this thread's scores, requested first
+    const int Csel = min(Cb, a.s_cols);
+    const bool use_filter = a.mode == 1 && a.top_k < Csel && a.top_k <= 64 && Csel <= kPer * kThreads;
+    float xs[kPer];
+    if (use_filter) {
+        const float* srow = a.s + (long)bh * a.s_cols;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int m = tid + u * kThreads;
+            xs[u] = m < Csel ? srow[m] : 0.f;
+        }
+    }
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -585,10 +607,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
             tma_load_3d(ring + kTile, &a.tv, full(0), 0, row0, bh);
             tma_load_3d(ring + kTile + kHalf, &a.tv, full(0), 64, row0, bh);
         }
-        const int Csel = min(Cb, a.s_cols);
         const int chunk = (Csel + CL - 1) / CL;
-        nsel = (a.top_k < Csel && a.top_k <= 64 && Csel <= kPer * kThreads) ? row_topk_filter(a, bh, Csel, base, list)
-                                                                            : -1;
+        nsel = use_filter ? row_topk_filter(a, Csel, xs, base, list) : -1;
         if (nsel < 0) {
             if (a.top_k < Csel && chunk <= (int)(kStage / 4) && CL * a.top_k <= (int)(kStage / 8))
                 nsel = cluster_topk_fast<CL>(a, bh, Csel, rank, base, list);
