@@ -166,11 +166,19 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         mbar_init(drain, 2 * MT);
         *abort_flag = 0;
         fence_barrier_init();
-        prefetch_tmap(&a.tq);
-        prefetch_tmap(&a.tdo);
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
+        // Q and dO of the query block do not depend on the selection: request them now
+        const int q_row = b * a.n + c * kBS;
+        mbar_arrive_expect_tx(q_full, 4 * L::kHalf);
+        for (int kh = 0; kh < 2; ++kh) {
+            tma_load_3d(sQ + kh * L::kHalf, &a.tq, q_full, kh * 64, h * G, q_row);
+            tma_load_3d(sDO + kh * L::kHalf, &a.tdo, q_full, kh * 64, h * G, q_row);
+        }
     }
+    // the score row is read again by the ds epilogue: have it in L2 by then
+    if (threadIdx.x < (a.Cq * 4 + 127) / 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.s + unit * a.Cq + threadIdx.x * 32) : "memory");
     if (warp == 0) {
         // attended history blocks (ascending) with their log-gate biases, then the
         // current block (bias 0); lanes read the selection in parallel
@@ -208,12 +216,6 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
 
     if (warp == 0) {
         if (lane == 0) {
-            const int q_row = b * a.n + c * kBS;
-            mbar_arrive_expect_tx(q_full, 4 * L::kHalf);
-            for (int kh = 0; kh < 2; ++kh) {
-                tma_load_3d(sQ + kh * L::kHalf, &a.tq, q_full, kh * 64, h * G, q_row);
-                tma_load_3d(sDO + kh * L::kHalf, &a.tdo, q_full, kh * 64, h * G, q_row);
-            }
             for (int t = 0; t < nlist; ++t) {
                 const int s = t % kStages;
                 if (t >= kStages && !mbar_wait(kv_empty(s), (t / kStages - 1) & 1, abort_flag, a.status)) break;
@@ -399,10 +401,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         part[t * 8] = acc;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (warp == 0) {
         float tot = 0.f;
-        for (int t = 0; t < nsel; ++t) tot += part[t * 8];
-        *tot_sh = tot;
+        for (int t = lane; t < nsel; t += 32) tot += part[t * 8];
+        tot = warp_sum(tot);
+        if (lane == 0) *tot_sh = tot;
     }
     __syncthreads();
     if (*abort_flag) return;
@@ -410,9 +413,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     const float* srow = a.s + unit * a.Cq;
     const float lse_c = a.lse_s[unit];
     float* dsrow = a.ds + unit * a.Cq;
+    // every block: -g_m * sum(dlogg) (0 from c on); then the attended ones are
+    // overwritten with dlogg_m - g_m * sum(dlogg), g_m from the bias kept in smem
     for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
     __syncthreads();
-    for (int t = threadIdx.x; t < nsel; t += kDqThreads) dsrow[list[t]] += part[t * 8];
+    for (int t = threadIdx.x; t < nsel; t += kDqThreads) dsrow[list[t]] = part[t * 8] - exp2f(bias2[t]) * tot;
 }
 
 // ============================================================================
@@ -489,17 +494,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long ubase = (long)bh * a.Cq;
 
-    // query blocks attending key block m: m itself, then every c > m holding m
-    list[0] = m;
-    int nlist = 1;
-    for (int c0 = m + 1; c0 < a.Cq; c0 += kKvThreads) {
-        const int cc = c0 + (int)threadIdx.x;
-        const int att = (cc < a.Cq && (a.full_scope || holds(a, ubase + cc, cc, m))) ? 1 : 0;
-        int cnt;
-        const int pos = block_exclusive_scan(att, scan, &cnt);
-        if (att) list[nlist + pos] = cc;
-        nlist += cnt;
-    }
     if (threadIdx.x == 0) {
         // arrival counts: commits of the chains that must all have completed
         mbar_init(kv_full, 1);
@@ -519,8 +513,25 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         fence_barrier_init();
         prefetch_tmap(&a.tq);
         prefetch_tmap(&a.tdo);
-        prefetch_tmap(&a.tk);
-        prefetch_tmap(&a.tv);
+        // K and V of the key block do not depend on the list: requested before it is built
+        mbar_arrive_expect_tx(kv_full, 4 * kSlab64);
+        const int krow = b * a.n + m * kBS;
+        for (int kh = 0; kh < 2; ++kh) {
+            tma_load_3d(sK + kh * kSlab64, &a.tk, kv_full, kh * 64, h, krow);
+            tma_load_3d(sV + kh * kSlab64, &a.tv, kv_full, kh * 64, h, krow);
+        }
+    }
+
+    // query blocks attending key block m: m itself, then every c > m holding m
+    list[0] = m;
+    int nlist = 1;
+    for (int c0 = m + 1; c0 < a.Cq; c0 += kKvThreads) {
+        const int cc = c0 + (int)threadIdx.x;
+        const int att = (cc < a.Cq && (a.full_scope || holds(a, ubase + cc, cc, m))) ? 1 : 0;
+        int cnt;
+        const int pos = block_exclusive_scan(att, scan, &cnt);
+        if (att) list[nlist + pos] = cc;
+        nlist += cnt;
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -534,12 +545,6 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
 
     if (warp == 0) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(kv_full, 4 * kSlab64);
-            const int krow = b * a.n + m * kBS;
-            for (int kh = 0; kh < 2; ++kh) {
-                tma_load_3d(sK + kh * kSlab64, &a.tk, kv_full, kh * 64, h, krow);
-                tma_load_3d(sV + kh * kSlab64, &a.tv, kv_full, kh * 64, h, krow);
-            }
             for (int j = 0; j < nitems; ++j) {
                 const int st = j % kStages;
                 if (j >= kStages && !mbar_wait(qd_empty(st), (j / kStages - 1) & 1, abort_flag, a.status)) break;

@@ -140,9 +140,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         mbar_init(stagger, 1);
         *abort_flag = 0;
         fence_barrier_init();
-        prefetch_tmap(&a.tq);
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
+        // Q of the query block does not depend on the selection: request it now
+        const int q_row = b * a.n + c * kBS;
+        mbar_arrive_expect_tx(q_full, 2 * L::kQHalf);
+        tma_load_3d(sQ, &a.tq, q_full, 0, h * G, q_row);
+        tma_load_3d(sQ + L::kQHalf, &a.tq, q_full, 64, h * G, q_row);
     }
     if (warp == 0) {
         // attended history blocks (ascending) with their log-gate biases, then the
@@ -182,10 +186,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const int q_row = b * a.n + c * kBS;
-            mbar_arrive_expect_tx(q_full, 2 * L::kQHalf);
-            tma_load_3d(sQ, &a.tq, q_full, 0, h * G, q_row);
-            tma_load_3d(sQ + L::kQHalf, &a.tq, q_full, 64, h * G, q_row);
             for (int t = 0; t < nlist; ++t) {
                 const int s = t % kStages;
                 if (t >= kStages && !mbar_wait(kv_empty(s), (t / kStages - 1) & 1, abort_flag, a.status)) break;
