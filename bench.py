@@ -313,8 +313,10 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
     """Median device time of one decode step with L2 flushed (a 512 MB read, so
     no dirty lines are written back inside the timed window) before every
     repetition.  mode: "fused" (sas_sparse_decode_select: selection + attention
-    in one launch), "two_call" (sas_topk_select then sas_sparse_decode), or
-    "dense" (sas_sparse_decode over every cached token)."""
+    in one launch), "two_call" (sas_topk_select then sas_sparse_decode), "dense"
+    (sas_sparse_decode over every cached token), or "paged" (the fused step on the
+    same cache scattered into a shuffled pool of one-block pages,
+    sas_sparse_decode_paged)."""
     import torch
 
     from trainable_block_sparse_sas_b200 import synthetic as syn
@@ -327,10 +329,30 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
     ws = api.workspace(api.sas_sparse_decode_workspace_size(desc), q.device)
     flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
     s4 = s.view(w.B, w.Hkv, 1, -1)
+    if mode == "paged":
+        pps = (w.T + w.bs - 1) // w.bs
+        g = torch.Generator(device="cpu")
+        g.manual_seed(3100)
+        table = torch.randperm(w.B * pps, generator=g).view(w.B, pps).to(torch.int32).cuda()
+        pools = []
+        for c in (kc, vc):
+            pool = torch.empty((w.B * pps, w.bs, w.Hkv, w.d), dtype=c.dtype, device="cuda")
+            for b in range(w.B):  # one sequence at a time keeps the temporaries small
+                pages = torch.nn.functional.pad(c[b], (0, 0, 0, pps * w.bs - w.T))
+                pool[table[b].long()] = pages.view(w.Hkv, pps, w.bs, w.d).permute(1, 2, 0, 3)
+                del pages
+            pools.append(pool)
+        inp["k_cache"] = inp["v_cache"] = kc = vc = c = None
+        torch.cuda.empty_cache()
+        kp, vp = pools
+        pdesc = api.paged_decode_desc(q, kp, w.bs, w.top_k, w.T)
 
     def run():
         if mode == "fused":
             api.sas_sparse_decode_select(desc, q, kc, vc, ctx, s, o, idx)
+            return
+        if mode == "paged":
+            api.sas_sparse_decode_paged(pdesc, q, kp, vp, table, ctx, o, s=s, idx_out=idx)
             return
         if mode == "two_call":
             api.sas_topk_select(s4, 1, s.shape[-1], w.top_k, idx=idx, ctx_len=ctx, block_size=w.bs)
@@ -488,7 +510,8 @@ def extras(api, args, peaks, peak_kind) -> dict:
         rec = {"ms": ms, "bytes": by, "gbs": gbs, "frac_of_hbm": gbs / hbm, "hbm_peak_gbs": hbm,
                "peak_source": f"{peak_kind} copy", "l2": "flushed (512 MB read) before every repetition",
                "includes": "Top-K selection + sparse decode in one launch (sas_sparse_decode_select)",
-               "two_call_ms": time_decode(api, w, steps=10, mode="two_call")}
+               "two_call_ms": time_decode(api, w, steps=10, mode="two_call"),
+               "paged_ms": time_decode(api, w, steps=10, mode="paged")}
         if w is syn.DECODE_512K:
             msd = time_decode(api, w, steps=5, mode="dense")
             byd = decode_bytes(w, dense=True)

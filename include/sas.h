@@ -195,6 +195,36 @@ sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, 
                                     void* o, int32_t* idx_out, sas_stream_t stream);
 
 /*
+ * sas_sparse_decode_paged -- the decode step over a paged KV cache, the form the
+ *   pages' serving backend uses (jaehun.me review, "Our Perspective: Strengths",
+ *   engineering completeness: paged KV cache, GQA, CUDA graphs; shibing624
+ *   review, engineering paragraph).  A page holds one block (block_size tokens)
+ *   of every kv head.  One launch, no workspace and no host synchronisation, so
+ *   the call can be captured in a CUDA graph and replayed with new q, s,
+ *   ctx_len and page_table contents.
+ * k_pages, v_pages  [num_pages, block_size, Hkv, d] pools (token-major within a
+ *          page, kv heads interleaved); 16-byte aligned.
+ * page_table  device int32 [B, pages_per_seq]: entry (b, j) is the page holding
+ *          block j (tokens j*block_size ..) of sequence b.  A page id outside
+ *          [0, num_pages), or a block at or past pages_per_seq, reads as zeros.
+ * ctx_len  device int32 [B], 1 <= ctx_len[b] <= desc->max_ctx, and
+ *          desc->max_ctx <= pages_per_seq * block_size (ragged lengths allowed).
+ * s, s_cols  when s != NULL the attended blocks are the Top-K of the scores, as
+ *          sas_sparse_decode_select (idx_out nullable, as there);
+ * idx      else when idx != NULL, the given blocks, as sas_sparse_decode;
+ *          else every block (dense comparator).
+ * q, o     as sas_sparse_decode.
+ * Errors: SAS_ERR_INVALID_VALUE (null pointers, pages_per_seq or num_pages <= 0,
+ *         max_ctx > pages_per_seq * block_size, s_cols <= 0 with s, unaligned
+ *         pools); SAS_ERR_UNSUPPORTED unless dtype is bf16, head_dim 128,
+ *         block_size 64 and at most 16 query heads per kv head.
+ */
+sas_status sas_sparse_decode_paged(const sas_decode_desc* desc, const void* q, const void* k_pages,
+                                   const void* v_pages, const int32_t* page_table, int32_t pages_per_seq,
+                                   int32_t num_pages, const int32_t* ctx_len, const int32_t* idx, const float* s,
+                                   int32_t s_cols, void* o, int32_t* idx_out, sas_stream_t stream);
+
+/*
  * sas_sparse_decode_noalloc -- the same decode as sas_sparse_decode (same
  *   arguments, layouts and results) for callers that cannot allocate device
  *   memory: a plugin whose host program owns all device memory, or a serving

@@ -133,3 +133,21 @@ def test_cuda_library_and_oracle_share_nothing(api):
     assert "#include \"" not in oracle_src and "sas.h" not in oracle_src
     deps = subprocess.run(["ldd", api._LIB_PATH], capture_output=True, text=True).stdout
     assert "oracle" not in deps
+
+
+def test_paged_decode_checks(api):
+    L = api.lib
+    d = api.DecodeDesc(2, 8, 2, 128, 64, 4, 1000, 1, 0.0)  # max_ctx 1000
+
+    def call(desc, pps=16, npages=64, kp=FAKE, s=FAKE, s_cols=16, table=FAKE):
+        return L.sas_sparse_decode_paged(ctypes.byref(desc), FAKE, kp, FAKE, table, pps, npages, FAKE, None, s,
+                                         s_cols, FAKE, None, None)
+
+    assert call(d, table=None) == 1
+    assert call(d, pps=0) == 1
+    assert call(d, npages=0) == 1
+    assert call(d, pps=15) == 1                       # 15 pages of 64 < max_ctx 1000
+    assert call(d, s_cols=0) == 1
+    assert call(d, kp=ctypes.c_void_p(0x1008)) == 1   # pool not 16-byte aligned
+    assert call(api.DecodeDesc(2, 8, 2, 128, 64, 4, 1000, 0, 0.0)) == 2         # fp32
+    assert call(api.DecodeDesc(2, 8, 2, 128, 32, 4, 1000, 1, 0.0), pps=32) == 2  # block 32

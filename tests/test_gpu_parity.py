@@ -373,3 +373,119 @@ def test_decode_selection_paths(api):
         for (b, h), (ro, ridx) in ref.items():
             np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx, err_msg=f"{name} idx[{b},{h}]")
             compare(f"{name} o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+
+
+def _paged_from_cache(kc, vc, bs, seed, spare=5):
+    """Scatter contiguous caches [B, Hkv, T, d] into shuffled page pools
+    [num_pages, bs, Hkv, d] (a few pages left unused) and the page table."""
+    B, Hkv, T, d = kc.shape
+    pps = (T + bs - 1) // bs
+    num = B * pps + spare
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    table = torch.randperm(num, generator=g)[: B * pps].view(B, pps).to(torch.int32)
+    pools = []
+    for c in (kc, vc):
+        padded = torch.nn.functional.pad(c, (0, 0, 0, pps * bs - T))  # [B, Hkv, pps*bs, d]
+        pages = padded.view(B, Hkv, pps, bs, d).permute(0, 2, 3, 1, 4).reshape(B * pps, bs, Hkv, d)
+        pool = torch.zeros((num, bs, Hkv, d), dtype=c.dtype, device=c.device)
+        pool[table.view(-1).long().to(c.device)] = pages
+        pools.append(pool)
+    return pools[0], pools[1], table.to(kc.device)
+
+
+def test_paged_decode_matches_oracle_and_contiguous(api):
+    """Paged cache, ragged lengths: the fused selection (bit-exact blocks), given
+    blocks, and dense attention against the oracle on the contiguous cache; given
+    blocks also bit-identical to the contiguous-cache call."""
+    bs, K = 64, 8
+    B, Hq, Hkv = 3, 8, 2
+    Tmax = bs * 40 + 7
+    inp = {
+        "q": _seeded((B, Hq, 128), 1.0, torch.bfloat16, 81),
+        "k_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 82),
+        "v_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 83),
+        "ctx_len": torch.tensor([Tmax, Tmax - 150, 700], dtype=torch.int32, device="cuda"),
+        "s": _seeded((B, Hkv, Tmax // bs), 1.0, torch.float32, 84),
+    }
+    kp, vp, table = _paged_from_cache(inp["k_cache"], inp["v_cache"], bs, 85)
+    q = inp["q"]
+    G = Hq // Hkv
+    rows = [(b, h) for b in range(B) for h in range(Hkv)]
+    desc = api.paged_decode_desc(q, kp, bs, K, Tmax)
+    # fused selection
+    o = torch.empty_like(q)
+    idx = torch.full((B, Hkv, K), -7, dtype=torch.int32, device="cuda")
+    api.sas_sparse_decode_paged(desc, q, kp, vp, table, inp["ctx_len"], o, s=inp["s"], idx_out=idx)
+    torch.cuda.synchronize()
+    ref = _oracle_decode_rows(inp, rows, bs, K, False)
+    for (b, h), (ro, ridx) in ref.items():
+        np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx)
+        compare(f"fused o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+    # given blocks: the same blocks, identical to the contiguous cache
+    o2 = torch.empty_like(q)
+    api.sas_sparse_decode_paged(desc, q, kp, vp, table, inp["ctx_len"], o2, idx=idx)
+    o3, _ = _run_decode(api, dict(inp), bs, K, fused=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, o3)
+    assert torch.equal(o, o3)
+    # dense
+    o4 = torch.empty_like(q)
+    api.sas_sparse_decode_paged(desc, q, kp, vp, table, inp["ctx_len"], o4)
+    torch.cuda.synchronize()
+    ref_d = _oracle_decode_rows(inp, rows, bs, K, True)
+    for (b, h), (ro, _) in ref_d.items():
+        compare(f"dense o[{b},{h}]", host(o4[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+
+
+def test_paged_decode_in_cuda_graph_and_missing_pages(api):
+    """The paged call captured in a CUDA graph replays with new q and scores; a
+    page id outside the pool reads as zeros (dense check against the oracle on a
+    cache with that block zeroed)."""
+    bs, K = 64, 6
+    B, Hq, Hkv = 2, 4, 1
+    Tmax = bs * 24 + 3
+    inp = {
+        "q": _seeded((B, Hq, 128), 1.0, torch.bfloat16, 91),
+        "k_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 92),
+        "v_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 93),
+        "ctx_len": torch.tensor([Tmax, Tmax - 70], dtype=torch.int32, device="cuda"),
+        "s": _seeded((B, Hkv, Tmax // bs), 1.0, torch.float32, 94),
+    }
+    kp, vp, table = _paged_from_cache(inp["k_cache"], inp["v_cache"], bs, 95)
+    q = inp["q"].clone()
+    s = inp["s"].clone()
+    desc = api.paged_decode_desc(q, kp, bs, K, Tmax)
+    o = torch.empty_like(q)
+    idx = torch.empty((B, Hkv, K), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        api.sas_sparse_decode_paged(desc, q, kp, vp, table, inp["ctx_len"], o, s=s, idx_out=idx)  # warm-up
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        api.sas_sparse_decode_paged(desc, q, kp, vp, table, inp["ctx_len"], o, s=s, idx_out=idx)
+    q.copy_(_seeded((B, Hq, 128), 1.0, torch.bfloat16, 96))
+    s.copy_(_seeded((B, Hkv, Tmax // bs), 1.0, torch.float32, 97))
+    graph.replay()
+    torch.cuda.synchronize()
+    o_ref = torch.empty_like(q)
+    idx_ref = torch.empty_like(idx)
+    api.sas_sparse_decode_paged(desc, q, kp, vp, table, inp["ctx_len"], o_ref, s=s, idx_out=idx_ref)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_ref) and torch.equal(o, o_ref)
+    del graph
+    # a missing page: block 5 of sequence 0 points outside the pool
+    table2 = table.clone()
+    table2[0, 5] = kp.shape[0] + 3
+    o_miss = torch.empty_like(q)
+    api.sas_sparse_decode_paged(desc, q, kp, vp, table2, inp["ctx_len"], o_miss)
+    torch.cuda.synchronize()
+    zeroed = dict(inp, q=q)
+    zeroed["k_cache"] = inp["k_cache"].clone()
+    zeroed["v_cache"] = inp["v_cache"].clone()
+    zeroed["k_cache"][0, :, 5 * bs:6 * bs] = 0
+    zeroed["v_cache"][0, :, 5 * bs:6 * bs] = 0
+    ref = _oracle_decode_rows(zeroed, [(0, 0)], bs, K, True)
+    G = Hq // Hkv
+    compare("missing-page o", host(o_miss[0, 0:G]), ref[(0, 0)][0], **BF16_TOL, bf16_out=True)

@@ -64,6 +64,9 @@ lib.sas_sparse_decode.restype = ctypes.c_int
 lib.sas_sparse_decode.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7 + [_sz, _vp]
 lib.sas_sparse_decode_select.restype = ctypes.c_int
 lib.sas_sparse_decode_select.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 5 + [_i32, _vp, _vp, _vp]
+lib.sas_sparse_decode_paged.restype = ctypes.c_int
+lib.sas_sparse_decode_paged.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32,
+                                        _vp, _vp, _vp]
 lib.sas_sparse_decode_noalloc.restype = ctypes.c_int
 lib.sas_sparse_decode_noalloc.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7
 lib.sas_selftest_bounded_wait.restype = ctypes.c_int
@@ -145,6 +148,23 @@ def sas_sparse_decode_select(desc, q, k_cache, v_cache, ctx_len, s, o, idx_out=N
     """Fused decode step: Top-K of s [B, Hkv, s_cols] and the gate-free attention."""
     _check(lib.sas_sparse_decode_select(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(s),
                                         s.shape[-1], _p(o), _p(idx_out), _stream(stream)), "sas_sparse_decode_select")
+
+
+def paged_decode_desc(q, k_pages, block_size: int, top_k: int, max_ctx: int, softmax_scale: float = 0.0) -> DecodeDesc:
+    """Descriptor of a paged-cache decode: k_pages [num_pages, block_size, Hkv, d]."""
+    B, Hq, d = q.shape
+    return DecodeDesc(B, Hq, k_pages.shape[2], d, block_size, top_k, max_ctx, _dtype_code(q), softmax_scale)
+
+
+def sas_sparse_decode_paged(desc, q, k_pages, v_pages, page_table, ctx_len, o, s=None, idx=None, idx_out=None,
+                            stream=None):
+    """Decode step over a paged cache: page_table [B, pages_per_seq] int32 maps a
+    sequence's blocks to pages of k_pages / v_pages [num_pages, block_size, Hkv, d].
+    Blocks from the Top-K of s (fused), from idx, or every block when both are None."""
+    _check(lib.sas_sparse_decode_paged(ctypes.byref(desc), _p(q), _p(k_pages), _p(v_pages), _p(page_table),
+                                       page_table.shape[1], k_pages.shape[0], _p(ctx_len), _p(idx), _p(s),
+                                       0 if s is None else s.shape[-1], _p(o), _p(idx_out), _stream(stream)),
+           "sas_sparse_decode_paged")
 
 
 def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream=None):

@@ -39,7 +39,9 @@ constexpr uint32_t kStage = 2 * kTile;  // K + V
 constexpr int kQLd = 136;              // padded row (bf16 elements) of the q tile in smem
 
 struct DecArgs {
-    CUtensorMap tk, tv;  // caches as {d, Tmax, B*Hkv}, box {64, 64, 1}
+    // contiguous caches as {d, Tmax, B*Hkv}, box {64, 64, 1}; paged pools as
+    // {d, Hkv, num_pages * 64}, box {64, 1, 64}; both land as 64 token rows x 128 B
+    CUtensorMap tk, tv;
     const __nv_bfloat16* q;
     const int32_t* ctx_len;
     const int32_t* idx;  // mode 0
@@ -49,7 +51,36 @@ struct DecArgs {
     int* status;
     int B, Hq, Hkv, Tmax, top_k, s_cols, mode;  // mode 0: given idx, 1: fused selection, 2: dense
     float scale_log2;
+    const int32_t* page_table;  // nullptr: contiguous caches
+    int pages_per_seq, num_pages;
 };
+
+// TMA coordinates of block `blk` of row (b, h): contiguous caches address it by
+// token row within the row's slab; a paged pool by the block's page (a page id
+// outside the pool, or a block past the table, lands outside the tensor map and
+// reads as zeros).
+__device__ __forceinline__ int page_of(const DecArgs& a, int b, int blk) {
+    if (blk >= a.pages_per_seq) return a.num_pages;
+    const int pg = a.page_table[(long)b * a.pages_per_seq + blk];
+    return (pg < 0 || pg >= a.num_pages) ? a.num_pages : pg;
+}
+
+__device__ __forceinline__ void load_block(const DecArgs& a, uint32_t dst, uint32_t bar, int b, int h, int bh,
+                                           int blk, int page) {
+    if (a.page_table) {
+        const int row0 = page * kBS;
+        tma_load_3d(dst, &a.tk, bar, 0, h, row0);
+        tma_load_3d(dst + kHalf, &a.tk, bar, 64, h, row0);
+        tma_load_3d(dst + kTile, &a.tv, bar, 0, h, row0);
+        tma_load_3d(dst + kTile + kHalf, &a.tv, bar, 64, h, row0);
+    } else {
+        const int row0 = blk * kBS;
+        tma_load_3d(dst, &a.tk, bar, 0, row0, bh);
+        tma_load_3d(dst + kHalf, &a.tk, bar, 64, row0, bh);
+        tma_load_3d(dst + kTile, &a.tv, bar, 0, row0, bh);
+        tma_load_3d(dst + kTile + kHalf, &a.tv, bar, 64, row0, bh);
+    }
+}
 
 struct Layout {
     static constexpr uint32_t kRing = 0;
@@ -600,12 +631,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         __syncthreads();
         // the current block (entry 0, on CTA 0) loads while the selection runs
         if (rank == 0 && tid == 0) {
-            const int row0 = Cb * kBS;
             mbar_arrive_expect_tx(full(0), kStage);
-            tma_load_3d(ring, &a.tk, full(0), 0, row0, bh);
-            tma_load_3d(ring + kHalf, &a.tk, full(0), 64, row0, bh);
-            tma_load_3d(ring + kTile, &a.tv, full(0), 0, row0, bh);
-            tma_load_3d(ring + kTile + kHalf, &a.tv, full(0), 64, row0, bh);
+            load_block(a, ring, full(0), b, h, bh, Cb, a.page_table ? page_of(a, b, Cb) : 0);
         }
         const int chunk = (Csel + CL - 1) / CL;
         nsel = use_filter ? row_topk_filter(a, Csel, xs, base, list) : -1;
@@ -624,18 +651,26 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     auto block_of = [&](int e) { return e == 0 ? Cb : (a.mode == 2 ? e - 1 : list[e]); };
 
     if (warp == 0) {
-        if (lane == 0) {
-            const int first = (a.mode == 1 && rank == 0) ? 1 : 0;  // entry 0 already in flight
-            for (int i = first; e0 + i < e1; ++i) {
-                const int st = i % kStages;
-                if (i >= kStages && !mbar_wait(empty(st), (i / kStages - 1) & 1, abort_flag, a.status)) break;
-                const int row0 = block_of(e0 + i) * kBS;
-                const uint32_t dst = ring + st * kStage;
-                mbar_arrive_expect_tx(full(st), kStage);
-                tma_load_3d(dst, &a.tk, full(st), 0, row0, bh);
-                tma_load_3d(dst + kHalf, &a.tk, full(st), 64, row0, bh);
-                tma_load_3d(dst + kTile, &a.tv, full(st), 0, row0, bh);
-                tma_load_3d(dst + kTile + kHalf, &a.tv, full(st), 64, row0, bh);
+        // lane 0 issues the loads; with a paged pool the warp first reads the next 32
+        // entries' page ids together (one round trip), so the table lookups do not
+        // serialise the stream
+        const int first = (a.mode == 1 && rank == 0) ? 1 : 0;  // entry 0 already in flight
+        bool ok = true;
+        for (int i0 = first; ok && e0 + i0 < e1; i0 += 32) {
+            int my_page = 0;
+            if (a.page_table && e0 + i0 + lane < e1) my_page = page_of(a, b, block_of(e0 + i0 + lane));
+            for (int j = 0; j < 32 && e0 + i0 + j < e1; ++j) {
+                const int page = __shfl_sync(0xffffffffu, my_page, j);
+                if (lane == 0) {
+                    const int i = i0 + j, st = i % kStages;
+                    if (i >= kStages && !mbar_wait(empty(st), (i / kStages - 1) & 1, abort_flag, a.status)) ok = false;
+                    if (ok) {
+                        mbar_arrive_expect_tx(full(st), kStage);
+                        load_block(a, ring + st * kStage, full(st), b, h, bh, block_of(e0 + i), page);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
             }
         }
     } else {
@@ -840,9 +875,17 @@ template <int CL>
 cudaError_t launch_cl(const DecArgs& a, int list_cap, cudaStream_t stream) {
     const int G = a.Hq / a.Hkv;
     const size_t smem = Layout::bytes(G, list_cap);
-    cudaError_t err =
-        cudaFuncSetAttribute(decode_cluster_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // raise the kernel's shared-memory limit only when a larger size is first needed
+    // (no attribute call on the steady path, e.g. inside a CUDA graph capture)
+    static size_t smem_set[64] = {};  // per device
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64 || smem > smem_set[dev]) {
+        err = cudaFuncSetAttribute(decode_cluster_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        if (dev >= 0 && dev < 64) smem_set[dev] = smem;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CL, a.B * a.Hkv, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -887,8 +930,16 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_col
     DecArgs a;
     memset(&a, 0, sizeof(a));
     const long rows = (long)p.B * p.Hkv;
-    if (!encode_cache(&a.tk, p.k, p.Tmax, rows) || !encode_cache(&a.tv, p.v, p.Tmax, rows))
+    if (p.page_table) {
+        const long pool_rows = (long)p.num_pages * kBS;
+        if (!encode_tma_rows(&a.tk, p.k, p.Hkv, pool_rows, 1, kBS) || !encode_tma_rows(&a.tv, p.v, p.Hkv, pool_rows, 1, kBS))
+            return cudaErrorInvalidValue;
+        a.page_table = p.page_table;
+        a.pages_per_seq = p.pages_per_seq;
+        a.num_pages = p.num_pages;
+    } else if (!encode_cache(&a.tk, p.k, p.Tmax, rows) || !encode_cache(&a.tv, p.v, p.Tmax, rows)) {
         return cudaErrorInvalidValue;
+    }
     a.q = static_cast<const __nv_bfloat16*>(p.q);
     a.ctx_len = p.ctx_len;
     a.idx = p.idx;

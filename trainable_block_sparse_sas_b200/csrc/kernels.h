@@ -44,6 +44,10 @@ struct DecodeParams {
     int* status;  // device status word (bounded waits)
     int B, Hq, Hkv, d, bs, top_k, Tmax, is_bf16, nsplit, per_split, list_max;
     float scale;
+    // paged cache (tensor-core decode only): k, v are [num_pages, bs, Hkv, d] pools and
+    // page_table[b * pages_per_seq + j] is the page of block j of sequence b
+    const int32_t* page_table;  // nullptr: contiguous [B, Hkv, Tmax, d] caches
+    int pages_per_seq, num_pages;
 };
 
 cudaError_t launch_topk_select(const float* s, int batch, int n_kv_heads, int n_rows, int row_len,

@@ -274,6 +274,34 @@ sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, 
     return from_cuda(launch_decode_sm100(p, s, s_cols, idx_out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+sas_status sas_sparse_decode_paged(const sas_decode_desc* desc, const void* q, const void* k_pages,
+                                   const void* v_pages, const int32_t* page_table, int32_t pages_per_seq,
+                                   int32_t num_pages, const int32_t* ctx_len, const int32_t* idx, const float* s,
+                                   int32_t s_cols, void* o, int32_t* idx_out, sas_stream_t stream) {
+    if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_pages || !v_pages || !page_table || !ctx_len || !o) return SAS_ERR_INVALID_VALUE;
+    if (pages_per_seq <= 0 || num_pages <= 0 || (s && s_cols <= 0)) return SAS_ERR_INVALID_VALUE;
+    if ((long)desc->max_ctx > (long)pages_per_seq * desc->block_size) return SAS_ERR_INVALID_VALUE;
+    if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15u)
+        return SAS_ERR_INVALID_VALUE;
+    DecodeParams p = make_decode(desc);
+    p.q = q;
+    p.k = k_pages;
+    p.v = v_pages;
+    p.ctx_len = ctx_len;
+    p.idx = (s || desc->top_k <= 0) ? nullptr : idx;
+    p.o = o;
+    p.page_table = page_table;
+    p.pages_per_seq = pages_per_seq;
+    p.num_pages = num_pages;
+    if (!supported_decode(desc) || !decode_sm100_supported(p)) return SAS_ERR_UNSUPPORTED;
+    if ((long)num_pages * desc->block_size > 0x7fffffffL) return SAS_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    if (device_info(&di) != cudaSuccess) return SAS_ERR_CUDA;
+    p.status = di.status;
+    return from_cuda(launch_decode_sm100(p, s, s_cols, s ? idx_out : nullptr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sas_status sas_device_status(sas_stream_t stream) {
     DeviceInfo di;
     cudaError_t err = device_info(&di);
