@@ -109,12 +109,23 @@ def train_select(s, top_k: int, full_scope: bool = False):
     return select(s, ncand, top_k, full_scope, idx_cols=top_k)
 
 
+GATES = {"off": 0, "softmax": 1, "sigmoid": 2, "raw": 3}
+
+
+def _gate_code(gate) -> int:
+    """True / "softmax": log g = s - LSE(s) (the method); False / "off": no bias;
+    "sigmoid": log g = log sigmoid(s); "raw": log g = s (the ablated activations)."""
+    if isinstance(gate, (bool, np.bool_)):
+        return 1 if gate else 0
+    return GATES[gate]
+
+
 def _desc(q, k, bs, top_k, full_scope, gate, sigma):
     B, n, Hq, d = q.shape
     Hkv = k.shape[2]
     if sigma is None:
         sigma = 1.0 / np.sqrt(d)
-    return _Desc(B, Hq, Hkv, d, n, bs, top_k, int(full_scope), int(gate), float(sigma))
+    return _Desc(B, Hq, Hkv, d, n, bs, top_k, int(full_scope), _gate_code(gate), float(sigma))
 
 
 def _same_code(*arrs):

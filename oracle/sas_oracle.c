@@ -167,7 +167,11 @@ int oracle_select(const void* s, int s_dt, long nrows, long row_stride, const in
 typedef struct {
     int B, Hq, Hkv, d, n, bs, top_k;
     int full_scope; /* 1: every history block is attended (gated) */
-    int gate;       /* 1: SAS log-gate bias on; 0: plain block-sparse attention */
+    int gate;       /* 0: plain block-sparse attention (no bias);
+                       1: log g = s - LSE(s) (softmax gate, the method);
+                       2: log g = log sigmoid(s); 3: log g = s (raw logit) -- the
+                       gate-activation variants the pages ablate (jaehun.me review,
+                       "Why the Four Design Choices Matter", gate activation) */
     double sigma;   /* softmax scale applied to q.k */
 } orc_desc;
 
@@ -206,8 +210,15 @@ static int gate_row_make(const orc_desc* D, const void* s, int s_dt, int b, int 
     for (int m = 0; m < c; ++m) row[m] = ld(s, s_dt, base + (size_t)m);
     out->lse_s = row_lse(row, c);
     for (int m = 0; m < c; ++m) {
-        out->logg[m] = row[m] - out->lse_s; /* log g_m = s_m - LSE(s) */
-        out->g[m] = exp(out->logg[m]);
+        double lg;
+        if (D->gate == 2)
+            lg = row[m] >= 0.0 ? -log1p(exp(-row[m])) : row[m] - log1p(exp(row[m])); /* log sigmoid(s_m) */
+        else if (D->gate == 3)
+            lg = row[m];                                                             /* raw logit */
+        else
+            lg = row[m] - out->lse_s;                                                /* s_m - LSE(s) */
+        out->logg[m] = lg;
+        out->g[m] = exp(lg);
     }
     out->cnt = select_row(row, c, D->top_k, D->full_scope, out->blocks);
     free(row);
@@ -418,11 +429,18 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
             }
         }
         if (D->gate) {
+            /* chain rule through log g: softmax d(log g_m)/ds_m' = [m = m'] - g_m';
+               log sigmoid: [m = m'] (1 - g_m); raw logit: [m = m'] */
             double tot = 0.0;
             for (int m = 0; m < c; ++m) tot += dlg[m];
             size_t rowoff = (size_t)u * Cq;
             for (int m = 0; m < c; ++m) {
-                ds[rowoff + m] = dlg[m] - gr.g[m] * tot;
+                if (D->gate == 2)
+                    ds[rowoff + m] = dlg[m] * (1.0 - gr.g[m]);
+                else if (D->gate == 3)
+                    ds[rowoff + m] = dlg[m];
+                else
+                    ds[rowoff + m] = dlg[m] - gr.g[m] * tot;
                 if (dlogg) dlogg[rowoff + m] = dlg[m];
             }
         }

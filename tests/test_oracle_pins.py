@@ -142,7 +142,8 @@ def test_select_full_scope_keeps_all_history():
 
 def _dense_masked_torch(q, k, v, s, bs, K, sigma, full_scope=False, gate=True):
     """Explicit dense formulation of Eq. 9 with torch: an n x n bias matrix holding
-    log_softmax(s) on the selected history blocks, 0 on the causal current block and
+    log g (log_softmax(s); or logsigmoid(s) / s for the "sigmoid" / "raw" gate
+    variants) on the selected history blocks, 0 on the causal current block and
     -inf elsewhere; softmax / matmul from torch.  Selection by brute force."""
     B, n, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -157,7 +158,12 @@ def _dense_masked_torch(q, k, v, s, bs, K, sigma, full_scope=False, gate=True):
             for c in range(Cq):
                 bias = torch.full((bs, n), float("-inf"), dtype=torch.float64)
                 if c > 0:
-                    logg = torch.log_softmax(s[b, h, c, :c], dim=0)
+                    if gate == "sigmoid":
+                        logg = torch.nn.functional.logsigmoid(s[b, h, c, :c])
+                    elif gate == "raw":
+                        logg = s[b, h, c, :c]
+                    else:
+                        logg = torch.log_softmax(s[b, h, c, :c], dim=0)
                     row = s[b, h, c, :c].detach().tolist()
                     sel = list(range(c)) if full_scope else _brute_select(row, c, K)
                     for m in sel:
@@ -429,3 +435,73 @@ def test_bf16_half_ulp_allowance():
     x = x.astype(np.float64)
     assert np.all(np.abs(r - x) <= bf16_half_ulp(x) * (1 + 1e-12))
     assert np.max(np.abs(r - x) / bf16_half_ulp(x)) > 0.99
+
+
+@pytest.mark.parametrize("gate", ["sigmoid", "raw"])
+def test_gate_activation_variants_vs_torch_dense_mask(gate):
+    """The ablated gate activations (jaehun.me review, "Why the Four Design Choices
+    Matter", gate activation): log g = log sigmoid(s) or the raw logit s inside the
+    softmax; every output and gradient against torch autograd of the dense form."""
+    rng = np.random.default_rng(31)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 4, 2, 16, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    sigma = 1 / np.sqrt(d)
+    for full in (False, True):
+        out = oracle.attn_bwd(q, k, v, dO, s, bs, K, full_scope=full, gate=gate, sigma=sigma)
+        T = [torch.tensor(x, requires_grad=True) for x in (q, k, v, s)]
+        o_t, lse_t = _dense_masked_torch(*T, bs, K, sigma, full_scope=full, gate=gate)
+        (o_t * torch.tensor(dO)).sum().backward()
+        np.testing.assert_allclose(out["o"], o_t.detach().numpy(), atol=1e-12, rtol=0)
+        np.testing.assert_allclose(out["lse"], lse_t.detach().numpy(), atol=1e-12, rtol=0)
+        for name, t in zip(("dq", "dk", "dv", "ds"), T):
+            np.testing.assert_allclose(out[name], t.grad.numpy(), atol=1e-11, rtol=0, err_msg=(gate, full, name))
+
+
+@pytest.mark.parametrize("gate", ["sigmoid", "raw"])
+def test_gate_activation_variants_finite_differences(gate):
+    rng = np.random.default_rng(32)
+    B, n, Hq, Hkv, d, bs, K = 1, 32, 2, 1, 4, 8, 2
+    q, k, v, _, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    Cq = n // bs
+    s = (rng.permutation(Cq * Cq).reshape(1, 1, Cq, Cq) * 0.05 + rng.uniform(0, 0.01, (1, 1, Cq, Cq))) - 0.3
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K, gate=gate)
+    eps = 1e-6
+
+    def loss(q_, s_):
+        o, _ = oracle.attn_fwd(q_, k, v, s_, bs, K, gate=gate)
+        return float((o * dO).sum())
+
+    for name, arr, pos in (("dq", q, 0), ("ds", s, 1)):
+        for fi in rng.choice(arr.size, size=min(arr.size, 30), replace=False):
+            ix = np.unravel_index(fi, arr.shape)
+            ap, am = arr.copy(), arr.copy()
+            ap[ix] += eps
+            am[ix] -= eps
+            args_p, args_m = [q, s], [q, s]
+            args_p[pos], args_m[pos] = ap, am
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - out[name][ix]) <= 1e-6 * max(1.0, abs(out[name][ix])), (gate, name, ix)
+
+
+def test_gate_variants_reduce_to_known_cases():
+    """The raw-logit gate fed log_softmax(s) is the softmax gate on s (forward); a
+    sigmoid gate saturated at 1 (s = 60) is plain block-sparse attention."""
+    rng = np.random.default_rng(33)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 4, 2, 8, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    Cq = n // bs
+    logg = np.zeros_like(s)
+    for c in range(1, Cq):
+        row = s[..., c, :c]
+        logg[..., c, :c] = row - np.log(np.exp(row - row.max(-1, keepdims=True)).sum(-1, keepdims=True)) \
+            - row.max(-1, keepdims=True)
+    o_soft, lse_soft = oracle.attn_fwd(q, k, v, s, bs, K, gate="softmax")
+    o_raw, lse_raw = oracle.attn_fwd(q, k, v, logg, bs, K, gate="raw")
+    np.testing.assert_allclose(o_raw, o_soft, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse_raw, lse_soft, atol=1e-12, rtol=0)
+    # selection depends only on the order of s: keep it, saturate the sigmoid
+    big = 60.0 + 1e-3 * (s - s.min())
+    o_sig = oracle.attn_bwd(q, k, v, dO, big, bs, K, gate="sigmoid")
+    o_off = oracle.attn_bwd(q, k, v, dO, big, bs, K, gate="off")
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_allclose(o_sig[name], o_off[name], atol=1e-12, rtol=0, err_msg=name)
