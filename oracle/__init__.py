@@ -156,10 +156,12 @@ def attn_fwd(q, k, v, s, bs: int, top_k: int, full_scope: bool = False, gate: bo
 
 
 def attn_bwd(q, k, v, dO, s, bs: int, top_k: int, full_scope: bool = False, gate: bool = True, sigma=None,
-             qmask=None, kvmask=None):
+             qmask=None, kvmask=None, o_store=None):
     """Backward of L = sum(dO * o).  Returns a dict with o, lse, dq, dk, dv, ds, dlogg
     (float64).  qmask / kvmask [B,Hkv,Cq] limit the query blocks (o, lse, dq, ds) and
-    the key blocks (dk, dv) computed."""
+    the key blocks (dk, dv) computed.  o_store="bf16": the backward reads o as a
+    bf16 output tensor holds it (the o of the inner-gate gradient, and of D_i =
+    dO_i . o_i, rounded to bf16); None: the exact o."""
     _same_code(np.asarray(q), np.asarray(k), np.asarray(v), np.asarray(dO))
     qa, code, qp = _in(q)
     ka, _, kp = _in(k)
@@ -177,7 +179,7 @@ def attn_bwd(q, k, v, dO, s, bs: int, top_k: int, full_scope: bool = False, gate
     km = None if kvmask is None else np.ascontiguousarray(kvmask, dtype=np.uint8)
     rc = lib().oracle_attn_bwd(ctypes.byref(D), qp, kp, vp, gp, ctypes.c_int(code), sp, ctypes.c_int(s_code),
                                None if qm is None else _ptr(qm), None if km is None else _ptr(km),
-                               _ptr(out["o"]), _ptr(out["lse"]), _ptr(out["dq"]), _ptr(out["dk"]),
+                               ctypes.c_int({None: 0, "bf16": 1}[o_store]), _ptr(out["o"]), _ptr(out["lse"]), _ptr(out["dq"]), _ptr(out["dk"]),
                                _ptr(out["dv"]), _ptr(out["ds"]), _ptr(out["dlogg"]))
     _check(rc, "attn_bwd")
     return out

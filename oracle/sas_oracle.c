@@ -59,6 +59,18 @@ static double ld(const void* p, int dt, size_t i) {
     return (double)f;
 }
 
+/* x rounded to the nearest bfloat16 value (8 significant bits, ties to even),
+ * kept as a double: the value a bf16 tensor holds after storing x.  Exponents
+ * below bf16's normal range keep its subnormal spacing of 2^-133. */
+static double round_bf16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    frexp(x, &e); /* |x| = f 2^e, f in [0.5, 1) */
+    int sh = e - 8;
+    if (sh < -133) sh = -133;
+    return ldexp(nearbyint(ldexp(x, -sh)), sh);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
@@ -325,7 +337,8 @@ int oracle_attn_fwd(const orc_desc* D, const void* q, const void* k, const void*
 }
 
 /* Backward of L = sum(dO * o) through Eq. 9.
- *   D_i   = dO_i . o_i
+ *   D_i   = dO_i . o_i   (o_i as the forward stored it: rounded to bf16 when
+ *                         o_store == 1, the exact value when o_store == 0)
  *   dS_ij = p_ij (dO_i . v_j - D_i)           (gradient of the logit z_ij)
  *   dq_i  = sigma sum_j dS_ij k_j
  *   dk_j  = sigma sum_{hq in group, i} dS_ij q_i,   dv_j = sum p_ij dO_i
@@ -339,8 +352,8 @@ int oracle_attn_fwd(const orc_desc* D, const void* q, const void* k, const void*
  * block must be in qmask (else ORC_ERR_MISSING_ROW_STATS).
  * dlogg (nullable): [B,Hkv,Cq,Cq] like ds.  Outputs outside the masks are 0. */
 int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void* v, const void* dO, int dt,
-                    const void* s, int s_dt, const unsigned char* qmask, const unsigned char* kvmask, double* o,
-                    double* lse, double* dq, double* dk, double* dv, double* ds, double* dlogg) {
+                    const void* s, int s_dt, const unsigned char* qmask, const unsigned char* kvmask, int o_store,
+                    double* o, double* lse, double* dq, double* dk, double* dv, double* ds, double* dlogg) {
     if (!check_desc(D) || !q || !k || !v || !dO || !s || !o || !lse || !dq || !dk || !dv || !ds) return ORC_ERR_ARG;
     int Cq = D->n / D->bs, G = D->Hq / D->Hkv, d = D->d, MK = max_keys(D);
     long units = (long)D->B * D->Hkv * Cq;
@@ -412,7 +425,8 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
                     for (int e = 0; e < d; ++e) o[ooff + e] += p * ld(v, dt, voff + e);
                 }
                 double Di = 0.0;
-                for (int e = 0; e < d; ++e) Di += ld(dO, dt, ooff + e) * o[ooff + e];
+                for (int e = 0; e < d; ++e)
+                    Di += ld(dO, dt, ooff + e) * (o_store == 1 ? round_bf16(o[ooff + e]) : o[ooff + e]);
                 size_t rix = ((size_t)b * D->Hq + hq) * D->n + i;
                 lse[rix] = L;
                 Drow[rix] = Di;

@@ -315,6 +315,71 @@ def test_inner_gate_gradient_identity_eq5():
                 assert abs(out["dlogg"][0, h, c, m] - want) < 1e-11
 
 
+def _nearest_bf16(x):
+    """Brute force: the nearest of all finite bfloat16 values (ties to the even
+    bit pattern), found by search in the sorted table of every pattern."""
+    pats = np.arange(1 << 16, dtype=np.uint32)
+    f32 = (pats << 16).view(np.float32)
+    keep = np.isfinite(f32) & (pats != 0x8000)  # one zero is enough
+    vals, pats = f32[keep].astype(np.float64), pats[keep]
+    order = np.argsort(vals, kind="stable")
+    vals, pats = vals[order], pats[order]
+    x = np.asarray(x, dtype=np.float64)
+    hi = np.clip(np.searchsorted(vals, x), 1, len(vals) - 1)
+    lo = hi - 1
+    dl, dh = x - vals[lo], vals[hi] - x
+    pick_hi = (dh < dl) | ((dh == dl) & (pats[hi] % 2 == 0))
+    return np.where(pick_hi, vals[hi], vals[lo])
+
+
+def test_nearest_bf16_table_agrees_with_torch_on_float_values():
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal(4096) * np.exp(rng.uniform(-20, 20, 4096))).astype(np.float32)
+    want = torch.tensor(x).to(torch.bfloat16).double().numpy()  # fp32 -> bf16 needs one rounding only
+    np.testing.assert_array_equal(_nearest_bf16(x.astype(np.float64)), want)
+
+
+def test_stored_bf16_output_in_eq5_and_D():
+    """With o_store="bf16" the backward reads o as a bf16 tensor holds it: Eq. 5's
+    d(log g)_m = sum_{i in B_m} p_i do.(v_i - o) with o rounded to the nearest bf16
+    value, and dq / dk through dS_ij = p_ij (dO_i.v_j - dO_i.o_i) with the same o."""
+    rng = np.random.default_rng(22)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 4, 2, 8, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    sigma = 1 / np.sqrt(d)
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K, sigma=sigma, o_store="bf16")
+    exact = oracle.attn_bwd(q, k, v, dO, s, bs, K, sigma=sigma)
+    np.testing.assert_array_equal(out["o"], exact["o"])  # o itself is reported exact
+    o, lse = oracle.attn_fwd(q, k, v, s, bs, K, sigma=sigma)
+    ot = _nearest_bf16(o)
+    assert np.any(ot != o)
+    G, Cq = Hq // Hkv, n // bs
+    dq_want = np.zeros_like(q)
+    for h in range(Hkv):
+        for c in range(Cq):
+            row = s[0, h, c, :c]
+            logg = row - scipy.special.logsumexp(row) if c else row
+            sel = _brute_select(row.tolist(), c, K) if c else []
+            for hq in range(h * G, (h + 1) * G):
+                for i in range(c * bs, (c + 1) * bs):
+                    keys = [(j, logg[m]) for m in sel for j in range(m * bs, (m + 1) * bs)]
+                    keys += [(j, 0.0) for j in range(c * bs, i + 1)]
+                    for j, bias in keys:
+                        p = np.exp(sigma * q[0, i, hq] @ k[0, j, h] + bias - lse[0, hq, i])
+                        dq_want[0, i, hq] += sigma * p * (dO[0, i, hq] @ (v[0, j, h] - ot[0, i, hq])) * k[0, j, h]
+            for m in range(c):
+                want = 0.0
+                if m in sel:
+                    for hq in range(h * G, (h + 1) * G):
+                        for i in range(c * bs, (c + 1) * bs):
+                            for j in range(m * bs, (m + 1) * bs):
+                                p = np.exp(sigma * q[0, i, hq] @ k[0, j, h] + logg[m] - lse[0, hq, i])
+                                want += p * dO[0, i, hq] @ (v[0, j, h] - ot[0, i, hq])
+                assert abs(out["dlogg"][0, h, c, m] - want) < 1e-11
+    np.testing.assert_allclose(out["dq"], dq_want, atol=1e-11, rtol=0)
+    assert np.abs(out["dq"] - exact["dq"]).max() > 1e-6  # the rounding is visible
+
+
 def test_ds_rows_sum_to_zero_and_unselected_share_one_ratio():
     """ds is the softmax VJP, so each row sums to zero; in sparse scope an
     unselected block m gets ds_m = -g_m * sum(dlogg), one common sign and a
