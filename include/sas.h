@@ -58,6 +58,11 @@ typedef enum {
 
 typedef enum { SAS_F32 = 0, SAS_BF16 = 1 } sas_dtype;
 typedef enum { SAS_SCOPE_SPARSE = 0, SAS_SCOPE_FULL = 1 } sas_scope;
+/* Gate activation (placed inside the attention softmax in every case).  SOFTMAX is
+ * the method: log g = s - LSE(s).  SIGMOID (log g = log sigmoid(s)) and RAW (log g
+ * = s) are the activations the pages ablate (jaehun.me review, "Why the Four
+ * Design Choices Matter", gate activation; shibing624 review, Fig. 2(b)). */
+typedef enum { SAS_GATE_SOFTMAX = 0, SAS_GATE_SIGMOID = 1, SAS_GATE_RAW = 2 } sas_gate;
 
 /* Training-shape problem.  Sparse scope attends the Top-K history blocks of each
  * query block plus the current block; full scope attends every history block,
@@ -71,6 +76,7 @@ typedef struct {
     int32_t scope;      /* sas_scope */
     int32_t dtype;      /* sas_dtype of q, k, v, o, dO, dq, dk, dv */
     float softmax_scale;
+    int32_t gate;       /* sas_gate; lse_s is read only by SAS_GATE_SOFTMAX */
 } sas_attn_desc;
 
 /* Decode-shape problem: one new token per sequence; ctx_len[b] counts the cached
@@ -115,11 +121,13 @@ sas_status sas_topk_select(const float* s, int32_t batch, int32_t n_kv_heads, in
  * sas_gated_attn_fwd -- o = softmax(sigma q K_S^T + log g_S) V_S for every query
  *   row (shibing624 review, SAS equation; jaehun.me review, Eq. 9 and the
  *   Kernel implementation paragraph).  Selected history block m of query block c
- *   adds log g_m = s[b,h,c,m] - lse_s[b,h,c] to the logits of its b tokens; the
- *   current block adds 0 and is causally masked; unselected blocks are skipped.
+ *   adds log g_m to the logits of its b tokens, per desc->gate:
+ *   s[b,h,c,m] - lse_s[b,h,c] (SOFTMAX), log sigmoid(s[b,h,c,m]) (SIGMOID) or
+ *   s[b,h,c,m] (RAW); the current block adds 0 and is causally masked;
+ *   unselected blocks are skipped.
  * q, k, v  bf16 or fp32 per desc->dtype; s [B,Hkv,Cq,Cq] fp32; lse_s [B,Hkv,Cq]
- *          fp32 (from sas_topk_select); idx [B,Hkv,Cq,K] (sparse scope; NULL in
- *          full scope).
+ *          fp32 (from sas_topk_select), may be NULL unless the gate is SOFTMAX;
+ *          idx [B,Hkv,Cq,K] (sparse scope; NULL in full scope).
  * o        out, same dtype and layout as q.   lse out [B,Hq,n] fp32.
  * Errors: SAS_ERR_INVALID_VALUE (null pointers, seq_len % block_size != 0,
  *         n_q_heads % n_kv_heads != 0, sizes <= 0, top_k < 0, idx NULL in
@@ -139,10 +147,13 @@ size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc);
  *   gradient of a selected block is the sum of the logit gradients of its tokens
  *   over the query rows and heads sharing the score row (jaehun.me review,
  *   Kernel implementation paragraph; inner-gate gradient, section 4.2.2 Eq. 5),
- *   carried to s through log g = s - LSE(s):
- *     ds[b,h,c,m] = dlogg_m - g_m * sum_{m'<c} dlogg_{m'}  (m < c), 0 (m >= c),
- *   so unselected blocks receive gradient only through the normaliser (jaehun.me
- *   review, "Training scope"; shibing624 review, Fig. 4).
+ *   carried to s through the gate's log g (0 for m >= c):
+ *     SOFTMAX  ds[b,h,c,m] = dlogg_m - g_m * sum_{m'<c} dlogg_{m'}  (m < c),
+ *              so unselected blocks receive gradient only through the
+ *              normaliser (jaehun.me review, "Training scope"; shibing624
+ *              review, Fig. 4);
+ *     SIGMOID  ds = dlogg_m * (1 - g_m);   RAW  ds = dlogg_m
+ *              (dlogg of an unselected block is 0, so so is its ds).
  * o, lse   the forward's outputs.   dq, dk, dv out (dtype of q), ds out fp32.
  * workspace, ws_bytes  caller scratch of at least the queried size.
  * Errors: as sas_gated_attn_fwd, plus SAS_ERR_WORKSPACE_TOO_SMALL.

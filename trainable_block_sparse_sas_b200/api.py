@@ -24,6 +24,8 @@ SAS_OK, SAS_ERR_INVALID_VALUE, SAS_ERR_UNSUPPORTED, SAS_ERR_WORKSPACE_TOO_SMALL,
     SAS_ERR_DEVICE_TIMEOUT = range(6)
 SAS_F32, SAS_BF16 = 0, 1
 SAS_SCOPE_SPARSE, SAS_SCOPE_FULL = 0, 1
+SAS_GATE_SOFTMAX, SAS_GATE_SIGMOID, SAS_GATE_RAW = 0, 1, 2
+GATES = {"softmax": SAS_GATE_SOFTMAX, "sigmoid": SAS_GATE_SIGMOID, "raw": SAS_GATE_RAW}
 
 
 class SasError(RuntimeError):
@@ -37,7 +39,7 @@ class AttnDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("block_size", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("scope", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("gate", ctypes.c_int32)]
 
 
 class DecodeDesc(ctypes.Structure):
@@ -99,10 +101,12 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def attn_desc(q, k, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0) -> AttnDesc:
+def attn_desc(q, k, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0,
+              gate: str = "softmax") -> AttnDesc:
+    """gate: "softmax" (log g = s - LSE(s)), "sigmoid" (log sigmoid(s)) or "raw" (s)."""
     B, n, Hq, d = q.shape
     return AttnDesc(B, Hq, k.shape[2], d, n, block_size, top_k, SAS_SCOPE_FULL if full_scope else SAS_SCOPE_SPARSE,
-                    _dtype_code(q), softmax_scale)
+                    _dtype_code(q), softmax_scale, GATES[gate])
 
 
 def decode_desc(q, k_cache, block_size: int, top_k: int, softmax_scale: float = 0.0) -> DecodeDesc:
@@ -210,9 +214,9 @@ def select_train(s, block_size: int, top_k: int, full_scope: bool = False, strea
 
 class _SASAttention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, s, block_size, top_k, full_scope, softmax_scale):
+    def forward(ctx, q, k, v, s, block_size, top_k, full_scope, softmax_scale, gate):
         q, k, v, s = (t.contiguous() for t in (q, k, v, s))
-        desc = attn_desc(q, k, block_size, top_k, full_scope, softmax_scale)
+        desc = attn_desc(q, k, block_size, top_k, full_scope, softmax_scale, gate)
         idx, lse_s = select_train(s, block_size, top_k, full_scope)
         o = torch.empty_like(q)
         lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=q.device)
@@ -231,14 +235,16 @@ class _SASAttention(torch.autograd.Function):
         ds = torch.empty_like(s)
         ws = workspace(sas_gated_attn_bwd_workspace_size(ctx.desc), q.device)
         sas_gated_attn_bwd(ctx.desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, ws)
-        return dq, dk, dv, ds, None, None, None, None
+        return dq, dk, dv, ds, None, None, None, None, None
 
 
-def sas_attention(q, k, v, s, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0):
+def sas_attention(q, k, v, s, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0,
+                  gate: str = "softmax"):
     """Differentiable SAS gated attention: o = softmax(sigma q K_S^T + log g_S) V_S.
 
-    q [B,n,Hq,d], k/v [B,n,Hkv,d] (bf16 or fp32), s [B,Hkv,n/b,n/b] fp32."""
-    return _SASAttention.apply(q, k, v, s, block_size, top_k, full_scope, softmax_scale)
+    q [B,n,Hq,d], k/v [B,n,Hkv,d] (bf16 or fp32), s [B,Hkv,n/b,n/b] fp32.
+    gate picks log g: "softmax" (the method), "sigmoid" or "raw" (ablations)."""
+    return _SASAttention.apply(q, k, v, s, block_size, top_k, full_scope, softmax_scale, gate)
 
 
 def default_scale(d: int) -> float:

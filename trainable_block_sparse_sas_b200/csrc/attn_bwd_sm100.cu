@@ -11,7 +11,13 @@
 //       -- the block-wise log-gate gradient dlogg[c,m] (jaehun.me review of SAS,
 //       Kernel implementation paragraph; inner-gate gradient, section 4.2.2)
 //     dQ_i += dS_i K                                  (TS MMA, dS read from TMEM)
-//   Epilogue: dq = sigma dQ, and ds[c,m] = dlogg_m - g_m sum(dlogg) for m < c.
+//   Epilogue: dq = sigma dQ, and ds[c,m] from dlogg per the gate.
+//   D enters dS first as dO_i . o_i from the stored (bf16) output; the row's
+//   probability-weighted D, sum_j P_ij dP_ij, differs from it by the row sum of
+//   that dS, delta_i.  With each block's mass M_it = sum_{j in t} P_ij (kept in
+//   the workspace as fp16) the epilogue takes delta_i M_it out of dlogg_t, so
+//   dlogg and ds do not carry the rounding of o (summed over G*64 rows, that
+//   rounding would otherwise reach several 1e-2 when one block holds a row's mass).
 //
 // bwd_dkdv_sm100: one CTA per (batch, kv head, key block m).  It walks the query
 //   blocks that attend m (m itself with the causal mask, and every later block
@@ -21,9 +27,12 @@
 //     dV^T += dO^T P and dK^T += Q^T dS               (SS MMAs, M = head_dim = 128)
 //   Epilogue: dk = sigma dK, dv = dV.
 //
-// D_i = dO_i . o_i is computed by the dq kernel's softmax threads (one row each)
-// and written to the workspace for the dk/dv kernel, which runs after it.
+// D_i is computed by the dq kernel's softmax threads (one row each): dO_i . o_i,
+// then corrected by delta_i; the corrected value is written to the workspace for
+// the dk/dv kernel, which runs after it.
 // Every wait is time-bounded and reports through the device status word.
+#include <cuda_fp16.h>
+
 #include <cstring>
 
 #include "kernels.h"
@@ -48,6 +57,7 @@ struct BwdArgs {
     const int32_t* idx;
     const float* lse;
     float* Dbuf;
+    __half* Mbuf;  // [CTA][list slot][row] block masses of the dq kernel
     const __nv_bfloat16* o;
     const __nv_bfloat16* dO;
     __nv_bfloat16* dq;
@@ -55,7 +65,7 @@ struct BwdArgs {
     __nv_bfloat16* dv;
     float* ds;
     int* status;
-    int B, Hq, Hkv, n, Cq, top_k, full_scope;
+    int B, Hq, Hkv, n, Cq, top_k, full_scope, gate;
     float scale, scale_log2;
 };
 
@@ -149,6 +159,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     const int bh = (int)(blockIdx.x / a.Cq);
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long unit = (long)bh * a.Cq + c;
+    // block masses M_t of the CTA's rows: [list slot][128 * MT rows], fp16
+    __half* mbase = a.Mbuf + (long)blockIdx.x * nl * (128 * MT);
+    float row_delta = 0.f;  // softmax threads: sum_j dS_ij of their row
+    int row_unit = -1;
 
     for (int i = threadIdx.x; i < 8 * nl; i += kDqThreads) part[i] = 0.f;
     if (threadIdx.x == 0) {
@@ -183,7 +197,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         // attended history blocks (ascending) with their log-gate biases, then the
         // current block (bias 0); lanes read the selection in parallel
         const float* srow = a.s + unit * a.Cq;
-        const float lse_c = a.lse_s[unit];
+        const float lse_c = a.gate == 0 ? a.lse_s[unit] : 0.f;
         int cnt = 0;
         const int kk = a.full_scope ? c : min(a.top_k, c);
         const int32_t* row = a.idx + unit * a.top_k;
@@ -195,7 +209,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             if (ok) {
                 const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
                 list[pos] = v;
-                bias2[pos] = (srow[v] - lse_c) * kLog2e;
+                bias2[pos] = gate_log(srow[v], lse_c, a.gate) * kLog2e;
             }
             cnt += __popc(bal);
         }
@@ -318,6 +332,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
             const uint32_t tS = tmem + lane_off + grp * 128, tP = tS + 64;
             const uint32_t tQ = tmem + lane_off + 256 + grp * 128;
+            __half* mrow = mbase + r_unit;  // stride 128 * MT per slot
+            float delta = 0.f;  // sum_j dS_ij of the row (dS taken with the stored-o D)
             bool ok = true;
             for (int t = 0; t < nlist; ++t) {
                 if (!warp_wait(s_full(grp), t & 1, abort_flag, a.status)) {
@@ -329,7 +345,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 const float off = bias2[t] - lse2;
                 const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
                 const uint64_t negD2 = f2_pack(-Drow, -Drow);
-                uint64_t rs2 = 0ull;
+                uint64_t rs2 = 0ull, m2 = 0ull;
                 uint32_t pk[32];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {  // 32 keys at a time
@@ -346,10 +362,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                             if (2 * jj > tok) p0 = 0.f;
                             if (2 * jj + 1 > tok) p1 = 0.f;
                         }
+                        const uint64_t p2 = f2_pack(p0, p1);
                         const uint64_t ds2 = f2_mul(
-                            f2_pack(p0, p1),
-                            f2_add(f2_pack(__uint_as_float(dr[2 * jq]), __uint_as_float(dr[2 * jq + 1])), negD2));
+                            p2, f2_add(f2_pack(__uint_as_float(dr[2 * jq]), __uint_as_float(dr[2 * jq + 1])), negD2));
                         rs2 = f2_add(rs2, ds2);
+                        m2 = f2_add(m2, p2);
                         float d0, d1;
                         f2_unpack(ds2, d0, d1);
                         pk[jj] = pack_bf16x2(d0, d1);
@@ -362,11 +379,18 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ds_ready(grp));
+                delta += rs;
                 if (!cur) {
+                    float ma, mb;
+                    f2_unpack(m2, ma, mb);
+                    mrow[t * (128 * MT)] = __float2half_rn(ma + mb);
                     rs = warp_sum(rs);
                     if (lane == 0) part[t * 8 + wi] = rs;
                 }
             }
+            a.Dbuf[ri] = Drow + delta;  // D for dk / dv
+            row_delta = delta;
+            row_unit = r_unit;
             if (ok && warp_wait(dq_done, 0, abort_flag, a.status)) {
                 tc_fence_after();
                 __nv_bfloat16* drow = a.dq + (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
@@ -392,13 +416,37 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-    // ds row: dlogg over the group's warps, then ds = dlogg - g * sum(dlogg)
+    // the MMAs are drained: the Q tile's smem holds the rows' delta from here on
+    float* delta_sh = reinterpret_cast<float*>(base + L::kQ);
+    if (row_unit >= 0) delta_sh[row_unit] = row_delta;
+    __syncthreads();
+    // dlogg_t: the group's warp partials, less sum_i delta_i M_it (one slot per thread)
     const int nsel = nlist - 1;
     for (int t = threadIdx.x; t < nsel; t += kDqThreads) {
         float acc = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) acc += part[t * 8 + w];
-        part[t * 8] = acc;
+        const uint4* mv = reinterpret_cast<const uint4*>(mbase + (long)t * (128 * MT));
+        const float4* dv4 = reinterpret_cast<const float4*>(delta_sh);
+        float corr = 0.f;
+#pragma unroll 4
+        for (int v = 0; v < 16 * MT; ++v) {  // 8 rows per 16-byte load
+            const uint4 x = mv[v];
+            const float4 d0 = dv4[2 * v], d1 = dv4[2 * v + 1];
+            const float2 m01 = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
+            const float2 m23 = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
+            const float2 m45 = __half22float2(*reinterpret_cast<const __half2*>(&x.z));
+            const float2 m67 = __half22float2(*reinterpret_cast<const __half2*>(&x.w));
+            corr = fmaf(d0.x, m01.x, corr);
+            corr = fmaf(d0.y, m01.y, corr);
+            corr = fmaf(d0.z, m23.x, corr);
+            corr = fmaf(d0.w, m23.y, corr);
+            corr = fmaf(d1.x, m45.x, corr);
+            corr = fmaf(d1.y, m45.y, corr);
+            corr = fmaf(d1.z, m67.x, corr);
+            corr = fmaf(d1.w, m67.y, corr);
+        }
+        part[t * 8] = acc - corr;
     }
     __syncthreads();
     if (warp == 0) {
@@ -411,13 +459,19 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     if (*abort_flag) return;
     const float tot = *tot_sh;
     const float* srow = a.s + unit * a.Cq;
-    const float lse_c = a.lse_s[unit];
     float* dsrow = a.ds + unit * a.Cq;
-    // every block: -g_m * sum(dlogg) (0 from c on); then the attended ones are
-    // overwritten with dlogg_m - g_m * sum(dlogg), g_m from the bias kept in smem
-    for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
+    // every block: ds of a block the row does not attend (dlogg 0: -g_m * sum(dlogg)
+    // for the softmax gate, 0 otherwise; 0 from c on); then the attended ones are
+    // overwritten with their ds, log g_m from the bias kept in smem
+    if (a.gate == 0) {
+        const float lse_c = a.lse_s[unit];
+        for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
+    } else {
+        for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = 0.f;
+    }
     __syncthreads();
-    for (int t = threadIdx.x; t < nsel; t += kDqThreads) dsrow[list[t]] = part[t * 8] - exp2f(bias2[t]) * tot;
+    for (int t = threadIdx.x; t < nsel; t += kDqThreads)
+        dsrow[list[t]] = gate_ds(part[t * 8], bias2[t] * kLn2, tot, a.gate);
 }
 
 // ============================================================================
@@ -623,7 +677,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             const int g = r_unit % G;
             const long ri = ((long)b * a.Hq + h * G + g) * a.n + c * kBS + tok;
             diag = (c == m);
-            const float bias = diag ? 0.f : (a.s[(ubase + c) * a.Cq + m] - a.lse_s[ubase + c]) * kLog2e;
+            const float bias =
+                diag ? 0.f
+                     : gate_log(a.s[(ubase + c) * a.Cq + m], a.gate == 0 ? a.lse_s[ubase + c] : 0.f, a.gate) * kLog2e;
             off = bias - a.lse[ri] * kLog2e;
             dneg = -a.Dbuf[ri];
         };
@@ -744,6 +800,7 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.idx = p.idx;
     a.lse = p.lse_in;
     a.Dbuf = p.Dbuf;
+    a.Mbuf = static_cast<__half*>(p.Mbuf);
     a.o = static_cast<const __nv_bfloat16*>(p.o_in);
     a.dO = static_cast<const __nv_bfloat16*>(p.dO);
     a.dq = static_cast<__nv_bfloat16*>(p.dq);
@@ -758,6 +815,7 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.Cq = p.Cq;
     a.top_k = p.top_k;
     a.full_scope = p.full_scope;
+    a.gate = p.gate;
     a.scale = p.scale;
     a.scale_log2 = p.scale * kLog2e;
     // query-major kernel: the whole query block (64 tokens x G heads) per box
@@ -777,10 +835,20 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-bool bwd_sm100_supported(const TrainParams& p) {
-    if (!p.is_bf16 || p.d != kD || p.bs != kBS) return false;
+static bool bwd_sm100_shape(const TrainParams& p) {
     const int G = p.Hq / p.Hkv;
-    if (G != 2 && G != 4) return false;
+    return p.is_bf16 && p.d == kD && p.bs == kBS && (G == 2 || G == 4);
+}
+
+size_t bwd_sm100_workspace(const TrainParams& p) {
+    // fp16 block masses: every query row once per list slot
+    if (!bwd_sm100_shape(p)) return 0;
+    return sizeof(__half) * (size_t)p.B * p.Hq * p.n * dq_list_max(p.Cq, p.top_k, p.full_scope);
+}
+
+bool bwd_sm100_supported(const TrainParams& p) {
+    if (!bwd_sm100_shape(p) || !p.Mbuf) return false;
+    const int G = p.Hq / p.Hkv;
     const uintptr_t al = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
                          reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.dO) |
                          reinterpret_cast<uintptr_t>(p.dq) | reinterpret_cast<uintptr_t>(p.dk) |

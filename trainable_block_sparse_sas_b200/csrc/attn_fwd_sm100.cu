@@ -58,7 +58,7 @@ struct FwdArgs {
     __nv_bfloat16* o;
     float* lse;
     int* status;
-    int B, Hq, Hkv, n, Cq, top_k, full_scope;
+    int B, Hq, Hkv, n, Cq, top_k, full_scope, gate;
     float scale_log2;
 };
 
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         // attended history blocks (ascending) with their log-gate biases, then the
         // current block (bias 0); lanes read the selection in parallel
         const float* srow = a.s + unit * a.Cq;
-        const float lse_c = a.lse_s[unit];
+        const float lse_c = a.gate == 0 ? a.lse_s[unit] : 0.f;
         int cnt = 0;
         const int kk = a.full_scope ? c : min(a.top_k, c);
         const int32_t* row = a.idx + unit * a.top_k;
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             if (ok) {
                 const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
                 list[pos] = v;
-                bias2[pos] = (srow[v] - lse_c) * kLog2e;
+                bias2[pos] = gate_log(srow[v], lse_c, a.gate) * kLog2e;
             }
             cnt += __popc(bal);
         }
@@ -418,6 +418,7 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.Cq = p.Cq;
     a.top_k = p.top_k;
     a.full_scope = p.full_scope;
+    a.gate = p.gate;
     a.scale_log2 = p.scale * kLog2e;
     const size_t smem = FwdLayout<MT>::bytes(p.Cq);
     cudaError_t err = cudaFuncSetAttribute(fwd_sm100_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
     const long unit = ((long)b * p.Hkv + h) * p.Cq + c;
     const int nsel = build_list(p, unit, c, blocks);
     const float* srow = p.s + unit * p.Cq;
-    const float lse_c = p.lse_s[unit];
+    const float lse_c = p.gate == 0 ? p.lse_s[unit] : 0.f;
 
     load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
     if (tid < BS) {
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
     for (int t = 0; t <= nsel; ++t) {
         const int blk = blocks[t];
         const bool cur = (t == nsel);
-        const float bias = cur ? 0.f : (srow[blk] - lse_c);
+        const float bias = cur ? 0.f : gate_log(srow[blk], lse_c, p.gate);
         __syncthreads();
         load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
         load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
     const long unit = ((long)b * p.Hkv + h) * p.Cq + c;
     const int nsel = build_list(p, unit, c, blocks);
     const float* srow = p.s + unit * p.Cq;
-    const float lse_c = p.lse_s[unit];
+    const float lse_c = p.gate == 0 ? p.lse_s[unit] : 0.f;
     for (int i = tid; i < nsel; i += kThreads) dlg[i] = 0.f;
     const int tr = tid / C::CG, tc = tid % C::CG;
 
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
         for (int t = 0; t <= nsel; ++t) {
             const int blk = blocks[t];
             const bool cur = (t == nsel);
-            const float bias = cur ? 0.f : (srow[blk] - lse_c);
+            const float bias = cur ? 0.f : gate_log(srow[blk], lse_c, p.gate);
             __syncthreads();
             load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
             load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
@@ -328,14 +328,17 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
         }
     }
     __syncthreads();
-    // ds[c, m] = dlogg_m - g_m * sum(dlogg) for m < c, 0 for m >= c
+    // ds[c, m] from dlogg (0 for blocks the row does not attend, and for m >= c):
+    // softmax gate dlogg_m - g_m * sum(dlogg); sigmoid dlogg_m (1 - g_m); raw dlogg_m
     float part = 0.f;
     for (int i = tid; i < nsel; i += kThreads) part += dlg[i];
     const float tot = block_sum(part, red);
     float* dsrow = p.ds + unit * p.Cq;
-    for (int m = tid; m < p.Cq; m += kThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
+    for (int m = tid; m < p.Cq; m += kThreads)
+        dsrow[m] = (m < c && p.gate == 0) ? -expf(srow[m] - lse_c) * tot : 0.f;
     __syncthreads();
-    for (int i = tid; i < nsel; i += kThreads) dsrow[blocks[i]] += dlg[i];
+    for (int i = tid; i < nsel; i += kThreads)
+        dsrow[blocks[i]] = gate_ds(dlg[i], gate_log(srow[blocks[i]], lse_c, p.gate), tot, p.gate);
 }
 
 // is history block m in the (ascending) selection of query block c?
@@ -393,7 +396,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
         for (int li = 0; li < cnt; ++li) {
             const int c = clist[li];
             const bool diag = (c == m);
-            const float bias = diag ? 0.f : (p.s[(ubase + c) * p.Cq + m] - p.lse_s[ubase + c]);
+            const float bias = diag ? 0.f : gate_log(p.s[(ubase + c) * p.Cq + m], p.gate == 0 ? p.lse_s[ubase + c] : 0.f, p.gate);
             for (int g = 0; g < G; ++g) {
                 const int hq = h * G + g;
                 __syncthreads();

@@ -24,6 +24,7 @@ struct TrainParams {
     const float* lse_in;
     const void* dO;
     float* Dbuf;  // [B, Hq, n] row dot(dO, o)
+    void* Mbuf;   // tensor-core backward: fp16 block masses (bwd_sm100_workspace bytes)
     void* dq;
     void* dk;
     void* dv;
@@ -31,7 +32,24 @@ struct TrainParams {
     int* status;  // device status word (bounded waits)
     int B, Hq, Hkv, d, n, bs, Cq, top_k, full_scope, is_bf16;
     float scale;
+    int gate;  // sas_gate: 0 softmax (log g = s - lse_s), 1 log sigmoid(s), 2 raw s
 };
+
+// log g of a history block from its score (natural log): the softmax gate needs
+// the row's LSE; the sigmoid and raw-logit variants do not
+__host__ __device__ __forceinline__ float gate_log(float s, float lse, int gate) {
+    if (gate == 1) return s >= 0.f ? -log1pf(expf(-s)) : s - log1pf(expf(s));
+    if (gate == 2) return s;
+    return s - lse;
+}
+
+// ds of one history block from its dlogg: the raw-logit gate passes it through,
+// the sigmoid gate scales by 1 - g; the softmax gate subtracts g * sum(dlogg)
+__host__ __device__ __forceinline__ float gate_ds(float dlogg, float logg, float tot, int gate) {
+    if (gate == 2) return dlogg;
+    if (gate == 1) return dlogg * (1.f - expf(logg));
+    return dlogg - expf(logg) * tot;
+}
 
 struct DecodeParams {
     const void* q;
@@ -57,6 +75,7 @@ cudaError_t launch_topk_select(const float* s, int batch, int n_kv_heads, int n_
 cudaError_t launch_fwd_simt(const TrainParams& p, cudaStream_t stream);
 bool fwd_sm100_supported(const TrainParams& p);
 bool bwd_sm100_supported(const TrainParams& p);
+size_t bwd_sm100_workspace(const TrainParams& p);
 cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream);
 cudaError_t launch_rowdot(const TrainParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_sm100(const TrainParams& p, cudaStream_t stream);

@@ -69,6 +69,7 @@ bool check_train(const sas_attn_desc* d) {
     if (d->scope != SAS_SCOPE_SPARSE && d->scope != SAS_SCOPE_FULL) return false;
     if (d->dtype != SAS_F32 && d->dtype != SAS_BF16) return false;
     if (!isfinite(d->softmax_scale)) return false;
+    if (d->gate != SAS_GATE_SOFTMAX && d->gate != SAS_GATE_SIGMOID && d->gate != SAS_GATE_RAW) return false;
     return true;
 }
 
@@ -89,6 +90,7 @@ TrainParams make_train(const sas_attn_desc* d) {
     p.Cq = d->seq_len / d->block_size;
     p.top_k = d->top_k;
     p.full_scope = d->scope == SAS_SCOPE_FULL ? 1 : 0;
+    p.gate = d->gate;
     p.is_bf16 = d->dtype == SAS_BF16 ? 1 : 0;
     p.scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->head_dim);
     return p;
@@ -158,7 +160,8 @@ sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const vo
                               const float* s, const float* lse_s, const int32_t* idx, void* o, float* lse,
                               sas_stream_t stream) {
     if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k || !v || !s || !lse_s || !o || !lse) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !s || !o || !lse) return SAS_ERR_INVALID_VALUE;
+    if (!lse_s && desc->gate == SAS_GATE_SOFTMAX) return SAS_ERR_INVALID_VALUE;
     if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
     if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
     DeviceInfo di;
@@ -183,7 +186,7 @@ sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const vo
 size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc) {
     if (!check_train(desc)) return 0;
     TrainParams p = make_train(desc);
-    return (bwd_simt_workspace(p) + 255) & ~(size_t)255;
+    return ((bwd_simt_workspace(p) + 255) & ~(size_t)255) + ((bwd_sm100_workspace(p) + 255) & ~(size_t)255);
 }
 
 sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
@@ -191,7 +194,8 @@ sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const vo
                               const int32_t* idx, void* dq, void* dk, void* dv, float* ds, void* workspace,
                               size_t ws_bytes, sas_stream_t stream) {
     if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k || !v || !o || !lse || !dO || !s || !lse_s || !dq || !dk || !dv || !ds) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !o || !lse || !dO || !s || !dq || !dk || !dv || !ds) return SAS_ERR_INVALID_VALUE;
+    if (!lse_s && desc->gate == SAS_GATE_SOFTMAX) return SAS_ERR_INVALID_VALUE;
     if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
     if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
     const size_t need = sas_gated_attn_bwd_workspace_size(desc);
@@ -217,6 +221,8 @@ sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const vo
     p.dv = dv;
     p.ds = ds;
     p.Dbuf = static_cast<float*>(workspace);
+    if (bwd_sm100_workspace(p) > 0)
+        p.Mbuf = static_cast<uint8_t*>(workspace) + ((bwd_simt_workspace(p) + 255) & ~(size_t)255);
     p.status = di.status;
     if (bwd_sm100_supported(p)) return from_cuda(launch_bwd_sm100(p, reinterpret_cast<cudaStream_t>(stream)));
     return from_cuda(launch_bwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
