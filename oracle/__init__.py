@@ -109,12 +109,14 @@ def train_select(s, top_k: int, full_scope: bool = False):
     return select(s, ncand, top_k, full_scope, idx_cols=top_k)
 
 
-GATES = {"off": 0, "softmax": 1, "sigmoid": 2, "raw": 3}
+GATES = {"off": 0, "softmax": 1, "sigmoid": 2, "raw": 3, "outer": 4, "ste": 5}
 
 
 def _gate_code(gate) -> int:
     """True / "softmax": log g = s - LSE(s) (the method); False / "off": no bias;
-    "sigmoid": log g = log sigmoid(s); "raw": log g = s (the ablated activations)."""
+    "sigmoid": log g = log sigmoid(s); "raw": log g = s (the ablated activations);
+    "outer": g = softmax(s) weights the values outside the attention softmax;
+    "ste": hard Top-K forward, backward straight through to g = softmax(s)."""
     if isinstance(gate, (bool, np.bool_)):
         return 1 if gate else 0
     return GATES[gate]

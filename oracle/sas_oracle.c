@@ -183,7 +183,12 @@ typedef struct {
                        1: log g = s - LSE(s) (softmax gate, the method);
                        2: log g = log sigmoid(s); 3: log g = s (raw logit) -- the
                        gate-activation variants the pages ablate (jaehun.me review,
-                       "Why the Four Design Choices Matter", gate activation) */
+                       "Why the Four Design Choices Matter", gate activation);
+                       4: outer gate, o = sum_j g_{m(j)} p_j v_j with p the gate-free
+                       softmax (gate placement, section 4.2.2 Eq. 5);
+                       5: hard STE gate, the forward a plain hard Top-K and the
+                       backward straight through to g (ranking preservation,
+                       section 4.2.2 Eq. 7).  4 and 5 use g = softmax(s). */
     double sigma;   /* softmax scale applied to q.k */
 } orc_desc;
 
@@ -237,27 +242,35 @@ static int gate_row_make(const orc_desc* D, const void* s, int s_dt, int b, int 
     return out->cnt < 0 ? ORC_ERR_NOMEM : ORC_OK;
 }
 
+/* Does the gate enter the logits (inner gate, Eq. 9)?  Not for the outer gate,
+ * which weights the values, nor for the hard STE gate, whose forward value is 1. */
+static int gate_in_logits(const orc_desc* D) { return D->gate >= 1 && D->gate <= 3; }
+
 /* The logits of query row i (block c) of head hq against its attended keys
  * (Eq. 9): z_j = sigma q_i.k_j + log g_{m(j)} for tokens of selected history
  * blocks, z_j = sigma q_i.k_j for tokens j <= i of the current block.
- * Fills keys[] and z[]; returns the number of keys. */
+ * Fills keys[], z[] and wv[], the weight of each key's value in o (g_{m(j)} for
+ * history keys under the outer gate, else 1); returns the number of keys. */
 static int row_logits(const orc_desc* D, const void* q, const void* k, int dt, int b, int hq, int i,
-                      const gate_row_t* gr, int* keys, double* z, double* biasv) {
+                      const gate_row_t* gr, int* keys, double* z, double* biasv, double* wv) {
     int G = D->Hq / D->Hkv, h = hq / G, c = i / D->bs, d = D->d;
     size_t qoff = (((size_t)b * D->n + i) * D->Hq + hq) * (size_t)d;
     int nk = 0;
     for (int t = 0; t < gr->cnt; ++t) {
         int m = gr->blocks[t];
-        double bias = D->gate ? gr->logg[m] : 0.0;
+        double bias = gate_in_logits(D) ? gr->logg[m] : 0.0;
+        double w = D->gate == 4 ? gr->g[m] : 1.0;
         for (int j = m * D->bs; j < (m + 1) * D->bs; ++j) {
             keys[nk] = j;
             biasv[nk] = bias;
+            wv[nk] = w;
             ++nk;
         }
     }
     for (int j = c * D->bs; j <= i; ++j) {
         keys[nk] = j;
         biasv[nk] = 0.0; /* current block: gate 1, bias log 1 = 0 */
+        wv[nk] = 1.0;
         ++nk;
     }
     for (int t = 0; t < nk; ++t) {
@@ -306,24 +319,26 @@ int oracle_attn_fwd(const orc_desc* D, const void* q, const void* k, const void*
         int* keys = (int*)malloc(sizeof(int) * MK);
         double* z = (double*)malloc(sizeof(double) * MK);
         double* bv = (double*)malloc(sizeof(double) * MK);
-        if (!keys || !z || !bv || gate_row_make(D, s, s_dt, b, h, c, &gr) != ORC_OK) {
+        double* wv = (double*)malloc(sizeof(double) * MK);
+        if (!keys || !z || !bv || !wv || gate_row_make(D, s, s_dt, b, h, c, &gr) != ORC_OK) {
             free(keys);
             free(z);
             free(bv);
+            free(wv);
             err = ORC_ERR_NOMEM;
             continue;
         }
         for (int g = 0; g < G; ++g) {
             int hq = h * G + g;
             for (int i = c * D->bs; i < (c + 1) * D->bs; ++i) {
-                int nk = row_logits(D, q, k, dt, b, hq, i, &gr, keys, z, bv);
+                int nk = row_logits(D, q, k, dt, b, hq, i, &gr, keys, z, bv, wv);
                 double L = lse_of(z, nk);
                 size_t ooff = (((size_t)b * D->n + i) * D->Hq + hq) * (size_t)d;
                 for (int e = 0; e < d; ++e) o[ooff + e] = 0.0;
                 for (int t = 0; t < nk; ++t) {
                     double p = exp(z[t] - L);
                     size_t voff = (((size_t)b * D->n + keys[t]) * D->Hkv + h) * (size_t)d;
-                    for (int e = 0; e < d; ++e) o[ooff + e] += p * ld(v, dt, voff + e);
+                    for (int e = 0; e < d; ++e) o[ooff + e] += p * wv[t] * ld(v, dt, voff + e);
                 }
                 lse[((size_t)b * D->Hq + hq) * D->n + i] = L;
             }
@@ -332,6 +347,7 @@ int oracle_attn_fwd(const orc_desc* D, const void* q, const void* k, const void*
         free(keys);
         free(z);
         free(bv);
+        free(wv);
     }
     return err;
 }
@@ -346,6 +362,12 @@ int oracle_attn_fwd(const orc_desc* D, const void* q, const void* k, const void*
  *                    of block m of dS_ij   (block-wise log-gate gradient)
  *   ds[b,h,c,m] = dlogg_m - g_m sum_{m' < c} dlogg_{m'}  for m < c, else 0
  *                 (chain rule through log g_m = s_m - LSE(s)).
+ * Gate variants: sigmoid / raw change log g and its chain rule.  The outer gate
+ * weights v_j by w_j = g_{m(j)}: dS_ij = p_ij (w_j dO_i.v_j - D_i), dv_j gets
+ * w_j p_ij dO_i, and dlogg_m = g_m sum_{i, j in m} p_ij dO_i.v_j.  The hard STE
+ * gate is plain block-sparse attention forward; its dlogg_m is g_m times
+ * sum_{i, j in m} exp(z_ij - lse_i) (dO_i.v_j - D_i) over every history block,
+ * dropped ones included.
  * Phase 1 runs per query block (b, h, c) selected by qmask and yields dq, ds,
  * dlogg and each row's lse and D.  Phase 2 runs per key block (b, h, m) selected
  * by kvmask and yields dk, dv; every query block that attends a requested key
@@ -366,11 +388,13 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
     if (dlogg) memset(dlogg, 0, (size_t)units * Cq * sizeof(double));
     size_t nrows = (size_t)D->B * D->Hq * D->n;
     double* Drow = (double*)malloc(nrows * sizeof(double));
-    double* logg_all = (double*)malloc((size_t)units * Cq * sizeof(double));
+    double* logg_all = (double*)malloc((size_t)units * Cq * sizeof(double)); /* logit bias of block m in row c */
+    double* w_all = (double*)malloc((size_t)units * Cq * sizeof(double));    /* value weight (outer gate) */
     int* sel_all = (int*)calloc((size_t)units * Cq, sizeof(int)); /* 1 if history block m is attended by c */
     unsigned char* have = (unsigned char*)calloc((size_t)units, 1);
-    if (!Drow || !logg_all || !sel_all || !have) {
+    if (!Drow || !logg_all || !w_all || !sel_all || !have) {
         free(Drow);
+        free(w_all);
         free(logg_all);
         free(sel_all);
         free(have);
@@ -389,7 +413,10 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
             err = ORC_ERR_NOMEM;
             continue;
         }
-        for (int m = 0; m < Cq; ++m) logg_all[u * Cq + m] = (m < c && D->gate) ? gr.logg[m] : 0.0;
+        for (int m = 0; m < Cq; ++m) {
+            logg_all[u * Cq + m] = (m < c && gate_in_logits(D)) ? gr.logg[m] : 0.0;
+            w_all[u * Cq + m] = (m < c && D->gate == 4) ? gr.g[m] : 1.0;
+        }
         for (int t = 0; t < gr.cnt; ++t) sel_all[u * Cq + gr.blocks[t]] = 1;
         gate_row_free(&gr);
     }
@@ -404,25 +431,30 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
         int* keys = (int*)malloc(sizeof(int) * MK);
         double* z = (double*)malloc(sizeof(double) * MK);
         double* bv = (double*)malloc(sizeof(double) * MK);
+        double* wv = (double*)malloc(sizeof(double) * MK);
         double* dlg = (double*)calloc((size_t)Cq, sizeof(double));
-        if (!keys || !z || !bv || !dlg || gate_row_make(D, s, s_dt, b, h, c, &gr) != ORC_OK) {
+        unsigned char* selm = (unsigned char*)calloc((size_t)Cq, 1);
+        if (!keys || !z || !bv || !wv || !dlg || !selm || gate_row_make(D, s, s_dt, b, h, c, &gr) != ORC_OK) {
             free(keys);
             free(z);
             free(bv);
+            free(wv);
             free(dlg);
+            free(selm);
             err = ORC_ERR_NOMEM;
             continue;
         }
+        for (int t = 0; t < gr.cnt; ++t) selm[gr.blocks[t]] = 1;
         for (int g = 0; g < G; ++g) {
             int hq = h * G + g;
             for (int i = c * D->bs; i < (c + 1) * D->bs; ++i) {
-                int nk = row_logits(D, q, k, dt, b, hq, i, &gr, keys, z, bv);
+                int nk = row_logits(D, q, k, dt, b, hq, i, &gr, keys, z, bv, wv);
                 double L = lse_of(z, nk);
                 size_t ooff = (((size_t)b * D->n + i) * D->Hq + hq) * (size_t)d;
                 for (int t = 0; t < nk; ++t) {
                     double p = exp(z[t] - L);
                     size_t voff = (((size_t)b * D->n + keys[t]) * D->Hkv + h) * (size_t)d;
-                    for (int e = 0; e < d; ++e) o[ooff + e] += p * ld(v, dt, voff + e);
+                    for (int e = 0; e < d; ++e) o[ooff + e] += p * wv[t] * ld(v, dt, voff + e);
                 }
                 double Di = 0.0;
                 for (int e = 0; e < d; ++e)
@@ -435,16 +467,39 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
                     size_t kvoff = (((size_t)b * D->n + keys[t]) * D->Hkv + h) * (size_t)d;
                     double dp = 0.0;
                     for (int e = 0; e < d; ++e) dp += ld(dO, dt, ooff + e) * ld(v, dt, kvoff + e);
-                    double dS = p * (dp - Di);
+                    /* o = sum_j w_j p_j v_j: dz_j = p_j (w_j dp_j - D) */
+                    double dS = p * (wv[t] * dp - Di);
                     for (int e = 0; e < d; ++e) dq[ooff + e] += D->sigma * dS * ld(k, dt, kvoff + e);
                     int m = keys[t] / D->bs;
-                    if (m != c) dlg[m] += dS; /* history token: its block's log-gate gradient */
+                    if (m == c) continue;
+                    /* history token: its block's log-gate gradient; the outer gate's
+                       dg_m = sum p_j dp_j (Eq. 5), times g_m for the log */
+                    dlg[m] += D->gate == 4 ? wv[t] * p * dp : dS;
+                }
+                if (D->gate == 5) {
+                    /* hard STE: dropped blocks get d h_m = sum_j exp(z_j - LSE_S) do.(v_j - o)
+                       with z_j = sigma q.k_j, normalised by the selected set's LSE (Eq. 7) */
+                    for (int m = 0; m < c; ++m) {
+                        if (selm[m]) continue;
+                        for (int j = m * D->bs; j < (m + 1) * D->bs; ++j) {
+                            size_t kvoff = (((size_t)b * D->n + j) * D->Hkv + h) * (size_t)d;
+                            double dot = 0.0, dp = 0.0;
+                            for (int e = 0; e < d; ++e) {
+                                dot += ld(q, dt, ooff + e) * ld(k, dt, kvoff + e);
+                                dp += ld(dO, dt, ooff + e) * ld(v, dt, kvoff + e);
+                            }
+                            dlg[m] += exp(D->sigma * dot - L) * (dp - Di);
+                        }
+                    }
                 }
             }
         }
+        if (D->gate == 5) /* straight through: dL/dg = dL/dh; as a log-gate gradient, g dL/dg */
+            for (int m = 0; m < c; ++m) dlg[m] *= gr.g[m];
         if (D->gate) {
             /* chain rule through log g: softmax d(log g_m)/ds_m' = [m = m'] - g_m';
-               log sigmoid: [m = m'] (1 - g_m); raw logit: [m = m'] */
+               log sigmoid: [m = m'] (1 - g_m); raw logit: [m = m'].  The outer and
+               STE gates use g = softmax(s) too, dlg holding g dL/dg */
             double tot = 0.0;
             for (int m = 0; m < c; ++m) tot += dlg[m];
             size_t rowoff = (size_t)u * Cq;
@@ -463,7 +518,9 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
         free(keys);
         free(z);
         free(bv);
+        free(wv);
         free(dlg);
+        free(selm);
     }
     if (err != ORC_OK) goto done;
 
@@ -481,6 +538,7 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
                 continue;
             }
             double bias = (c == m) ? 0.0 : logg_all[(ubase + c) * Cq + m];
+            double w = (c == m) ? 1.0 : w_all[(ubase + c) * Cq + m];
             for (int g = 0; g < G; ++g) {
                 int hq = h * G + g;
                 for (int i = c * D->bs; i < (c + 1) * D->bs; ++i) {
@@ -495,10 +553,10 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
                             dp += ld(dO, dt, qoff + e) * ld(v, dt, kvoff + e);
                         }
                         double p = exp(D->sigma * dot + bias - lse[rix]);
-                        double dS = p * (dp - Drow[rix]);
+                        double dS = p * (w * dp - Drow[rix]);
                         for (int e = 0; e < d; ++e) {
                             dk[kvoff + e] += D->sigma * dS * ld(q, dt, qoff + e);
-                            dv[kvoff + e] += p * ld(dO, dt, qoff + e);
+                            dv[kvoff + e] += p * w * ld(dO, dt, qoff + e);
                         }
                     }
                 }
@@ -507,6 +565,7 @@ int oracle_attn_bwd(const orc_desc* D, const void* q, const void* k, const void*
     }
 done:
     free(Drow);
+    free(w_all);
     free(logg_all);
     free(sel_all);
     free(have);

@@ -522,7 +522,7 @@ def test_gate_activation_variants_vs_torch_dense_mask(gate):
             np.testing.assert_allclose(out[name], t.grad.numpy(), atol=1e-11, rtol=0, err_msg=(gate, full, name))
 
 
-@pytest.mark.parametrize("gate", ["sigmoid", "raw"])
+@pytest.mark.parametrize("gate", ["sigmoid", "raw", "outer"])
 def test_gate_activation_variants_finite_differences(gate):
     rng = np.random.default_rng(32)
     B, n, Hq, Hkv, d, bs, K = 1, 32, 2, 1, 4, 8, 2
@@ -546,6 +546,141 @@ def test_gate_activation_variants_finite_differences(gate):
             args_p[pos], args_m[pos] = ap, am
             fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
             assert abs(fd - out[name][ix]) <= 1e-6 * max(1.0, abs(out[name][ix])), (gate, name, ix)
+
+
+def _dense_torch_outer_or_ste(q, k, v, s, bs, K, sigma, gate, full_scope=False):
+    """Dense torch forms of the two other ablations (shibing624 review, Fig. 2(a)
+    and 2(c); jaehun.me review, section 4.2.2 Eq. 5 and Eq. 7), g = softmax(s):
+    "outer": o = (p * W) V with p the gate-free causal softmax over the selected
+      history blocks and the current block, W[i, j] = g_{m(j)} (1 on the current
+      block);
+    "ste": every history block's keys enter the softmax numerator weighted by
+      h_m = g_m + (hard_m - g_m).detach(), hard_m = 1 for the selected blocks and
+      0 otherwise (1 on the current block): the value is hard Top-K attention and
+      the gradient reaches g as if h were g."""
+    B, n, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    Cq = n // bs
+    outs, lses = [], []
+    for b in range(B):
+        oh, lh = [], []
+        for hq in range(Hq):
+            h = hq // G
+            z = sigma * q[b, :, hq] @ k[b, :, h].T
+            rows_o, rows_l = [], []
+            for c in range(Cq):
+                zc = z[c * bs:(c + 1) * bs]
+                keep = torch.zeros((bs, n), dtype=torch.bool)
+                weight = [torch.ones((), dtype=torch.float64)] * Cq
+                if c > 0:
+                    g = torch.softmax(s[b, h, c, :c], dim=0)
+                    row = s[b, h, c, :c].detach().tolist()
+                    sel = list(range(c)) if full_scope else _brute_select(row, c, K)
+                    for m in range(c):
+                        if gate == "outer":
+                            if m in sel:
+                                keep[:, m * bs:(m + 1) * bs] = True
+                                weight[m] = g[m]
+                        else:
+                            keep[:, m * bs:(m + 1) * bs] = True
+                            hard = 1.0 if m in sel else 0.0
+                            weight[m] = g[m] + (hard - g[m]).detach()
+                keep[:, c * bs:(c + 1) * bs] = torch.ones((bs, bs), dtype=torch.bool).tril()
+                wcol = torch.stack([weight[m] for m in range(Cq) for _ in range(bs)])
+                zm = zc.masked_fill(~keep, float("-inf"))
+                mx = zm.max(dim=-1, keepdim=True).values.detach()
+                e = torch.exp(zm - mx)
+                if gate == "outer":
+                    p = e / e.sum(-1, keepdim=True)
+                    rows_o.append((p * wcol) @ v[b, :, h])
+                    rows_l.append(torch.log(e.sum(-1)) + mx[:, 0])
+                else:
+                    eh = e * wcol
+                    rows_o.append(eh @ v[b, :, h] / eh.sum(-1, keepdim=True))
+                    rows_l.append(torch.log(eh.sum(-1)) + mx[:, 0])
+            oh.append(torch.cat(rows_o, 0))
+            lh.append(torch.cat(rows_l, 0))
+        outs.append(torch.stack(oh, 1))
+        lses.append(torch.stack(lh, 0))
+    return torch.stack(outs, 0), torch.stack(lses, 0)
+
+
+@pytest.mark.parametrize("gate", ["outer", "ste"])
+def test_outer_and_ste_gates_vs_torch_dense(gate):
+    rng = np.random.default_rng(34)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 4, 2, 16, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    sigma = 1 / np.sqrt(d)
+    for full in ((False, True) if gate == "outer" else (False,)):
+        out = oracle.attn_bwd(q, k, v, dO, s, bs, K, full_scope=full, gate=gate, sigma=sigma)
+        T = [torch.tensor(x, requires_grad=True) for x in (q, k, v, s)]
+        o_t, lse_t = _dense_torch_outer_or_ste(*T, bs, K, sigma, gate, full_scope=full)
+        (o_t * torch.tensor(dO)).sum().backward()
+        np.testing.assert_allclose(out["o"], o_t.detach().numpy(), atol=1e-12, rtol=0)
+        np.testing.assert_allclose(out["lse"], lse_t.detach().numpy(), atol=1e-12, rtol=0)
+        for name, t in zip(("dq", "dk", "dv", "ds"), T):
+            np.testing.assert_allclose(out[name], t.grad.numpy(), atol=1e-11, rtol=0, err_msg=(gate, full, name))
+
+
+def test_ste_forward_is_hard_topk_and_outer_gradient_is_eq5():
+    """STE: the forward equals plain block-sparse attention (gate off).  Outer:
+    d(log g)_m = g_m dg_m with dg_m = sum_{i in B_m} p_i do.v_i (Eq. 5, outer),
+    p the gate-free attention probabilities."""
+    rng = np.random.default_rng(35)
+    B, n, Hq, Hkv, d, bs, K = 1, 64, 4, 2, 8, 8, 3
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    sigma = 1 / np.sqrt(d)
+    ste = oracle.attn_bwd(q, k, v, dO, s, bs, K, gate="ste", sigma=sigma)
+    off = oracle.attn_bwd(q, k, v, dO, s, bs, K, gate="off", sigma=sigma)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_allclose(ste[name], off[name], atol=1e-12, rtol=0, err_msg=name)
+    out = oracle.attn_bwd(q, k, v, dO, s, bs, K, gate="outer", sigma=sigma)
+    G, Cq = Hq // Hkv, n // bs
+    for h in range(Hkv):
+        for c in range(1, Cq):
+            row = s[0, h, c, :c]
+            g = np.exp(row - scipy.special.logsumexp(row))
+            sel = _brute_select(row.tolist(), c, K)
+            keys = [j for m in sel for j in range(m * bs, (m + 1) * bs)]
+            for m in range(c):
+                want = 0.0
+                if m in sel:
+                    for hq in range(h * G, (h + 1) * G):
+                        for i in range(c * bs, (c + 1) * bs):
+                            kk = keys + list(range(c * bs, i + 1))
+                            z = np.array([sigma * q[0, i, hq] @ k[0, j, h] for j in kk])
+                            p = np.exp(z - scipy.special.logsumexp(z))
+                            for t, j in enumerate(kk):
+                                if j // bs == m:
+                                    want += p[t] * dO[0, i, hq] @ v[0, j, h]
+                assert abs(out["dlogg"][0, h, c, m] - g[m] * want) < 1e-11, (h, c, m)
+
+
+def test_ste_dropped_block_weights_are_unbounded():
+    """Eq. 7: a dropped block's implied weights exp(z - LSE_S) are normalised by
+    the selected set only.  Scaling the dropped block's keys along the queries'
+    mean direction leaves the forward and the selected block's gradient as they
+    are, while the dropped block's straight-through gradient grows without bound."""
+    rng = np.random.default_rng(36)
+    B, n, Hq, Hkv, d, bs, K = 1, 32, 1, 1, 8, 8, 1
+    q, k, v, s, dO = _rand_train(rng, B, n, Hq, Hkv, d, bs)
+    s[0, 0, 3, :3] = [0.0, 5.0, 0.0]  # query block 3 selects block 1 only
+    qm = q[0, 24:32, 0].mean(0)
+    qm /= np.linalg.norm(qm)
+    g0 = np.exp(s[0, 0, 3, 0] - scipy.special.logsumexp(s[0, 0, 3, :3]))
+    grads, ref = [], None
+    for alpha in (0.0, 8.0, 16.0, 32.0):
+        ka = k.copy()
+        ka[0, 0:8, 0] = qm * alpha  # block 0: dropped by query block 3
+        out = oracle.attn_bwd(q, ka, v, dO, s, bs, K, gate="ste")
+        if ref is None:
+            ref = out
+        np.testing.assert_allclose(out["o"][0, 24:32], ref["o"][0, 24:32], atol=1e-12, rtol=0)
+        assert abs(out["dlogg"][0, 0, 3, 1] - ref["dlogg"][0, 0, 3, 1]) < 1e-12
+        grads.append(abs(out["dlogg"][0, 0, 3, 0]) / g0)
+    assert all(b > a for a, b in zip(grads, grads[1:])), grads
+    assert grads[-1] > 100 * grads[0], grads
 
 
 def test_gate_variants_reduce_to_known_cases():
