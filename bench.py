@@ -273,14 +273,14 @@ def workload_config(w, n_gpus: int) -> dict:
 class TrainRunner:
     """Preallocated buffers and the three ABI calls of one training step."""
 
-    def __init__(self, api, w, inp):
+    def __init__(self, api, w, inp, gate: str = "softmax"):
         import torch
 
         self.api, self.w = api, w
         self.inp = inp
         q, k = inp["q"], inp["k"]
         dev = q.device
-        self.desc = api.attn_desc(q, k, w.bs, w.top_k, w.full_scope)
+        self.desc = api.attn_desc(q, k, w.bs, w.top_k, w.full_scope, gate=gate)
         self.lse_s = torch.empty((w.B, w.Hkv, w.Cq), dtype=torch.float32, device=dev)
         self.idx = None if (w.full_scope or w.top_k == 0) else torch.empty(
             (w.B, w.Hkv, w.Cq, w.top_k), dtype=torch.int32, device=dev)
@@ -501,6 +501,29 @@ def extras(api, args, peaks, peak_kind) -> dict:
     out[w.name] = {"ms_per_step": ms, "tflops": fl["total"] / (ms * 1e-3) / 1e12,
                    "frac_of_bf16_peak": fl["total"] / (ms * 1e-3) / 1e12 / peak}
     del r, inp
+    torch.cuda.empty_cache()
+    # the ablated gates on the headline training workload (same FLOP convention;
+    # the hard STE gate's dq kernel also walks every dropped block, uncounted)
+    w = syn.TRAIN_SPARSE_32K
+    inp = syn.train_inputs(w, device="cuda", seed=1600)
+    fl = train_flops(w)
+    gates = {}
+    for gate in ("sigmoid", "raw", "outer", "ste"):
+        r = TrainRunner(api, w, inp, gate=gate)
+        for _ in range(2):
+            r.step()
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(n):
+            r.step()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / n
+        gates[gate] = {"ms_per_step": ms, "tflops": fl["total"] / (ms * 1e-3) / 1e12}
+        del r
+        torch.cuda.empty_cache()
+    out["gate_variants_" + w.name] = gates
+    del inp
     torch.cuda.empty_cache()
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     for w in (syn.DECODE_128K, syn.DECODE_512K):

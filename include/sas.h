@@ -58,11 +58,25 @@ typedef enum {
 
 typedef enum { SAS_F32 = 0, SAS_BF16 = 1 } sas_dtype;
 typedef enum { SAS_SCOPE_SPARSE = 0, SAS_SCOPE_FULL = 1 } sas_scope;
-/* Gate activation (placed inside the attention softmax in every case).  SOFTMAX is
- * the method: log g = s - LSE(s).  SIGMOID (log g = log sigmoid(s)) and RAW (log g
- * = s) are the activations the pages ablate (jaehun.me review, "Why the Four
- * Design Choices Matter", gate activation; shibing624 review, Fig. 2(b)). */
-typedef enum { SAS_GATE_SOFTMAX = 0, SAS_GATE_SIGMOID = 1, SAS_GATE_RAW = 2 } sas_gate;
+/* Gate.  SOFTMAX is the method: log g = s - LSE(s) added to the logits inside the
+ * attention softmax.  The others are the ablations of the pages' design choices
+ * (jaehun.me review, "Why the Four Design Choices Matter"; shibing624 review,
+ * Fig. 2):
+ *   SIGMOID  log g = log sigmoid(s), inside the softmax   (gate activation)
+ *   RAW      log g = s, inside the softmax                (gate activation)
+ *   OUTER    g = softmax(s) weights each selected block's values outside a
+ *            gate-free softmax: o = sum_j g_m(j) p_j v_j  (gate placement, Eq. 5)
+ *   STE      hard gate: the forward is plain Top-K attention; the backward passes
+ *            dL/dh straight through to g = softmax(s), for every history block,
+ *            a dropped block's keys weighted exp(z - lse) with the forward's lse
+ *            (ranking preservation, Eq. 7). */
+typedef enum {
+    SAS_GATE_SOFTMAX = 0,
+    SAS_GATE_SIGMOID = 1,
+    SAS_GATE_RAW = 2,
+    SAS_GATE_OUTER = 3,
+    SAS_GATE_STE = 4
+} sas_gate;
 
 /* Training-shape problem.  Sparse scope attends the Top-K history blocks of each
  * query block plus the current block; full scope attends every history block,
@@ -76,7 +90,7 @@ typedef struct {
     int32_t scope;      /* sas_scope */
     int32_t dtype;      /* sas_dtype of q, k, v, o, dO, dq, dk, dv */
     float softmax_scale;
-    int32_t gate;       /* sas_gate; lse_s is read only by SAS_GATE_SOFTMAX */
+    int32_t gate;       /* sas_gate; lse_s is read by SOFTMAX, OUTER and STE */
 } sas_attn_desc;
 
 /* Decode-shape problem: one new token per sequence; ctx_len[b] counts the cached
@@ -126,7 +140,7 @@ sas_status sas_topk_select(const float* s, int32_t batch, int32_t n_kv_heads, in
  *   s[b,h,c,m] (RAW); the current block adds 0 and is causally masked;
  *   unselected blocks are skipped.
  * q, k, v  bf16 or fp32 per desc->dtype; s [B,Hkv,Cq,Cq] fp32; lse_s [B,Hkv,Cq]
- *          fp32 (from sas_topk_select), may be NULL unless the gate is SOFTMAX;
+ *          fp32 (from sas_topk_select), may be NULL for the SIGMOID and RAW gates;
  *          idx [B,Hkv,Cq,K] (sparse scope; NULL in full scope).
  * o        out, same dtype and layout as q.   lse out [B,Hq,n] fp32.
  * Errors: SAS_ERR_INVALID_VALUE (null pointers, seq_len % block_size != 0,
@@ -153,7 +167,10 @@ size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc);
  *              normaliser (jaehun.me review, "Training scope"; shibing624
  *              review, Fig. 4);
  *     SIGMOID  ds = dlogg_m * (1 - g_m);   RAW  ds = dlogg_m
- *              (dlogg of an unselected block is 0, so so is its ds).
+ *              (dlogg of an unselected block is 0, so so is its ds);
+ *     OUTER    as SOFTMAX with dlogg_m = g_m sum_{i, j in m} p_ij dO_i.v_j;
+ *     STE      as SOFTMAX with dlogg_m = g_m sum_{i, j in m} exp(z_ij - lse_i)
+ *              (dO_i.v_j - D_i) over every history block m < c.
  * o, lse   the forward's outputs.   dq, dk, dv out (dtype of q), ds out fp32.
  * workspace, ws_bytes  caller scratch of at least the queried size.
  * Errors: as sas_gated_attn_fwd, plus SAS_ERR_WORKSPACE_TOO_SMALL.

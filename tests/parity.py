@@ -51,8 +51,8 @@ def run_train(api, inp: dict, bs: int, top_k: int, full_scope: bool, backward: b
     q, k, v, s, dO = (inp[x] for x in ("q", "k", "v", "s", "dO"))
     desc = api.attn_desc(q, k, bs, top_k, full_scope, gate=gate)
     idx, lse_s = api.select_train(s, bs, top_k, full_scope)
-    if gate != "softmax":
-        lse_s = None  # only the softmax gate reads the score LSE
+    if gate in ("sigmoid", "raw"):
+        lse_s = None  # these gates do not read the score LSE
     o = torch.empty_like(q)
     lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=q.device)
     api.sas_gated_attn_fwd(desc, q, k, v, s, lse_s, idx, o, lse)

@@ -63,7 +63,7 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every case below fails val
 
 @pytest.mark.parametrize("kw,status", [
     (dict(batch=0), 1), (dict(n_q_heads=3), 1), (dict(seq_len=100), 1), (dict(top_k=-1), 1),
-    (dict(scope=7), 1), (dict(dtype=5), 1), (dict(gate=3), 1), (dict(gate=-1), 1), (dict(head_dim=96), 2), (dict(block_size=48, seq_len=96), 2), (dict(block_size=128), 2),
+    (dict(scope=7), 1), (dict(dtype=5), 1), (dict(gate=5), 1), (dict(gate=-1), 1), (dict(head_dim=96), 2), (dict(block_size=48, seq_len=96), 2), (dict(block_size=128), 2),
 ])
 def test_fwd_rejects_bad_descriptors(api, kw, status):
     d = _desc(api, **kw)

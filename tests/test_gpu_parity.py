@@ -155,7 +155,7 @@ def test_unsupported_block_size_is_refused(api):
     assert e.value.status == api.SAS_ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("gate", ["sigmoid", "raw"])
+@pytest.mark.parametrize("gate", ["sigmoid", "raw", "outer", "ste"])
 @pytest.mark.parametrize("dtype,d,bs,K,full", [
     (torch.bfloat16, 128, 64, 3, False),  # tcgen05 kernels, sparse scope
     (torch.bfloat16, 128, 64, 0, True),   # tcgen05 kernels, full scope
@@ -163,11 +163,13 @@ def test_unsupported_block_size_is_refused(api):
     (torch.float32, 128, 32, 3, False),   # SIMT kernels, fp32
 ])
 def test_gate_variants(api, gate, dtype, d, bs, K, full):
-    """log sigmoid(s) and raw-logit gates: outputs and every gradient against the
-    oracle.  Unlike log_softmax these gates are not normalised, so one history
-    block can hold nearly all of a row's mass (raw: weight e^s against the
-    current block's 1); its dlogg then sums D_i over all G*b rows of the query
-    block, which is what the stored-o correction of D is tested on here."""
+    """The ablated gates against the oracle, every output and gradient: log
+    sigmoid(s) and raw-logit gates inside the softmax, the outer gate, and the hard
+    STE gate (whose backward also walks the dropped blocks).  Unlike log_softmax
+    the sigmoid and raw gates are not normalised, so one history block can hold
+    nearly all of a row's mass (raw: weight e^s against the current block's 1);
+    its dlogg then sums D_i over all G*b rows of the query block, which is what
+    the stored-o correction of D is tested on here."""
     B, n, Hq, Hkv = 1, 512, 4, 2
     Cq = n // bs
     qk_std = 1.0 if dtype == torch.bfloat16 else 0.3

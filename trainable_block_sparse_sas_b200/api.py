@@ -24,8 +24,9 @@ SAS_OK, SAS_ERR_INVALID_VALUE, SAS_ERR_UNSUPPORTED, SAS_ERR_WORKSPACE_TOO_SMALL,
     SAS_ERR_DEVICE_TIMEOUT = range(6)
 SAS_F32, SAS_BF16 = 0, 1
 SAS_SCOPE_SPARSE, SAS_SCOPE_FULL = 0, 1
-SAS_GATE_SOFTMAX, SAS_GATE_SIGMOID, SAS_GATE_RAW = 0, 1, 2
-GATES = {"softmax": SAS_GATE_SOFTMAX, "sigmoid": SAS_GATE_SIGMOID, "raw": SAS_GATE_RAW}
+SAS_GATE_SOFTMAX, SAS_GATE_SIGMOID, SAS_GATE_RAW, SAS_GATE_OUTER, SAS_GATE_STE = 0, 1, 2, 3, 4
+GATES = {"softmax": SAS_GATE_SOFTMAX, "sigmoid": SAS_GATE_SIGMOID, "raw": SAS_GATE_RAW, "outer": SAS_GATE_OUTER,
+         "ste": SAS_GATE_STE}
 
 
 class SasError(RuntimeError):
@@ -103,7 +104,9 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 def attn_desc(q, k, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0,
               gate: str = "softmax") -> AttnDesc:
-    """gate: "softmax" (log g = s - LSE(s)), "sigmoid" (log sigmoid(s)) or "raw" (s)."""
+    """gate: "softmax" (log g = s - LSE(s), the method), "sigmoid" (log sigmoid(s)),
+    "raw" (s), "outer" (g = softmax(s) weighting the values outside the softmax) or
+    "ste" (hard Top-K forward, straight-through backward to g = softmax(s))."""
     B, n, Hq, d = q.shape
     return AttnDesc(B, Hq, k.shape[2], d, n, block_size, top_k, SAS_SCOPE_FULL if full_scope else SAS_SCOPE_SPARSE,
                     _dtype_code(q), softmax_scale, GATES[gate])
@@ -243,7 +246,7 @@ def sas_attention(q, k, v, s, block_size: int, top_k: int, full_scope: bool = Fa
     """Differentiable SAS gated attention: o = softmax(sigma q K_S^T + log g_S) V_S.
 
     q [B,n,Hq,d], k/v [B,n,Hkv,d] (bf16 or fp32), s [B,Hkv,n/b,n/b] fp32.
-    gate picks log g: "softmax" (the method), "sigmoid" or "raw" (ablations)."""
+    gate: "softmax" (the method); "sigmoid", "raw", "outer", "ste" (ablations)."""
     return _SASAttention.apply(q, k, v, s, block_size, top_k, full_scope, softmax_scale, gate)
 
 

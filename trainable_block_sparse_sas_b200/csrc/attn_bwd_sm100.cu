@@ -15,7 +15,7 @@
 //   D enters dS first as dO_i . o_i from the stored (bf16) output; the row's
 //   probability-weighted D, sum_j P_ij dP_ij, differs from it by the row sum of
 //   that dS, delta_i.  With each block's mass M_it = sum_{j in t} P_ij (kept in
-//   the workspace as fp16) the epilogue takes delta_i M_it out of dlogg_t, so
+//   the workspace as bf16) the epilogue takes delta_i M_it out of dlogg_t, so
 //   dlogg and ds do not carry the rounding of o (summed over G*64 rows, that
 //   rounding would otherwise reach several 1e-2 when one block holds a row's mass).
 //
@@ -30,8 +30,12 @@
 // D_i is computed by the dq kernel's softmax threads (one row each): dO_i . o_i,
 // then corrected by delta_i; the corrected value is written to the workspace for
 // the dk/dv kernel, which runs after it.
+//
+// Gate variants (the pages' ablations): sigmoid and raw logit change log g; the
+// outer gate scales P by g (dS = P (g dP - D), dV from g P, dlogg = g sum P dP);
+// the hard STE gate has bias 0 and its dq kernel also walks the dropped history
+// blocks, whose dS feeds dlogg but not dQ.
 // Every wait is time-bounded and reports through the device status word.
-#include <cuda_fp16.h>
 
 #include <cstring>
 
@@ -57,7 +61,7 @@ struct BwdArgs {
     const int32_t* idx;
     const float* lse;
     float* Dbuf;
-    __half* Mbuf;  // [CTA][list slot][row] block masses of the dq kernel
+    __nv_bfloat16* Mbuf;  // [CTA][list slot][row] block masses of the dq kernel
     const __nv_bfloat16* o;
     const __nv_bfloat16* dO;
     __nv_bfloat16* dq;
@@ -116,14 +120,17 @@ struct DqLayout {
     static constexpr int kNumBars = 1 + 2 * ST + 2 + 2 + 1 + 1 + 2;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
     static constexpr uint32_t kList = kMisc + 16;
-    // list [nl] ints, biases [nl] floats, then the per-warp dlogg partials [nl][8];
-    // nl = the longest list (attended history blocks + the current block)
-    __host__ __device__ static uint32_t part_off(int nl) { return (kList + 8 * (uint32_t)nl + 15) & ~15u; }
+    // list [nl] ints, biases [nl] floats, value weights [nl] floats, then the
+    // per-warp dlogg partials [nl][8]; nl = the longest list (attended history
+    // blocks + the current block)
+    __host__ __device__ static uint32_t part_off(int nl) { return (kList + 12 * (uint32_t)nl + 15) & ~15u; }
     static size_t bytes(int nl) { return 1024 + part_off(nl) + 32 * (size_t)nl; }
 };
 
-__host__ __device__ inline int dq_list_max(int Cq, int top_k, int full_scope) {
-    return (full_scope ? Cq : min(top_k, Cq)) + 1;
+// the hard STE gate's dq kernel walks every history block (dropped ones give
+// their straight-through gradient only)
+__host__ __device__ inline int dq_list_max(int Cq, int top_k, int full_scope, int gate) {
+    return (full_scope || gate == kGateSte ? Cq : min(top_k, Cq)) + 1;
 }
 
 template <int MT, int ST>
@@ -149,9 +156,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
     float* tot_sh = reinterpret_cast<float*>(base + L::kMisc + 12);
     int* list = reinterpret_cast<int*>(base + L::kList);
-    const int nl = dq_list_max(a.Cq, a.top_k, a.full_scope);
+    const int nl = dq_list_max(a.Cq, a.top_k, a.full_scope, a.gate);
     float* part = reinterpret_cast<float*>(base + L::part_off(nl));  // [slot][8 softmax warps]
     float* bias2 = reinterpret_cast<float*>(base + L::kList + 4 * nl);  // log-gate, log2 units
+    // value weight: g for the outer gate; for the hard STE gate 1 on selected and
+    // 0 on dropped blocks; else 1
+    float* wgt = reinterpret_cast<float*>(base + L::kList + 8 * nl);
+    const bool ste = a.gate == kGateSte;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // head-major order (concurrent CTAs share one KV head in L2), long query blocks first
@@ -159,9 +170,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     const int bh = (int)(blockIdx.x / a.Cq);
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long unit = (long)bh * a.Cq + c;
-    // block masses M_t of the CTA's rows: [list slot][128 * MT rows], fp16
-    __half* mbase = a.Mbuf + (long)blockIdx.x * nl * (128 * MT);
-    float row_delta = 0.f;  // softmax threads: sum_j dS_ij of their row
+    // block masses M_t of the CTA's rows: [list slot][128 * MT rows], bf16
+    __nv_bfloat16* mbase = a.Mbuf + (long)blockIdx.x * nl * (128 * MT);
+    // softmax threads: the coefficient of their row's block masses in the dlogg
+    // correction (delta = sum_j dS_ij; for the outer gate -D)
+    float row_delta = 0.f;
     int row_unit = -1;
 
     for (int i = threadIdx.x; i < 8 * nl; i += kDqThreads) part[i] = 0.f;
@@ -197,25 +210,44 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         // attended history blocks (ascending) with their log-gate biases, then the
         // current block (bias 0); lanes read the selection in parallel
         const float* srow = a.s + unit * a.Cq;
-        const float lse_c = a.gate == 0 ? a.lse_s[unit] : 0.f;
+        const float lse_c = gate_softmax_family(a.gate) ? a.lse_s[unit] : 0.f;
         int cnt = 0;
         const int kk = a.full_scope ? c : min(a.top_k, c);
         const int32_t* row = a.idx + unit * a.top_k;
-        for (int base_i = 0; base_i < kk; base_i += 32) {
-            const int i = base_i + lane;
-            const int v = i < kk ? (a.full_scope ? i : row[i]) : -1;
-            const bool ok = v >= 0 && v < c;
-            const unsigned bal = __ballot_sync(0xffffffffu, ok);
-            if (ok) {
-                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-                list[pos] = v;
-                bias2[pos] = gate_log(srow[v], lse_c, a.gate) * kLog2e;
+        if (ste && !a.full_scope) {
+            // every history block in order, flagged by the selection
+            for (int m = lane; m < c; m += 32) {
+                list[m] = m;
+                bias2[m] = 0.f;
+                wgt[m] = 0.f;
             }
-            cnt += __popc(bal);
+            __syncwarp();
+            for (int i = lane; i < kk; i += 32) {
+                const int v = row[i];
+                if (v >= 0 && v < c) wgt[v] = 1.f;
+            }
+            __syncwarp();
+            cnt = c;
+        } else {
+            for (int base_i = 0; base_i < kk; base_i += 32) {
+                const int i = base_i + lane;
+                const int v = i < kk ? (a.full_scope ? i : row[i]) : -1;
+                const bool ok = v >= 0 && v < c;
+                const unsigned bal = __ballot_sync(0xffffffffu, ok);
+                if (ok) {
+                    const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                    const float lg = gate_log(srow[v], lse_c, a.gate);
+                    list[pos] = v;
+                    bias2[pos] = gate_in_logits(a.gate) ? lg * kLog2e : 0.f;
+                    wgt[pos] = a.gate == kGateOuter ? expf(lg) : 1.f;
+                }
+                cnt += __popc(bal);
+            }
         }
         if (lane == 0) {
             list[cnt] = c;
             bias2[cnt] = 0.f;
+            wgt[cnt] = 1.f;
             *list_count = cnt + 1;
         }
     }
@@ -332,7 +364,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
             const uint32_t tS = tmem + lane_off + grp * 128, tP = tS + 64;
             const uint32_t tQ = tmem + lane_off + 256 + grp * 128;
-            __half* mrow = mbase + r_unit;  // stride 128 * MT per slot
+            __nv_bfloat16* mrow = mbase + r_unit;  // stride 128 * MT per slot
             float delta = 0.f;  // sum_j dS_ij of the row (dS taken with the stored-o D)
             bool ok = true;
             for (int t = 0; t < nlist; ++t) {
@@ -345,6 +377,12 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 const float off = bias2[t] - lse2;
                 const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
                 const uint64_t negD2 = f2_pack(-Drow, -Drow);
+                // dS = P (w dP - D); a dropped block of the STE gate takes w = 1 for its
+                // straight-through gradient and gives dQ nothing
+                const float wt = wgt[t];
+                const bool dropped = ste && wt == 0.f;
+                const float wd = dropped ? 1.f : wt;
+                const uint64_t w2 = f2_pack(wd, wd);
                 uint64_t rs2 = 0ull, m2 = 0ull;
                 uint32_t pk[32];
 #pragma unroll
@@ -364,7 +402,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                         }
                         const uint64_t p2 = f2_pack(p0, p1);
                         const uint64_t ds2 = f2_mul(
-                            p2, f2_add(f2_pack(__uint_as_float(dr[2 * jq]), __uint_as_float(dr[2 * jq + 1])), negD2));
+                            p2, f2_fma(f2_pack(__uint_as_float(dr[2 * jq]), __uint_as_float(dr[2 * jq + 1])), w2, negD2));
                         rs2 = f2_add(rs2, ds2);
                         m2 = f2_add(m2, p2);
                         float d0, d1;
@@ -375,21 +413,27 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 float rsa, rsb;
                 f2_unpack(rs2, rsa, rsb);
                 float rs = rsa + rsb;
+                if (dropped) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) pk[jj] = 0u;
+                }
                 tmem_st32(tP, pk);  // dS over dP, for dQ = dS K
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(ds_ready(grp));
-                delta += rs;
+                if (!dropped) delta += rs;  // the row's P sum to 1 over the attended keys
                 if (!cur) {
                     float ma, mb;
                     f2_unpack(m2, ma, mb);
-                    mrow[t * (128 * MT)] = __float2half_rn(ma + mb);
+                    mrow[t * (128 * MT)] = __float2bfloat16_rn(ma + mb);
                     rs = warp_sum(rs);
                     if (lane == 0) part[t * 8 + wi] = rs;
                 }
             }
             a.Dbuf[ri] = Drow + delta;  // D for dk / dv
-            row_delta = delta;
+            // dlogg_t = sum_i (dS-sum_it - coef_i M_it): the exact-D correction, or
+            // for the outer gate g_t sum P dP = dS-sum + D M
+            row_delta = a.gate == kGateOuter ? -Drow : delta;
             row_unit = r_unit;
             if (ok && warp_wait(dq_done, 0, abort_flag, a.status)) {
                 tc_fence_after();
@@ -433,10 +477,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         for (int v = 0; v < 16 * MT; ++v) {  // 8 rows per 16-byte load
             const uint4 x = mv[v];
             const float4 d0 = dv4[2 * v], d1 = dv4[2 * v + 1];
-            const float2 m01 = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
-            const float2 m23 = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
-            const float2 m45 = __half22float2(*reinterpret_cast<const __half2*>(&x.z));
-            const float2 m67 = __half22float2(*reinterpret_cast<const __half2*>(&x.w));
+            const float2 m01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
+            const float2 m23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
+            const float2 m45 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.z));
+            const float2 m67 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.w));
             corr = fmaf(d0.x, m01.x, corr);
             corr = fmaf(d0.y, m01.y, corr);
             corr = fmaf(d0.z, m23.x, corr);
@@ -446,7 +490,10 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             corr = fmaf(d1.z, m67.x, corr);
             corr = fmaf(d1.w, m67.y, corr);
         }
-        part[t * 8] = acc - corr;
+        float dl = acc - corr;
+        // STE: the straight-through dL/dg of the block, as a log-gate gradient g dL/dg
+        if (ste) dl *= expf(a.s[unit * a.Cq + list[t]] - a.lse_s[unit]);
+        part[t * 8] = dl;
     }
     __syncthreads();
     if (warp == 0) {
@@ -463,15 +510,17 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     // every block: ds of a block the row does not attend (dlogg 0: -g_m * sum(dlogg)
     // for the softmax gate, 0 otherwise; 0 from c on); then the attended ones are
     // overwritten with their ds, log g_m from the bias kept in smem
-    if (a.gate == 0) {
-        const float lse_c = a.lse_s[unit];
+    const float lse_c = gate_softmax_family(a.gate) ? a.lse_s[unit] : 0.f;
+    if (gate_softmax_family(a.gate)) {
         for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
     } else {
         for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = 0.f;
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < nsel; t += kDqThreads)
-        dsrow[list[t]] = gate_ds(part[t * 8], bias2[t] * kLn2, tot, a.gate);
+    for (int t = threadIdx.x; t < nsel; t += kDqThreads) {
+        const float lg = gate_in_logits(a.gate) ? bias2[t] * kLn2 : gate_log(srow[list[t]], lse_c, a.gate);
+        dsrow[list[t]] = gate_ds(part[t * 8], lg, tot, a.gate);
+    }
 }
 
 // ============================================================================
@@ -515,7 +564,9 @@ __device__ __forceinline__ bool holds(const BwdArgs& a, long uc, int c, int m) {
     return false;
 }
 
-template <int MT>
+// kOuter: the outer gate, P and dP scaled by g of the (query block, key block)
+// pair: dV += (g P)^T dO, dS = P (g dP - D)
+template <int MT, bool kOuter>
 __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __grid_constant__ BwdArgs a) {
     using L = DkvLayout;
     constexpr int G = 2 * MT;
@@ -670,36 +721,38 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
         bool ok = true;
         // per-item row statistics, fetched one item ahead
-        auto fetch = [&](int j, float& off, float& dneg, int& tok, bool& diag) {
+        auto fetch = [&](int j, float& off, float& dneg, float& w, int& tok, bool& diag) {
             const int c = list[j / MT], i = j % MT;
             const int r_unit = 128 * i + row;
             tok = r_unit / G;
             const int g = r_unit % G;
             const long ri = ((long)b * a.Hq + h * G + g) * a.n + c * kBS + tok;
             diag = (c == m);
-            const float bias =
+            const float lg =
                 diag ? 0.f
-                     : gate_log(a.s[(ubase + c) * a.Cq + m], a.gate == 0 ? a.lse_s[ubase + c] : 0.f, a.gate) * kLog2e;
-            off = bias - a.lse[ri] * kLog2e;
+                     : gate_log(a.s[(ubase + c) * a.Cq + m],
+                                gate_softmax_family(a.gate) ? a.lse_s[ubase + c] : 0.f, a.gate);
+            off = (gate_in_logits(a.gate) ? lg * kLog2e : 0.f) - a.lse[ri] * kLog2e;
             dneg = -a.Dbuf[ri];
+            w = (kOuter && !diag) ? expf(lg) : 1.f;
         };
-        float off = 0.f, dneg = 0.f;
+        float off = 0.f, dneg = 0.f, w = 1.f;
         int tok = 0;
         bool diag = false;
-        if (nitems > 0) fetch(0, off, dneg, tok, diag);
+        if (nitems > 0) fetch(0, off, dneg, w, tok, diag);
         for (int j = 0; j < nitems; ++j) {
             const int buf = j & 1;
-            float n_off = 0.f, n_dneg = 0.f;
+            float n_off = 0.f, n_dneg = 0.f, n_w = 1.f;
             int n_tok = 0;
             bool n_diag = false;
-            if (j + 1 < nitems) fetch(j + 1, n_off, n_dneg, n_tok, n_diag);
+            if (j + 1 < nitems) fetch(j + 1, n_off, n_dneg, n_w, n_tok, n_diag);
             if (!warp_wait(s_full(buf), (j >> 1) & 1, abort_flag, a.status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
-            const uint64_t dn2 = f2_pack(dneg, dneg);
+            const uint64_t dn2 = f2_pack(dneg, dneg), w2 = f2_pack(w, w);
             uint32_t pp[16], dd[16];
             {
                 uint32_t sr[32], dr[32];
@@ -720,14 +773,15 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                     }
                     float d0, d1;
                     f2_unpack(f2_mul(f2_pack(p0, p1),
-                                     f2_add(f2_pack(__uint_as_float(dr[2 * jj]), __uint_as_float(dr[2 * jj + 1])), dn2)),
+                                     f2_fma(f2_pack(__uint_as_float(dr[2 * jj]), __uint_as_float(dr[2 * jj + 1])), w2, dn2)),
                               d0, d1);
-                    pp[jj] = pack_bf16x2(p0, p1);
+                    pp[jj] = kOuter ? pack_bf16x2(p0 * w, p1 * w) : pack_bf16x2(p0, p1);
                     dd[jj] = pack_bf16x2(d0, d1);
                 }
             }
             off = n_off;
             dneg = n_dneg;
+            w = n_w;
             tok = n_tok;
             diag = n_diag;
             tc_fence_before();
@@ -800,7 +854,7 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.idx = p.idx;
     a.lse = p.lse_in;
     a.Dbuf = p.Dbuf;
-    a.Mbuf = static_cast<__half*>(p.Mbuf);
+    a.Mbuf = static_cast<__nv_bfloat16*>(p.Mbuf);
     a.o = static_cast<const __nv_bfloat16*>(p.o_in);
     a.dO = static_cast<const __nv_bfloat16*>(p.dO);
     a.dq = static_cast<__nv_bfloat16*>(p.dq);
@@ -822,7 +876,7 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, kBS) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, kBS) ||
         !encode_tma_rows(&a.tk, p.k, p.Hkv, rows, 1, kBS) || !encode_tma_rows(&a.tv, p.v, p.Hkv, rows, 1, kBS))
         return cudaErrorInvalidValue;
-    const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope);
+    const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
     cudaError_t err = DqLayout<MT, 3>::bytes(nl) <= kSmemLimit
                           ? launch_kernel(bwd_dq_sm100_kernel<MT, 3>, grid, kDqThreads, DqLayout<MT, 3>::bytes(nl), a, stream)
                           : launch_kernel(bwd_dq_sm100_kernel<MT, 2>, grid, kDqThreads, DqLayout<MT, 2>::bytes(nl), a, stream);
@@ -830,7 +884,9 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     // key-major kernel: 128-row items (128/G tokens x G heads) per box
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, 128 / G) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, 128 / G))
         return cudaErrorInvalidValue;
-    return launch_kernel(bwd_dkdv_sm100_kernel<MT>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream);
+    return p.gate == kGateOuter
+               ? launch_kernel(bwd_dkdv_sm100_kernel<MT, true>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream)
+               : launch_kernel(bwd_dkdv_sm100_kernel<MT, false>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream);
 }
 
 }  // namespace
@@ -841,9 +897,9 @@ static bool bwd_sm100_shape(const TrainParams& p) {
 }
 
 size_t bwd_sm100_workspace(const TrainParams& p) {
-    // fp16 block masses: every query row once per list slot
+    // bf16 block masses: every query row once per list slot
     if (!bwd_sm100_shape(p)) return 0;
-    return sizeof(__half) * (size_t)p.B * p.Hq * p.n * dq_list_max(p.Cq, p.top_k, p.full_scope);
+    return sizeof(__nv_bfloat16) * (size_t)p.B * p.Hq * p.n * dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
 }
 
 bool bwd_sm100_supported(const TrainParams& p) {
@@ -855,7 +911,7 @@ bool bwd_sm100_supported(const TrainParams& p) {
                          reinterpret_cast<uintptr_t>(p.dv) | reinterpret_cast<uintptr_t>(p.o_in);
     if (al & 15u) return false;
     if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq > 0x7fffffffL) return false;
-    const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope);
+    const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
     return DqLayout<2, 2>::bytes(nl) <= kSmemLimit && DkvLayout::bytes(p.Cq) <= kSmemLimit;
 }
 

@@ -74,8 +74,8 @@ struct FwdLayout {
     // PV, so no waiter can fall two phases behind.
     static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4 + 4 + 1 + 1;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;  // tmem base, abort flag, list count
-    static constexpr uint32_t kList = kMisc + 16;  // [Cq + 1] ints, then [Cq + 1] biases
-    static size_t bytes(int Cq) { return 1024 + kList + 8 * (size_t)(Cq + 1); }
+    static constexpr uint32_t kList = kMisc + 16;  // [Cq + 1] ints, [Cq + 1] biases, [Cq + 1] value weights
+    static size_t bytes(int Cq) { return 1024 + kList + 12 * (size_t)(Cq + 1); }
 };
 
 __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
@@ -90,7 +90,9 @@ __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]
                  : "memory");
 }
 
-template <int MT>
+// kOuter: the outer gate, g scaling each history block's P before P.V (the row
+// sum l stays that of the gate-free P)
+template <int MT, bool kOuter>
 __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_constant__ FwdArgs a) {
     using L = FwdLayout<MT>;
     constexpr int G = L::G;
@@ -114,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     int* list_count = reinterpret_cast<int*>(base + L::kMisc + 8);
     int* list = reinterpret_cast<int*>(base + L::kList);
     float* bias2 = reinterpret_cast<float*>(base + L::kList + 4 * (a.Cq + 1));  // log-gate, log2 units
+    float* wgt = reinterpret_cast<float*>(base + L::kList + 8 * (a.Cq + 1));    // outer gate: g
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // head-major order: concurrent CTAs share one KV head's K/V in L2; within a
@@ -152,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         // attended history blocks (ascending) with their log-gate biases, then the
         // current block (bias 0); lanes read the selection in parallel
         const float* srow = a.s + unit * a.Cq;
-        const float lse_c = a.gate == 0 ? a.lse_s[unit] : 0.f;
+        const float lse_c = gate_softmax_family(a.gate) ? a.lse_s[unit] : 0.f;
         int cnt = 0;
         const int kk = a.full_scope ? c : min(a.top_k, c);
         const int32_t* row = a.idx + unit * a.top_k;
@@ -163,14 +166,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             const unsigned bal = __ballot_sync(0xffffffffu, ok);
             if (ok) {
                 const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                const float lg = gate_log(srow[v], lse_c, a.gate);
                 list[pos] = v;
-                bias2[pos] = gate_log(srow[v], lse_c, a.gate) * kLog2e;
+                bias2[pos] = gate_in_logits(a.gate) ? lg * kLog2e : 0.f;
+                if (kOuter) wgt[pos] = expf(lg);
             }
             cnt += __popc(bal);
         }
         if (lane == 0) {
             list[cnt] = c;
             bias2[cnt] = 0.f;
+            if (kOuter) wgt[cnt] = 1.f;
             *list_count = cnt + 1;
         }
     }
@@ -311,6 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                 // pairs over the first 32 columns of this buffer
                 const float off = bias2[t] - m_used;
                 const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
+                const float w = kOuter ? wgt[t] : 1.f;
                 uint64_t rs2 = 0ull;
                 uint32_t pk[32];
 #pragma unroll
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                         if (2 * jj + 1 > tok) p1 = 0.f;
                     }
                     rs2 = f2_add(rs2, f2_pack(p0, p1));
-                    pk[jj] = pack_bf16x2(p0, p1);
+                    pk[jj] = kOuter ? pack_bf16x2(p0 * w, p1 * w) : pack_bf16x2(p0, p1);
                 }
                 tmem_st32(tS + bf * 64, pk);
                 float rsa, rsb;
@@ -421,10 +428,11 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.gate = p.gate;
     a.scale_log2 = p.scale * kLog2e;
     const size_t smem = FwdLayout<MT>::bytes(p.Cq);
-    cudaError_t err = cudaFuncSetAttribute(fwd_sm100_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = p.gate == kGateOuter ? fwd_sm100_kernel<MT, true> : fwd_sm100_kernel<MT, false>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const long grid = (long)p.B * p.Hkv * p.Cq;
-    fwd_sm100_kernel<MT><<<(unsigned)grid, kThreads, smem, stream>>>(a);
+    kern<<<(unsigned)grid, kThreads, smem, stream>>>(a);
     err = cudaGetLastError();
     if (err == cudaSuccess) count_launch();
     return err;

@@ -83,6 +83,25 @@ __device__ __forceinline__ int build_list(const TrainParams& p, long unit, int c
     return cnt_sh;
 }
 
+// Every history block of query block c in order, for the hard STE gate's
+// backward: blocks[m] = m when the selection holds m, -(m + 1) when it dropped m;
+// the current block at blocks[c].  Returns c.
+__device__ __forceinline__ int build_list_all(const TrainParams& p, long unit, int c, int* blocks) {
+    for (int i = threadIdx.x; i < c; i += kThreads) blocks[i] = p.full_scope ? i : -(i + 1);
+    if (threadIdx.x == 0) blocks[c] = c;
+    __syncthreads();
+    if (!p.full_scope && threadIdx.x == 0) {
+        const int kk = min(p.top_k, c);
+        const int32_t* row = p.idx + unit * p.top_k;
+        for (int i = 0; i < kk; ++i) {
+            const int v = row[i];
+            if (v >= 0 && v < c) blocks[v] = v;
+        }
+    }
+    __syncthreads();
+    return c;
+}
+
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
     using C = Cfg<D, BS>;
@@ -104,7 +123,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
     const long unit = ((long)b * p.Hkv + h) * p.Cq + c;
     const int nsel = build_list(p, unit, c, blocks);
     const float* srow = p.s + unit * p.Cq;
-    const float lse_c = p.gate == 0 ? p.lse_s[unit] : 0.f;
+    const float lse_c = gate_softmax_family(p.gate) ? p.lse_s[unit] : 0.f;
 
     load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
     if (tid < BS) {
@@ -121,7 +140,9 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
     for (int t = 0; t <= nsel; ++t) {
         const int blk = blocks[t];
         const bool cur = (t == nsel);
-        const float bias = cur ? 0.f : gate_log(srow[blk], lse_c, p.gate);
+        const float lg = cur ? 0.f : gate_log(srow[blk], lse_c, p.gate);
+        const float bias = gate_in_logits(p.gate) ? lg : 0.f;
+        const float w = (p.gate == kGateOuter && !cur) ? expf(lg) : 1.f;  // outer gate: g weights V
         __syncthreads();
         load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
         load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
@@ -176,7 +197,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
         for (int j = 0; j < BS; ++j) {
             float pv[4];
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) pv[ii] = Ss[(tr + C::RG * ii) * C::LDS + j];
+            for (int ii = 0; ii < 4; ++ii) pv[ii] = Ss[(tr + C::RG * ii) * C::LDS + j] * w;
 #pragma unroll
             for (int ee = 0; ee < C::COLS; ++ee) {
                 const float vv = Vs[j * C::LD + tc + C::CG * ee];
@@ -236,9 +257,10 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
     const int b = (int)(blockIdx.x / ((long)p.Cq * p.Hkv));
     const int G = p.Hq / p.Hkv;
     const long unit = ((long)b * p.Hkv + h) * p.Cq + c;
-    const int nsel = build_list(p, unit, c, blocks);
+    const bool ste = p.gate == kGateSte;
+    const int nsel = ste ? build_list_all(p, unit, c, blocks) : build_list(p, unit, c, blocks);
     const float* srow = p.s + unit * p.Cq;
-    const float lse_c = p.gate == 0 ? p.lse_s[unit] : 0.f;
+    const float lse_c = gate_softmax_family(p.gate) ? p.lse_s[unit] : 0.f;
     for (int i = tid; i < nsel; i += kThreads) dlg[i] = 0.f;
     const int tr = tid / C::CG, tc = tid % C::CG;
 
@@ -259,9 +281,13 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
             for (int ee = 0; ee < C::COLS; ++ee) acc[ii][ee] = 0.f;
 
         for (int t = 0; t <= nsel; ++t) {
-            const int blk = blocks[t];
+            const int code = blocks[t];
+            const bool dropped = code < 0;  // STE: a block the selection dropped
+            const int blk = dropped ? -code - 1 : code;
             const bool cur = (t == nsel);
-            const float bias = cur ? 0.f : gate_log(srow[blk], lse_c, p.gate);
+            const float lg = cur ? 0.f : gate_log(srow[blk], lse_c, p.gate);
+            const float bias = gate_in_logits(p.gate) ? lg : 0.f;
+            const float w = (p.gate == kGateOuter && !cur) ? expf(lg) : 1.f;
             __syncthreads();
             load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
             load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
@@ -297,9 +323,10 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
                         const int r = ttr + C::RG * ii, j = ttc + C::RG * jj;
                         const float z = fmaf(p.scale, sacc[ii][jj], bias);
                         const float pr = (cur && j > r) ? 0.f : expf(z - rowL[r]);
-                        const float dS = pr * (pacc[ii][jj] - rowD[r]);
+                        const float dS = pr * (w * pacc[ii][jj] - rowD[r]);
                         Ss[r * C::LDS + j] = dS;
-                        local += dS;
+                        // the block's log-gate gradient: sum dS (the outer gate: g sum P dP)
+                        local += p.gate == kGateOuter ? w * pr * pacc[ii][jj] : dS;
                     }
             }
             if (!cur) {
@@ -307,6 +334,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
                 if (tid == 0) dlg[t] += tot;
             }
             __syncthreads();
+            if (dropped) continue;  // its dS reaches dlogg only
             for (int j = 0; j < BS; ++j) {
                 float sv[4];
 #pragma unroll
@@ -328,17 +356,23 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
         }
     }
     __syncthreads();
+    // STE: dlg holds the straight-through dL/dg; as a log-gate gradient, g dL/dg
+    if (ste)
+        for (int i = tid; i < nsel; i += kThreads) dlg[i] *= expf(srow[i] - lse_c);
+    __syncthreads();
     // ds[c, m] from dlogg (0 for blocks the row does not attend, and for m >= c):
-    // softmax gate dlogg_m - g_m * sum(dlogg); sigmoid dlogg_m (1 - g_m); raw dlogg_m
+    // g = softmax(s): dlogg_m - g_m * sum(dlogg); sigmoid dlogg_m (1 - g_m); raw dlogg_m
     float part = 0.f;
     for (int i = tid; i < nsel; i += kThreads) part += dlg[i];
     const float tot = block_sum(part, red);
     float* dsrow = p.ds + unit * p.Cq;
     for (int m = tid; m < p.Cq; m += kThreads)
-        dsrow[m] = (m < c && p.gate == 0) ? -expf(srow[m] - lse_c) * tot : 0.f;
+        dsrow[m] = (m < c && gate_softmax_family(p.gate)) ? -expf(srow[m] - lse_c) * tot : 0.f;
     __syncthreads();
-    for (int i = tid; i < nsel; i += kThreads)
-        dsrow[blocks[i]] = gate_ds(dlg[i], gate_log(srow[blocks[i]], lse_c, p.gate), tot, p.gate);
+    for (int i = tid; i < nsel; i += kThreads) {
+        const int m = blocks[i] < 0 ? -blocks[i] - 1 : blocks[i];
+        dsrow[m] = gate_ds(dlg[i], gate_log(srow[m], lse_c, p.gate), tot, p.gate);
+    }
 }
 
 // is history block m in the (ascending) selection of query block c?
@@ -396,7 +430,12 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
         for (int li = 0; li < cnt; ++li) {
             const int c = clist[li];
             const bool diag = (c == m);
-            const float bias = diag ? 0.f : gate_log(p.s[(ubase + c) * p.Cq + m], p.gate == 0 ? p.lse_s[ubase + c] : 0.f, p.gate);
+            const float lg =
+                diag ? 0.f
+                     : gate_log(p.s[(ubase + c) * p.Cq + m], gate_softmax_family(p.gate) ? p.lse_s[ubase + c] : 0.f,
+                                p.gate);
+            const float bias = gate_in_logits(p.gate) ? lg : 0.f;
+            const float w = (p.gate == kGateOuter && !diag) ? expf(lg) : 1.f;  // outer gate: g weights V
             for (int g = 0; g < G; ++g) {
                 const int hq = h * G + g;
                 __syncthreads();
@@ -438,8 +477,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
                             const int r = ttr + C::RG * ii, j = ttc + C::RG * jj;
                             const float z = fmaf(p.scale, sacc[ii][jj], bias);
                             const float pr = (diag && j > r) ? 0.f : expf(z - rowL[r]);
-                            Ps[r * C::LDS + j] = pr;
-                            dSs[r * C::LDS + j] = pr * (pacc[ii][jj] - rowD[r]);
+                            Ps[r * C::LDS + j] = pr * w;
+                            dSs[r * C::LDS + j] = pr * (w * pacc[ii][jj] - rowD[r]);
                         }
                 }
                 __syncthreads();

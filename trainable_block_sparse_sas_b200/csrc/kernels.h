@@ -32,11 +32,19 @@ struct TrainParams {
     int* status;  // device status word (bounded waits)
     int B, Hq, Hkv, d, n, bs, Cq, top_k, full_scope, is_bf16;
     float scale;
-    int gate;  // sas_gate: 0 softmax (log g = s - lse_s), 1 log sigmoid(s), 2 raw s
+    int gate;  // sas_gate: 0 softmax, 1 sigmoid, 2 raw logit, 3 outer, 4 hard STE
 };
 
-// log g of a history block from its score (natural log): the softmax gate needs
-// the row's LSE; the sigmoid and raw-logit variants do not
+constexpr int kGateOuter = 3, kGateSte = 4;
+
+// does log g enter the logits (inner gates 0-2)?  The outer gate weights the
+// values instead; the hard STE gate's forward value is 1 (bias 0)
+__host__ __device__ __forceinline__ bool gate_in_logits(int gate) { return gate <= 2; }
+// is g = softmax(s) (so that lse_s is needed)?
+__host__ __device__ __forceinline__ bool gate_softmax_family(int gate) { return gate == 0 || gate >= 3; }
+
+// log g of a history block from its score (natural log): g = softmax(s) needs the
+// row's LSE; the sigmoid and raw-logit variants do not
 __host__ __device__ __forceinline__ float gate_log(float s, float lse, int gate) {
     if (gate == 1) return s >= 0.f ? -log1pf(expf(-s)) : s - log1pf(expf(s));
     if (gate == 2) return s;
@@ -44,7 +52,7 @@ __host__ __device__ __forceinline__ float gate_log(float s, float lse, int gate)
 }
 
 // ds of one history block from its dlogg: the raw-logit gate passes it through,
-// the sigmoid gate scales by 1 - g; the softmax gate subtracts g * sum(dlogg)
+// the sigmoid gate scales by 1 - g; g = softmax(s) subtracts g * sum(dlogg)
 __host__ __device__ __forceinline__ float gate_ds(float dlogg, float logg, float tot, int gate) {
     if (gate == 2) return dlogg;
     if (gate == 1) return dlogg * (1.f - expf(logg));

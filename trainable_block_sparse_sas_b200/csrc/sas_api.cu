@@ -69,7 +69,7 @@ bool check_train(const sas_attn_desc* d) {
     if (d->scope != SAS_SCOPE_SPARSE && d->scope != SAS_SCOPE_FULL) return false;
     if (d->dtype != SAS_F32 && d->dtype != SAS_BF16) return false;
     if (!isfinite(d->softmax_scale)) return false;
-    if (d->gate != SAS_GATE_SOFTMAX && d->gate != SAS_GATE_SIGMOID && d->gate != SAS_GATE_RAW) return false;
+    if (d->gate < SAS_GATE_SOFTMAX || d->gate > SAS_GATE_STE) return false;
     return true;
 }
 
@@ -161,7 +161,7 @@ sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const vo
                               sas_stream_t stream) {
     if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
     if (!q || !k || !v || !s || !o || !lse) return SAS_ERR_INVALID_VALUE;
-    if (!lse_s && desc->gate == SAS_GATE_SOFTMAX) return SAS_ERR_INVALID_VALUE;
+    if (!lse_s && gate_softmax_family(desc->gate)) return SAS_ERR_INVALID_VALUE;
     if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
     if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
     DeviceInfo di;
@@ -195,7 +195,7 @@ sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const vo
                               size_t ws_bytes, sas_stream_t stream) {
     if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
     if (!q || !k || !v || !o || !lse || !dO || !s || !dq || !dk || !dv || !ds) return SAS_ERR_INVALID_VALUE;
-    if (!lse_s && desc->gate == SAS_GATE_SOFTMAX) return SAS_ERR_INVALID_VALUE;
+    if (!lse_s && gate_softmax_family(desc->gate)) return SAS_ERR_INVALID_VALUE;
     if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
     if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
     const size_t need = sas_gated_attn_bwd_workspace_size(desc);
