@@ -211,3 +211,51 @@ def decode(q, k_cache, v_cache, ctx_len, s, bs: int, top_k: int, dense: bool = F
                              ctypes.c_int(sa.shape[-1]), ctypes.c_int(int(dense)), _ptr(o), _ptr(idx))
     _check(rc, "decode")
     return o, idx[..., :top_k]
+
+
+def pool_scores(q, k, bs: int, sigma=None):
+    """Pooled-key scorer, training shape: q [B,n,Hq,d], k [B,n,Hkv,d] ->
+    s [B,Hkv,Cq,Cq] float64 with s[c,m] = sigma mean_q(block c) . mean_k(block m)
+    for m < c, 0 for m >= c."""
+    _same_code(np.asarray(q), np.asarray(k))
+    qa, code, qp = _in(q)
+    ka, _, kp = _in(k)
+    B, n, Hq, d = qa.shape
+    Hkv = ka.shape[2]
+    if sigma is None:
+        sigma = 1.0 / np.sqrt(d)
+    Cq = n // bs
+    s = np.zeros((B, Hkv, Cq, Cq), dtype=np.float64)
+    rc = lib().oracle_pool_scores(B, n, Hq, Hkv, d, bs, ctypes.c_double(sigma), qp, kp, ctypes.c_int(code), _ptr(s))
+    _check(rc, "pool_scores")
+    return s
+
+
+def pool_keys(k_cache, bs: int, m0: int, m1: int, nsum: int, round_bf16: bool = False, ksum=None):
+    """Mean-pooled key summaries of full blocks [m0, m1) of k_cache [B,Hkv,Tmax,d]
+    into ksum [B,Hkv,nsum,d] float64 (rounded to bf16 values when round_bf16)."""
+    ka, code, kp = _in(k_cache)
+    B, Hkv, Tmax, d = ka.shape
+    if ksum is None:
+        ksum = np.zeros((B, Hkv, nsum, d), dtype=np.float64)
+    rc = lib().oracle_pool_keys(B, Hkv, Tmax, d, bs, kp, ctypes.c_int(code), m0, m1, nsum, int(round_bf16),
+                                _ptr(ksum))
+    _check(rc, "pool_keys")
+    return ksum
+
+
+def decode_scores(q, ksum, ctx_len, bs: int, s_cols: int, sigma=None):
+    """Decode scores s [B,Hkv,s_cols] float64: sigma (mean over the group's heads of
+    q) . ksum[b,h,m] for the full history blocks m < (ctx_len-1)//bs, else 0."""
+    qa, code, qp = _in(q)
+    B, Hq, d = qa.shape
+    ks = np.ascontiguousarray(ksum, dtype=np.float64)
+    Hkv, nsum = ks.shape[1], ks.shape[2]
+    if sigma is None:
+        sigma = 1.0 / np.sqrt(d)
+    cl = np.ascontiguousarray(ctx_len, dtype=np.int32)
+    s = np.zeros((B, Hkv, s_cols), dtype=np.float64)
+    rc = lib().oracle_decode_scores(B, Hq, Hkv, d, bs, ctypes.c_double(sigma), qp, ctypes.c_int(code), _ptr(ks),
+                                    nsum, _ptr(cl), s_cols, _ptr(s))
+    _check(rc, "decode_scores")
+    return s

@@ -656,3 +656,112 @@ int oracle_decode(int B, int Hq, int Hkv, int d, int bs, int Tmax, int top_k, do
     }
     return err;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Parameter-free pooled-key scorer: block summaries by mean pooling          */
+/* (jaehun.me review, walkthrough Step 1 and Limitations: the selector scores  */
+/* a query against per-block key summaries, pooling-based).                   */
+/* ------------------------------------------------------------------------- */
+
+/* Training shape.  q [B,n,Hq,d], k [B,n,Hkv,d]; s [B,Hkv,Cq,Cq] out:
+ *   qbar[b,h,c] = mean over the b tokens of block c and the G heads of group h of q
+ *   kbar[b,h,m] = mean over the b tokens of block m of k
+ *   s[b,h,c,m]  = sigma qbar[b,h,c] . kbar[b,h,m]  for m < c, 0 for m >= c. */
+int oracle_pool_scores(int B, int n, int Hq, int Hkv, int d, int bs, double sigma, const void* q, const void* k,
+                       int dt, double* s) {
+    if (B <= 0 || n <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || d <= 0 || bs <= 0 || n % bs || !q || !k || !s)
+        return ORC_ERR_ARG;
+    int G = Hq / Hkv, Cq = n / bs;
+    int err = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long u = 0; u < (long)B * Hkv; ++u) {
+        int b = (int)(u / Hkv), h = (int)(u % Hkv);
+        double* qbar = (double*)calloc((size_t)Cq * d, sizeof(double));
+        double* kbar = (double*)calloc((size_t)Cq * d, sizeof(double));
+        if (!qbar || !kbar) {
+            free(qbar);
+            free(kbar);
+            err = ORC_ERR_NOMEM;
+            continue;
+        }
+        for (int c = 0; c < Cq; ++c) {
+            for (int i = c * bs; i < (c + 1) * bs; ++i) {
+                for (int g = 0; g < G; ++g) {
+                    size_t qoff = (((size_t)b * n + i) * Hq + h * G + g) * (size_t)d;
+                    for (int e = 0; e < d; ++e) qbar[(size_t)c * d + e] += ld(q, dt, qoff + e);
+                }
+                size_t koff = (((size_t)b * n + i) * Hkv + h) * (size_t)d;
+                for (int e = 0; e < d; ++e) kbar[(size_t)c * d + e] += ld(k, dt, koff + e);
+            }
+            for (int e = 0; e < d; ++e) {
+                qbar[(size_t)c * d + e] /= (double)bs * G;
+                kbar[(size_t)c * d + e] /= (double)bs;
+            }
+        }
+        for (int c = 0; c < Cq; ++c)
+            for (int m = 0; m < Cq; ++m) {
+                double dot = 0.0;
+                if (m < c)
+                    for (int e = 0; e < d; ++e) dot += qbar[(size_t)c * d + e] * kbar[(size_t)m * d + e];
+                s[(u * Cq + c) * (size_t)Cq + m] = m < c ? sigma * dot : 0.0;
+            }
+        free(qbar);
+        free(kbar);
+    }
+    return err;
+}
+
+/* Decode shape.  Key summaries of the full blocks [m0, m1) of a cache
+ * [B,Hkv,Tmax,d]: ksum[b,h,m] = mean over the block's b tokens, kept in the
+ * summary array's dtype (rounded to bf16 when round_out != 0).  ksum is
+ * [B,Hkv,nsum,d] doubles; blocks outside [m0, m1) are left as they are. */
+int oracle_pool_keys(int B, int Hkv, int Tmax, int d, int bs, const void* kc, int dt, int m0, int m1, int nsum,
+                     int round_out, double* ksum) {
+    if (B <= 0 || Hkv <= 0 || Tmax <= 0 || d <= 0 || bs <= 0 || !kc || !ksum || m0 < 0 || m1 < m0 || m1 > nsum ||
+        (long)m1 * bs > Tmax)
+        return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (long u = 0; u < (long)B * Hkv; ++u) {
+        for (int m = m0; m < m1; ++m) {
+            for (int e = 0; e < d; ++e) {
+                double acc = 0.0;
+                for (int j = m * bs; j < (m + 1) * bs; ++j) acc += ld(kc, dt, ((size_t)u * Tmax + j) * (size_t)d + e);
+                acc /= (double)bs;
+                ksum[((size_t)u * nsum + m) * (size_t)d + e] = round_out ? round_bf16(acc) : acc;
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* Decode scores: q [B,Hq,d]; ksum [B,Hkv,nsum,d] doubles; ctx_len[b] = T:
+ *   s[b,h,m] = sigma qbar[b,h] . ksum[b,h,m] for the Cb = floor((T-1)/b) full
+ *   history blocks, 0 for m >= Cb; qbar = mean of q over the group's G heads.
+ * s: [B,Hkv,s_cols], s_cols >= every Cb. */
+int oracle_decode_scores(int B, int Hq, int Hkv, int d, int bs, double sigma, const void* q, int dt,
+                         const double* ksum, int nsum, const int* ctx_len, int s_cols, double* s) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || d <= 0 || bs <= 0 || !q || !ksum || !ctx_len || !s)
+        return ORC_ERR_ARG;
+    int G = Hq / Hkv;
+    int err = ORC_OK;
+    for (long u = 0; u < (long)B * Hkv; ++u) {
+        int b = (int)(u / Hkv), h = (int)(u % Hkv);
+        int T = ctx_len[b];
+        int Cb = T > 0 ? (T - 1) / bs : 0;
+        if (T <= 0 || Cb > s_cols || Cb > nsum) {
+            err = ORC_ERR_ARG;
+            continue;
+        }
+        for (int m = 0; m < s_cols; ++m) {
+            double dot = 0.0;
+            if (m < Cb)
+                for (int e = 0; e < d; ++e) {
+                    double qb = 0.0;
+                    for (int g = 0; g < G; ++g) qb += ld(q, dt, ((size_t)b * Hq + h * G + g) * (size_t)d + e);
+                    dot += qb / G * ksum[((size_t)u * nsum + m) * (size_t)d + e];
+                }
+            s[u * (size_t)s_cols + m] = m < Cb ? sigma * dot : 0.0;
+        }
+    }
+    return err;
+}

@@ -705,3 +705,67 @@ def test_gate_variants_reduce_to_known_cases():
     o_off = oracle.attn_bwd(q, k, v, dO, big, bs, K, gate="off")
     for name in ("o", "lse", "dq", "dk", "dv"):
         np.testing.assert_allclose(o_sig[name], o_off[name], atol=1e-12, rtol=0, err_msg=name)
+
+
+def test_pooled_scores_are_block_means_of_the_dense_logits():
+    """The pooled-key scorer: by bilinearity, sigma qbar_c . kbar_m is the mean of
+    the dense logits sigma q_i . k_j over the tokens i of block c (all G heads of
+    the group) and j of block m.  Computed here from a dense torch QK^T."""
+    rng = np.random.default_rng(40)
+    B, n, Hq, Hkv, d, bs = 2, 64, 4, 2, 16, 8
+    q = rng.standard_normal((B, n, Hq, d))
+    k = rng.standard_normal((B, n, Hkv, d))
+    sigma = 0.3
+    s = oracle.pool_scores(q, k, bs, sigma=sigma)
+    G, Cq = Hq // Hkv, n // bs
+    qt, kt = torch.tensor(q), torch.tensor(k)
+    for b in range(B):
+        for h in range(Hkv):
+            z = torch.stack([sigma * qt[b, :, h * G + g] @ kt[b, :, h].T for g in range(G)])  # [G, n, n]
+            zb = z.reshape(G, Cq, bs, Cq, bs).mean(dim=(0, 2, 4)).numpy()
+            want = np.tril(zb, -1)
+            np.testing.assert_allclose(s[b, h], want, atol=1e-12, rtol=0)
+
+
+def test_pooled_scores_closed_form_constant_blocks():
+    """Blocks whose tokens are all one vector: the summaries are those vectors."""
+    B, n, Hq, Hkv, d, bs = 1, 32, 2, 1, 4, 8
+    Cq = n // bs
+    u = np.arange(Cq * d, dtype=np.float64).reshape(Cq, d) / 8.0  # dyadic: every mean and dot exact
+    w = (np.arange(Cq * d, dtype=np.float64).reshape(Cq, d) % 3) - 1.0
+    k = np.repeat(u, bs, axis=0)[None, :, None, :]
+    q = np.repeat(np.repeat(w, bs, axis=0)[None, :, None, :], Hq, axis=2)
+    s = oracle.pool_scores(q, k, bs, sigma=1.0)
+    for c in range(Cq):
+        for m in range(Cq):
+            assert s[0, 0, c, m] == (float(w[c] @ u[m]) if m < c else 0.0)
+
+
+def test_decode_pooled_scores_brute_force():
+    """Decode: key summaries of the full blocks, then sigma (mean over the group's
+    heads of q) . kbar_m, equal to the mean of the dense logits over the heads and
+    the block's tokens; 0 beyond the history; bf16 summaries are the nearest bf16
+    values of the exact means."""
+    rng = np.random.default_rng(41)
+    B, Hq, Hkv, d, bs, Tmax = 3, 4, 2, 8, 8, 64
+    G = Hq // Hkv
+    q = rng.standard_normal((B, Hq, d))
+    kc = rng.standard_normal((B, Hkv, Tmax, d))
+    ctx = np.array([1, 30, 64], dtype=np.int32)  # 0, 3 and 7 full history blocks
+    nsum = Tmax // bs
+    ksum = oracle.pool_keys(kc, bs, 0, nsum, nsum)
+    s = oracle.decode_scores(q, ksum, ctx, bs, nsum, sigma=0.5)
+    for b in range(B):
+        Cb = (ctx[b] - 1) // bs
+        for h in range(Hkv):
+            for m in range(nsum):
+                want = 0.0
+                if m < Cb:
+                    want = np.mean([0.5 * q[b, h * G + g] @ kc[b, h, j] for g in range(G)
+                                    for j in range(m * bs, (m + 1) * bs)])
+                assert abs(s[b, h, m] - want) < 1e-12, (b, h, m)
+    part = oracle.pool_keys(kc, bs, 2, 5, nsum)
+    assert np.all(part[:, :, :2] == 0) and np.all(part[:, :, 5:] == 0)
+    np.testing.assert_array_equal(part[:, :, 2:5], ksum[:, :, 2:5])
+    r = oracle.pool_keys(kc, bs, 0, nsum, nsum, round_bf16=True)
+    np.testing.assert_array_equal(r, _nearest_bf16(ksum))
