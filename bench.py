@@ -374,6 +374,37 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
     return statistics.median(times)
 
 
+def time_decode_scores(api, w, hbm: float) -> dict:
+    """Pooled-key decode scores over the workload's block summaries (one bf16 row
+    per full block): the selector-scoring pass that precedes selection."""
+    import torch
+
+    g = torch.Generator(device="cpu")
+    g.manual_seed(3100)
+    Cb = (w.T - 1) // w.bs
+    q = (torch.randn((w.B, w.Hq, w.d), generator=g)).to(w.dtype).cuda()
+    ksum = (torch.randn((w.B, w.Hkv, Cb, w.d), generator=g) * 0.2).to(w.dtype).cuda()
+    ctx = torch.full((w.B,), w.T, dtype=torch.int32, device="cuda")
+    s = torch.empty((w.B, w.Hkv, Cb), dtype=torch.float32, device="cuda")
+    desc = api.DecodeDesc(w.B, w.Hq, w.Hkv, w.d, w.bs, w.top_k, w.T, api.SAS_BF16, 0.0)
+    flush = torch.empty(128 << 20, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        api.sas_decode_scores(desc, q, ksum, ctx, s)
+    ts = []
+    for _ in range(10):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        api.sas_decode_scores(desc, q, ksum, ctx, s)
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    us = sorted(ts)[len(ts) // 2]
+    by = ksum.numel() * ksum.element_size() + s.numel() * 4 + q.numel() * q.element_size()
+    return {"us": us, "bytes": by, "gbs": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm,
+            "l2": "flushed (512 MB write) before every repetition"}
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -523,7 +554,25 @@ def extras(api, args, peaks, peak_kind) -> dict:
         del r
         torch.cuda.empty_cache()
     out["gate_variants_" + w.name] = gates
-    del inp
+    # pooled-key scorer on the same workload: one pass over q and k (HBM bound)
+    desc = api.attn_desc(inp["q"], inp["k"], w.bs, w.top_k)
+    s = torch.empty_like(inp["s"])
+    ws = api.workspace(api.sas_pooled_scores_workspace_size(desc), inp["q"].device)
+    for _ in range(3):
+        api.sas_pooled_scores(desc, inp["q"], inp["k"], s, ws)
+    reps = 10
+    a.record()
+    for _ in range(reps):
+        api.sas_pooled_scores(desc, inp["q"], inp["k"], s, ws)
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) / reps * 1e3
+    by = inp["q"].numel() * inp["q"].element_size() + inp["k"].numel() * inp["k"].element_size()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out["pooled_scores_" + w.name] = {"us": us, "bytes": by, "gbs": by / (us * 1e-6) / 1e9,
+                                      "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm,
+                                      "l2": "q and k (335 MB) exceed L2"}
+    del inp, s, ws
     torch.cuda.empty_cache()
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     for w in (syn.DECODE_128K, syn.DECODE_512K):
@@ -535,6 +584,7 @@ def extras(api, args, peaks, peak_kind) -> dict:
                "includes": "Top-K selection + sparse decode in one launch (sas_sparse_decode_select)",
                "two_call_ms": time_decode(api, w, steps=10, mode="two_call"),
                "paged_ms": time_decode(api, w, steps=10, mode="paged")}
+        rec["decode_scores"] = time_decode_scores(api, w, hbm)
         if w is syn.DECODE_512K:
             msd = time_decode(api, w, steps=5, mode="dense")
             byd = decode_bytes(w, dense=True)

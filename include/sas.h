@@ -180,6 +180,52 @@ sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const vo
                               const int32_t* idx, void* dq, void* dk, void* dv, float* ds, void* workspace,
                               size_t ws_bytes, sas_stream_t stream);
 
+/*
+ * Parameter-free pooled-key scorer (jaehun.me review, walkthrough Step 1: scores
+ * from the query and per-block key summaries; Limitations: pooling-based block
+ * summaries).  The pages' trained selector is not given; this is its weight-free
+ * form, mean pooling on both sides, producing the score array s the selection
+ * and the gate read.
+ *
+ * sas_pooled_scores -- training shape:
+ *   s[b,h,c,m] = sigma qbar[b,h,c] . kbar[b,h,m] for m < c, 0 for m >= c, with
+ *   qbar the mean of q over query block c's tokens and the G query heads of kv
+ *   head h, kbar the mean of k over block m's tokens, sigma = desc->softmax_scale
+ *   (1/sqrt(d) when 0).  Only batch, heads, head_dim, seq_len, block_size, dtype
+ *   and softmax_scale of desc are read.
+ * q [B,n,Hq,d], k [B,n,Hkv,d] (16-byte aligned); s out [B,Hkv,Cq,Cq] fp32.
+ * workspace of sas_pooled_scores_workspace_size bytes (256-byte aligned).
+ * Errors: SAS_ERR_INVALID_VALUE (bad desc or pointers, misalignment);
+ *   SAS_ERR_UNSUPPORTED (d * elem not a multiple of 16, d > 256, or
+ *   G * d * elem > 2 KB); SAS_ERR_WORKSPACE_TOO_SMALL.
+ */
+size_t sas_pooled_scores_workspace_size(const sas_attn_desc* desc);
+sas_status sas_pooled_scores(const sas_attn_desc* desc, const void* q, const void* k, float* s, void* workspace,
+                             size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * sas_pool_key_blocks -- decode shape: block summaries of a contiguous cache,
+ *   ksum[b,h,m] = mean of k_cache[b,h,m*b:(m+1)*b] for m in [block_begin,
+ *   block_end), stored in desc->dtype (bf16 rounded to nearest); other entries
+ *   are left as they are, so a caller extends the summaries as blocks fill.
+ * k_cache [B,Hkv,max_ctx,d] (16-byte aligned); ksum [B,Hkv,nsum,d], caller-owned.
+ * Errors: SAS_ERR_INVALID_VALUE (bad desc, pointers, range outside [0, nsum] or
+ *   past max_ctx); SAS_ERR_UNSUPPORTED (d * elem not a multiple of 16, d > 256).
+ *
+ * sas_decode_scores -- s[b,h,m] = sigma qbar[b,h] . ksum[b,h,m] for the
+ *   floor((ctx_len[b]-1)/b) full history blocks, 0 for the rest of the row;
+ *   qbar = mean of the new token's q over the G heads of kv head h.
+ * q [B,Hq,d]; ksum [B,Hkv,nsum,d] in desc->dtype (16-byte aligned); ctx_len
+ *   device int32 [B]; s out [B,Hkv,s_cols] fp32, ready for sas_topk_select or
+ *   sas_sparse_decode_select.
+ * Errors: SAS_ERR_INVALID_VALUE (bad desc or pointers, nsum or s_cols <= 0);
+ *   SAS_ERR_UNSUPPORTED (head_dim not 64 or 128).
+ */
+sas_status sas_pool_key_blocks(const sas_decode_desc* desc, const void* k_cache, int32_t block_begin,
+                               int32_t block_end, void* ksum, int32_t nsum, sas_stream_t stream);
+sas_status sas_decode_scores(const sas_decode_desc* desc, const void* q, const void* ksum, int32_t nsum,
+                             const int32_t* ctx_len, float* s, int32_t s_cols, sas_stream_t stream);
+
 /* Bytes of workspace sas_sparse_decode needs for this problem (0 on bad desc). */
 size_t sas_sparse_decode_workspace_size(const sas_decode_desc* desc);
 

@@ -151,3 +151,26 @@ def test_paged_decode_checks(api):
     assert call(d, kp=ctypes.c_void_p(0x1008)) == 1   # pool not 16-byte aligned
     assert call(api.DecodeDesc(2, 8, 2, 128, 64, 4, 1000, 0, 0.0)) == 2         # fp32
     assert call(api.DecodeDesc(2, 8, 2, 128, 32, 4, 1000, 1, 0.0), pps=32) == 2  # block 32
+
+
+def test_scorer_checks(api):
+    """Argument checks of the pooled-key scorer entry points (nothing is launched)."""
+    L = api.lib
+    d = _desc(api)
+    need = L.sas_pooled_scores_workspace_size(ctypes.byref(d))
+    assert need > 0 and need % 256 == 0
+    assert L.sas_pooled_scores(ctypes.byref(d), None, FAKE, FAKE, FAKE, need, None) == 1
+    assert L.sas_pooled_scores(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, need - 1, None) == 3
+    assert L.sas_pooled_scores(ctypes.byref(_desc(api, seq_len=100)), FAKE, FAKE, FAKE, FAKE, need, None) == 1
+    wide = _desc(api, n_q_heads=16, n_kv_heads=1, dtype=0)  # fp32, G d = 2048 elements: 8 KB per row
+    assert L.sas_pooled_scores(ctypes.byref(wide), FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 2
+    assert L.sas_pooled_scores(ctypes.byref(_desc(api, head_dim=20)), FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == 2
+    dd = api.DecodeDesc(2, 8, 2, 128, 64, 4, 1000, 1, 0.0)  # max_ctx 1000: 15 full blocks
+    assert L.sas_pool_key_blocks(ctypes.byref(dd), None, 0, 4, FAKE, 16, None) == 1
+    assert L.sas_pool_key_blocks(ctypes.byref(dd), FAKE, 3, 2, FAKE, 16, None) == 1   # empty-negative range
+    assert L.sas_pool_key_blocks(ctypes.byref(dd), FAKE, 0, 17, FAKE, 16, None) == 1  # past nsum
+    assert L.sas_pool_key_blocks(ctypes.byref(dd), FAKE, 0, 16, FAKE, 16, None) == 1  # past max_ctx
+    assert L.sas_decode_scores(ctypes.byref(dd), FAKE, FAKE, 0, FAKE, FAKE, 16, None) == 1
+    assert L.sas_decode_scores(ctypes.byref(dd), FAKE, FAKE, 16, None, FAKE, 16, None) == 1
+    d96 = api.DecodeDesc(2, 8, 2, 96, 64, 4, 1000, 1, 0.0)
+    assert L.sas_decode_scores(ctypes.byref(d96), FAKE, FAKE, 16, FAKE, FAKE, 16, None) == 2

@@ -538,3 +538,75 @@ def test_paged_decode_in_cuda_graph_and_missing_pages(api):
     ref = _oracle_decode_rows(zeroed, [(0, 0)], bs, K, True)
     G = Hq // Hkv
     compare("missing-page o", host(o_miss[0, 0:G]), ref[(0, 0)][0], **BF16_TOL, bf16_out=True)
+
+
+# --------------------------------------------------------------------------
+# pooled-key scorer
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,n,Hq,Hkv,d,bs,dtype", [
+    (1, 1024, 8, 2, 128, 64, torch.bfloat16),  # G 4, the training workloads' geometry
+    (2, 480, 5, 1, 64, 32, torch.bfloat16),    # G 5, ragged count of 32-blocks (Cq 15)
+    (1, 256, 4, 2, 64, 16, torch.float32),
+    (1, 192, 2, 2, 128, 64, torch.float32),    # Cq 3: one tile
+])
+def test_pooled_scores_match_oracle(api, B, n, Hq, Hkv, d, bs, dtype):
+    q = _seeded((B, n, Hq, d), 1.0, dtype, 51)
+    k = _seeded((B, n, Hkv, d), 1.0, dtype, 52)
+    desc = api.attn_desc(q, k, bs, 0)
+    s = torch.full((B, Hkv, n // bs, n // bs), float("nan"), device="cuda")
+    ws = api.workspace(api.sas_pooled_scores_workspace_size(desc), q.device)
+    api.sas_pooled_scores(desc, q, k, s, ws)
+    torch.cuda.synchronize()
+    want = oracle.pool_scores(bits(q), bits(k), bs)
+    compare("s", host(s), want, **F32_TOL)
+    assert torch.all(torch.triu(s) == 0)  # m >= c: exactly 0
+
+
+def test_pooled_scores_full_size_and_selection(api):
+    """train_sparse_32k geometry: scores of two KV heads against the oracle, then
+    the selection of the GPU's scores, bit for bit against the oracle's."""
+    w = syn.TRAIN_SPARSE_32K
+    inp = syn.train_inputs(w, device="cuda", seed=2100)
+    desc = api.attn_desc(inp["q"], inp["k"], w.bs, w.top_k)
+    s = torch.empty((w.B, w.Hkv, w.Cq, w.Cq), device="cuda")
+    ws = api.workspace(api.sas_pooled_scores_workspace_size(desc), inp["q"].device)
+    api.sas_pooled_scores(desc, inp["q"], inp["k"], s, ws)
+    idx, _ = api.select_train(s, w.bs, w.top_k)
+    torch.cuda.synchronize()
+    G = w.Hq // w.Hkv
+    for h in (0, w.Hkv - 1):
+        want = oracle.pool_scores(bits(inp["q"][:, :, h * G:(h + 1) * G]), bits(inp["k"][:, :, h:h + 1]), w.bs)
+        compare(f"s[h{h}]", host(s[:, h:h + 1]), want, **F32_TOL)
+        want_idx, _ = oracle.train_select(bits(s[:, h:h + 1]), w.top_k)
+        np.testing.assert_array_equal(idx[:, h:h + 1].cpu().numpy(), want_idx)
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_decode_scores_match_oracle(api, dtype, d):
+    """Block summaries (built in two calls, as a cache grows), then the decode
+    scores: summaries within half a bf16 ulp of the oracle's rounding of the
+    exact mean, scores against the oracle on the GPU's summaries and on its own."""
+    B, Hq, Hkv, bs, Tmax = 4, 8, 2, 64, 64 * 40 + 5
+    q = _seeded((B, Hq, d), 1.0, dtype, 61)
+    kc = _seeded((B, Hkv, Tmax, d), 1.0, dtype, 62)
+    ctx = torch.tensor([1, 65, 64 * 17 + 3, Tmax], dtype=torch.int32, device="cuda")  # 0, 1, 17, 40 blocks
+    nsum = 40
+    desc = api.decode_desc(q, kc, bs, 4)
+    ksum = torch.zeros((B, Hkv, nsum, d), dtype=dtype, device="cuda")
+    api.sas_pool_key_blocks(desc, kc, 0, 25, ksum)
+    api.sas_pool_key_blocks(desc, kc, 25, 40, ksum)
+    s_cols = 48
+    s = torch.full((B, Hkv, s_cols), float("nan"), device="cuda")
+    api.sas_decode_scores(desc, q, ksum, ctx, s)
+    torch.cuda.synchronize()
+    want_sum = oracle.pool_keys(bits(kc), bs, 0, nsum, nsum, round_bf16=dtype == torch.bfloat16)
+    compare("ksum", host(ksum), want_sum, rel_l2=1e-6, max_abs=1e-6, bf16_out=dtype == torch.bfloat16)
+    got_sum = host(ksum)
+    compare("s (GPU summaries)", host(s), oracle.decode_scores(bits(q), got_sum, ctx.cpu().numpy(), bs, s_cols),
+            **F32_TOL)
+    compare("s", host(s), oracle.decode_scores(bits(q), want_sum, ctx.cpu().numpy(), bs, s_cols),
+            **(BF16_TOL if dtype == torch.bfloat16 else F32_TOL))
+    Cb = (ctx.cpu().numpy() - 1) // bs
+    for b in range(B):
+        assert torch.all(s[b, :, int(Cb[b]):] == 0)

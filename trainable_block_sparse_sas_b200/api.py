@@ -78,6 +78,14 @@ lib.sas_launch_count.restype = ctypes.c_uint64
 lib.sas_launch_count.argtypes = []
 lib.sas_device_status.restype = ctypes.c_int
 lib.sas_device_status.argtypes = [_vp]
+lib.sas_pooled_scores_workspace_size.restype = _sz
+lib.sas_pooled_scores_workspace_size.argtypes = [ctypes.POINTER(AttnDesc)]
+lib.sas_pooled_scores.restype = ctypes.c_int
+lib.sas_pooled_scores.argtypes = [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _sz, _vp]
+lib.sas_pool_key_blocks.restype = ctypes.c_int
+lib.sas_pool_key_blocks.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _i32, _i32, _vp, _i32, _vp]
+lib.sas_decode_scores.restype = ctypes.c_int
+lib.sas_decode_scores.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _vp, _i32, _vp, _vp, _i32, _vp]
 
 
 def _p(t):
@@ -172,6 +180,31 @@ def sas_sparse_decode_paged(desc, q, k_pages, v_pages, page_table, ctx_len, o, s
                                        page_table.shape[1], k_pages.shape[0], _p(ctx_len), _p(idx), _p(s),
                                        0 if s is None else s.shape[-1], _p(o), _p(idx_out), _stream(stream)),
            "sas_sparse_decode_paged")
+
+
+def sas_pooled_scores_workspace_size(desc) -> int:
+    return int(lib.sas_pooled_scores_workspace_size(ctypes.byref(desc)))
+
+
+def sas_pooled_scores(desc, q, k, s, workspace, stream=None):
+    """Pooled-key scores, training shape: s [B,Hkv,Cq,Cq] fp32 (m < c), from the
+    mean of q over each query block and group and the mean of k over each block."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.sas_pooled_scores(ctypes.byref(desc), _p(q), _p(k), _p(s), _p(workspace), ws_bytes, _stream(stream)),
+           "sas_pooled_scores")
+
+
+def sas_pool_key_blocks(desc, k_cache, block_begin: int, block_end: int, ksum, stream=None):
+    """Mean-pooled summaries of the full blocks [block_begin, block_end) of a
+    contiguous cache into ksum [B,Hkv,nsum,d] (the cache's dtype)."""
+    _check(lib.sas_pool_key_blocks(ctypes.byref(desc), _p(k_cache), block_begin, block_end, _p(ksum), ksum.shape[2],
+                                   _stream(stream)), "sas_pool_key_blocks")
+
+
+def sas_decode_scores(desc, q, ksum, ctx_len, s, stream=None):
+    """Decode scores s [B,Hkv,s_cols] fp32 from the block summaries ksum."""
+    _check(lib.sas_decode_scores(ctypes.byref(desc), _p(q), _p(ksum), ksum.shape[2], _p(ctx_len), _p(s), s.shape[-1],
+                                 _stream(stream)), "sas_decode_scores")
 
 
 def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream=None):

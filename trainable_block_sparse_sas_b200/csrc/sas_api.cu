@@ -228,6 +228,58 @@ sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const vo
     return from_cuda(launch_bwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// ---------------------------------------------------------------------------
+// pooled-key scorer
+// ---------------------------------------------------------------------------
+
+size_t sas_pooled_scores_workspace_size(const sas_attn_desc* desc) {
+    if (!check_train(desc)) return 0;
+    return (pooled_scores_workspace(make_train(desc)) + 255) & ~(size_t)255;
+}
+
+sas_status sas_pooled_scores(const sas_attn_desc* desc, const void* q, const void* k, float* s, void* workspace,
+                             size_t ws_bytes, sas_stream_t stream) {
+    if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k || !s) return SAS_ERR_INVALID_VALUE;
+    const int eb = desc->dtype == SAS_BF16 ? 2 : 4;
+    if (!pool_shape_ok(desc->head_dim, desc->n_q_heads / desc->n_kv_heads, eb)) return SAS_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k)) & 15u) return SAS_ERR_INVALID_VALUE;
+    const size_t need = sas_pooled_scores_workspace_size(desc);
+    if (ws_bytes < need) return SAS_ERR_WORKSPACE_TOO_SMALL;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SAS_ERR_INVALID_VALUE;
+    TrainParams p = make_train(desc);
+    p.q = q;
+    p.k = k;
+    return from_cuda(launch_pooled_scores(p, s, workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_pool_key_blocks(const sas_decode_desc* desc, const void* k_cache, int32_t block_begin,
+                               int32_t block_end, void* ksum, int32_t nsum, sas_stream_t stream) {
+    if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!k_cache || !ksum) return SAS_ERR_INVALID_VALUE;
+    if (block_begin < 0 || block_end < block_begin || block_end > nsum ||
+        (long)block_end * desc->block_size > desc->max_ctx)
+        return SAS_ERR_INVALID_VALUE;
+    const int eb = desc->dtype == SAS_BF16 ? 2 : 4;
+    if (!pool_shape_ok(desc->head_dim, 1, eb)) return SAS_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(k_cache) & 15u) return SAS_ERR_INVALID_VALUE;
+    DecodeParams p = make_decode(desc);
+    p.k = k_cache;
+    return from_cuda(launch_pool_keys(p, block_begin, block_end, ksum, nsum, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_decode_scores(const sas_decode_desc* desc, const void* q, const void* ksum, int32_t nsum,
+                             const int32_t* ctx_len, float* s, int32_t s_cols, sas_stream_t stream) {
+    if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !ksum || !ctx_len || !s || nsum <= 0 || s_cols <= 0) return SAS_ERR_INVALID_VALUE;
+    if (desc->head_dim != 64 && desc->head_dim != 128) return SAS_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(ksum) & 15u) return SAS_ERR_INVALID_VALUE;
+    DecodeParams p = make_decode(desc);
+    p.q = q;
+    p.ctx_len = ctx_len;
+    return from_cuda(launch_decode_scores(p, ksum, nsum, s, s_cols, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t sas_sparse_decode_workspace_size(const sas_decode_desc* desc) {
     if (!check_decode(desc)) return 0;
     return decode_ws_bytes(make_decode(desc));
