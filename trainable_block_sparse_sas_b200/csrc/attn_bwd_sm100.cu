@@ -62,6 +62,7 @@ struct BwdArgs {
     const float* lse;
     float* Dbuf;
     __nv_bfloat16* Mbuf;  // [CTA][list slot][row] block masses of the dq kernel
+    float* Cbuf;          // [CTA][row] the rows' coefficients of those masses in dlogg
     const __nv_bfloat16* o;
     const __nv_bfloat16* dO;
     __nv_bfloat16* dq;
@@ -133,7 +134,8 @@ __host__ __device__ inline int dq_list_max(int Cq, int top_k, int full_scope, in
     return (full_scope || gate == kGateSte ? Cq : min(top_k, Cq)) + 1;
 }
 
-template <int MT, int ST>
+// kOuter: the outer gate (dS = P (g dP - D)); the other gates keep dS = P (dP - D)
+template <int MT, int ST, bool kOuter>
 __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __grid_constant__ BwdArgs a) {
     using L = DqLayout<MT, ST>;
     constexpr int kStages = ST;
@@ -172,10 +174,6 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     const long unit = (long)bh * a.Cq + c;
     // block masses M_t of the CTA's rows: [list slot][128 * MT rows], bf16
     __nv_bfloat16* mbase = a.Mbuf + (long)blockIdx.x * nl * (128 * MT);
-    // softmax threads: the coefficient of their row's block masses in the dlogg
-    // correction (delta = sum_j dS_ij; for the outer gate -D)
-    float row_delta = 0.f;
-    int row_unit = -1;
 
     for (int i = threadIdx.x; i < 8 * nl; i += kDqThreads) part[i] = 0.f;
     if (threadIdx.x == 0) {
@@ -377,12 +375,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 const float off = bias2[t] - lse2;
                 const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
                 const uint64_t negD2 = f2_pack(-Drow, -Drow);
-                // dS = P (w dP - D); a dropped block of the STE gate takes w = 1 for its
-                // straight-through gradient and gives dQ nothing
+                // dS = P (w dP - D), w = g for the outer gate; a dropped block of the STE
+                // gate (w = 0 in the list) gives dQ nothing
                 const float wt = wgt[t];
                 const bool dropped = ste && wt == 0.f;
-                const float wd = dropped ? 1.f : wt;
-                const uint64_t w2 = f2_pack(wd, wd);
+                const uint64_t w2 = f2_pack(wt, wt);
                 uint64_t rs2 = 0ull, m2 = 0ull;
                 uint32_t pk[32];
 #pragma unroll
@@ -401,8 +398,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                             if (2 * jj + 1 > tok) p1 = 0.f;
                         }
                         const uint64_t p2 = f2_pack(p0, p1);
-                        const uint64_t ds2 = f2_mul(
-                            p2, f2_fma(f2_pack(__uint_as_float(dr[2 * jq]), __uint_as_float(dr[2 * jq + 1])), w2, negD2));
+                        const uint64_t dp2 = f2_pack(__uint_as_float(dr[2 * jq]), __uint_as_float(dr[2 * jq + 1]));
+                        const uint64_t ds2 = f2_mul(p2, kOuter ? f2_fma(dp2, w2, negD2) : f2_add(dp2, negD2));
                         rs2 = f2_add(rs2, ds2);
                         m2 = f2_add(m2, p2);
                         float d0, d1;
@@ -433,8 +430,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             a.Dbuf[ri] = Drow + delta;  // D for dk / dv
             // dlogg_t = sum_i (dS-sum_it - coef_i M_it): the exact-D correction, or
             // for the outer gate g_t sum P dP = dS-sum + D M
-            row_delta = a.gate == kGateOuter ? -Drow : delta;
-            row_unit = r_unit;
+            a.Cbuf[(long)blockIdx.x * (128 * MT) + r_unit] = kOuter ? -Drow : delta;
             if (ok && warp_wait(dq_done, 0, abort_flag, a.status)) {
                 tc_fence_after();
                 __nv_bfloat16* drow = a.dq + (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
@@ -460,21 +456,17 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-    // the MMAs are drained: the Q tile's smem holds the rows' delta from here on
-    float* delta_sh = reinterpret_cast<float*>(base + L::kQ);
-    if (row_unit >= 0) delta_sh[row_unit] = row_delta;
-    __syncthreads();
-    // dlogg_t: the group's warp partials, less sum_i delta_i M_it (one slot per thread)
+    // dlogg_t: the group's warp partials, less sum_i delta_i M_it; eight threads per
+    // slot, each a strip of the rows (2 MT 16-byte loads), summed over the eight
     const int nsel = nlist - 1;
-    for (int t = threadIdx.x; t < nsel; t += kDqThreads) {
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) acc += part[t * 8 + w];
-        const uint4* mv = reinterpret_cast<const uint4*>(mbase + (long)t * (128 * MT));
-        const float4* dv4 = reinterpret_cast<const float4*>(delta_sh);
+    const int sub = threadIdx.x & 7;
+    const unsigned grp_mask = 0xffu << (threadIdx.x & 24);  // the 8 lanes sharing a slot
+    for (int t = threadIdx.x >> 3; t < nsel; t += kDqThreads / 8) {
+        const uint4* mv = reinterpret_cast<const uint4*>(mbase + (long)t * (128 * MT)) + sub * 2 * MT;
+        const float4* dv4 = reinterpret_cast<const float4*>(a.Cbuf + (long)blockIdx.x * (128 * MT)) + sub * 4 * MT;
         float corr = 0.f;
-#pragma unroll 4
-        for (int v = 0; v < 16 * MT; ++v) {  // 8 rows per 16-byte load
+#pragma unroll
+        for (int v = 0; v < 2 * MT; ++v) {  // 8 rows per 16-byte load
             const uint4 x = mv[v];
             const float4 d0 = dv4[2 * v], d1 = dv4[2 * v + 1];
             const float2 m01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
@@ -490,6 +482,12 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             corr = fmaf(d1.z, m67.x, corr);
             corr = fmaf(d1.w, m67.y, corr);
         }
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) corr += __shfl_xor_sync(grp_mask, corr, o);
+        if (sub != 0) continue;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc += part[t * 8 + w];
         float dl = acc - corr;
         // STE: the straight-through dL/dg of the block, as a log-gate gradient g dL/dg
         if (ste) dl *= expf(a.s[unit * a.Cq + list[t]] - a.lse_s[unit]);
@@ -842,6 +840,12 @@ cudaError_t launch_kernel(Kern kern, long grid, int threads, size_t smem, const 
     return err;
 }
 
+// bf16 block masses: every query row once per list slot (256-byte multiple)
+static size_t bwd_sm100_mass_bytes(const TrainParams& p) {
+    const size_t b = sizeof(__nv_bfloat16) * (size_t)p.B * p.Hq * p.n * dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
+    return (b + 255) & ~(size_t)255;
+}
+
 template <int MT>
 cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     constexpr int G = 2 * MT;
@@ -855,6 +859,7 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.lse = p.lse_in;
     a.Dbuf = p.Dbuf;
     a.Mbuf = static_cast<__nv_bfloat16*>(p.Mbuf);
+    a.Cbuf = reinterpret_cast<float*>(static_cast<uint8_t*>(p.Mbuf) + bwd_sm100_mass_bytes(p));
     a.o = static_cast<const __nv_bfloat16*>(p.o_in);
     a.dO = static_cast<const __nv_bfloat16*>(p.dO);
     a.dq = static_cast<__nv_bfloat16*>(p.dq);
@@ -877,9 +882,12 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
         !encode_tma_rows(&a.tk, p.k, p.Hkv, rows, 1, kBS) || !encode_tma_rows(&a.tv, p.v, p.Hkv, rows, 1, kBS))
         return cudaErrorInvalidValue;
     const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
-    cudaError_t err = DqLayout<MT, 3>::bytes(nl) <= kSmemLimit
-                          ? launch_kernel(bwd_dq_sm100_kernel<MT, 3>, grid, kDqThreads, DqLayout<MT, 3>::bytes(nl), a, stream)
-                          : launch_kernel(bwd_dq_sm100_kernel<MT, 2>, grid, kDqThreads, DqLayout<MT, 2>::bytes(nl), a, stream);
+    const bool outer = p.gate == kGateOuter;
+    const bool st3 = DqLayout<MT, 3>::bytes(nl) <= kSmemLimit;
+    const size_t smem = st3 ? DqLayout<MT, 3>::bytes(nl) : DqLayout<MT, 2>::bytes(nl);
+    auto kern = st3 ? (outer ? bwd_dq_sm100_kernel<MT, 3, true> : bwd_dq_sm100_kernel<MT, 3, false>)
+                    : (outer ? bwd_dq_sm100_kernel<MT, 2, true> : bwd_dq_sm100_kernel<MT, 2, false>);
+    cudaError_t err = launch_kernel(kern, grid, kDqThreads, smem, a, stream);
     if (err != cudaSuccess) return err;
     // key-major kernel: 128-row items (128/G tokens x G heads) per box
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, 128 / G) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, 128 / G))
@@ -897,9 +905,9 @@ static bool bwd_sm100_shape(const TrainParams& p) {
 }
 
 size_t bwd_sm100_workspace(const TrainParams& p) {
-    // bf16 block masses: every query row once per list slot
+    // the block masses, then one fp32 coefficient per query row
     if (!bwd_sm100_shape(p)) return 0;
-    return sizeof(__nv_bfloat16) * (size_t)p.B * p.Hq * p.n * dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
+    return bwd_sm100_mass_bytes(p) + sizeof(float) * (size_t)p.B * p.Hq * p.n;
 }
 
 bool bwd_sm100_supported(const TrainParams& p) {
