@@ -232,9 +232,9 @@ def _slice_inputs(inp, h, G):
     }
 
 
-def _sampled_full_size(api, w, q_blocks, kv_blocks, heads):
+def _sampled_full_size(api, w, q_blocks, kv_blocks, heads, gate="softmax"):
     inp = syn.train_inputs(w, device="cuda", seed=2000)
-    got = run_train(api, inp, w.bs, w.top_k, w.full_scope)
+    got = run_train(api, inp, w.bs, w.top_k, w.full_scope, gate=gate)
     G, Cq, bs = w.Hq // w.Hkv, w.Cq, w.bs
     for h in heads:
         si = _slice_inputs(inp, h, G)
@@ -252,7 +252,7 @@ def _sampled_full_size(api, w, q_blocks, kv_blocks, heads):
                 if w.full_scope or m in sel[0, 0, c].tolist():
                     qmask[0, 0, c] = True
         want = oracle.attn_bwd(si["q"], si["k"], si["v"], si["dO"], si["s"], bs, w.top_k, full_scope=w.full_scope,
-                               qmask=qmask, kvmask=kvmask,
+                               qmask=qmask, kvmask=kvmask, gate=gate,
                                o_store="bf16" if _reads_stored_o(w.dtype, w.d, bs, G) else None)
         rows = np.concatenate([np.arange(c * bs, (c + 1) * bs) for c in q_blocks])
         hs = slice(h * G, (h + 1) * G)
@@ -268,6 +268,14 @@ def _sampled_full_size(api, w, q_blocks, kv_blocks, heads):
 def test_train_sparse_32k_sampled(api):
     w = syn.TRAIN_SPARSE_32K
     _sampled_full_size(api, w, q_blocks=(0, 1, 31, 32, 33, 257, 511), kv_blocks=(511, 480, 350), heads=(0, 5))
+
+
+@pytest.mark.parametrize("gate,kv_blocks", [("outer", (480, 100)), ("ste", (480,))])
+def test_train_sparse_32k_gate_variants_sampled(api, gate, kv_blocks):
+    """The outer and hard-STE gates on the full 32K workload, as the benchmark
+    times them; the STE's dq kernel walks up to 511 dropped blocks per row."""
+    w = syn.TRAIN_SPARSE_32K
+    _sampled_full_size(api, w, q_blocks=(0, 1, 33, 257, 511), kv_blocks=kv_blocks, heads=(3,), gate=gate)
 
 
 def test_train_full_16k_sampled(api):
