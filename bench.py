@@ -316,7 +316,8 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
     in one launch), "two_call" (sas_topk_select then sas_sparse_decode), "dense"
     (sas_sparse_decode over every cached token), or "paged" (the fused step on the
     same cache scattered into a shuffled pool of one-block pages,
-    sas_sparse_decode_paged)."""
+    sas_sparse_decode_paged).  Repetitions rotate among 4 score tensors, so the
+    attended blocks change from one repetition to the next."""
     import torch
 
     from trainable_block_sparse_sas_b200 import synthetic as syn
@@ -328,7 +329,10 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
     o = torch.empty_like(q)
     ws = api.workspace(api.sas_sparse_decode_workspace_size(desc), q.device)
     flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
-    s4 = s.view(w.B, w.Hkv, 1, -1)
+    gs = torch.Generator(device="cuda")
+    gs.manual_seed(3200)
+    s_rot = [s] + [torch.randn(s.shape, generator=gs, device="cuda") * w.s_std for _ in range(3)]
+    cur = {"s": s}
     if mode == "paged":
         pps = (w.T + w.bs - 1) // w.bs
         g = torch.Generator(device="cpu")
@@ -348,20 +352,23 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
         pdesc = api.paged_decode_desc(q, kp, w.bs, w.top_k, w.T)
 
     def run():
+        sc = cur["s"]
         if mode == "fused":
-            api.sas_sparse_decode_select(desc, q, kc, vc, ctx, s, o, idx)
+            api.sas_sparse_decode_select(desc, q, kc, vc, ctx, sc, o, idx)
             return
         if mode == "paged":
-            api.sas_sparse_decode_paged(pdesc, q, kp, vp, table, ctx, o, s=s, idx_out=idx)
+            api.sas_sparse_decode_paged(pdesc, q, kp, vp, table, ctx, o, s=sc, idx_out=idx)
             return
         if mode == "two_call":
-            api.sas_topk_select(s4, 1, s.shape[-1], w.top_k, idx=idx, ctx_len=ctx, block_size=w.bs)
+            api.sas_topk_select(sc.view(w.B, w.Hkv, 1, -1), 1, sc.shape[-1], w.top_k, idx=idx, ctx_len=ctx,
+                                block_size=w.bs)
         api.sas_sparse_decode(desc, q, kc, vc, ctx, None if mode == "dense" else idx, o, ws)
 
     for _ in range(3):
         run()
     times = []
-    for _ in range(steps):
+    for i in range(steps):
+        cur["s"] = s_rot[i % 4]
         flush.sum()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
