@@ -11,8 +11,9 @@
 //   s[b,h,c,m]  = sigma qbar[b,h,c] . kbar[b,h,m] for m < c, 0 for m >= c.
 //   pool_train_kernel: one CTA per (b, block, kv head), 16-byte loads over the
 //     block's rows, fp32 sums: a single pass over q and k, bound by HBM.
-//   pool_scores_kernel: 32 x 32 tiles of the strictly lower triangle in fp32 on
-//     the CUDA cores (Cq^2 d / 2 FMAs per head: small next to the pooling pass).
+//   pool_scores_kernel: 64 x 64 tiles of the strictly lower triangle in fp32 on
+//     the CUDA cores, 4 x 4 outputs per thread (Cq^2 d / 2 FMAs per head: small
+//     next to the pooling pass).
 //
 // Decode shape:
 //   pool_keys_kernel: ksum[b,h,m] = mean of the cache's block m (full blocks in
@@ -62,14 +63,14 @@ __device__ __forceinline__ void add_vec<float>(float* acc, const uint4 x) {
 // Sum of `rows` rows of `span` elements (row r at base + r * stride, 16-byte
 // aligned), folded over `fold` equal parts of the span (the G heads of a query
 // row): out[e] = sum_r sum_f row_r[f * (span / fold) + e], e < span / fold.
-// All threads of the CTA take part; red is shared scratch of kPoolThreads * 8
-// floats; the result is written by threads e < span / fold.
-template <typename T>
+// All NT threads of the CTA take part; red is shared scratch of NT * 8 floats;
+// the result is written by threads e < span / fold.
+template <typename T, int NT = kPoolThreads>
 __device__ __forceinline__ void pool_rows(const T* base, long stride, int rows, int span, int fold, float* red,
                                           float scale, float* out) {
     constexpr int V = Vec<T>::N;
     const int nv = span / V;                    // vectors per row
-    const int rg = kPoolThreads / nv;           // rows in flight; threads from rg * nv on idle
+    const int rg = NT / nv;                     // rows in flight; threads from rg * nv on idle
     const int tid = threadIdx.x;
     const int r0 = tid / nv, v = tid % nv;
     float acc[V];
@@ -87,7 +88,7 @@ __device__ __forceinline__ void pool_rows(const T* base, long stride, int rows, 
     for (int i = 0; i < V; ++i) red[tid * V + i] = acc[i];
     __syncthreads();
     const int part = span / fold;
-    for (int e = tid; e < part; e += kPoolThreads) {
+    for (int e = tid; e < part; e += NT) {
         float s = 0.f;
         for (int f = 0; f < fold; ++f) {
             const int el = f * part + e;  // element of the span
@@ -99,60 +100,77 @@ __device__ __forceinline__ void pool_rows(const T* base, long stride, int rows, 
     __syncthreads();
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kPoolThreads) pool_train_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                                                                  int n, int Hq, int Hkv, int d, int bs, int Cq,
-                                                                  float* __restrict__ qbar, float* __restrict__ kbar) {
-    __shared__ float red[kPoolThreads * 8];
+// NT threads per (b, block, kv head): 64 when a query row's G heads fit in 64
+// 16-byte vectors, so that every CTA of a training problem is resident at once
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) pool_train_kernel(const T* __restrict__ q, const T* __restrict__ k, int n, int Hq,
+                                                        int Hkv, int d, int bs, int Cq, float* __restrict__ qbar,
+                                                        float* __restrict__ kbar) {
+    __shared__ float red[NT * 8];
     const int h = (int)(blockIdx.x % Hkv);
     const int c = (int)((blockIdx.x / Hkv) % Cq);
     const int b = (int)(blockIdx.x / ((long)Hkv * Cq));
     const int G = Hq / Hkv;
     const long row0 = (long)b * n + (long)c * bs;
     const long u = ((long)b * Hkv + h) * Cq + c;
-    pool_rows<T>(q + (row0 * Hq + (long)h * G) * d, (long)Hq * d, bs, G * d, G, red, 1.f / (float)(bs * G),
-                 qbar + u * d);
-    pool_rows<T>(k + (row0 * Hkv + h) * d, (long)Hkv * d, bs, d, 1, red, 1.f / (float)bs, kbar + u * d);
+    pool_rows<T, NT>(q + (row0 * Hq + (long)h * G) * d, (long)Hq * d, bs, G * d, G, red, 1.f / (float)(bs * G),
+                     qbar + u * d);
+    pool_rows<T, NT>(k + (row0 * Hkv + h) * d, (long)Hkv * d, bs, d, 1, red, 1.f / (float)bs, kbar + u * d);
 }
 
-constexpr int kTile = 32;
+constexpr int kTile = 64;   // output tile (query blocks x key blocks)
+constexpr int kTileE = 32;  // head-dim chunk staged in shared memory
 
-// s[b,h,c,m] for one 32 x 32 tile; 256 threads, 4 outputs each
+// s[b,h,c,m] for one 64 x 64 tile; 256 threads, a 4 x 4 register tile each
+// (rows ty + 16 i, columns tx + 16 j), so a thread reads 8 shared values per 16 FMAs
 __global__ void __launch_bounds__(256) pool_scores_kernel(const float* __restrict__ qbar,
                                                           const float* __restrict__ kbar, int Cq, int d, float sigma,
                                                           float* __restrict__ s) {
-    __shared__ float qs[kTile][kTile + 1], ks[kTile][kTile + 1];
+    __shared__ float qs[kTile][kTileE + 1], ks[kTile][kTileE + 1];
     const int tiles = (Cq + kTile - 1) / kTile;
     const int tc = (int)(blockIdx.x % tiles), tm = (int)((blockIdx.x / tiles) % tiles);
     const long bh = blockIdx.x / ((long)tiles * tiles);
     const int tid = threadIdx.x;
-    const int ty = tid / kTile, tx = tid % kTile;  // ty 0..7: rows ty, ty + 8, ...
+    const int ty = tid / 16, tx = tid % 16;
     const int c0 = tc * kTile, m0 = tm * kTile;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
     if (m0 < c0 + kTile - 1) {  // the tile holds some m < c
         const float* qb = qbar + bh * Cq * d;
         const float* kb = kbar + bh * Cq * d;
-        for (int e0 = 0; e0 < d; e0 += kTile) {
-            for (int i = ty; i < kTile; i += 8) {
-                const int cr = c0 + i, mr = m0 + i, e = e0 + tx;
-                qs[i][tx] = (cr < Cq && e < d) ? qb[(long)cr * d + e] : 0.f;
-                ks[i][tx] = (mr < Cq && e < d) ? kb[(long)mr * d + e] : 0.f;
+        for (int e0 = 0; e0 < d; e0 += kTileE) {
+            // 64 rows x 32 columns of each side: 8 elements per thread, coalesced rows
+            for (int idx = tid; idx < kTile * kTileE; idx += 256) {
+                const int r = idx / kTileE, e = e0 + idx % kTileE;
+                qs[r][idx % kTileE] = (c0 + r < Cq && e < d) ? qb[(long)(c0 + r) * d + e] : 0.f;
+                ks[r][idx % kTileE] = (m0 + r < Cq && e < d) ? kb[(long)(m0 + r) * d + e] : 0.f;
             }
             __syncthreads();
 #pragma unroll 8
-            for (int e = 0; e < kTile; ++e) {
-                const float kv = ks[tx][e];
+            for (int e = 0; e < kTileE; ++e) {
+                float qv[4], kv[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[j] = fmaf(qs[ty + 8 * j][e], kv, acc[j]);
+                for (int i = 0; i < 4; ++i) qv[i] = qs[ty + 16 * i][e];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) kv[j] = ks[tx + 16 * j][e];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qv[i], kv[j], acc[i][j]);
             }
             __syncthreads();
         }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int c = c0 + ty + 8 * j, m = m0 + tx;
-        if (c < Cq && m < Cq) s[(bh * Cq + c) * Cq + m] = m < c ? sigma * acc[j] : 0.f;
-    }
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = c0 + ty + 16 * i, m = m0 + tx + 16 * j;
+            if (c < Cq && m < Cq) s[(bh * Cq + c) * Cq + m] = m < c ? sigma * acc[i][j] : 0.f;
+        }
 }
 
 // ksum[b,h,m] = mean of the cache block m, m in [m0, m1); one CTA per (b, h, m)
@@ -259,8 +277,12 @@ template <typename T>
 cudaError_t pooled_scores_t(const TrainParams& p, float* qbar, float* kbar, float* s, cudaStream_t stream) {
     const long units = (long)p.B * p.Hkv * p.Cq;
     if (units <= 0) return cudaSuccess;
-    pool_train_kernel<T><<<(unsigned)units, kPoolThreads, 0, stream>>>(
-        static_cast<const T*>(p.q), static_cast<const T*>(p.k), p.n, p.Hq, p.Hkv, p.d, p.bs, p.Cq, qbar, kbar);
+    if (p.Hq / p.Hkv * p.d / Vec<T>::N <= 64)
+        pool_train_kernel<T, 64><<<(unsigned)units, 64, 0, stream>>>(
+            static_cast<const T*>(p.q), static_cast<const T*>(p.k), p.n, p.Hq, p.Hkv, p.d, p.bs, p.Cq, qbar, kbar);
+    else
+        pool_train_kernel<T, kPoolThreads><<<(unsigned)units, kPoolThreads, 0, stream>>>(
+            static_cast<const T*>(p.q), static_cast<const T*>(p.k), p.n, p.Hq, p.Hkv, p.d, p.bs, p.Cq, qbar, kbar);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     count_launch();
