@@ -223,6 +223,19 @@ sas_status sas_pooled_scores(const sas_attn_desc* desc, const void* q, const voi
  */
 sas_status sas_pool_key_blocks(const sas_decode_desc* desc, const void* k_cache, int32_t block_begin,
                                int32_t block_end, void* ksum, int32_t nsum, sas_stream_t stream);
+
+/*
+ * sas_pool_key_blocks_paged -- the same summaries from a paged cache (the layout
+ *   of sas_sparse_decode_paged: pages of one block, [num_pages, block_size, Hkv,
+ *   d], page_table [B, pages_per_seq] device int32).  A page id outside [0,
+ *   num_pages) gives a zero summary.
+ * Errors: SAS_ERR_INVALID_VALUE (bad desc or pointers, pages_per_seq or
+ *   num_pages <= 0, range outside [0, min(nsum, pages_per_seq)], k_pages not
+ *   16-byte aligned); SAS_ERR_UNSUPPORTED as sas_pool_key_blocks.
+ */
+sas_status sas_pool_key_blocks_paged(const sas_decode_desc* desc, const void* k_pages, const int32_t* page_table,
+                                     int32_t pages_per_seq, int32_t num_pages, int32_t block_begin, int32_t block_end,
+                                     void* ksum, int32_t nsum, sas_stream_t stream);
 sas_status sas_decode_scores(const sas_decode_desc* desc, const void* q, const void* ksum, int32_t nsum,
                              const int32_t* ctx_len, float* s, int32_t s_cols, sas_stream_t stream);
 

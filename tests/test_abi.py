@@ -174,3 +174,9 @@ def test_scorer_checks(api):
     assert L.sas_decode_scores(ctypes.byref(dd), FAKE, FAKE, 16, None, FAKE, 16, None) == 1
     d96 = api.DecodeDesc(2, 8, 2, 96, 64, 4, 1000, 1, 0.0)
     assert L.sas_decode_scores(ctypes.byref(d96), FAKE, FAKE, 16, FAKE, FAKE, 16, None) == 2
+    P = L.sas_pool_key_blocks_paged
+    assert P(ctypes.byref(dd), None, FAKE, 16, 40, 0, 4, FAKE, 16, None) == 1
+    assert P(ctypes.byref(dd), FAKE, FAKE, 0, 40, 0, 4, FAKE, 16, None) == 1    # pages_per_seq
+    assert P(ctypes.byref(dd), FAKE, FAKE, 16, 40, 0, 17, FAKE, 20, None) == 1  # past pages_per_seq
+    assert P(ctypes.byref(dd), FAKE, FAKE, 16, 40, 0, 17, FAKE, 16, None) == 1  # past nsum
+    assert P(ctypes.byref(dd), ctypes.c_void_p(0x1008), FAKE, 16, 40, 0, 4, FAKE, 16, None) == 1  # misaligned

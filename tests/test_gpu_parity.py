@@ -621,3 +621,30 @@ def test_decode_scores_match_oracle(api, dtype, d):
     Cb = (ctx.cpu().numpy() - 1) // bs
     for b in range(B):
         assert torch.all(s[b, :, int(Cb[b]):] == 0)
+
+
+def test_paged_key_summaries_match_contiguous(api):
+    """Summaries pooled from a shuffled page pool equal, bit for bit, those pooled
+    from the contiguous cache (same rows, same order of the sums); a page id
+    outside the pool gives a zero summary."""
+    B, Hq, Hkv, d, bs, Tmax = 3, 8, 2, 128, 64, 64 * 40 + 5
+    q = _seeded((B, Hq, d), 1.0, torch.bfloat16, 81)
+    kc = _seeded((B, Hkv, Tmax, d), 1.0, torch.bfloat16, 82)
+    vc = _seeded((B, Hkv, Tmax, d), 1.0, torch.bfloat16, 83)
+    kp, _, table = _paged_from_cache(kc, vc, bs, 84)
+    desc = api.decode_desc(q, kc, bs, 4)
+    nsum = 40
+    want = torch.zeros((B, Hkv, nsum, d), dtype=torch.bfloat16, device="cuda")
+    got = torch.full_like(want, float("nan"))
+    api.sas_pool_key_blocks(desc, kc, 0, nsum, want)
+    api.sas_pool_key_blocks_paged(desc, kp, table, 0, 17, got)
+    api.sas_pool_key_blocks_paged(desc, kp, table, 17, nsum, got)
+    bad = table.clone()
+    bad[1, 5] = kp.shape[0] + 7
+    got_bad = torch.full_like(want, float("nan"))
+    api.sas_pool_key_blocks_paged(desc, kp, bad, 0, nsum, got_bad)
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
+    assert torch.all(got_bad[1, :, 5] == 0)
+    got_bad[1, :, 5] = want[1, :, 5]
+    assert torch.equal(got_bad, want)

@@ -84,6 +84,8 @@ lib.sas_pooled_scores.restype = ctypes.c_int
 lib.sas_pooled_scores.argtypes = [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _sz, _vp]
 lib.sas_pool_key_blocks.restype = ctypes.c_int
 lib.sas_pool_key_blocks.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _i32, _i32, _vp, _i32, _vp]
+lib.sas_pool_key_blocks_paged.restype = ctypes.c_int
+lib.sas_pool_key_blocks_paged.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp]
 lib.sas_decode_scores.restype = ctypes.c_int
 lib.sas_decode_scores.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _vp, _i32, _vp, _vp, _i32, _vp]
 
@@ -199,6 +201,14 @@ def sas_pool_key_blocks(desc, k_cache, block_begin: int, block_end: int, ksum, s
     contiguous cache into ksum [B,Hkv,nsum,d] (the cache's dtype)."""
     _check(lib.sas_pool_key_blocks(ctypes.byref(desc), _p(k_cache), block_begin, block_end, _p(ksum), ksum.shape[2],
                                    _stream(stream)), "sas_pool_key_blocks")
+
+
+def sas_pool_key_blocks_paged(desc, k_pages, page_table, block_begin: int, block_end: int, ksum, stream=None):
+    """Block summaries from a paged pool k_pages [num_pages, block_size, Hkv, d]
+    with page_table [B, pages_per_seq] int32, into ksum [B,Hkv,nsum,d]."""
+    _check(lib.sas_pool_key_blocks_paged(ctypes.byref(desc), _p(k_pages), _p(page_table), page_table.shape[1],
+                                         k_pages.shape[0], block_begin, block_end, _p(ksum), ksum.shape[2],
+                                         _stream(stream)), "sas_pool_key_blocks_paged")
 
 
 def sas_decode_scores(desc, q, ksum, ctx_len, s, stream=None):

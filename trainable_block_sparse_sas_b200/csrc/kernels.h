@@ -94,6 +94,7 @@ bool pool_shape_ok(int d, int G, int elem_bytes);
 size_t pooled_scores_workspace(const TrainParams& p);
 cudaError_t launch_pooled_scores(const TrainParams& p, float* s, void* ws, cudaStream_t stream);
 cudaError_t launch_pool_keys(const DecodeParams& p, int m0, int m1, void* ksum, int nsum, cudaStream_t stream);
+cudaError_t launch_pool_keys_paged(const DecodeParams& p, int m0, int m1, void* ksum, int nsum, cudaStream_t stream);
 cudaError_t launch_decode_scores(const DecodeParams& p, const void* ksum, int nsum, float* s, int s_cols,
                                  cudaStream_t stream);
 size_t simt_max_smem(int D, int BS, int Cq);

@@ -268,6 +268,25 @@ sas_status sas_pool_key_blocks(const sas_decode_desc* desc, const void* k_cache,
     return from_cuda(launch_pool_keys(p, block_begin, block_end, ksum, nsum, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+sas_status sas_pool_key_blocks_paged(const sas_decode_desc* desc, const void* k_pages, const int32_t* page_table,
+                                     int32_t pages_per_seq, int32_t num_pages, int32_t block_begin, int32_t block_end,
+                                     void* ksum, int32_t nsum, sas_stream_t stream) {
+    if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!k_pages || !page_table || !ksum || pages_per_seq <= 0 || num_pages <= 0) return SAS_ERR_INVALID_VALUE;
+    if (block_begin < 0 || block_end < block_begin || block_end > nsum || block_end > pages_per_seq)
+        return SAS_ERR_INVALID_VALUE;
+    const int eb = desc->dtype == SAS_BF16 ? 2 : 4;
+    if (!pool_shape_ok(desc->head_dim, 1, eb)) return SAS_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(k_pages) & 15u) return SAS_ERR_INVALID_VALUE;
+    DecodeParams p = make_decode(desc);
+    p.k = k_pages;
+    p.page_table = page_table;
+    p.pages_per_seq = pages_per_seq;
+    p.num_pages = num_pages;
+    return from_cuda(
+        launch_pool_keys_paged(p, block_begin, block_end, ksum, nsum, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sas_status sas_decode_scores(const sas_decode_desc* desc, const void* q, const void* ksum, int32_t nsum,
                              const int32_t* ctx_len, float* s, int32_t s_cols, sas_stream_t stream) {
     if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;

@@ -187,6 +187,27 @@ __global__ void __launch_bounds__(kPoolThreads) pool_keys_kernel(const T* __rest
     for (int e = threadIdx.x; e < d; e += kPoolThreads) ksum[(bh * nsum + m) * d + e] = from_f32<T>(mean[e]);
 }
 
+// The same over a paged pool [num_pages, b, Hkv, d]: block m of sequence b is the
+// page page_table[b * pps + m]; a page id outside the pool gives a zero summary
+template <typename T>
+__global__ void __launch_bounds__(kPoolThreads) pool_keys_paged_kernel(const T* __restrict__ kp,
+                                                                       const int32_t* __restrict__ table, int pps,
+                                                                       int num_pages, int Hkv, int d, int bs, int m0,
+                                                                       int nblk, int nsum, T* __restrict__ ksum) {
+    __shared__ float red[kPoolThreads * 8];
+    __shared__ float mean[256];
+    const long bh = blockIdx.x / nblk;
+    const int m = m0 + (int)(blockIdx.x % nblk);
+    const int b = (int)(bh / Hkv), h = (int)(bh % Hkv);
+    const int page = table[(long)b * pps + m];
+    if (page < 0 || page >= num_pages) {
+        for (int e = threadIdx.x; e < d; e += kPoolThreads) ksum[(bh * nsum + m) * d + e] = from_f32<T>(0.f);
+        return;
+    }
+    pool_rows<T>(kp + ((long)page * bs * Hkv + h) * d, (long)Hkv * d, bs, d, 1, red, 1.f / (float)bs, mean);
+    for (int e = threadIdx.x; e < d; e += kPoolThreads) ksum[(bh * nsum + m) * d + e] = from_f32<T>(mean[e]);
+}
+
 // EPL consecutive elements (2 or 4) as floats, one vector load
 template <typename T, int EPL>
 __device__ __forceinline__ void load_lane(const T* p, float* x) {
@@ -327,6 +348,23 @@ cudaError_t launch_pool_keys(const DecodeParams& p, int m0, int m1, void* ksum, 
     else
         pool_keys_kernel<float><<<(unsigned)grid, kPoolThreads, 0, stream>>>(
             static_cast<const float*>(p.k), p.Hkv, p.Tmax, p.d, p.bs, m0, m1 - m0, nsum, static_cast<float*>(ksum));
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) count_launch();
+    return err;
+}
+
+cudaError_t launch_pool_keys_paged(const DecodeParams& p, int m0, int m1, void* ksum, int nsum, cudaStream_t stream) {
+    const long grid = (long)p.B * p.Hkv * (m1 - m0);
+    if (grid <= 0) return cudaSuccess;
+    if (grid > 0x7fffffffL) return cudaErrorInvalidValue;
+    if (p.is_bf16)
+        pool_keys_paged_kernel<__nv_bfloat16><<<(unsigned)grid, kPoolThreads, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(p.k), p.page_table, p.pages_per_seq, p.num_pages, p.Hkv, p.d, p.bs, m0,
+            m1 - m0, nsum, static_cast<__nv_bfloat16*>(ksum));
+    else
+        pool_keys_paged_kernel<float><<<(unsigned)grid, kPoolThreads, 0, stream>>>(
+            static_cast<const float*>(p.k), p.page_table, p.pages_per_seq, p.num_pages, p.Hkv, p.d, p.bs, m0, m1 - m0,
+            nsum, static_cast<float*>(ksum));
     cudaError_t err = cudaGetLastError();
     if (err == cudaSuccess) count_launch();
     return err;
