@@ -180,3 +180,20 @@ def test_scorer_checks(api):
     assert P(ctypes.byref(dd), FAKE, FAKE, 16, 40, 0, 17, FAKE, 20, None) == 1  # past pages_per_seq
     assert P(ctypes.byref(dd), FAKE, FAKE, 16, 40, 0, 17, FAKE, 16, None) == 1  # past nsum
     assert P(ctypes.byref(dd), ctypes.c_void_p(0x1008), FAKE, 16, 40, 0, 4, FAKE, 16, None) == 1  # misaligned
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """A copy of the package without libsas.so cannot be imported: the binding
+    raises instead of falling back to anything."""
+    import shutil
+    import sys
+
+    src = os.path.join(ROOT, "trainable_block_sparse_sas_b200")
+    dst = tmp_path / "trainable_block_sparse_sas_b200"
+    dst.mkdir()
+    for f in ("__init__.py", "api.py", "synthetic.py"):
+        shutil.copy(os.path.join(src, f), dst / f)
+    r = subprocess.run([sys.executable, "-c", "import trainable_block_sparse_sas_b200.api"], cwd=tmp_path,
+                       capture_output=True, text=True, env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode != 0
+    assert "libsas.so not built" in r.stderr
