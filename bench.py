@@ -381,6 +381,28 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
     return statistics.median(times)
 
 
+def decode_oracle_sample(w) -> dict:
+    """The oracle's decode (selection + attention, fp64) timed on the host cores
+    on a bounded sample of the workload: sequence 0 and kv head 0 (its G query
+    heads) at the full context length, reported as GB/s of that row's algorithmic
+    bytes (the decode_bytes count for one row)."""
+    import oracle
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    inp = syn.decode_inputs(w, device="cuda", seed=3000)
+    G = w.Hq // w.Hkv
+    host = {"q": syn.bf16_bits(inp["q"][0:1, 0:G]), "k": syn.bf16_bits(inp["k_cache"][0:1, 0:1]),
+            "v": syn.bf16_bits(inp["v_cache"][0:1, 0:1]), "s": inp["s"][0:1, 0:1].cpu().numpy(),
+            "ctx": inp["ctx_len"][0:1].cpu().numpy()}
+    del inp
+    t0 = time.perf_counter()
+    oracle.decode(host["q"], host["k"], host["v"], host["ctx"], host["s"], w.bs, w.top_k)
+    dt = time.perf_counter() - t0
+    by = decode_bytes(w) // (w.B * w.Hkv)
+    return {"value": by / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"sequence 0, kv head 0 ({G} query heads) at {w.T} tokens: {dt * 1e3:.1f} ms"}
+
+
 def time_decode_scores(api, w, hbm: float) -> dict:
     """Pooled-key decode scores over the workload's block summaries (one bf16 row
     per full block): the selector-scoring pass that precedes selection."""
@@ -618,6 +640,7 @@ def extras(api, args, peaks, peak_kind) -> dict:
                "two_call_ms": time_decode(api, w, steps=10, mode="two_call"),
                "paged_ms": time_decode(api, w, steps=10, mode="paged")}
         rec["decode_scores"] = time_decode_scores(api, w, hbm)
+        rec["cpu_oracle"] = decode_oracle_sample(w)
         if w is syn.DECODE_512K:
             msd = time_decode(api, w, steps=5, mode="dense")
             byd = decode_bytes(w, dense=True)
