@@ -569,6 +569,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     using L = DkvLayout;
     constexpr int G = 2 * MT;
     constexpr int kRowsTok = 128 / G;  // tokens per 128-row item
+    constexpr int kPreItems = kStages < MT ? kStages : MT;  // items of query block m, loaded up front
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(base);
@@ -623,6 +624,15 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             tma_load_3d(sK + kh * kSlab64, &a.tk, kv_full, kh * 64, h, krow);
             tma_load_3d(sV + kh * kSlab64, &a.tv, kv_full, kh * 64, h, krow);
         }
+        // so are the first items: query block m itself, which always attends m
+        for (int j = 0; j < kPreItems; ++j) {
+            const int qrow = b * a.n + m * kBS + j * kRowsTok;
+            mbar_arrive_expect_tx(qd_full(j), 4 * kSlab128);
+            for (int kh = 0; kh < 2; ++kh) {
+                tma_load_3d(sQ + (j * 2 + kh) * kSlab128, &a.tq, qd_full(j), kh * 64, h * G, qrow);
+                tma_load_3d(sDO + (j * 2 + kh) * kSlab128, &a.tdo, qd_full(j), kh * 64, h * G, qrow);
+            }
+        }
     }
 
     // query blocks attending key block m: m itself, then every c > m holding m
@@ -648,7 +658,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
 
     if (warp == 0) {
         if (lane == 0) {
-            for (int j = 0; j < nitems; ++j) {
+            for (int j = kPreItems; j < nitems; ++j) {
                 const int st = j % kStages;
                 if (j >= kStages && !mbar_wait(qd_empty(st), (j / kStages - 1) & 1, abort_flag, a.status)) break;
                 const int c = list[j / MT], i = j % MT;

@@ -150,10 +150,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         mbar_arrive_expect_tx(q_full, 2 * L::kQHalf);
         tma_load_3d(sQ, &a.tq, q_full, 0, h * G, q_row);
         tma_load_3d(sQ + L::kQHalf, &a.tq, q_full, 64, h * G, q_row);
+        // the current block is the list's first entry: its K and V go out now too
+        mbar_arrive_expect_tx(kv_full(0), kStage);
+        for (int kh = 0; kh < 2; ++kh) {
+            tma_load_3d(sKV + kh * kSlab, &a.tk, kv_full(0), kh * 64, h, q_row);
+            tma_load_3d(sKV + 2 * kSlab + kh * kSlab, &a.tv, kv_full(0), kh * 64, h, q_row);
+        }
     }
     if (warp == 0) {
-        // attended history blocks (ascending) with their log-gate biases, then the
-        // current block (bias 0); lanes read the selection in parallel
+        // the current block (bias 0), then the attended history blocks (ascending)
+        // with their log-gate biases; lanes read the selection in parallel
         const float* srow = a.s + unit * a.Cq;
         const float lse_c = gate_softmax_family(a.gate) ? a.lse_s[unit] : 0.f;
         int cnt = 0;
@@ -165,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             const bool ok = v >= 0 && v < c;
             const unsigned bal = __ballot_sync(0xffffffffu, ok);
             if (ok) {
-                const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+                const int pos = 1 + cnt + __popc(bal & ((1u << lane) - 1u));
                 const float lg = gate_log(srow[v], lse_c, a.gate);
                 list[pos] = v;
                 bias2[pos] = gate_in_logits(a.gate) ? lg * kLog2e : 0.f;
@@ -174,9 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             cnt += __popc(bal);
         }
         if (lane == 0) {
-            list[cnt] = c;
-            bias2[cnt] = 0.f;
-            if (kOuter) wgt[cnt] = 1.f;
+            list[0] = c;
+            bias2[0] = 0.f;
+            if (kOuter) wgt[0] = 1.f;
             *list_count = cnt + 1;
         }
     }
@@ -192,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            for (int t = 0; t < nlist; ++t) {
+            for (int t = 1; t < nlist; ++t) {  // block 0 (the current block) was requested at start
                 const int s = t % kStages;
                 if (t >= kStages && !mbar_wait(kv_empty(s), (t / kStages - 1) & 1, abort_flag, a.status)) break;
                 mbar_arrive_expect_tx(kv_full(s), kStage);
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                 }
                 if (t == 0 && grp == 0 && quad == 0 && lane == 0) mbar_arrive(stagger);
                 tc_fence_after();
-                const bool cur = (t == nlist - 1);
+                const bool cur = (t == 0);
                 uint32_t r0[32], r1[32];
                 tmem_ld64_sync(tS + bf * 64, r0, r1);
                 // row max over the raw logits (sigma > 0), causal mask on the current block
