@@ -4,15 +4,17 @@
 //
 // o = softmax(sigma q K_S^T + log g_S) V_S (jaehun.me review of SAS, Eq. 9 and the
 // Kernel implementation paragraph): for query block c the attended key blocks
-// are its selected history blocks, each adding log g_m = s[c,m] - lse_s[c] to
-// its logits, then the current block c with bias 0 and a causal mask.
+// are the current block c with bias 0 and a causal mask (processed first, so its
+// K and V are requested before the list is built) and its selected history
+// blocks, each adding log g_m = s[c,m] - lse_s[c] to its logits.
 //
 // One CTA per (batch, kv head, query block).  The G query heads of the group
 // share the selection, so their 64 rows each are stacked into G*64 query rows
 // (row r = token * G + head, exactly the order of a TMA box over [token, head,
 // d]) and processed as G/2 M-tiles of 128 rows.  Attended key blocks go one at a
 // time (N = 64 keys) through a 4-stage shared-memory ring of K and V.
-//   warp 0      TMA producer: Q once, then K and V blocks by block index
+//   warp 0      TMA producer: K and V blocks of the list after the first (Q and the
+//               current block's K and V are requested at the start)
 //   warps 1..4  MMA issuers, two per M-tile (a single thread's chain of small
 //               MMAs is latency-bound; the chains run concurrently):
 //                 S_i = Q_i K^T   (SS MMA into TMEM buffer t mod 2 of tile i)
