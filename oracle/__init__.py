@@ -7,9 +7,11 @@ shares no code with the CUDA library: the arithmetic lives in ``sas_oracle.c``
 
 Every function follows a definition on the pages about SAS ("SAS: Simple
 Attention Sparsification via End-to-End Optimization of Context Ranking"); the
-C file cites each one.  Parity status: every function here is pinned by the
-``-m "not gpu"`` tests in ``tests/test_oracle_pins.py`` (worked example, closed
-forms, brute force, library special cases, finite differences).
+C file cites each one.  Parity status: every function here (selection, the
+gated forward and backward with every gate variant and the bf16-stored-output
+option, decode, and the pooled-key scorer) is pinned by the ``-m "not gpu"``
+tests in ``tests/test_oracle_pins.py`` (worked example, closed forms, brute
+force, dense torch formulations, finite differences, library special cases).
 """
 from __future__ import annotations
 

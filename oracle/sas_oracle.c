@@ -20,13 +20,22 @@
  *     (jaehun.me review, Kernel implementation paragraph) and carried to s
  *     through log g = s - LSE(s);
  *   - the inference rule I = Top-K(s, K) with no gate (jaehun.me review,
- *     walkthrough Step 6).
+ *     walkthrough Step 6);
+ *   - the ablated gates: log sigmoid(s) and raw logits inside the softmax, the
+ *     outer gate weighting the values, and the hard STE gate (jaehun.me review,
+ *     "Why the Four Design Choices Matter", Eq. 5 and Eq. 7; shibing624 review,
+ *     Fig. 2);
+ *   - a weight-free pooled-key scorer: mean-pooled query and key block summaries
+ *     and their scaled dot product (jaehun.me review, walkthrough Step 1 and
+ *     Limitations: pooling-based block summaries).
  * Readings where the pages are silent (all listed in the design notes):
  *   softmax scale sigma (default 1/sqrt(d)); one score row per (kv head, query
  *   block) shared by the query heads of a GQA group; 0-based blocks, history of
  *   query block c is m < c, current block causally masked token by token; ties in
  *   Top-K go to the lower block index (-0.0 == +0.0); selected lists ascending,
- *   padded with -1; ds = dlogg - g * sum(dlogg) over the history blocks.
+ *   padded with -1; ds = dlogg - g * sum(dlogg) over the history blocks; the
+ *   backward may read o as a bf16 tensor stores it (o_store); the STE passes
+ *   dL/dh straight through to g; the scorer pools by plain means.
  *
  * Everything is computed in double.  Inputs may be given as double, float or
  * bfloat16 bits; they are widened exactly on load.  Parallelism (OpenMP) only
