@@ -25,7 +25,8 @@
 //     S = Q K_m^T and dP = dO V_m^T                   (SS MMAs, double-buffered TMEM)
 //     softmax warps: P and dS as above, written as bf16 rows into swizzled smem
 //     dV^T += dO^T P and dK^T += Q^T dS               (SS MMAs, M = head_dim = 128)
-//   Epilogue: dk = sigma dK, dv = dV.
+//   Epilogue: dk = sigma dK, dv = dV.  The first items (query block m itself) are
+//   requested together with K and V, before the list of attending blocks is built.
 //
 // D_i is computed by the dq kernel's softmax threads (one row each): dO_i . o_i,
 // then corrected by delta_i; the corrected value is written to the workspace for

@@ -15,6 +15,13 @@
 //                P (dP - D), dq = sigma dS K, and the block-wise log-gate gradient
 //                dlogg[c,m] = sum of dS over the tile (jaehun.me review, Kernel
 //                implementation paragraph), then ds[c,:] = dlogg - g sum(dlogg).
+//                D here is dO . o of the stored output.
+//
+// Gate variants: the sigmoid and raw-logit gates change the bias and ds; the
+// outer gate weights V by g (dS = P (g dP - D), dv from g P, dlogg = g sum P dP);
+// the hard STE gate has bias 0, and its dq kernel also walks the dropped history
+// blocks (flagged negative in the block list) for their straight-through
+// gradient, giving dq nothing from them.
 //   bwd_dkdv     one CTA per (batch, kv head, key block m), looping over the query
 //                blocks that attend m (m itself, and every c > m whose selection
 //                holds m) and the group's heads: dv = P^T dO, dk = sigma dS^T Q.
