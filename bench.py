@@ -103,6 +103,7 @@ def kernel_sources_sha(names) -> str:
         with open(os.path.join(ROOT, "trainable_block_sparse_sas_b200", "csrc", n), encoding="utf-8") as f:
             code = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
         code = re.sub(r"//[^\n]*", "", code)
+        code = "\n".join(ln.strip() for ln in code.splitlines() if ln.strip())  # blank lines, indentation
         h.update(code.encode())
     return h.hexdigest()[:16]
 
