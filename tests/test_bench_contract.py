@@ -34,3 +34,23 @@ def test_reference_arm_prints_the_contract_line():
 def test_too_few_warmup_steps_are_refused():
     r = _run("--impl", "reference", "--steps", "1", "--warmup", "2")
     assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    """The traffic record stays valid through comment and blank-line edits and is
+    retired by any change to the code itself."""
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    csrc = tmp_path / "trainable_block_sparse_sas_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f = csrc / "k.cu"
+    f.write_text("int f(int a) {\n    return a + 1;  // one\n}\n")
+    base = bench.kernel_sources_sha(["k.cu"])
+    f.write_text("/* header */\nint f(int a) {\n\n    // a new comment line\n  return a + 1;\n}\n")
+    assert bench.kernel_sources_sha(["k.cu"]) == base
+    f.write_text("int f(int a) {\n    return a + 2;  // one\n}\n")
+    assert bench.kernel_sources_sha(["k.cu"]) != base
