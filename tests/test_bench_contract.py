@@ -54,3 +54,21 @@ def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     assert bench.kernel_sources_sha(["k.cu"]) == base
     f.write_text("int f(int a) {\n    return a + 2;  // one\n}\n")
     assert bench.kernel_sources_sha(["k.cu"]) != base
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Launched as the harness launches N > 1 (torchrun, one process per rank):
+    rank 0 alone prints the line and every rank exits 0."""
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+                        "--reference-tokens", "256"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["impl"] == "reference"
