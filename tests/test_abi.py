@@ -197,3 +197,41 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
                        capture_output=True, text=True, env={**os.environ, "PYTHONPATH": str(tmp_path)})
     assert r.returncode != 0
     assert "libsas.so not built" in r.stderr
+
+
+def test_binding_refuses_short_mistyped_strided_or_host_buffers(api):
+    """The binding checks each buffer against the descriptor before the C call
+    (the ABI sees pointers only, so a short buffer would be accessed out of
+    bounds on the GPU): size, then dtype, then layout, then device."""
+    import torch
+
+    q = torch.zeros((1, 256, 4, 128), dtype=torch.bfloat16)
+    k = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16)
+    desc = api.attn_desc(q, k, 64, 2)
+    s, lse_s = torch.zeros((1, 2, 4, 4)), torch.zeros((1, 2, 4))
+    idx = torch.zeros((1, 2, 4, 2), dtype=torch.int32)
+    o, lse = torch.zeros_like(q), torch.zeros((1, 4, 256))
+    with pytest.raises(ValueError, match="q holds"):
+        api.sas_gated_attn_fwd(desc, q[:, :128], k, k, s, lse_s, idx, o, lse)
+    with pytest.raises(ValueError, match="idx holds"):
+        api.sas_gated_attn_fwd(desc, q, k, k, s, lse_s, idx[..., :1], o, lse)
+    with pytest.raises(TypeError, match="k is torch.float32"):
+        api.sas_gated_attn_fwd(desc, q, k.float(), k, s, lse_s, idx, o, lse)
+    with pytest.raises(ValueError, match="contiguous"):
+        api.sas_gated_attn_fwd(desc, q.transpose(2, 3), k, k, s, lse_s, idx, o, lse)
+    with pytest.raises(ValueError, match="CUDA device"):
+        api.sas_gated_attn_fwd(desc, q, k, k, s, lse_s, idx, o, lse)
+    ds = torch.zeros_like(s)
+    with pytest.raises(ValueError, match="ds holds"):
+        api.sas_gated_attn_bwd(desc, q, k, k, o, lse, q, s, lse_s, idx, q, k, k, ds[:, :1], None)
+    qd = torch.zeros((2, 8, 128), dtype=torch.bfloat16)
+    kc = torch.zeros((2, 2, 1000, 128), dtype=torch.bfloat16)
+    dd = api.decode_desc(qd, kc, 64, 4)
+    ctx = torch.zeros((2,), dtype=torch.int32)
+    with pytest.raises(ValueError, match="v_cache holds"):
+        api.sas_sparse_decode(dd, qd, kc, kc[:1], ctx, None, torch.zeros_like(qd), None)
+    with pytest.raises(ValueError, match="idx holds"):
+        api.sas_sparse_decode(dd, qd, kc, kc, ctx, torch.zeros((2, 2, 3), dtype=torch.int32), torch.zeros_like(qd),
+                              None)
+    with pytest.raises(TypeError, match="ctx_len is torch.int64"):
+        api.sas_sparse_decode_select(dd, qd, kc, kc, ctx.long(), torch.zeros((2, 2, 15)), torch.zeros_like(qd))

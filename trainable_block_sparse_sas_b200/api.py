@@ -91,7 +91,13 @@ lib.sas_decode_scores.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _vp, _i32, _v
 
 
 def _p(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device pointer of a tensor for the C ABI (every libsas pointer is device
+    memory: a host tensor here would be dereferenced by a kernel)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libsas must be on a CUDA device")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream=None):
@@ -112,6 +118,61 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+# ---------------------------------------------------------------------------
+# buffer checks: the C ABI sees pointers only, so before each call the binding
+# makes sure every tensor holds the elements the descriptor implies, contiguously
+# and in the expected dtype (a short buffer would be read or written out of
+# bounds on the GPU); _p then refuses host tensors
+# ---------------------------------------------------------------------------
+
+_I32 = (torch.int32,)
+_F32 = (torch.float32,)
+
+
+def _dt(desc):
+    return (torch.bfloat16,) if desc.dtype == SAS_BF16 else (torch.float32,)
+
+
+def _need(t, numel: int, dtypes, name: str, optional: bool = False):
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call uses {numel}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} is {t.dtype}; expected {' or '.join(str(d) for d in dtypes)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _train_sizes(desc):
+    Cq = desc.seq_len // desc.block_size if desc.block_size > 0 else 0
+    q = desc.batch * desc.seq_len * desc.n_q_heads * desc.head_dim
+    kv = desc.batch * desc.seq_len * desc.n_kv_heads * desc.head_dim
+    return Cq, q, kv
+
+
+def _check_train(desc, q, k, v, s, lse_s, idx):
+    Cq, nq, nkv = _train_sizes(desc)
+    dt = _dt(desc)
+    _need(q, nq, dt, "q")
+    _need(k, nkv, dt, "k")
+    _need(v, nkv, dt, "v")
+    _need(s, desc.batch * desc.n_kv_heads * Cq * Cq, _F32, "s")
+    _need(lse_s, desc.batch * desc.n_kv_heads * Cq, _F32, "lse_s", optional=True)
+    _need(idx, desc.batch * desc.n_kv_heads * Cq * max(desc.top_k, 0), _I32, "idx", optional=True)
+    return Cq, nq, nkv
+
+
+def _check_decode(desc, q, o, ctx_len):
+    dt = _dt(desc)
+    nq = desc.batch * desc.n_q_heads * desc.head_dim
+    _need(q, nq, dt, "q")
+    _need(o, nq, dt, "o", optional=o is None)
+    _need(ctx_len, desc.batch, _I32, "ctx_len")
+
+
 def attn_desc(q, k, block_size: int, top_k: int, full_scope: bool = False, softmax_scale: float = 0.0,
               gate: str = "softmax") -> AttnDesc:
     """gate: "softmax" (log g = s - LSE(s), the method), "sigmoid" (log sigmoid(s)),
@@ -130,12 +191,19 @@ def decode_desc(q, k_cache, block_size: int, top_k: int, softmax_scale: float = 
 def sas_topk_select(s, n_rows, row_len, top_k, idx=None, lse_s=None, ctx_len=None, block_size=0, stream=None):
     """s [B, Hkv, n_rows, row_len] fp32 -> writes idx [B,Hkv,n_rows,top_k] int32 and/or lse_s."""
     B, Hkv = s.shape[0], s.shape[1]
+    _need(s, B * Hkv * n_rows * row_len, _F32, "s")
+    _need(idx, B * Hkv * n_rows * max(top_k, 0), _I32, "idx", optional=True)
+    _need(lse_s, B * Hkv * n_rows, _F32, "lse_s", optional=True)
+    _need(ctx_len, B, _I32, "ctx_len", optional=True)
     st = lib.sas_topk_select(_p(s), B, Hkv, n_rows, row_len, _p(ctx_len), block_size, top_k, _p(idx), _p(lse_s),
                              _stream(stream))
     _check(st, "sas_topk_select")
 
 
 def sas_gated_attn_fwd(desc, q, k, v, s, lse_s, idx, o, lse, stream=None):
+    _, nq, _ = _check_train(desc, q, k, v, s, lse_s, idx)
+    _need(o, nq, _dt(desc), "o")
+    _need(lse, desc.batch * desc.n_q_heads * desc.seq_len, _F32, "lse")
     _check(lib.sas_gated_attn_fwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(s), _p(lse_s), _p(idx), _p(o), _p(lse),
                                   _stream(stream)), "sas_gated_attn_fwd")
 
@@ -145,6 +213,12 @@ def sas_gated_attn_bwd_workspace_size(desc) -> int:
 
 
 def sas_gated_attn_bwd(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, workspace, stream=None):
+    Cq, nq, nkv = _check_train(desc, q, k, v, s, lse_s, idx)
+    dt = _dt(desc)
+    for t, n, name in ((o, nq, "o"), (dO, nq, "dO"), (dq, nq, "dq"), (dk, nkv, "dk"), (dv, nkv, "dv")):
+        _need(t, n, dt, name)
+    _need(lse, desc.batch * desc.n_q_heads * desc.seq_len, _F32, "lse")
+    _need(ds, desc.batch * desc.n_kv_heads * Cq * Cq, _F32, "ds")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.sas_gated_attn_bwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dO), _p(s), _p(lse_s),
                                   _p(idx), _p(dq), _p(dk), _p(dv), _p(ds), _p(workspace), ws_bytes, _stream(stream)),
@@ -155,7 +229,16 @@ def sas_sparse_decode_workspace_size(desc) -> int:
     return int(lib.sas_sparse_decode_workspace_size(ctypes.byref(desc)))
 
 
+def _check_cache(desc, k_cache, v_cache):
+    n = desc.batch * desc.n_kv_heads * desc.max_ctx * desc.head_dim
+    _need(k_cache, n, _dt(desc), "k_cache")
+    _need(v_cache, n, _dt(desc), "v_cache")
+
+
 def sas_sparse_decode(desc, q, k_cache, v_cache, ctx_len, idx, o, workspace, stream=None):
+    _check_decode(desc, q, o, ctx_len)
+    _check_cache(desc, k_cache, v_cache)
+    _need(idx, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx", optional=True)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.sas_sparse_decode(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx), _p(o),
                                  _p(workspace), ws_bytes, _stream(stream)), "sas_sparse_decode")
@@ -163,6 +246,10 @@ def sas_sparse_decode(desc, q, k_cache, v_cache, ctx_len, idx, o, workspace, str
 
 def sas_sparse_decode_select(desc, q, k_cache, v_cache, ctx_len, s, o, idx_out=None, stream=None):
     """Fused decode step: Top-K of s [B, Hkv, s_cols] and the gate-free attention."""
+    _check_decode(desc, q, o, ctx_len)
+    _check_cache(desc, k_cache, v_cache)
+    _need(s, desc.batch * desc.n_kv_heads * s.shape[-1], _F32, "s")
+    _need(idx_out, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx_out", optional=True)
     _check(lib.sas_sparse_decode_select(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(s),
                                         s.shape[-1], _p(o), _p(idx_out), _stream(stream)), "sas_sparse_decode_select")
 
@@ -178,6 +265,15 @@ def sas_sparse_decode_paged(desc, q, k_pages, v_pages, page_table, ctx_len, o, s
     """Decode step over a paged cache: page_table [B, pages_per_seq] int32 maps a
     sequence's blocks to pages of k_pages / v_pages [num_pages, block_size, Hkv, d].
     Blocks from the Top-K of s (fused), from idx, or every block when both are None."""
+    _check_decode(desc, q, o, ctx_len)
+    pool = k_pages.shape[0] * desc.block_size * desc.n_kv_heads * desc.head_dim
+    _need(k_pages, pool, _dt(desc), "k_pages")
+    _need(v_pages, pool, _dt(desc), "v_pages")
+    _need(page_table, desc.batch * page_table.shape[1], _I32, "page_table")
+    if s is not None:
+        _need(s, desc.batch * desc.n_kv_heads * s.shape[-1], _F32, "s")
+    _need(idx, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx", optional=True)
+    _need(idx_out, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx_out", optional=True)
     _check(lib.sas_sparse_decode_paged(ctypes.byref(desc), _p(q), _p(k_pages), _p(v_pages), _p(page_table),
                                        page_table.shape[1], k_pages.shape[0], _p(ctx_len), _p(idx), _p(s),
                                        0 if s is None else s.shape[-1], _p(o), _p(idx_out), _stream(stream)),
@@ -191,6 +287,10 @@ def sas_pooled_scores_workspace_size(desc) -> int:
 def sas_pooled_scores(desc, q, k, s, workspace, stream=None):
     """Pooled-key scores, training shape: s [B,Hkv,Cq,Cq] fp32 (m < c), from the
     mean of q over each query block and group and the mean of k over each block."""
+    Cq, nq, nkv = _train_sizes(desc)
+    _need(q, nq, _dt(desc), "q")
+    _need(k, nkv, _dt(desc), "k")
+    _need(s, desc.batch * desc.n_kv_heads * Cq * Cq, _F32, "s")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.sas_pooled_scores(ctypes.byref(desc), _p(q), _p(k), _p(s), _p(workspace), ws_bytes, _stream(stream)),
            "sas_pooled_scores")
@@ -199,6 +299,8 @@ def sas_pooled_scores(desc, q, k, s, workspace, stream=None):
 def sas_pool_key_blocks(desc, k_cache, block_begin: int, block_end: int, ksum, stream=None):
     """Mean-pooled summaries of the full blocks [block_begin, block_end) of a
     contiguous cache into ksum [B,Hkv,nsum,d] (the cache's dtype)."""
+    _need(k_cache, desc.batch * desc.n_kv_heads * desc.max_ctx * desc.head_dim, _dt(desc), "k_cache")
+    _need(ksum, desc.batch * desc.n_kv_heads * ksum.shape[2] * desc.head_dim, _dt(desc), "ksum")
     _check(lib.sas_pool_key_blocks(ctypes.byref(desc), _p(k_cache), block_begin, block_end, _p(ksum), ksum.shape[2],
                                    _stream(stream)), "sas_pool_key_blocks")
 
@@ -206,6 +308,9 @@ def sas_pool_key_blocks(desc, k_cache, block_begin: int, block_end: int, ksum, s
 def sas_pool_key_blocks_paged(desc, k_pages, page_table, block_begin: int, block_end: int, ksum, stream=None):
     """Block summaries from a paged pool k_pages [num_pages, block_size, Hkv, d]
     with page_table [B, pages_per_seq] int32, into ksum [B,Hkv,nsum,d]."""
+    _need(k_pages, k_pages.shape[0] * desc.block_size * desc.n_kv_heads * desc.head_dim, _dt(desc), "k_pages")
+    _need(page_table, desc.batch * page_table.shape[1], _I32, "page_table")
+    _need(ksum, desc.batch * desc.n_kv_heads * ksum.shape[2] * desc.head_dim, _dt(desc), "ksum")
     _check(lib.sas_pool_key_blocks_paged(ctypes.byref(desc), _p(k_pages), _p(page_table), page_table.shape[1],
                                          k_pages.shape[0], block_begin, block_end, _p(ksum), ksum.shape[2],
                                          _stream(stream)), "sas_pool_key_blocks_paged")
@@ -213,6 +318,9 @@ def sas_pool_key_blocks_paged(desc, k_pages, page_table, block_begin: int, block
 
 def sas_decode_scores(desc, q, ksum, ctx_len, s, stream=None):
     """Decode scores s [B,Hkv,s_cols] fp32 from the block summaries ksum."""
+    _check_decode(desc, q, None, ctx_len)
+    _need(ksum, desc.batch * desc.n_kv_heads * ksum.shape[2] * desc.head_dim, _dt(desc), "ksum")
+    _need(s, desc.batch * desc.n_kv_heads * s.shape[-1], _F32, "s")
     _check(lib.sas_decode_scores(ctypes.byref(desc), _p(q), _p(ksum), ksum.shape[2], _p(ctx_len), _p(s), s.shape[-1],
                                  _stream(stream)), "sas_decode_scores")
 
@@ -221,6 +329,9 @@ def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream
     """sas_sparse_decode without a workspace, for callers that cannot allocate
     device memory: the partials use a fixed 4 MiB array inside the library.
     Overlapping calls race on that array."""
+    _check_decode(desc, q, o, ctx_len)
+    _check_cache(desc, k_cache, v_cache)
+    _need(idx, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx", optional=True)
     _check(lib.sas_sparse_decode_noalloc(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx),
                                          _p(o), _stream(stream)), "sas_sparse_decode_noalloc")
 
