@@ -39,7 +39,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_agree_on_max_timing():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of this multi-threaded process
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     for rank in range(world):
         ms_max, value, same_batch = out[rank]
