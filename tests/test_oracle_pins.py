@@ -769,3 +769,25 @@ def test_decode_pooled_scores_brute_force():
     np.testing.assert_array_equal(part[:, :, 2:5], ksum[:, :, 2:5])
     r = oracle.pool_keys(kc, bs, 0, nsum, nsum, round_bf16=True)
     np.testing.assert_array_equal(r, _nearest_bf16(ksum))
+
+
+@pytest.mark.parametrize("gate", ["softmax", "outer", "ste"])
+def test_softmax_family_ds_rows_sum_to_zero_on_random_shapes(gate):
+    """Every gate built on g = softmax(s) passes its gradient to s through the
+    softmax's vector-Jacobian product, so each ds row sums to zero, whatever the
+    shape, budget or scope."""
+    rng = np.random.default_rng(50)
+    for _ in range(4):
+        bs = int(rng.choice([4, 8]))
+        Cq = int(rng.integers(2, 7))
+        Hkv = int(rng.integers(1, 3))
+        G = int(rng.choice([1, 2, 3]))
+        d = int(rng.choice([4, 8]))
+        K = int(rng.integers(0, Cq + 1))
+        full = bool(rng.integers(0, 2)) and gate != "ste"
+        q, k, v, s, dO = _rand_train(rng, 1, Cq * bs, Hkv * G, Hkv, d, bs)
+        out = oracle.attn_bwd(q, k, v, dO, s, bs, K, full_scope=full, gate=gate)
+        for h in range(Hkv):
+            for c in range(Cq):
+                assert abs(out["ds"][0, h, c, :c].sum()) < 1e-12, (gate, bs, Cq, K, full, h, c)
+                assert np.all(out["ds"][0, h, c, c:] == 0)
