@@ -6,8 +6,12 @@ One step = the whole training hot path over one batch of the 32K workload
 Top-K selection, the gated forward, and the backward with dq/dk/dv and ds.
 The metric counts tensor-core FLOPs on selected blocks only (4d per attended
 (query, key) pair forward, 10d backward; the current block counts its causal
-b(b+1)/2 pairs).  Extras (single GPU): full-scope 16K training, and the two
-decode workloads (selection included) in GB/s of algorithmic bytes.
+b(b+1)/2 pairs).  Extras (single GPU): full-scope 16K training, the four
+ablated gates on the 32K workload, the pooled-key scorer, and the two decode
+workloads (selection included; contiguous, two-call, paged and dense forms) in
+GB/s of algorithmic bytes, each decode workload with the oracle timed on a
+bounded host sample.  `e2e` repeats the 32K step through pinned host buffers,
+every step copying its inputs in and its outputs out.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
