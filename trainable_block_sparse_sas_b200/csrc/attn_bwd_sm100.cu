@@ -923,7 +923,6 @@ size_t bwd_sm100_workspace(const TrainParams& p) {
 
 bool bwd_sm100_supported(const TrainParams& p) {
     if (!bwd_sm100_shape(p) || !p.Mbuf) return false;
-    const int G = p.Hq / p.Hkv;
     const uintptr_t al = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
                          reinterpret_cast<uintptr_t>(p.v) | reinterpret_cast<uintptr_t>(p.dO) |
                          reinterpret_cast<uintptr_t>(p.dq) | reinterpret_cast<uintptr_t>(p.dk) |
