@@ -18,6 +18,16 @@
  *   - Arguments are checked on the host before anything is launched; a failed
  *     check returns an error code and has no side effect.  Launch failures
  *     return SAS_ERR_CUDA.  Nothing aborts, traps or throws across the ABI.
+ *   - Device-side failures are reported through a status word the caller owns:
+ *     one int32 of device memory, passed as `status` to every call whose kernels
+ *     wait on one another inside the GPU (the attention forward and backward,
+ *     and the decode calls).  Every such wait gives up after a bounded time; the
+ *     kernel then writes SAS_ERR_DEVICE_TIMEOUT into the word it was given, stops
+ *     its work (its outputs are then undefined) and returns, leaving the context
+ *     usable.  The word must hold 0 before its first use; sas_get_device_status
+ *     reads and clears it.  A call writes only the word it is given, so callers
+ *     that want their own report (a stream each, a thread each) pass their own
+ *     word; the library keeps no mutable state of its own.
  *   - Layouts are row-major with the last index contiguous:
  *       training  q, o, dO, dq : [B, n, Hq, d]     k, v, dk, dv : [B, n, Hkv, d]
  *                 s, ds        : [B, Hkv, Cq, Cq]  (Cq = n / b; row c scores the
@@ -143,6 +153,7 @@ sas_status sas_topk_select(const float* s, int32_t batch, int32_t n_kv_heads, in
  *          fp32 (from sas_topk_select), may be NULL for the SIGMOID and RAW gates;
  *          idx [B,Hkv,Cq,K] (sparse scope; NULL in full scope).
  * o        out, same dtype and layout as q.   lse out [B,Hq,n] fp32.
+ * status   the caller's device status word (see the conventions above).
  * Errors: SAS_ERR_INVALID_VALUE (null pointers, seq_len % block_size != 0,
  *         n_q_heads % n_kv_heads != 0, sizes <= 0, top_k < 0, idx NULL in
  *         sparse scope with top_k > 0); SAS_ERR_UNSUPPORTED (head_dim not 64 or
@@ -150,7 +161,7 @@ sas_status sas_topk_select(const float* s, int32_t batch, int32_t n_kv_heads, in
  */
 sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
                               const float* s, const float* lse_s, const int32_t* idx, void* o, float* lse,
-                              sas_stream_t stream);
+                              int32_t* status, sas_stream_t stream);
 
 /* Bytes of workspace sas_gated_attn_bwd needs for this problem (0 on bad desc). */
 size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc);
@@ -173,12 +184,27 @@ size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc);
  *              (dO_i.v_j - D_i) over every history block m < c.
  * o, lse   the forward's outputs.   dq, dk, dv out (dtype of q), ds out fp32.
  * workspace, ws_bytes  caller scratch of at least the queried size.
+ * status   the caller's device status word.
  * Errors: as sas_gated_attn_fwd, plus SAS_ERR_WORKSPACE_TOO_SMALL.
  */
 sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
                               const void* o, const float* lse, const void* dO, const float* s, const float* lse_s,
                               const int32_t* idx, void* dq, void* dk, void* dv, float* ds, void* workspace,
-                              size_t ws_bytes, sas_stream_t stream);
+                              size_t ws_bytes, int32_t* status, sas_stream_t stream);
+
+/*
+ * sas_gated_attn_bwd_timed -- sas_gated_attn_bwd with CUDA events recorded on
+ *   `stream` around its two kernels, so that each can be timed live: events[0]
+ *   before the first (dq and ds, query-major), events[1] between it and the
+ *   second (dk and dv, key-major), events[2] after the second.  events holds
+ *   three cudaEvent_t (as void*) the caller created; nothing else differs.
+ * Errors: as sas_gated_attn_bwd; SAS_ERR_INVALID_VALUE for NULL events.
+ */
+sas_status sas_gated_attn_bwd_timed(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
+                                    const void* o, const float* lse, const void* dO, const float* s,
+                                    const float* lse_s, const int32_t* idx, void* dq, void* dk, void* dv, float* ds,
+                                    void* workspace, size_t ws_bytes, void* const* events, int32_t* status,
+                                    sas_stream_t stream);
 
 /*
  * Parameter-free pooled-key scorer (jaehun.me review, walkthrough Step 1: scores
@@ -253,14 +279,15 @@ size_t sas_sparse_decode_workspace_size(const sas_decode_desc* desc);
  *          decode mode, or NULL for dense attention over all ctx_len[b] tokens
  *          (the full-attention comparator).
  * o        out [B,Hq,d], dtype of q.
+ * status   the caller's device status word.
  * Errors: SAS_ERR_INVALID_VALUE (null pointers, sizes <= 0, heads not divisible,
- *         top_k < 0); SAS_ERR_UNSUPPORTED (head_dim != 128 for bf16 / not 64 or
- *         128 for fp32, block_size not a multiple of 16 up to 256);
- *         SAS_ERR_WORKSPACE_TOO_SMALL.
+ *         top_k < 0); SAS_ERR_UNSUPPORTED (head_dim not 64 or 128, block_size
+ *         not a multiple of 16 up to 256, more than 16 query heads per kv
+ *         head); SAS_ERR_WORKSPACE_TOO_SMALL.
  */
 sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* ctx_len, const int32_t* idx, void* o, void* workspace, size_t ws_bytes,
-                             sas_stream_t stream);
+                             int32_t* status, sas_stream_t stream);
 
 /*
  * sas_sparse_decode_select -- the decode step with its selection fused: the
@@ -275,11 +302,12 @@ sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const v
  *          -1 padded.
  * Other arguments as sas_sparse_decode.
  * Errors: as sas_sparse_decode; SAS_ERR_UNSUPPORTED unless dtype is bf16,
- *         head_dim 128, block_size 64 and at most 16 query heads per kv head.
+ *         head_dim 128, block_size 64, at most 16 query heads per kv head and
+ *         every pointer 16-byte aligned.
  */
 sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, const void* k_cache,
                                     const void* v_cache, const int32_t* ctx_len, const float* s, int32_t s_cols,
-                                    void* o, int32_t* idx_out, sas_stream_t stream);
+                                    void* o, int32_t* idx_out, int32_t* status, sas_stream_t stream);
 
 /*
  * sas_sparse_decode_paged -- the decode step over a paged KV cache, the form the
@@ -300,7 +328,7 @@ sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, 
  *          sas_sparse_decode_select (idx_out nullable, as there);
  * idx      else when idx != NULL, the given blocks, as sas_sparse_decode;
  *          else every block (dense comparator).
- * q, o     as sas_sparse_decode.
+ * q, o, status  as sas_sparse_decode.
  * Errors: SAS_ERR_INVALID_VALUE (null pointers, pages_per_seq or num_pages <= 0,
  *         max_ctx > pages_per_seq * block_size, s_cols <= 0 with s, unaligned
  *         pools); SAS_ERR_UNSUPPORTED unless dtype is bf16, head_dim 128,
@@ -309,24 +337,29 @@ sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, 
 sas_status sas_sparse_decode_paged(const sas_decode_desc* desc, const void* q, const void* k_pages,
                                    const void* v_pages, const int32_t* page_table, int32_t pages_per_seq,
                                    int32_t num_pages, const int32_t* ctx_len, const int32_t* idx, const float* s,
-                                   int32_t s_cols, void* o, int32_t* idx_out, sas_stream_t stream);
+                                   int32_t s_cols, void* o, int32_t* idx_out, int32_t* status, sas_stream_t stream);
 
 /*
- * sas_sparse_decode_noalloc -- the same decode as sas_sparse_decode (same
- *   arguments, layouts and results) for callers that cannot allocate device
- *   memory: a plugin whose host program owns all device memory, or a serving
- *   loop that may not call cudaMalloc (which synchronises the device) between
- *   steps.  It takes no workspace.  The paper has no counterpart to this entry
- *   point; it exists for those callers only.
- * Scratch: the split-K partials live in a fixed 4 MiB array inside the library
- *   (every GPU that loads the library holds it until the process exits).
- *   Problems whose partials need more than 4 MiB return
- *   SAS_ERR_WORKSPACE_TOO_SMALL before any launch; sparse calls of the Qwen3
- *   decode shapes need about 1.4 MiB, long dense calls may exceed the limit.
- * The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any stream
- *   capture.  It allocates nothing (no cudaMalloc or cudaFree, no allocating
- *   library routine).
+ * sas_sparse_decode_noalloc -- the decode of sas_sparse_decode (same arguments
+ *   apart from the workspace, same kernels, same results) for callers that
+ *   cannot allocate device memory: a plugin inside a host program that owns
+ *   every byte of device memory, or a serving loop that may not call cudaMalloc
+ *   (which synchronises the device) between decode steps.  It takes no
+ *   workspace.  The paper has no counterpart to this entry point; it exists for
+ *   those callers only.
+ * Scratch: problems the tensor-core decode kernel takes (bf16, head_dim 128,
+ *   block_size 64, at most 16 query heads per kv head, 16-byte aligned
+ *   pointers) need none.  The others run the split-K kernels, whose partials
+ *   live in a fixed 4 MiB array inside the library (every GPU that loads the
+ *   library holds it until the process exits); a problem whose partials need
+ *   more returns SAS_ERR_WORKSPACE_TOO_SMALL before any launch (long dense
+ *   calls can; sparse calls of the Qwen3 decode shapes need about 1.4 MiB).
+ * The first call on a device looks up the array's device address, once per
+ *   device, with that device current; make that first call before any stream
+ *   capture.  The address is kept for the life of the process, so a program
+ *   that resets a device (cudaDeviceReset) must not call this entry point on
+ *   that device afterwards.  Nothing is allocated (no cudaMalloc or cudaFree,
+ *   no allocating library routine).
  * All calls share the one array: each call writes every partial it later reads,
  *   so nothing has to start at zero, but calls that overlap on the GPU (other
  *   streams, other host threads) race on it and must be serialised by the caller.
@@ -335,20 +368,29 @@ sas_status sas_sparse_decode_paged(const sas_decode_desc* desc, const void* q, c
  */
 sas_status sas_sparse_decode_noalloc(const sas_decode_desc* desc, const void* q, const void* k_cache,
                                      const void* v_cache, const int32_t* ctx_len, const int32_t* idx, void* o,
-                                     sas_stream_t stream);
+                                     int32_t* status, sas_stream_t stream);
 
-/* Synchronises `stream`, then reports and clears the device-side status word that
- * bounded waits inside the kernels set when they give up: SAS_OK or
- * SAS_ERR_DEVICE_TIMEOUT (SAS_ERR_CUDA if the synchronisation itself fails). */
-sas_status sas_device_status(sas_stream_t stream);
+/* sas_get_device_status -- synchronises `stream`, then reads the caller's device
+ * status word and clears it: SAS_OK (the word held 0) or the code a kernel wrote
+ * there (SAS_ERR_DEVICE_TIMEOUT: a bounded wait gave up; the outputs of the calls
+ * since the last read are undefined).  SAS_ERR_CUDA if the synchronisation or the
+ * copy fails; SAS_ERR_INVALID_VALUE for a NULL word. */
+sas_status sas_get_device_status(int32_t* status, sas_stream_t stream);
 
-/* Self-test of the failure path: launches one thread that waits on an mbarrier
- * nothing ever arrives at, bounded by limit_ms (1..10000), exactly as the
- * tensor-core kernels bound their waits.  The wait gives up, records a timeout
- * in the device status word and returns: sas_device_status then reports
- * SAS_ERR_DEVICE_TIMEOUT once, and the context stays usable.  No fault, trap or
- * hang is involved.  Errors: SAS_ERR_INVALID_VALUE for a limit out of range. */
-sas_status sas_selftest_bounded_wait(int32_t limit_ms, sas_stream_t stream);
+/* sas_selftest_bounded_wait -- self-test of the failure path of the tensor-core
+ * kernels, without a fault.  One CTA allocates tensor memory, issues a
+ * tensor-core MMA and, from its MMA-issuing thread, waits on an mbarrier that
+ * nothing ever arrives at, through the same bounded-wait routine the kernels
+ * use, limited to limit_ms (1..10000) instead of their fixed limit.  The wait
+ * gives up and records SAS_ERR_DEVICE_TIMEOUT in *status; a second warp waiting
+ * on another such barrier sees the abort flag and leaves; the issuing thread
+ * drains its MMAs and the tensor memory is freed, exactly as in the kernels.
+ * trace (nullable, device int32 [4]) receives 1s for the phases reached: the
+ * wait gave up, the other warp left on the abort flag, the MMAs drained, the
+ * tensor memory was freed.  The context stays usable; no fault, trap or hang is
+ * involved.  Errors: SAS_ERR_INVALID_VALUE for a limit out of range or a NULL
+ * status word. */
+sas_status sas_selftest_bounded_wait(int32_t limit_ms, int32_t* status, int32_t* trace, sas_stream_t stream);
 
 /* Number of kernels this library has launched in this process (all devices),
  * counted on the host at each successful launch. */

@@ -67,22 +67,19 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every case below fails val
 ])
 def test_fwd_rejects_bad_descriptors(api, kw, status):
     d = _desc(api, **kw)
-    st = api.lib.sas_gated_attn_fwd(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None)
+    st = api.lib.sas_gated_attn_fwd(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None)
     assert st == status
 
 
 def test_fwd_rejects_null_pointers(api):
+    """Every pointer of the forward is required (idx only in sparse scope with
+    top_k > 0), the device status word included."""
     d = _desc(api)
-    args = [FAKE] * 8
-    for i in range(8):
+    args = [FAKE] * 9
+    for i in range(9):
         a = list(args)
         a[i] = None
-        if i == 5:  # idx
-            continue
         assert api.lib.sas_gated_attn_fwd(ctypes.byref(d), *a, None) == 1, i
-    a = list(args)
-    a[5] = None  # idx missing in sparse scope with top_k > 0
-    assert api.lib.sas_gated_attn_fwd(ctypes.byref(d), *a, None) == 1
 
 
 def test_bwd_checks_workspace(api):
@@ -90,8 +87,10 @@ def test_bwd_checks_workspace(api):
     need = api.lib.sas_gated_attn_bwd_workspace_size(ctypes.byref(d))
     assert need > 0 and need % 256 == 0
     args = [FAKE] * 13
-    st = api.lib.sas_gated_attn_bwd(ctypes.byref(d), *args, FAKE, need - 1, None)
+    st = api.lib.sas_gated_attn_bwd(ctypes.byref(d), *args, FAKE, need - 1, FAKE, None)
     assert st == 3
+    st = api.lib.sas_gated_attn_bwd(ctypes.byref(d), *args, FAKE, need, None, None)  # no status word
+    assert st == 1
     assert api.lib.sas_gated_attn_bwd_workspace_size(None) == 0
     bad = _desc(api, seq_len=100)
     assert api.lib.sas_gated_attn_bwd_workspace_size(ctypes.byref(bad)) == 0
@@ -101,14 +100,19 @@ def test_decode_checks(api):
     d = api.DecodeDesc(2, 8, 2, 128, 64, 4, 1000, 1, 0.0)
     need = api.lib.sas_sparse_decode_workspace_size(ctypes.byref(d))
     assert need > 0 and need % 256 == 0
-    st = api.lib.sas_sparse_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None)
-    assert st == 3
-    st = api.lib.sas_sparse_decode(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None)
-    assert st == 1
+    dec = api.lib.sas_sparse_decode
+    assert dec(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, FAKE, None) == 3
+    assert dec(ctypes.byref(d), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, FAKE, None) == 1
+    assert dec(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None, None) == 1  # no status word
     bad = api.DecodeDesc(2, 8, 3, 128, 64, 4, 1000, 1, 0.0)
-    assert api.lib.sas_sparse_decode(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 1
+    assert dec(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, FAKE, None) == 1
     uns = api.DecodeDesc(2, 8, 2, 96, 64, 4, 1000, 1, 0.0)
-    assert api.lib.sas_sparse_decode(ctypes.byref(uns), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 2
+    assert dec(ctypes.byref(uns), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, FAKE, None) == 2
+    sel = api.lib.sas_sparse_decode_select
+    assert sel(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 16, FAKE, None, None, None) == 1  # no status word
+    na = api.lib.sas_sparse_decode_noalloc
+    assert na(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None) == 1  # no status word
+    assert na(ctypes.byref(uns), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None) == 2
 
 
 def test_select_checks(api):
@@ -118,6 +122,16 @@ def test_select_checks(api):
     assert L.sas_topk_select(FAKE, 1, 1, 4, 4, None, 0, 2, None, None, None) == 1
     assert L.sas_topk_select(FAKE, 1, 1, 2, 4, FAKE, 64, 2, FAKE, None, None) == 1  # decode rows need n_rows 1
     assert L.sas_topk_select(FAKE, 1, 1, 1, 4, FAKE, 0, 2, FAKE, None, None) == 1   # decode rows need block_size
+
+
+def test_status_word_and_selftest_checks(api):
+    """The status reader and the failure self-test refuse a missing word or an
+    out-of-range limit before touching the device."""
+    L = api.lib
+    assert L.sas_get_device_status(None, None) == 1
+    assert L.sas_selftest_bounded_wait(50, None, None, None) == 1
+    for bad in (0, -5, 20000):
+        assert L.sas_selftest_bounded_wait(bad, FAKE, None, None) == 1
 
 
 def test_cuda_library_and_oracle_share_nothing(api):
@@ -141,7 +155,7 @@ def test_paged_decode_checks(api):
 
     def call(desc, pps=16, npages=64, kp=FAKE, s=FAKE, s_cols=16, table=FAKE):
         return L.sas_sparse_decode_paged(ctypes.byref(desc), FAKE, kp, FAKE, table, pps, npages, FAKE, None, s,
-                                         s_cols, FAKE, None, None)
+                                         s_cols, FAKE, None, FAKE, None)
 
     assert call(d, table=None) == 1
     assert call(d, pps=0) == 1

@@ -72,3 +72,42 @@ def test_reference_arm_under_torchrun_prints_once():
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
     assert json.loads(lines[0])["impl"] == "reference"
+
+
+def _bench():
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("bench_mod2", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    return bench
+
+
+def test_tensor_peak_follows_the_clock_record():
+    """Burst peak when the timed region ran at the maximum clock with no throttle
+    reason; the sustained (power-capped) figure otherwise or without a record."""
+    bench = _bench()
+    peaks = {"bf16_tflops": 1595.8, "bf16_tflops_sustained": 1385.2}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.tensor_peak(peaks, at_max)[0] == 1595.8
+    assert bench.tensor_peak(peaks, dict(at_max, reasons=["sw_power_cap"]))[0] == 1385.2
+    assert bench.tensor_peak(peaks, dict(at_max, sm_mhz=1500.0))[0] == 1385.2
+    assert bench.tensor_peak(peaks, None)[0] == 1385.2
+
+
+def test_kernel_breakdown_is_reproducible_from_the_times():
+    """Per-kernel executed FLOPs (4d, 6d, 8d per attended pair) over the live
+    times, as fractions of the named peak."""
+    bench = _bench()
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    w = syn.TRAIN_SPARSE_32K
+    fl = bench.train_flops(w)
+    per_call = {"sas_topk_select": 0.04, "sas_gated_attn_fwd": 1.1, "sas_gated_attn_bwd": 5.0}
+    out = bench.kernel_breakdown(fl, w, per_call, {"bwd_dq": 2.0, "bwd_dkdv": 3.0}, 1595.8)
+    assert set(out) == {"fwd_sm100", "bwd_dq_sm100", "bwd_dkdv_sm100"}
+    k = out["bwd_dkdv_sm100"]
+    assert k["executed_flops"] == 8 * w.d * fl["pairs"]
+    assert abs(k["executed_tflops"] - k["executed_flops"] / 3.0e-3 / 1e12) < 1e-6
+    assert abs(k["frac_executed"] - k["executed_tflops"] / 1595.8) < 1e-12
+    assert abs(sum(v["share_of_step"] for v in out.values()) - (1.1 + 5.0) / 6.14) < 1e-9

@@ -81,20 +81,12 @@ def test_select_decode_rows_bit_exact(api):
 # training-shape forward + backward, whole problems
 # --------------------------------------------------------------------------
 
-def _reads_stored_o(dtype, d, bs, G):
-    """The SIMT backward takes D_i = dO_i . o_i from the bf16 output the forward
-    stored, so its oracle rounds o the same way; the tensor-core backward
-    (bf16, d 128, b 64, G 2 or 4) corrects D by the row sum of dS and is held
-    to the exact oracle."""
-    return dtype == torch.bfloat16 and not (d == 128 and bs == 64 and G in (2, 4))
-
-
 def _oracle_train(inp, bs, top_k, full_scope, gate="softmax"):
-    q = inp["q"]
-    G = q.shape[2] // inp["k"].shape[2]
-    o_store = "bf16" if _reads_stored_o(q.dtype, q.shape[3], bs, G) else None
+    """The exact oracle (fp64 on the inputs' bits, D_i = dO_i . o_i from the exact
+    output) for every path: the tensor-core and the SIMT backward both take D from
+    the exact output rather than from the rounded o the forward stored."""
     return oracle.attn_bwd(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]), bits(inp["dO"]), bits(inp["s"]), bs,
-                           top_k, full_scope=full_scope, gate=gate, o_store=o_store)
+                           top_k, full_scope=full_scope, gate=gate)
 
 
 def _compare_train(got, want, tol, idx_want=None):
@@ -156,21 +148,24 @@ def test_unsupported_block_size_is_refused(api):
 
 
 @pytest.mark.parametrize("gate", ["sigmoid", "raw", "outer", "ste"])
-@pytest.mark.parametrize("dtype,d,bs,K,full", [
-    (torch.bfloat16, 128, 64, 3, False),  # tcgen05 kernels, sparse scope
-    (torch.bfloat16, 128, 64, 0, True),   # tcgen05 kernels, full scope
-    (torch.bfloat16, 64, 32, 4, False),   # SIMT kernels (d = 64)
-    (torch.float32, 128, 32, 3, False),   # SIMT kernels, fp32
+@pytest.mark.parametrize("dtype,d,bs,K,full,G", [
+    (torch.bfloat16, 128, 64, 3, False, 2),  # tcgen05 kernels, sparse scope
+    (torch.bfloat16, 128, 64, 0, True, 2),   # tcgen05 kernels, full scope
+    (torch.bfloat16, 64, 32, 4, False, 2),   # SIMT kernels (d = 64)
+    (torch.bfloat16, 64, 32, 4, False, 5),   # SIMT kernels, GQA 5
+    (torch.bfloat16, 128, 16, 5, False, 4),  # SIMT kernels, 16-token blocks
+    (torch.float32, 128, 32, 3, False, 2),   # SIMT kernels, fp32
 ])
-def test_gate_variants(api, gate, dtype, d, bs, K, full):
+def test_gate_variants(api, gate, dtype, d, bs, K, full, G):
     """The ablated gates against the oracle, every output and gradient: log
     sigmoid(s) and raw-logit gates inside the softmax, the outer gate, and the hard
     STE gate (whose backward also walks the dropped blocks).  Unlike log_softmax
     the sigmoid and raw gates are not normalised, so one history block can hold
     nearly all of a row's mass (raw: weight e^s against the current block's 1);
     its dlogg then sums D_i over all G*b rows of the query block, which is what
-    the stored-o correction of D is tested on here."""
-    B, n, Hq, Hkv = 1, 512, 4, 2
+    the exact D of both backward paths is tested on here."""
+    B, n, Hkv = 1, 512, 2 if G < 5 else 1
+    Hq = G * Hkv
     Cq = n // bs
     qk_std = 1.0 if dtype == torch.bfloat16 else 0.3
     inp = {
@@ -252,8 +247,7 @@ def _sampled_full_size(api, w, q_blocks, kv_blocks, heads, gate="softmax"):
                 if w.full_scope or m in sel[0, 0, c].tolist():
                     qmask[0, 0, c] = True
         want = oracle.attn_bwd(si["q"], si["k"], si["v"], si["dO"], si["s"], bs, w.top_k, full_scope=w.full_scope,
-                               qmask=qmask, kvmask=kvmask, gate=gate,
-                               o_store="bf16" if _reads_stored_o(w.dtype, w.d, bs, G) else None)
+                               qmask=qmask, kvmask=kvmask, gate=gate)
         rows = np.concatenate([np.arange(c * bs, (c + 1) * bs) for c in q_blocks])
         hs = slice(h * G, (h + 1) * G)
         compare(f"o[h{h}]", host(got["o"][:, rows, hs]), want["o"][:, rows], **BF16_TOL, bf16_out=True)
@@ -346,9 +340,17 @@ def test_decode_full_size_sampled(api, w):
             compare(f"dense o[{b},{h}]", host(od[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
 
 
-@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64), (torch.float32, 128)])
-def test_decode_edge_cases(api, dtype, d):
-    B, Hq, Hkv, bs, K, Tmax = 7, 10, 2, 64, 3, 1100
+@pytest.mark.parametrize("dtype,d,bs", [
+    (torch.bfloat16, 128, 64),  # cluster kernel (tensor cores)
+    (torch.bfloat16, 64, 64),   # split-K SIMT kernels, bf16
+    (torch.bfloat16, 128, 32),  # split-K SIMT kernels, bf16, 32-token blocks
+    (torch.float32, 64, 64),
+    (torch.float32, 128, 64),
+])
+def test_decode_edge_cases(api, dtype, d, bs):
+    """Ragged lengths (1 token, a block boundary, one token past it, ...), sparse,
+    dense and fused-selection decode against the oracle, on every decode kernel."""
+    B, Hq, Hkv, K, Tmax = 7, 10, 2, 3, 1100
     ctx = torch.tensor([1, 2, 64, 65, 129, 300, 1100], dtype=torch.int32, device="cuda")
     inp = {
         "q": _seeded((B, Hq, d), 1.0, dtype, 41),
@@ -361,7 +363,7 @@ def test_decode_edge_cases(api, dtype, d):
     G = Hq // Hkv
     rows = [(b, h) for b in range(B) for h in range(Hkv)]
     modes = [("sparse", False, False), ("dense", True, False)]
-    if dtype == torch.bfloat16:
+    if dtype == torch.bfloat16 and d == 128 and bs == 64:
         modes.append(("fused", False, True))
     for name, dense, fused in modes:
         o, idx = _run_decode(api, inp, bs, K, dense=dense, fused=fused)

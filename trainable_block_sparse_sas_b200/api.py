@@ -56,28 +56,30 @@ lib.sas_version.restype = ctypes.c_int32
 lib.sas_topk_select.restype = ctypes.c_int
 lib.sas_topk_select.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _vp, _vp]
 lib.sas_gated_attn_fwd.restype = ctypes.c_int
-lib.sas_gated_attn_fwd.argtypes = [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.sas_gated_attn_fwd.argtypes = [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.sas_gated_attn_bwd_workspace_size.restype = _sz
 lib.sas_gated_attn_bwd_workspace_size.argtypes = [ctypes.POINTER(AttnDesc)]
 lib.sas_gated_attn_bwd.restype = ctypes.c_int
-lib.sas_gated_attn_bwd.argtypes = [ctypes.POINTER(AttnDesc)] + [_vp] * 14 + [_sz, _vp]
+lib.sas_gated_attn_bwd.argtypes = [ctypes.POINTER(AttnDesc)] + [_vp] * 14 + [_sz, _vp, _vp]
+lib.sas_gated_attn_bwd_timed.restype = ctypes.c_int
+lib.sas_gated_attn_bwd_timed.argtypes = [ctypes.POINTER(AttnDesc)] + [_vp] * 14 + [_sz, _vp, _vp, _vp]
 lib.sas_sparse_decode_workspace_size.restype = _sz
 lib.sas_sparse_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeDesc)]
 lib.sas_sparse_decode.restype = ctypes.c_int
-lib.sas_sparse_decode.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7 + [_sz, _vp]
+lib.sas_sparse_decode.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7 + [_sz, _vp, _vp]
 lib.sas_sparse_decode_select.restype = ctypes.c_int
-lib.sas_sparse_decode_select.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 5 + [_i32, _vp, _vp, _vp]
+lib.sas_sparse_decode_select.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 5 + [_i32, _vp, _vp, _vp, _vp]
 lib.sas_sparse_decode_paged.restype = ctypes.c_int
 lib.sas_sparse_decode_paged.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32,
-                                        _vp, _vp, _vp]
+                                        _vp, _vp, _vp, _vp]
 lib.sas_sparse_decode_noalloc.restype = ctypes.c_int
-lib.sas_sparse_decode_noalloc.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7
+lib.sas_sparse_decode_noalloc.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 8
 lib.sas_selftest_bounded_wait.restype = ctypes.c_int
-lib.sas_selftest_bounded_wait.argtypes = [_i32, _vp]
+lib.sas_selftest_bounded_wait.argtypes = [_i32, _vp, _vp, _vp]
 lib.sas_launch_count.restype = ctypes.c_uint64
 lib.sas_launch_count.argtypes = []
-lib.sas_device_status.restype = ctypes.c_int
-lib.sas_device_status.argtypes = [_vp]
+lib.sas_get_device_status.restype = ctypes.c_int
+lib.sas_get_device_status.argtypes = [_vp, _vp]
 lib.sas_pooled_scores_workspace_size.restype = _sz
 lib.sas_pooled_scores_workspace_size.argtypes = [ctypes.POINTER(AttnDesc)]
 lib.sas_pooled_scores.restype = ctypes.c_int
@@ -108,6 +110,32 @@ def _stream(stream=None):
 def _check(status: int, where: str):
     if status != SAS_OK:
         raise SasError(status, where)
+
+
+# The C ABI reports device-side failures (a bounded wait that gave up) through a
+# caller-owned int32 status word.  Calls take it as `status=`; without one the
+# binding passes a word of its own, one per device, created zeroed on first use
+# (make a first call on a device outside any CUDA-graph capture).
+_default_words = {}
+
+
+def status_word(device=None) -> torch.Tensor:
+    """A zeroed device status word for the C ABI (int32, one element)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return torch.zeros(1, dtype=torch.int32, device=dev)
+
+
+def _status(status, ref: torch.Tensor):
+    if status is not None:
+        _need(status, 1, _I32, "status")
+        return _p(status)
+    dev = ref.device
+    idx = dev.index if dev.index is not None else torch.cuda.current_device()
+    word = _default_words.get(idx)
+    if word is None:
+        word = status_word(torch.device("cuda", idx))
+        _default_words[idx] = word
+    return _p(word)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -200,19 +228,19 @@ def sas_topk_select(s, n_rows, row_len, top_k, idx=None, lse_s=None, ctx_len=Non
     _check(st, "sas_topk_select")
 
 
-def sas_gated_attn_fwd(desc, q, k, v, s, lse_s, idx, o, lse, stream=None):
+def sas_gated_attn_fwd(desc, q, k, v, s, lse_s, idx, o, lse, stream=None, status=None):
     _, nq, _ = _check_train(desc, q, k, v, s, lse_s, idx)
     _need(o, nq, _dt(desc), "o")
     _need(lse, desc.batch * desc.n_q_heads * desc.seq_len, _F32, "lse")
     _check(lib.sas_gated_attn_fwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(s), _p(lse_s), _p(idx), _p(o), _p(lse),
-                                  _stream(stream)), "sas_gated_attn_fwd")
+                                  _status(status, q), _stream(stream)), "sas_gated_attn_fwd")
 
 
 def sas_gated_attn_bwd_workspace_size(desc) -> int:
     return int(lib.sas_gated_attn_bwd_workspace_size(ctypes.byref(desc)))
 
 
-def sas_gated_attn_bwd(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, workspace, stream=None):
+def sas_gated_attn_bwd(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, workspace, stream=None, status=None):
     Cq, nq, nkv = _check_train(desc, q, k, v, s, lse_s, idx)
     dt = _dt(desc)
     for t, n, name in ((o, nq, "o"), (dO, nq, "dO"), (dq, nq, "dq"), (dk, nkv, "dk"), (dv, nkv, "dv")):
@@ -221,8 +249,32 @@ def sas_gated_attn_bwd(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds,
     _need(ds, desc.batch * desc.n_kv_heads * Cq * Cq, _F32, "ds")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.sas_gated_attn_bwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dO), _p(s), _p(lse_s),
-                                  _p(idx), _p(dq), _p(dk), _p(dv), _p(ds), _p(workspace), ws_bytes, _stream(stream)),
-           "sas_gated_attn_bwd")
+                                  _p(idx), _p(dq), _p(dk), _p(dv), _p(ds), _p(workspace), ws_bytes,
+                                  _status(status, q), _stream(stream)), "sas_gated_attn_bwd")
+
+
+def sas_gated_attn_bwd_timed(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, workspace, events, stream=None,
+                             status=None):
+    """sas_gated_attn_bwd with three torch.cuda.Event (timing enabled) recorded by
+    the library on the stream: before the dq/ds kernel, between it and the dk/dv
+    kernel, and after the latter."""
+    Cq, nq, nkv = _check_train(desc, q, k, v, s, lse_s, idx)
+    dt = _dt(desc)
+    for t, n, name in ((o, nq, "o"), (dO, nq, "dO"), (dq, nq, "dq"), (dk, nkv, "dk"), (dv, nkv, "dv")):
+        _need(t, n, dt, name)
+    _need(lse, desc.batch * desc.n_q_heads * desc.seq_len, _F32, "lse")
+    _need(ds, desc.batch * desc.n_kv_heads * Cq * Cq, _F32, "ds")
+    if len(events) != 3:
+        raise ValueError("events: three torch.cuda.Event")
+    st = stream if stream is not None else torch.cuda.current_stream()
+    for e in events:
+        if not e.cuda_event:
+            e.record(st)  # torch creates the CUDA event on its first record
+    handles = (ctypes.c_void_p * 3)(*(e.cuda_event for e in events))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.sas_gated_attn_bwd_timed(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(lse), _p(dO), _p(s),
+                                        _p(lse_s), _p(idx), _p(dq), _p(dk), _p(dv), _p(ds), _p(workspace), ws_bytes,
+                                        handles, _status(status, q), _stream(stream)), "sas_gated_attn_bwd_timed")
 
 
 def sas_sparse_decode_workspace_size(desc) -> int:
@@ -235,23 +287,24 @@ def _check_cache(desc, k_cache, v_cache):
     _need(v_cache, n, _dt(desc), "v_cache")
 
 
-def sas_sparse_decode(desc, q, k_cache, v_cache, ctx_len, idx, o, workspace, stream=None):
+def sas_sparse_decode(desc, q, k_cache, v_cache, ctx_len, idx, o, workspace, stream=None, status=None):
     _check_decode(desc, q, o, ctx_len)
     _check_cache(desc, k_cache, v_cache)
     _need(idx, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx", optional=True)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.sas_sparse_decode(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx), _p(o),
-                                 _p(workspace), ws_bytes, _stream(stream)), "sas_sparse_decode")
+                                 _p(workspace), ws_bytes, _status(status, q), _stream(stream)), "sas_sparse_decode")
 
 
-def sas_sparse_decode_select(desc, q, k_cache, v_cache, ctx_len, s, o, idx_out=None, stream=None):
+def sas_sparse_decode_select(desc, q, k_cache, v_cache, ctx_len, s, o, idx_out=None, stream=None, status=None):
     """Fused decode step: Top-K of s [B, Hkv, s_cols] and the gate-free attention."""
     _check_decode(desc, q, o, ctx_len)
     _check_cache(desc, k_cache, v_cache)
     _need(s, desc.batch * desc.n_kv_heads * s.shape[-1], _F32, "s")
     _need(idx_out, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx_out", optional=True)
     _check(lib.sas_sparse_decode_select(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(s),
-                                        s.shape[-1], _p(o), _p(idx_out), _stream(stream)), "sas_sparse_decode_select")
+                                        s.shape[-1], _p(o), _p(idx_out), _status(status, q), _stream(stream)),
+           "sas_sparse_decode_select")
 
 
 def paged_decode_desc(q, k_pages, block_size: int, top_k: int, max_ctx: int, softmax_scale: float = 0.0) -> DecodeDesc:
@@ -261,7 +314,7 @@ def paged_decode_desc(q, k_pages, block_size: int, top_k: int, max_ctx: int, sof
 
 
 def sas_sparse_decode_paged(desc, q, k_pages, v_pages, page_table, ctx_len, o, s=None, idx=None, idx_out=None,
-                            stream=None):
+                            stream=None, status=None):
     """Decode step over a paged cache: page_table [B, pages_per_seq] int32 maps a
     sequence's blocks to pages of k_pages / v_pages [num_pages, block_size, Hkv, d].
     Blocks from the Top-K of s (fused), from idx, or every block when both are None."""
@@ -276,8 +329,8 @@ def sas_sparse_decode_paged(desc, q, k_pages, v_pages, page_table, ctx_len, o, s
     _need(idx_out, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx_out", optional=True)
     _check(lib.sas_sparse_decode_paged(ctypes.byref(desc), _p(q), _p(k_pages), _p(v_pages), _p(page_table),
                                        page_table.shape[1], k_pages.shape[0], _p(ctx_len), _p(idx), _p(s),
-                                       0 if s is None else s.shape[-1], _p(o), _p(idx_out), _stream(stream)),
-           "sas_sparse_decode_paged")
+                                       0 if s is None else s.shape[-1], _p(o), _p(idx_out), _status(status, q),
+                                       _stream(stream)), "sas_sparse_decode_paged")
 
 
 def sas_pooled_scores_workspace_size(desc) -> int:
@@ -325,23 +378,42 @@ def sas_decode_scores(desc, q, ksum, ctx_len, s, stream=None):
                                  _stream(stream)), "sas_decode_scores")
 
 
-def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream=None):
+def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, ctx_len, idx, o, stream=None, status=None):
     """sas_sparse_decode without a workspace, for callers that cannot allocate
-    device memory: the partials use a fixed 4 MiB array inside the library.
+    device memory: shapes the tensor-core decode takes need no scratch; the
+    split-K kernels put their partials in a fixed 4 MiB array inside the library.
     Overlapping calls race on that array."""
     _check_decode(desc, q, o, ctx_len)
     _check_cache(desc, k_cache, v_cache)
     _need(idx, desc.batch * desc.n_kv_heads * max(desc.top_k, 0), _I32, "idx", optional=True)
     _check(lib.sas_sparse_decode_noalloc(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(idx),
-                                         _p(o), _stream(stream)), "sas_sparse_decode_noalloc")
+                                         _p(o), _status(status, q), _stream(stream)), "sas_sparse_decode_noalloc")
 
 
-def sas_device_status(stream=None):
-    _check(lib.sas_device_status(_stream(stream)), "sas_device_status")
+def sas_get_device_status(status=None, stream=None):
+    """Synchronise the stream, then read and clear a device status word (the
+    binding's word of the current device when status is None); raises SasError
+    (SAS_ERR_DEVICE_TIMEOUT) when a bounded device-side wait gave up."""
+    if status is None:
+        word = _default_words.get(torch.cuda.current_device())
+        if word is None:
+            return  # nothing has run on this device through the default word
+        status = word
+    _need(status, 1, _I32, "status")
+    _check(lib.sas_get_device_status(_p(status), _stream(stream)), "sas_get_device_status")
 
 
-def sas_selftest_bounded_wait(limit_ms: int, stream=None):
-    _check(lib.sas_selftest_bounded_wait(limit_ms, _stream(stream)), "sas_selftest_bounded_wait")
+def sas_selftest_bounded_wait(limit_ms: int, status=None, trace=None, stream=None):
+    """Run the failure path of the tensor-core kernels with a wait limit of
+    limit_ms; the timeout lands in `status` (the binding's word when None) and the
+    phases reached in `trace` (int32 [4]) when given."""
+    if status is not None:
+        _need(status, 1, _I32, "status")
+    else:
+        status = _default_words.setdefault(torch.cuda.current_device(), status_word())
+    _need(trace, 4, _I32, "trace", optional=True)
+    _check(lib.sas_selftest_bounded_wait(limit_ms, _p(status), _p(trace), _stream(stream)),
+           "sas_selftest_bounded_wait")
 
 
 def sas_launch_count() -> int:

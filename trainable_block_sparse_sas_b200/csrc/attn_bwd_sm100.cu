@@ -900,6 +900,8 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
                     : (outer ? bwd_dq_sm100_kernel<MT, 2, true> : bwd_dq_sm100_kernel<MT, 2, false>);
     cudaError_t err = launch_kernel(kern, grid, kDqThreads, smem, a, stream);
     if (err != cudaSuccess) return err;
+    if (p.phase_event && (err = cudaEventRecord(static_cast<cudaEvent_t>(p.phase_event), stream)) != cudaSuccess)
+        return err;
     // key-major kernel: 128-row items (128/G tokens x G heads) per box
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, 128 / G) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, 128 / G))
         return cudaErrorInvalidValue;

@@ -9,13 +9,19 @@
 // bias 0 and a causal mask -- through shared memory with an online softmax.
 //
 // Backward, without atomics and therefore deterministic:
-//   bwd_rowdot   D_i = dO_i . o_i
 //   bwd_dq       one CTA per (batch, kv head, query block c), looping over the
 //                group's query heads: recomputes P from the saved lse, dS =
 //                P (dP - D), dq = sigma dS K, and the block-wise log-gate gradient
 //                dlogg[c,m] = sum of dS over the tile (jaehun.me review, Kernel
 //                implementation paragraph), then ds[c,:] = dlogg - g sum(dlogg).
-//                D here is dO . o of the stored output.
+//                D_i = dO_i . o_i is taken from the exact output, not from the
+//                rounded o the forward stored: a first pass over the attended
+//                blocks sums D_i = sum_j P_ij w_j dP_ij (the identity o_i =
+//                sum_j P_ij w_j v_j; w = 1 except for the outer gate's g), and
+//                the row's D goes to the workspace for the dk/dv kernel.  With
+//                the sigmoid and raw-logit gates one history block can hold most
+//                of a row's mass, and dlogg of that block then sums the rounding
+//                error of the stored o over every row of the query block.
 //
 // Gate variants: the sigmoid and raw-logit gates change the bias and ds; the
 // outer gate weights V by g (dS = P (g dP - D), dv from g P, dlogg = g sum P dP);
@@ -225,21 +231,35 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
     if (tid < BS) p.lse[((long)b * p.Hq + hq) * p.n + c * BS + tid] = row_m[tid] + logf(row_l[tid]);
 }
 
-// D_i = dO_i . o_i, one warp per row.
-template <typename T>
-__global__ void __launch_bounds__(kThreads) bwd_rowdot_kernel(TrainParams p) {
-    const long rows = (long)p.B * p.n * p.Hq;
-    const long row = (long)blockIdx.x * (kThreads / 32) + threadIdx.x / 32;
-    if (row >= rows) return;
-    const int lane = threadIdx.x & 31;
-    float acc = 0.f;
-    for (int e = lane; e < p.d; e += 32) acc += ldg<T>(p.dO, row * p.d + e) * ldg<T>(p.o_in, row * p.d + e);
-    acc = warp_sum(acc);
-    if (lane == 0) {
-        const int hq = (int)(row % p.Hq);
-        const long bi = row / p.Hq;  // b * n + i
-        const int b = (int)(bi / p.n), i = (int)(bi % p.n);
-        p.Dbuf[((long)b * p.Hq + hq) * p.n + i] = acc;
+// One 4x4 micro-tile of S = Q K^T (unscaled) and dP = dO V^T: rows ttr + RG*ii
+// of the [BS][D] query-side tiles against rows ttc + RG*jj of the key-side tiles.
+template <int D, int BS>
+__device__ __forceinline__ void tile_s_dp(const float* Qs, const float* dOs, const float* Ks, const float* Vs,
+                                          int ttr, int ttc, float (&sacc)[4][4], float (&pacc)[4][4]) {
+    using C = Cfg<D, BS>;
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) sacc[ii][jj] = pacc[ii][jj] = 0.f;
+    for (int e = 0; e < D; ++e) {
+        float qv[4], gv[4], kv[4], vv[4];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            qv[ii] = Qs[(ttr + C::RG * ii) * C::LD + e];
+            gv[ii] = dOs[(ttr + C::RG * ii) * C::LD + e];
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            kv[jj] = Ks[(ttc + C::RG * jj) * C::LD + e];
+            vv[jj] = Vs[(ttc + C::RG * jj) * C::LD + e];
+        }
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                sacc[ii][jj] = fmaf(qv[ii], kv[jj], sacc[ii][jj]);
+                pacc[ii][jj] = fmaf(gv[ii], vv[jj], pacc[ii][jj]);
+            }
     }
 }
 
@@ -277,16 +297,51 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
         load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
         load_rows<T, D, BS>(dOs, p.dO, b, p.n, p.Hq, hq, c * BS);
         if (tid < BS) {
-            const long ri = ((long)b * p.Hq + hq) * p.n + c * BS + tid;
-            rowL[tid] = p.lse_in[ri];
-            rowD[tid] = p.Dbuf[ri];
+            rowL[tid] = p.lse_in[((long)b * p.Hq + hq) * p.n + c * BS + tid];
+            rowD[tid] = 0.f;
         }
+        // pass 1: D_i = sum_j P_ij w_j dP_ij over the blocks the forward attended
+        for (int t = 0; t <= nsel; ++t) {
+            const int code = blocks[t];
+            if (code < 0) continue;  // STE: a block the selection dropped is not part of o
+            const bool cur = (t == nsel);
+            const float lg = cur ? 0.f : gate_log(srow[code], lse_c, p.gate);
+            const float bias = gate_in_logits(p.gate) ? lg : 0.f;
+            const float w = (p.gate == kGateOuter && !cur) ? expf(lg) : 1.f;
+            __syncthreads();
+            load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, code * BS);
+            load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, code * BS);
+            __syncthreads();
+            for (int tile = tid; tile < C::NT_S; tile += kThreads) {
+                const int ttr = tile / C::RG, ttc = tile % C::RG;
+                float sacc[4][4], pacc[4][4];
+                tile_s_dp<D, BS>(Qs, dOs, Ks, Vs, ttr, ttc, sacc, pacc);
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int r = ttr + C::RG * ii, j = ttc + C::RG * jj;
+                        const float z = fmaf(p.scale, sacc[ii][jj], bias);
+                        const float pr = (cur && j > r) ? 0.f : expf(z - rowL[r]);
+                        Ss[r * C::LDS + j] = pr * w * pacc[ii][jj];
+                    }
+            }
+            __syncthreads();
+            if (tid < BS) {
+                float a = 0.f;
+                for (int j = 0; j < BS; ++j) a += Ss[tid * C::LDS + j];
+                rowD[tid] += a;
+            }
+        }
+        __syncthreads();
+        if (tid < BS) p.Dbuf[((long)b * p.Hq + hq) * p.n + c * BS + tid] = rowD[tid];  // for dk / dv
         float acc[4][C::COLS];
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
             for (int ee = 0; ee < C::COLS; ++ee) acc[ii][ee] = 0.f;
 
+        // pass 2: dS, dq and the blocks' log-gate gradients
         for (int t = 0; t <= nsel; ++t) {
             const int code = blocks[t];
             const bool dropped = code < 0;  // STE: a block the selection dropped
@@ -302,27 +357,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
             float local = 0.f;
             for (int tile = tid; tile < C::NT_S; tile += kThreads) {
                 const int ttr = tile / C::RG, ttc = tile % C::RG;
-                float sacc[4][4] = {}, pacc[4][4] = {};
-                for (int e = 0; e < D; ++e) {
-                    float qv[4], gv[4], kv[4], vv[4];
-#pragma unroll
-                    for (int ii = 0; ii < 4; ++ii) {
-                        qv[ii] = Qs[(ttr + C::RG * ii) * C::LD + e];
-                        gv[ii] = dOs[(ttr + C::RG * ii) * C::LD + e];
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        kv[jj] = Ks[(ttc + C::RG * jj) * C::LD + e];
-                        vv[jj] = Vs[(ttc + C::RG * jj) * C::LD + e];
-                    }
-#pragma unroll
-                    for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            sacc[ii][jj] = fmaf(qv[ii], kv[jj], sacc[ii][jj]);
-                            pacc[ii][jj] = fmaf(gv[ii], vv[jj], pacc[ii][jj]);
-                        }
-                }
+                float sacc[4][4], pacc[4][4];
+                tile_s_dp<D, BS>(Qs, dOs, Ks, Vs, ttr, ttc, sacc, pacc);
 #pragma unroll
                 for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
@@ -456,27 +492,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
                 __syncthreads();
                 for (int tile = tid; tile < C::NT_S; tile += kThreads) {
                     const int ttr = tile / C::RG, ttc = tile % C::RG;  // query rows, keys
-                    float sacc[4][4] = {}, pacc[4][4] = {};
-                    for (int e = 0; e < D; ++e) {
-                        float qv[4], gv[4], kv[4], vv[4];
-#pragma unroll
-                        for (int ii = 0; ii < 4; ++ii) {
-                            qv[ii] = Qs[(ttr + C::RG * ii) * C::LD + e];
-                            gv[ii] = dOs[(ttr + C::RG * ii) * C::LD + e];
-                        }
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            kv[jj] = Ks[(ttc + C::RG * jj) * C::LD + e];
-                            vv[jj] = Vs[(ttc + C::RG * jj) * C::LD + e];
-                        }
-#pragma unroll
-                        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                            for (int jj = 0; jj < 4; ++jj) {
-                                sacc[ii][jj] = fmaf(qv[ii], kv[jj], sacc[ii][jj]);
-                                pacc[ii][jj] = fmaf(gv[ii], vv[jj], pacc[ii][jj]);
-                            }
-                    }
+                    float sacc[4][4], pacc[4][4];
+                    tile_s_dp<D, BS>(Qs, dOs, Ks, Vs, ttr, ttc, sacc, pacc);
 #pragma unroll
                     for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
@@ -607,28 +624,14 @@ size_t simt_max_smem(int D, int BS, int Cq) {
 cudaError_t launch_fwd_simt(const TrainParams& p, cudaStream_t stream) { return launch_fwd_impl(p, stream); }
 
 size_t bwd_simt_workspace(const TrainParams& p) {
-    return sizeof(float) * (size_t)p.B * p.Hq * p.n;  // D rows
-}
-
-cudaError_t launch_rowdot(const TrainParams& p, cudaStream_t stream) {
-    const long rows = (long)p.B * p.n * p.Hq;
-    const long grid = (rows + kThreads / 32 - 1) / (kThreads / 32);
-    if (grid <= 0) return cudaSuccess;
-    if (grid > 0x7fffffffL) return cudaErrorInvalidValue;
-    if (p.is_bf16)
-        bwd_rowdot_kernel<__nv_bfloat16><<<(unsigned)grid, kThreads, 0, stream>>>(p);
-    else
-        bwd_rowdot_kernel<float><<<(unsigned)grid, kThreads, 0, stream>>>(p);
-    cudaError_t err = cudaGetLastError();
-    if (err == cudaSuccess) count_launch();
-    return err;
+    return sizeof(float) * (size_t)p.B * p.Hq * p.n;  // D rows, written by the dq kernel
 }
 
 cudaError_t launch_bwd_simt(const TrainParams& p, cudaStream_t stream) {
-    cudaError_t err = launch_rowdot(p, stream);
+    cudaError_t err = launch_dq_impl(p, stream);
     if (err != cudaSuccess) return err;
-    err = launch_dq_impl(p, stream);
-    if (err != cudaSuccess) return err;
+    if (p.phase_event && (err = cudaEventRecord(static_cast<cudaEvent_t>(p.phase_event), stream)) != cudaSuccess)
+        return err;
     return launch_dkdv_impl(p, stream);
 }
 

@@ -5,8 +5,12 @@
 // inside a host program that owns every byte of device memory, a serving loop
 // that must not call cudaMalloc (it synchronises the device) between decode
 // steps, or a caller with no spare pool to carve a workspace from.  Such a
-// caller passes only its inputs and outputs; the split-K partials live in a
-// fixed array compiled into this library instead of a caller workspace.
+// caller passes only its inputs and outputs.
+//
+// The dispatch is that of sas_sparse_decode: the tensor-core decode kernel,
+// which keeps its partials in shared memory and needs no scratch, takes the
+// shapes it supports; the split-K kernels take the rest, and their partials live
+// in a fixed array compiled into this library instead of a caller workspace.
 //
 // The array is file-scope device memory of kScratchFloats floats (4 MiB); every
 // GPU that loads the library holds it until the process exits.  Host code may
@@ -68,10 +72,10 @@ bool supported(const sas_decode_desc* d) {
 
 extern "C" sas_status sas_sparse_decode_noalloc(const sas_decode_desc* desc, const void* q, const void* k_cache,
                                                 const void* v_cache, const int32_t* ctx_len, const int32_t* idx,
-                                                void* o, sas_stream_t stream) {
+                                                void* o, int32_t* status, sas_stream_t stream) {
     using namespace sas;
     if (!valid(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k_cache || !v_cache || !ctx_len || !o) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_cache || !v_cache || !ctx_len || !o || !status) return SAS_ERR_INVALID_VALUE;
     if (!supported(desc)) return SAS_ERR_UNSUPPORTED;
     DecodeParams p = {};
     p.B = desc->batch;
@@ -89,12 +93,19 @@ extern "C" sas_status sas_sparse_decode_noalloc(const sas_decode_desc* desc, con
     p.ctx_len = ctx_len;
     p.idx = (desc->top_k > 0 && idx) ? idx : nullptr;
     p.o = o;
-    decode_plan(p);
-    if (decode_workspace(p) > kScratchFloats * sizeof(float)) return SAS_ERR_WORKSPACE_TOO_SMALL;
-    float* scratch = nullptr;
-    if (scratch_address(&scratch) != cudaSuccess) return SAS_ERR_CUDA;
-    p.part = scratch;
-    const cudaError_t err = launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+    p.status = status;
+    cudaError_t err;
+    if (decode_sm100_supported(p)) {
+        // partials in shared memory: no scratch at all
+        err = launch_decode_sm100(p, nullptr, 0, nullptr, reinterpret_cast<cudaStream_t>(stream));
+    } else {
+        decode_plan(p);
+        if (decode_workspace(p) > kScratchFloats * sizeof(float)) return SAS_ERR_WORKSPACE_TOO_SMALL;
+        float* scratch = nullptr;
+        if (scratch_address(&scratch) != cudaSuccess) return SAS_ERR_CUDA;
+        p.part = scratch;
+        err = launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+    }
     if (err == cudaSuccess) return SAS_OK;
     return err == cudaErrorNotSupported ? SAS_ERR_UNSUPPORTED : SAS_ERR_CUDA;
 }

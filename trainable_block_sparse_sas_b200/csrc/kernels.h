@@ -30,6 +30,7 @@ struct TrainParams {
     void* dv;
     float* ds;
     int* status;  // device status word (bounded waits)
+    void* phase_event;  // host only: cudaEvent_t recorded between the backward's two kernels (nullable)
     int B, Hq, Hkv, d, n, bs, Cq, top_k, full_scope, is_bf16;
     float scale;
     int gate;  // sas_gate: 0 softmax, 1 sigmoid, 2 raw logit, 3 outer, 4 hard STE
@@ -85,7 +86,6 @@ bool fwd_sm100_supported(const TrainParams& p);
 bool bwd_sm100_supported(const TrainParams& p);
 size_t bwd_sm100_workspace(const TrainParams& p);
 cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream);
-cudaError_t launch_rowdot(const TrainParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_sm100(const TrainParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_simt(const TrainParams& p, cudaStream_t stream);
 size_t bwd_simt_workspace(const TrainParams& p);
@@ -102,7 +102,7 @@ size_t simt_max_smem(int D, int BS, int Cq);
 void decode_plan(DecodeParams& p);
 size_t decode_workspace(const DecodeParams& p);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
-cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);
+cudaError_t launch_selftest_wait(int* status, int* trace, unsigned long long limit_ns, cudaStream_t stream);
 bool decode_sm100_supported(const DecodeParams& p);
 // s != nullptr: fused Top-K selection from s [B, Hkv, s_cols] (idx_out nullable)
 cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,

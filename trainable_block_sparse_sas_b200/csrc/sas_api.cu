@@ -1,6 +1,7 @@
 // sas_api.cu -- the C ABI declared in include/sas.h: argument checks (before any
-// launch, no side effects on failure), kernel dispatch, and the device status
-// word that bounded device-side waits set when they give up.
+// launch, no side effects on failure), kernel dispatch, and the reading of the
+// caller's device status word (which bounded device-side waits set when they
+// give up).
 #include <math.h>
 
 #include <atomic>
@@ -18,21 +19,18 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-// Per-device status word: kernels with bounded waits write a non-zero code here.
-__device__ int g_status_word;
-
+// Read-only device properties, looked up once per device.
 struct DeviceInfo {
     bool init = false;
     int n_sm = 0;
     int max_smem_optin = 0;
-    int* status = nullptr;  // device address of g_status_word
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 
-// Set-up once per device, with that device current: SM count, shared-memory
-// limit and the device address of the status word.
+// Set-up once per device, with that device current: SM count and shared-memory
+// limit.
 cudaError_t device_info(DeviceInfo* out) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -45,10 +43,6 @@ cudaError_t device_info(DeviceInfo* out) {
         if (err != cudaSuccess) return err;
         err = cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (err != cudaSuccess) return err;
-        void* addr = nullptr;
-        err = cudaGetSymbolAddress(&addr, g_status_word);
-        if (err != cudaSuccess) return err;
-        di.status = static_cast<int*>(addr);
         di.init = true;
     }
     *out = di;
@@ -158,9 +152,9 @@ sas_status sas_topk_select(const float* s, int32_t batch, int32_t n_kv_heads, in
 
 sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
                               const float* s, const float* lse_s, const int32_t* idx, void* o, float* lse,
-                              sas_stream_t stream) {
+                              int32_t* status, sas_stream_t stream) {
     if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k || !v || !s || !o || !lse) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !s || !o || !lse || !status) return SAS_ERR_INVALID_VALUE;
     if (!lse_s && gate_softmax_family(desc->gate)) return SAS_ERR_INVALID_VALUE;
     if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
     if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
@@ -178,7 +172,7 @@ sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const vo
     if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k == 0) p.idx = nullptr;
     p.o = o;
     p.lse = lse;
-    p.status = di.status;
+    p.status = status;
     if (fwd_sm100_supported(p)) return from_cuda(launch_fwd_sm100(p, reinterpret_cast<cudaStream_t>(stream)));
     return from_cuda(launch_fwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -189,12 +183,12 @@ size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc) {
     return ((bwd_simt_workspace(p) + 255) & ~(size_t)255) + ((bwd_sm100_workspace(p) + 255) & ~(size_t)255);
 }
 
-sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
-                              const void* o, const float* lse, const void* dO, const float* s, const float* lse_s,
-                              const int32_t* idx, void* dq, void* dk, void* dv, float* ds, void* workspace,
-                              size_t ws_bytes, sas_stream_t stream) {
+static sas_status bwd_impl(const sas_attn_desc* desc, const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dO, const float* s, const float* lse_s, const int32_t* idx,
+                           void* dq, void* dk, void* dv, float* ds, void* workspace, size_t ws_bytes, int32_t* status,
+                           void* const* events, sas_stream_t stream) {
     if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k || !v || !o || !lse || !dO || !s || !dq || !dk || !dv || !ds) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k || !v || !o || !lse || !dO || !s || !dq || !dk || !dv || !ds || !status) return SAS_ERR_INVALID_VALUE;
     if (!lse_s && gate_softmax_family(desc->gate)) return SAS_ERR_INVALID_VALUE;
     if (desc->scope == SAS_SCOPE_SPARSE && desc->top_k > 0 && !idx) return SAS_ERR_INVALID_VALUE;
     if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
@@ -223,9 +217,35 @@ sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const vo
     p.Dbuf = static_cast<float*>(workspace);
     if (bwd_sm100_workspace(p) > 0)
         p.Mbuf = static_cast<uint8_t*>(workspace) + ((bwd_simt_workspace(p) + 255) & ~(size_t)255);
-    p.status = di.status;
-    if (bwd_sm100_supported(p)) return from_cuda(launch_bwd_sm100(p, reinterpret_cast<cudaStream_t>(stream)));
-    return from_cuda(launch_bwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
+    p.status = status;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (events) {
+        if (!events[0] || !events[1] || !events[2]) return SAS_ERR_INVALID_VALUE;
+        p.phase_event = events[1];
+        if (cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st) != cudaSuccess) return SAS_ERR_CUDA;
+    }
+    err = bwd_sm100_supported(p) ? launch_bwd_sm100(p, st) : launch_bwd_simt(p, st);
+    if (err != cudaSuccess) return from_cuda(err);
+    if (events && cudaEventRecord(static_cast<cudaEvent_t>(events[2]), st) != cudaSuccess) return SAS_ERR_CUDA;
+    return SAS_OK;
+}
+
+sas_status sas_gated_attn_bwd(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
+                              const void* o, const float* lse, const void* dO, const float* s, const float* lse_s,
+                              const int32_t* idx, void* dq, void* dk, void* dv, float* ds, void* workspace,
+                              size_t ws_bytes, int32_t* status, sas_stream_t stream) {
+    return bwd_impl(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, workspace, ws_bytes, status, nullptr,
+                    stream);
+}
+
+sas_status sas_gated_attn_bwd_timed(const sas_attn_desc* desc, const void* q, const void* k, const void* v,
+                                    const void* o, const float* lse, const void* dO, const float* s,
+                                    const float* lse_s, const int32_t* idx, void* dq, void* dk, void* dv, float* ds,
+                                    void* workspace, size_t ws_bytes, void* const* events, int32_t* status,
+                                    sas_stream_t stream) {
+    if (!events) return SAS_ERR_INVALID_VALUE;
+    return bwd_impl(desc, q, k, v, o, lse, dO, s, lse_s, idx, dq, dk, dv, ds, workspace, ws_bytes, status, events,
+                    stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -306,17 +326,14 @@ size_t sas_sparse_decode_workspace_size(const sas_decode_desc* desc) {
 
 sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const void* k_cache, const void* v_cache,
                              const int32_t* ctx_len, const int32_t* idx, void* o, void* workspace, size_t ws_bytes,
-                             sas_stream_t stream) {
+                             int32_t* status, sas_stream_t stream) {
     if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k_cache || !v_cache || !ctx_len || !o) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_cache || !v_cache || !ctx_len || !o || !status) return SAS_ERR_INVALID_VALUE;
     if (!supported_decode(desc)) return SAS_ERR_UNSUPPORTED;
     DecodeParams p = make_decode(desc);
     const size_t need = decode_ws_bytes(p);
     if (ws_bytes < need) return SAS_ERR_WORKSPACE_TOO_SMALL;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SAS_ERR_INVALID_VALUE;
-    DeviceInfo di;
-    cudaError_t err = device_info(&di);
-    if (err != cudaSuccess) return SAS_ERR_CUDA;
     p.q = q;
     p.k = k_cache;
     p.v = v_cache;
@@ -325,7 +342,7 @@ sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const v
     if (!idx) p.idx = nullptr;
     p.o = o;
     p.part = static_cast<float*>(workspace);
-    p.status = di.status;
+    p.status = status;
     if (decode_sm100_supported(p))
         return from_cuda(launch_decode_sm100(p, nullptr, 0, nullptr, reinterpret_cast<cudaStream_t>(stream)));
     decode_plan(p);
@@ -334,9 +351,9 @@ sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const v
 
 sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, const void* k_cache,
                                     const void* v_cache, const int32_t* ctx_len, const float* s, int32_t s_cols,
-                                    void* o, int32_t* idx_out, sas_stream_t stream) {
+                                    void* o, int32_t* idx_out, int32_t* status, sas_stream_t stream) {
     if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k_cache || !v_cache || !ctx_len || !s || !o || s_cols <= 0) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_cache || !v_cache || !ctx_len || !s || !o || !status || s_cols <= 0) return SAS_ERR_INVALID_VALUE;
     DecodeParams p = make_decode(desc);
     p.q = q;
     p.k = k_cache;
@@ -345,18 +362,16 @@ sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, 
     p.idx = nullptr;
     p.o = o;
     if (!supported_decode(desc) || !decode_sm100_supported(p)) return SAS_ERR_UNSUPPORTED;
-    DeviceInfo di;
-    if (device_info(&di) != cudaSuccess) return SAS_ERR_CUDA;
-    p.status = di.status;
+    p.status = status;
     return from_cuda(launch_decode_sm100(p, s, s_cols, idx_out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_sparse_decode_paged(const sas_decode_desc* desc, const void* q, const void* k_pages,
                                    const void* v_pages, const int32_t* page_table, int32_t pages_per_seq,
                                    int32_t num_pages, const int32_t* ctx_len, const int32_t* idx, const float* s,
-                                   int32_t s_cols, void* o, int32_t* idx_out, sas_stream_t stream) {
+                                   int32_t s_cols, void* o, int32_t* idx_out, int32_t* status, sas_stream_t stream) {
     if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
-    if (!q || !k_pages || !v_pages || !page_table || !ctx_len || !o) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_pages || !v_pages || !page_table || !ctx_len || !o || !status) return SAS_ERR_INVALID_VALUE;
     if (pages_per_seq <= 0 || num_pages <= 0 || (s && s_cols <= 0)) return SAS_ERR_INVALID_VALUE;
     if ((long)desc->max_ctx > (long)pages_per_seq * desc->block_size) return SAS_ERR_INVALID_VALUE;
     if ((reinterpret_cast<uintptr_t>(k_pages) | reinterpret_cast<uintptr_t>(v_pages)) & 15u)
@@ -373,32 +388,26 @@ sas_status sas_sparse_decode_paged(const sas_decode_desc* desc, const void* q, c
     p.num_pages = num_pages;
     if (!supported_decode(desc) || !decode_sm100_supported(p)) return SAS_ERR_UNSUPPORTED;
     if ((long)num_pages * desc->block_size > 0x7fffffffL) return SAS_ERR_UNSUPPORTED;
-    DeviceInfo di;
-    if (device_info(&di) != cudaSuccess) return SAS_ERR_CUDA;
-    p.status = di.status;
+    p.status = status;
     return from_cuda(launch_decode_sm100(p, s, s_cols, s ? idx_out : nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-sas_status sas_device_status(sas_stream_t stream) {
-    DeviceInfo di;
-    cudaError_t err = device_info(&di);
-    if (err != cudaSuccess) return SAS_ERR_CUDA;
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SAS_ERR_CUDA;
-    int word = 0;
-    if (cudaMemcpy(&word, di.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SAS_ERR_CUDA;
-    if (word != 0) {
-        const int zero = 0;
-        if (cudaMemcpy(di.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SAS_ERR_CUDA;
-        return SAS_ERR_DEVICE_TIMEOUT;
-    }
-    return SAS_OK;
+sas_status sas_get_device_status(int32_t* status, sas_stream_t stream) {
+    if (!status) return SAS_ERR_INVALID_VALUE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SAS_ERR_CUDA;
+    int32_t word = 0;
+    if (cudaMemcpyAsync(&word, status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SAS_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SAS_ERR_CUDA;
+    if (word == 0) return SAS_OK;
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return SAS_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SAS_ERR_CUDA;
+    return word == SAS_ERR_DEVICE_TIMEOUT ? SAS_ERR_DEVICE_TIMEOUT : SAS_ERR_CUDA;
 }
 
-sas_status sas_selftest_bounded_wait(int32_t limit_ms, sas_stream_t stream) {
-    if (limit_ms <= 0 || limit_ms > 10000) return SAS_ERR_INVALID_VALUE;
-    DeviceInfo di;
-    if (device_info(&di) != cudaSuccess) return SAS_ERR_CUDA;
-    return from_cuda(launch_selftest_wait(di.status, (unsigned long long)limit_ms * 1000000ull,
+sas_status sas_selftest_bounded_wait(int32_t limit_ms, int32_t* status, int32_t* trace, sas_stream_t stream) {
+    if (limit_ms <= 0 || limit_ms > 10000 || !status) return SAS_ERR_INVALID_VALUE;
+    return from_cuda(launch_selftest_wait(status, trace, (unsigned long long)limit_ms * 1000000ull,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 

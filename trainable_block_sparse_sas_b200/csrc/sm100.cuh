@@ -13,10 +13,11 @@
 namespace sas {
 namespace sm100 {
 
-// Status code a timed-out wait writes to the library's device status word.
+// Status code a timed-out wait writes to the caller's device status word.
 constexpr int kStatusTimeout = 5;
-// A wait gives up after this long (ns of %globaltimer): far above any healthy
-// wait in these kernels, short enough to return control to the host.
+// A kernel's waits give up after this long (ns of %globaltimer): far above any
+// healthy wait in these kernels, short enough to return control to the host.
+// The self-test passes a shorter limit to the same routines.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -60,12 +61,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                                   uint64_t limit_ns) {
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort = 1;
             if (status) atomicExch(status, kStatusTimeout);
             return false;
@@ -74,27 +76,30 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
 }
 
 // Wait for the phase of parity `parity` to complete.  Gives up when `abort`
-// is set by another thread, or after kWaitLimitNs (then sets `abort` and the
+// is set by another thread, or after limit_ns (then sets `abort` and the
 // device status word).  Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
-    return mbar_wait_slow(bar, parity, abort, status);
+    return mbar_wait_slow(bar, parity, abort, status, limit_ns);
 }
 
 
 // Whole-warp wait with a warp-uniform outcome; the warp leaves it converged,
 // ready for .aligned instructions (tcgen05.ld, ldmatrix, mma.sync).
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status) {
-    const bool ok = mbar_wait(bar, parity, abort, status);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+    const bool ok = mbar_wait(bar, parity, abort, status, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
 // Time-bounded wait that ignores the abort flag (used to drain in-flight work
 // before TMEM is released).  Returns false on timeout.
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, int* status) {
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, int* status,
+                                                uint64_t limit_ns = kWaitLimitNs) {
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             if (status) atomicExch(status, kStatusTimeout);
             return false;
         }
