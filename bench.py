@@ -720,6 +720,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4096, help="tokens of the oracle's CPU-baseline sample")
     ap.add_argument("--reference-tokens", type=int, default=1024, help="tokens of the reference arm's sample")
+    ap.add_argument("--profile-train", type=int, default=0, metavar="N",
+                    help="only run training steps of the 32K workload's geometry at sequence length N (a small "
+                         "case for profiler captures) and print the per-kernel timing")
     ap.add_argument("--profile-decode", type=int, default=0, metavar="T",
                     help="only run the fused decode of the 128K workload's geometry with a T-token cache "
                          "(a small case for profiler captures) and print its timing")
@@ -731,6 +734,24 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.profile_train:
+        import torch
+
+        from trainable_block_sparse_sas_b200 import api
+        from trainable_block_sparse_sas_b200 import synthetic as syn
+
+        w = dataclasses.replace(syn.TRAIN_SPARSE_32K, name="train_sparse_geometry", n=args.profile_train)
+        r = TrainRunner(api, w, syn.train_inputs(w, device="cuda", seed=1000))
+        for _ in range(args.warmup):
+            r.step()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            r.step(evs[i])
+        torch.cuda.synchronize()
+        ms = {k: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+              for k, (a, b) in {"select": (0, 1), "fwd": (1, 2), "bwd_dq": (2, 3), "bwd_dkdv": (3, 4)}.items()}
+        print(json.dumps({"workload": w.name, "n": w.n, "ms": ms}))
         return
     if args.profile_decode:
         from trainable_block_sparse_sas_b200 import api

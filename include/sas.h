@@ -63,7 +63,10 @@ typedef enum {
     SAS_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. head_dim) */
     SAS_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_size query */
     SAS_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed */
-    SAS_ERR_DEVICE_TIMEOUT = 5       /* a bounded device-side wait gave up */
+    SAS_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up */
+    SAS_ERR_DEVICE_BOUNDS = 6        /* debug-bounds build only: a kernel's index check failed (the
+                                        access was skipped); the status word holds the source line
+                                        in its bits 8 and up */
 } sas_status;
 
 typedef enum { SAS_F32 = 0, SAS_BF16 = 1 } sas_dtype;
@@ -372,9 +375,10 @@ sas_status sas_sparse_decode_noalloc(const sas_decode_desc* desc, const void* q,
 
 /* sas_get_device_status -- synchronises `stream`, then reads the caller's device
  * status word and clears it: SAS_OK (the word held 0) or the code a kernel wrote
- * there (SAS_ERR_DEVICE_TIMEOUT: a bounded wait gave up; the outputs of the calls
- * since the last read are undefined).  SAS_ERR_CUDA if the synchronisation or the
- * copy fails; SAS_ERR_INVALID_VALUE for a NULL word. */
+ * there (SAS_ERR_DEVICE_TIMEOUT: a bounded wait gave up; SAS_ERR_DEVICE_BOUNDS: in
+ * the debug-bounds build, an index check failed; either way the outputs of the
+ * calls since the last read are undefined).  SAS_ERR_CUDA if the synchronisation
+ * or the copy fails; SAS_ERR_INVALID_VALUE for a NULL word. */
 sas_status sas_get_device_status(int32_t* status, sas_stream_t stream);
 
 /* sas_selftest_bounded_wait -- self-test of the failure path of the tensor-core

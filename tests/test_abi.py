@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(api):
 
 
 def test_status_strings(api):
-    for st in range(6):
+    for st in range(7):
         assert api.lib.sas_status_string(st)
     assert api.lib.sas_version() >= 100
 

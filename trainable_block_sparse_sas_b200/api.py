@@ -15,13 +15,15 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas.so")
+# SAS_LIBRARY names another build of the same library (the debug-bounds build,
+# libsas_debug.so, made by `python -m trainable_block_sparse_sas_b200.build --debug-bounds`)
+_LIB_PATH = os.environ.get("SAS_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsas.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"libsas.so not built at {_LIB_PATH}: run python -m trainable_block_sparse_sas_b200.build")
 lib = ctypes.CDLL(_LIB_PATH)
 
 SAS_OK, SAS_ERR_INVALID_VALUE, SAS_ERR_UNSUPPORTED, SAS_ERR_WORKSPACE_TOO_SMALL, SAS_ERR_CUDA, \
-    SAS_ERR_DEVICE_TIMEOUT = range(6)
+    SAS_ERR_DEVICE_TIMEOUT, SAS_ERR_DEVICE_BOUNDS = range(7)
 SAS_F32, SAS_BF16 = 0, 1
 SAS_SCOPE_SPARSE, SAS_SCOPE_FULL = 0, 1
 SAS_GATE_SOFTMAX, SAS_GATE_SIGMOID, SAS_GATE_RAW, SAS_GATE_OUTER, SAS_GATE_STE = 0, 1, 2, 3, 4

@@ -1,9 +1,13 @@
 """Build libsas.so (the CUDA kernels and their C ABI) in-tree for sm_100a.
 
-    python -m trainable_block_sparse_sas_b200.build [--force] [-v]
+    python -m trainable_block_sparse_sas_b200.build [--force] [-v] [--debug-bounds]
 
 Each csrc/*.cu is compiled to an object under _build/ (in parallel, skipped when
-up to date), then linked into trainable_block_sparse_sas_b200/libsas.so.
+up to date), then linked into trainable_block_sparse_sas_b200/libsas.so.  With
+--debug-bounds the same sources are built with -DSAS_DEBUG_BOUNDS (every kernel
+checks the global-memory indices it computes against its buffers' extents and
+records a failure in the caller's status word instead of making the access) into
+libsas_debug.so, objects under _build/debug_bounds/.
 """
 from __future__ import annotations
 
@@ -20,6 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsas.so")
+LIB_DEBUG = os.path.join(PKG, "libsas_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -39,8 +44,8 @@ def _deps_mtime() -> float:
     return max((os.path.getmtime(f) for f in files), default=0.0)
 
 
-def _compile(src: str, obj: str, verbose: bool) -> str:
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+def _compile(src: str, obj: str, verbose: bool, extra=()) -> str:
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -49,30 +54,33 @@ def _compile(src: str, obj: str, verbose: bool) -> str:
     return r.stderr
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False) -> str:
+    out_dir = os.path.join(BUILD, "debug_bounds") if debug_bounds else BUILD
+    lib = LIB_DEBUG if debug_bounds else LIB
+    extra = ("-DSAS_DEBUG_BOUNDS",) if debug_bounds else ()
+    os.makedirs(out_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     deps = _deps_mtime()
     jobs = []
     objs = []
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(out_dir, os.path.basename(src) + ".o")
         objs.append(obj)
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), deps):
             jobs.append((src, obj))
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, max(1, len(jobs)))) as ex:
-        for (src, _), log in zip(jobs, ex.map(lambda j: _compile(j[0], j[1], verbose), jobs)):
+        for (src, _), log in zip(jobs, ex.map(lambda j: _compile(j[0], j[1], verbose, extra), jobs)):
             if verbose and log:
                 sys.stderr.write(f"== {os.path.basename(src)}\n{log}")
-    if jobs or force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        tmp = LIB + ".tmp"
+    if jobs or force or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        tmp = lib + ".tmp"
         cmd = [nvcc(), *ARCH, "-shared", *objs, "-o", tmp, "-lcuda"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))

@@ -209,7 +209,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         // attended history blocks (ascending) with their log-gate biases, then the
         // current block (bias 0); lanes read the selection in parallel
         const float* srow = a.s + unit * a.Cq;
-        const float lse_c = gate_softmax_family(a.gate) ? a.lse_s[unit] : 0.f;
+        const long n_units = (long)a.B * a.Hkv * a.Cq;
+        const float lse_c =
+            gate_softmax_family(a.gate) && SAS_IN_BOUNDS(unit, n_units, a.status) ? a.lse_s[unit] : 0.f;
         int cnt = 0;
         const int kk = a.full_scope ? c : min(a.top_k, c);
         const int32_t* row = a.idx + unit * a.top_k;
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             }
             __syncwarp();
             for (int i = lane; i < kk; i += 32) {
-                const int v = row[i];
+                const int v = SAS_IN_BOUNDS(unit * a.top_k + i, n_units * a.top_k, a.status) ? row[i] : -1;
                 if (v >= 0 && v < c) wgt[v] = 1.f;
             }
             __syncwarp();
@@ -230,8 +232,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         } else {
             for (int base_i = 0; base_i < kk; base_i += 32) {
                 const int i = base_i + lane;
-                const int v = i < kk ? (a.full_scope ? i : row[i]) : -1;
-                const bool ok = v >= 0 && v < c;
+                const int v = i < kk ? (a.full_scope ? i
+                                        : SAS_IN_BOUNDS(unit * a.top_k + i, n_units * a.top_k, a.status) ? row[i]
+                                                                                                          : -1)
+                                     : -1;
+                const bool ok = v >= 0 && v < c && SAS_IN_BOUNDS(unit * a.Cq + v, n_units * a.Cq, a.status);
                 const unsigned bal = __ballot_sync(0xffffffffu, ok);
                 if (ok) {
                     const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
@@ -249,6 +254,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             wgt[cnt] = 1.f;
             *list_count = cnt + 1;
         }
+        __syncwarp();  // the warp reaches the CTA barrier converged
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -272,6 +278,9 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 }
             }
         }
+        // every warp reaches the CTA barrier below converged: a barrier reached by a
+        // warp in diverged pieces can release it before the other warps arrive
+        __syncwarp();
     } else if (warp < kDqSoftmaxWarp0) {
         const int i = (warp - 1) >> 1;       // M-tile
         const bool dp_chain = ((warp - 1) & 1) != 0;
@@ -325,6 +334,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             mma_commit(drain);
             mbar_wait_drain(drain, 0, a.status);
         }
+        __syncwarp();
     } else {
         const int wi = warp - kDqSoftmaxWarp0;  // 0..7
         const int grp = wi >> 2;
@@ -335,12 +345,15 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             const int tok = r_unit / G, g = r_unit % G;
             const int hq = h * G + g;
             const long ri = ((long)b * a.Hq + hq) * a.n + c * kBS + tok;
-            const float lse2 = a.lse[ri] * kLog2e;
+            const long e0 = (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
+            // debug-bounds build: this row's global indices (o, dO, dq rows; lse, D)
+            const bool inb = SAS_IN_BOUNDS(e0 + kD - 1, (long)a.B * a.n * a.Hq * kD, a.status) &&
+                             SAS_IN_BOUNDS(ri, (long)a.B * a.Hq * a.n, a.status);
+            const float lse2 = inb ? a.lse[ri] * kLog2e : 0.f;
             // D = dO . o of this row (fp32 sum of the bf16 products), kept for the
             // dk/dv kernel as well
-            float Drow;
-            {
-                const long e0 = (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
+            float Drow = 0.f;
+            if (inb) {
                 const uint4* po = reinterpret_cast<const uint4*>(a.o + e0);
                 const uint4* pd = reinterpret_cast<const uint4*>(a.dO + e0);
                 uint64_t acc2 = 0ull;
@@ -360,6 +373,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 Drow = da + db;
                 a.Dbuf[ri] = Drow;
             }
+            const long n_mass = (long)gridDim.x * dq_list_max(a.Cq, a.top_k, a.full_scope, a.gate) * (128 * MT);
             const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
             const uint32_t tS = tmem + lane_off + grp * 128, tP = tS + 64;
             const uint32_t tQ = tmem + lane_off + 256 + grp * 128;
@@ -423,12 +437,13 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                 if (!cur) {
                     float ma, mb;
                     f2_unpack(m2, ma, mb);
-                    mrow[t * (128 * MT)] = __float2bfloat16_rn(ma + mb);
+                    if (SAS_IN_BOUNDS((mrow - a.Mbuf) + (long)t * (128 * MT), n_mass, a.status))
+                        mrow[t * (128 * MT)] = __float2bfloat16_rn(ma + mb);
                     rs = warp_sum(rs);
                     if (lane == 0) part[t * 8 + wi] = rs;
                 }
             }
-            a.Dbuf[ri] = Drow + delta;  // D for dk / dv
+            if (inb) a.Dbuf[ri] = Drow + delta;  // D for dk / dv
             // dlogg_t = sum_i (dS-sum_it - coef_i M_it): the exact-D correction, or
             // for the outer gate g_t sum P dP = dS-sum + D M
             a.Cbuf[(long)blockIdx.x * (128 * MT) + r_unit] = kOuter ? -Drow : delta;
@@ -444,8 +459,11 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
                     for (int j = 0; j < 16; ++j)
                         o[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * a.scale, __uint_as_float(r[2 * j + 1]) * a.scale);
                     uint4* dst = reinterpret_cast<uint4*>(drow + ch * 32);
+                    if (inb) {
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+                    }
                 }
             }
         }
@@ -503,6 +521,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     }
     __syncthreads();
     if (*abort_flag) return;
+    if (!SAS_IN_BOUNDS((unit + 1) * a.Cq - 1, (long)a.B * a.Hkv * a.Cq * a.Cq, a.status)) return;
     const float tot = *tot_sh;
     const float* srow = a.s + unit * a.Cq;
     float* dsrow = a.ds + unit * a.Cq;
@@ -552,6 +571,7 @@ struct DkvLayout {
 // is history block m in the ascending selection of query block c (unit uc)?
 __device__ __forceinline__ bool holds(const BwdArgs& a, long uc, int c, int m) {
     int lo = 0, hi = min(a.top_k, c) - 1;
+    if (!SAS_IN_BOUNDS(uc * a.top_k + hi, (long)a.B * a.Hkv * a.Cq * a.top_k, a.status)) return false;
     const int32_t* row = a.idx + uc * a.top_k;
     while (lo <= hi) {
         const int mid = (lo + hi) >> 1;
@@ -671,6 +691,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                 }
             }
         }
+        // every warp reaches the CTA barrier below converged: a barrier reached by a
+        // warp in diverged pieces can release it before the other warps arrive
+        __syncwarp();
     } else if (warp < kKvSoftmaxWarp0) {
         const int chain = warp - 1;  // 0 S, 1 dP, 2 dV, 3 dK
         if (lane < (chain < 2 ? 1 : 2)) {
@@ -723,6 +746,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             mma_commit(drain);
             mbar_wait_drain(drain, 0, a.status);
         }
+        __syncwarp();
     } else {
         const int quad = warp & 3;
         const int kw = (warp - kKvSoftmaxWarp0) >> 2;  // key half of the block handled by this group
@@ -737,12 +761,15 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             const int g = r_unit % G;
             const long ri = ((long)b * a.Hq + h * G + g) * a.n + c * kBS + tok;
             diag = (c == m);
+            const long n_units = (long)a.B * a.Hkv * a.Cq;
+            const bool inb = SAS_IN_BOUNDS((ubase + c) * a.Cq + m, n_units * a.Cq, a.status) &&
+                             SAS_IN_BOUNDS(ri, (long)a.B * a.Hq * a.n, a.status);
             const float lg =
-                diag ? 0.f
-                     : gate_log(a.s[(ubase + c) * a.Cq + m],
-                                gate_softmax_family(a.gate) ? a.lse_s[ubase + c] : 0.f, a.gate);
-            off = (gate_in_logits(a.gate) ? lg * kLog2e : 0.f) - a.lse[ri] * kLog2e;
-            dneg = -a.Dbuf[ri];
+                (diag || !inb) ? 0.f
+                               : gate_log(a.s[(ubase + c) * a.Cq + m],
+                                          gate_softmax_family(a.gate) ? a.lse_s[ubase + c] : 0.f, a.gate);
+            off = (gate_in_logits(a.gate) ? lg * kLog2e : 0.f) - (inb ? a.lse[ri] : 0.f) * kLog2e;
+            dneg = inb ? -a.Dbuf[ri] : 0.f;
             w = (kOuter && !diag) ? expf(lg) : 1.f;
         };
         float off = 0.f, dneg = 0.f, w = 1.f;
@@ -825,8 +852,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
 #pragma unroll
                 for (int jx = 0; jx < 32; ++jx) {
                     const int key = ch * 32 + jx;
-                    dst[(((long)b * a.n + m * kBS + key) * a.Hkv + h) * kD + d] =
-                        __float2bfloat16_rn((__uint_as_float(r0[jx]) + __uint_as_float(r1[jx])) * mul);
+                    const long di = (((long)b * a.n + m * kBS + key) * a.Hkv + h) * kD + d;
+                    if (SAS_IN_BOUNDS(di, (long)a.B * a.n * a.Hkv * kD, a.status))
+                        dst[di] = __float2bfloat16_rn((__uint_as_float(r0[jx]) + __uint_as_float(r1[jx])) * mul);
                 }
             }
         }

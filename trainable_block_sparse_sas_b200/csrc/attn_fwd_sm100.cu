@@ -163,14 +163,18 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         // the current block (bias 0), then the attended history blocks (ascending)
         // with their log-gate biases; lanes read the selection in parallel
         const float* srow = a.s + unit * a.Cq;
-        const float lse_c = gate_softmax_family(a.gate) ? a.lse_s[unit] : 0.f;
+        const long n_units = (long)a.B * a.Hkv * a.Cq;
+        const float lse_c =
+            gate_softmax_family(a.gate) && SAS_IN_BOUNDS(unit, n_units, a.status) ? a.lse_s[unit] : 0.f;
         int cnt = 0;
         const int kk = a.full_scope ? c : min(a.top_k, c);
         const int32_t* row = a.idx + unit * a.top_k;
         for (int base_i = 0; base_i < kk; base_i += 32) {
             const int i = base_i + lane;
-            const int v = i < kk ? (a.full_scope ? i : row[i]) : -1;
-            const bool ok = v >= 0 && v < c;
+            const int v = i < kk ? (a.full_scope ? i
+                                    : SAS_IN_BOUNDS(unit * a.top_k + i, n_units * a.top_k, a.status) ? row[i] : -1)
+                                 : -1;
+            const bool ok = v >= 0 && v < c && SAS_IN_BOUNDS(unit * a.Cq + v, n_units * a.Cq, a.status);
             const unsigned bal = __ballot_sync(0xffffffffu, ok);
             if (ok) {
                 const int pos = 1 + cnt + __popc(bal & ((1u << lane) - 1u));
@@ -187,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             if (kOuter) wgt[0] = 1.f;
             *list_count = cnt + 1;
         }
+        __syncwarp();  // the warp reaches the CTA barrier converged
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -212,6 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                 }
             }
         }
+        // every warp reaches the CTA barrier below converged: a barrier reached by a
+        // warp in diverged pieces can release it before the other warps arrive
+        __syncwarp();
     } else if (warp <= 4) {
         // ------------------------------------------------------------ MMA issuers
         // warps 1, 3: S_i = Q_i K^T for tile i = (warp - 1) / 2; warps 2, 4: O_i += P_i V
@@ -258,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             mma_commit(drain);
             mbar_wait_drain(drain, 0, a.status);
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
         const int grp = (warp - kSoftmaxWarp0) >> 2;
@@ -351,6 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                 mbar_arrive(p_ready(grp, bf));
             }
             const int tl = nlist - 1;
+            // the row's outputs (the checks of the debug-bounds build skip the stores
+            // only: the TMEM loads below are whole-warp instructions)
+            const long orow_i = (((long)b * a.n + c * kBS + tok) * a.Hq + h * G + g) * kD;
+            const long lse_i = ((long)b * a.Hq + h * G + g) * a.n + c * kBS + tok;
+            const bool inb = SAS_IN_BOUNDS(orow_i + kD - 1, (long)a.B * a.n * a.Hq * kD, a.status) &&
+                             SAS_IN_BOUNDS(lse_i, (long)a.B * a.Hq * a.n, a.status);
             if (ok && warp_wait(pv_done(grp, tl & 1), (tl >> 1) & 1, abort_flag, a.status)) {
                 tc_fence_after();
                 const float inv_l = 1.f / l;
@@ -365,11 +380,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
                     for (int j = 0; j < 16; ++j)
                         pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * inv_l, __uint_as_float(r[2 * j + 1]) * inv_l);
                     uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+                    if (inb) {
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                    }
                 }
-                a.lse[((long)b * a.Hq + hq) * a.n + c * kBS + tok] = m_used * kLn2 + logf(l);
+                if (inb) a.lse[lse_i] = m_used * kLn2 + logf(l);
             }
         }
     }

@@ -60,13 +60,22 @@ __device__ __forceinline__ void stg(void* p, long i, float v) {
     static_cast<T*>(p)[i] = from_f32<T>(v);
 }
 
+// a store of element i of a tensor of n elements (checked in the debug-bounds build)
+template <typename T>
+__device__ __forceinline__ void stg_chk(void* p, long i, long n, float v, int* status) {
+    if (SAS_IN_BOUNDS(i, n, status)) static_cast<T*>(p)[i] = from_f32<T>(v);
+}
+
 // rows [BS] of head `head` (of `H` heads) starting at token t0 -> smem [BS][LD]
+// (the debug-bounds build checks each index against the tensor's B n H D elements)
 template <typename T, int D, int BS>
-__device__ __forceinline__ void load_rows(float* dst, const void* src, int b, int n, int H, int head, int t0) {
+__device__ __forceinline__ void load_rows(float* dst, const void* src, int b, int n, int H, int head, int t0,
+                                          const TrainParams& p) {
     using C = Cfg<D, BS>;
     for (int i = threadIdx.x; i < BS * D; i += kThreads) {
         const int r = i / D, e = i % D;
-        dst[r * C::LD + e] = ldg<T>(src, (((long)b * n + t0 + r) * H + head) * D + e);
+        const long gi = (((long)b * n + t0 + r) * H + head) * D + e;
+        dst[r * C::LD + e] = SAS_IN_BOUNDS(gi, (long)p.B * n * H * D, p.status) ? ldg<T>(src, gi) : 0.f;
     }
 }
 
@@ -85,8 +94,9 @@ __device__ __forceinline__ int build_list(const TrainParams& p, long unit, int c
         const int kk = min(p.top_k, c);
         const int32_t* row = p.idx + unit * p.top_k;
         int cnt = 0;
+        const long n_idx = (long)p.B * p.Hkv * p.Cq * p.top_k;
         for (int i = 0; i < kk; ++i) {
-            const int v = row[i];
+            const int v = SAS_IN_BOUNDS(unit * p.top_k + i, n_idx, p.status) ? row[i] : -1;
             if (v >= 0 && v < c) blocks[cnt++] = v;
         }
         blocks[cnt] = c;
@@ -106,8 +116,9 @@ __device__ __forceinline__ int build_list_all(const TrainParams& p, long unit, i
     if (!p.full_scope && threadIdx.x == 0) {
         const int kk = min(p.top_k, c);
         const int32_t* row = p.idx + unit * p.top_k;
+        const long n_idx = (long)p.B * p.Hkv * p.Cq * p.top_k;
         for (int i = 0; i < kk; ++i) {
-            const int v = row[i];
+            const int v = SAS_IN_BOUNDS(unit * p.top_k + i, n_idx, p.status) ? row[i] : -1;
             if (v >= 0 && v < c) blocks[v] = v;
         }
     }
@@ -138,7 +149,7 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
     const float* srow = p.s + unit * p.Cq;
     const float lse_c = gate_softmax_family(p.gate) ? p.lse_s[unit] : 0.f;
 
-    load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
+    load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS, p);
     if (tid < BS) {
         row_m[tid] = -INFINITY;
         row_l[tid] = 0.f;
@@ -157,8 +168,8 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
         const float bias = gate_in_logits(p.gate) ? lg : 0.f;
         const float w = (p.gate == kGateOuter && !cur) ? expf(lg) : 1.f;  // outer gate: g weights V
         __syncthreads();
-        load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
-        load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
+        load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS, p);
+        load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS, p);
         __syncthreads();
         for (int tile = tid; tile < C::NT_S; tile += kThreads) {
             const int ttr = tile / C::RG, ttc = tile % C::RG;
@@ -226,9 +237,11 @@ __global__ void __launch_bounds__(kThreads) fwd_simt_kernel(TrainParams p) {
         const float inv = 1.f / row_l[r];
         const long base = (((long)b * p.n + c * BS + r) * p.Hq + hq) * D;
 #pragma unroll
-        for (int ee = 0; ee < C::COLS; ++ee) stg<T>(p.o, base + tc + C::CG * ee, acc[ii][ee] * inv);
+        for (int ee = 0; ee < C::COLS; ++ee)
+            stg_chk<T>(p.o, base + tc + C::CG * ee, (long)p.B * p.n * p.Hq * D, acc[ii][ee] * inv, p.status);
     }
-    if (tid < BS) p.lse[((long)b * p.Hq + hq) * p.n + c * BS + tid] = row_m[tid] + logf(row_l[tid]);
+    const long li = ((long)b * p.Hq + hq) * p.n + c * BS + tid;
+    if (tid < BS && SAS_IN_BOUNDS(li, (long)p.B * p.Hq * p.n, p.status)) p.lse[li] = row_m[tid] + logf(row_l[tid]);
 }
 
 // One 4x4 micro-tile of S = Q K^T (unscaled) and dP = dO V^T: rows ttr + RG*ii
@@ -294,10 +307,12 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
     for (int g = 0; g < G; ++g) {
         const int hq = h * G + g;
         __syncthreads();
-        load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
-        load_rows<T, D, BS>(dOs, p.dO, b, p.n, p.Hq, hq, c * BS);
+        load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS, p);
+        load_rows<T, D, BS>(dOs, p.dO, b, p.n, p.Hq, hq, c * BS, p);
+        const long ri = ((long)b * p.Hq + hq) * p.n + c * BS + tid;
+        const bool ri_ok = tid < BS && SAS_IN_BOUNDS(ri, (long)p.B * p.Hq * p.n, p.status);
         if (tid < BS) {
-            rowL[tid] = p.lse_in[((long)b * p.Hq + hq) * p.n + c * BS + tid];
+            rowL[tid] = ri_ok ? p.lse_in[ri] : 0.f;
             rowD[tid] = 0.f;
         }
         // pass 1: D_i = sum_j P_ij w_j dP_ij over the blocks the forward attended
@@ -309,8 +324,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
             const float bias = gate_in_logits(p.gate) ? lg : 0.f;
             const float w = (p.gate == kGateOuter && !cur) ? expf(lg) : 1.f;
             __syncthreads();
-            load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, code * BS);
-            load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, code * BS);
+            load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, code * BS, p);
+            load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, code * BS, p);
             __syncthreads();
             for (int tile = tid; tile < C::NT_S; tile += kThreads) {
                 const int ttr = tile / C::RG, ttc = tile % C::RG;
@@ -334,7 +349,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
             }
         }
         __syncthreads();
-        if (tid < BS) p.Dbuf[((long)b * p.Hq + hq) * p.n + c * BS + tid] = rowD[tid];  // for dk / dv
+        if (ri_ok) p.Dbuf[ri] = rowD[tid];  // for dk / dv
         float acc[4][C::COLS];
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii)
@@ -351,8 +366,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
             const float bias = gate_in_logits(p.gate) ? lg : 0.f;
             const float w = (p.gate == kGateOuter && !cur) ? expf(lg) : 1.f;
             __syncthreads();
-            load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS);
-            load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS);
+            load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, blk * BS, p);
+            load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, blk * BS, p);
             __syncthreads();
             float local = 0.f;
             for (int tile = tid; tile < C::NT_S; tile += kThreads) {
@@ -395,7 +410,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
             const int r = tr + C::RG * ii;
             const long base = (((long)b * p.n + c * BS + r) * p.Hq + hq) * D;
 #pragma unroll
-            for (int ee = 0; ee < C::COLS; ++ee) stg<T>(p.dq, base + tc + C::CG * ee, p.scale * acc[ii][ee]);
+            for (int ee = 0; ee < C::COLS; ++ee)
+                stg_chk<T>(p.dq, base + tc + C::CG * ee, (long)p.B * p.n * p.Hq * D, p.scale * acc[ii][ee], p.status);
         }
     }
     __syncthreads();
@@ -409,6 +425,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
     for (int i = tid; i < nsel; i += kThreads) part += dlg[i];
     const float tot = block_sum(part, red);
     float* dsrow = p.ds + unit * p.Cq;
+    if (!SAS_IN_BOUNDS((unit + 1) * p.Cq - 1, (long)p.B * p.Hkv * p.Cq * p.Cq, p.status)) return;
     for (int m = tid; m < p.Cq; m += kThreads)
         dsrow[m] = (m < c && gate_softmax_family(p.gate)) ? -expf(srow[m] - lse_c) * tot : 0.f;
     __syncthreads();
@@ -422,6 +439,7 @@ __global__ void __launch_bounds__(kThreads) bwd_dq_kernel(TrainParams p) {
 __device__ __forceinline__ bool selected(const TrainParams& p, long unit_c, int c, int m) {
     if (p.full_scope) return m < c;
     int lo = 0, hi = min(p.top_k, c) - 1;
+    if (!SAS_IN_BOUNDS(unit_c * p.top_k + hi, (long)p.B * p.Hkv * p.Cq * p.top_k, p.status)) return false;
     const int32_t* row = p.idx + unit_c * p.top_k;
     while (lo <= hi) {
         const int mid = (lo + hi) >> 1;
@@ -454,8 +472,8 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
     const int b = (int)(blockIdx.x / ((long)p.Cq * p.Hkv));
     const int G = p.Hq / p.Hkv;
     const long ubase = ((long)b * p.Hkv + h) * p.Cq;
-    load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, m * BS);
-    load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, m * BS);
+    load_rows<T, D, BS>(Ks, p.k, b, p.n, p.Hkv, h, m * BS, p);
+    load_rows<T, D, BS>(Vs, p.v, b, p.n, p.Hkv, h, m * BS, p);
     const int tr = tid / C::CG, tc = tid % C::CG;  // rows here are keys j
     float dk[4][C::COLS], dv[4][C::COLS];
 #pragma unroll
@@ -482,12 +500,13 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
             for (int g = 0; g < G; ++g) {
                 const int hq = h * G + g;
                 __syncthreads();
-                load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS);
-                load_rows<T, D, BS>(dOs, p.dO, b, p.n, p.Hq, hq, c * BS);
+                load_rows<T, D, BS>(Qs, p.q, b, p.n, p.Hq, hq, c * BS, p);
+                load_rows<T, D, BS>(dOs, p.dO, b, p.n, p.Hq, hq, c * BS, p);
                 if (tid < BS) {
                     const long ri = ((long)b * p.Hq + hq) * p.n + c * BS + tid;
-                    rowL[tid] = p.lse_in[ri];
-                    rowD[tid] = p.Dbuf[ri];
+                    const bool ok = SAS_IN_BOUNDS(ri, (long)p.B * p.Hq * p.n, p.status);
+                    rowL[tid] = ok ? p.lse_in[ri] : 0.f;
+                    rowD[tid] = ok ? p.Dbuf[ri] : 0.f;
                 }
                 __syncthreads();
                 for (int tile = tid; tile < C::NT_S; tile += kThreads) {
@@ -534,8 +553,9 @@ __global__ void __launch_bounds__(kThreads) bwd_dkdv_kernel(TrainParams p) {
         const long base = (((long)b * p.n + m * BS + j) * p.Hkv + h) * D;
 #pragma unroll
         for (int ee = 0; ee < C::COLS; ++ee) {
-            stg<T>(p.dk, base + tc + C::CG * ee, p.scale * dk[ii][ee]);
-            stg<T>(p.dv, base + tc + C::CG * ee, dv[ii][ee]);
+            const long n_kv = (long)p.B * p.n * p.Hkv * D;
+            stg_chk<T>(p.dk, base + tc + C::CG * ee, n_kv, p.scale * dk[ii][ee], p.status);
+            stg_chk<T>(p.dv, base + tc + C::CG * ee, n_kv, dv[ii][ee], p.status);
         }
     }
 }

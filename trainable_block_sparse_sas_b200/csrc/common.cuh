@@ -7,6 +7,24 @@
 
 namespace sas {
 
+// Index checks of the debug-bounds build (compiled with -DSAS_DEBUG_BOUNDS): a
+// global-memory index the kernel computed is compared with the extent the
+// problem shape gives its buffer; an index outside it records
+// SAS_ERR_DEVICE_BOUNDS (6) and the source line (bits 8 and up) in the caller's
+// device status word -- the first failure wins -- and the access is skipped.
+// Nothing traps.  Release builds compile every check to `true`.
+constexpr int kStatusBounds = 6;
+#ifdef SAS_DEBUG_BOUNDS
+__device__ __noinline__ inline bool bounds_fail(int* status, int line) {
+    if (status) atomicCAS(status, 0, kStatusBounds | (line << 8));
+    return false;
+}
+#define SAS_IN_BOUNDS(i, n, status) \
+    (((long long)(i) >= 0 && (long long)(i) < (long long)(n)) || ::sas::bounds_fail((status), __LINE__))
+#else
+#define SAS_IN_BOUNDS(i, n, status) ((void)(i), (void)(n), (void)(status), true)
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -33,7 +33,10 @@ __device__ __forceinline__ DecodeList decode_list(const DecodeParams& p, int b, 
     } else {
         const int32_t* row = p.idx + ((long)b * p.Hkv + h) * p.top_k;
         int cnt = 0;
-        while (cnt < p.top_k && row[cnt] >= 0 && row[cnt] < L.cur_blk) ++cnt;
+        const long n_idx = (long)p.B * p.Hkv * p.top_k;
+        while (cnt < p.top_k && SAS_IN_BOUNDS(((long)b * p.Hkv + h) * p.top_k + cnt, n_idx, p.status) &&
+               row[cnt] >= 0 && row[cnt] < L.cur_blk)
+            ++cnt;
         L.nsel = cnt;
     }
     return L;
@@ -60,10 +63,16 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeParams p
     const DecodeList L = decode_list(p, b, h);
     const int li0 = split * p.per_split, li1 = min(L.nsel + 1, li0 + p.per_split);
     float* part = p.part + ((long)bh * p.nsplit + split) * G * (D + 2);
+    // the partials of this CTA, within the workspace (or the built-in scratch)
+    const long n_part = (long)p.B * p.Hkv * p.nsplit * G * (D + 2);
+    if (!SAS_IN_BOUNDS(((long)bh * p.nsplit + split + 1) * G * (D + 2) - 1, n_part, p.status)) return;
 
     for (int i = tid; i < G * D; i += kThreads) {
         const int g = i / D, e = i % D;
-        qs[i] = to_f32<T>(static_cast<const T*>(p.q)[((long)b * p.Hq + h * G + g) * D + e]) * p.scale;
+        const long qi = ((long)b * p.Hq + h * G + g) * D + e;
+        qs[i] = SAS_IN_BOUNDS(qi, (long)p.B * p.Hq * D, p.status)
+                    ? to_f32<T>(static_cast<const T*>(p.q)[qi]) * p.scale
+                    : 0.f;
     }
     __syncthreads();
     const T* kc = static_cast<const T*>(p.k) + (long)bh * p.Tmax * D;
@@ -77,7 +86,11 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeParams p
         for (int j = j0 + warp; j < j1; j += kThreads / 32) {
             float kv[D / 32];
 #pragma unroll
-            for (int u = 0; u < D / 32; ++u) kv[u] = to_f32<T>(kc[(long)j * D + lane + 32 * u]);
+            for (int u = 0; u < D / 32; ++u)
+                kv[u] = SAS_IN_BOUNDS(((long)bh * p.Tmax + j) * D + lane + 32 * u, (long)p.B * p.Hkv * p.Tmax * D,
+                                      p.status)
+                            ? to_f32<T>(kc[(long)j * D + lane + 32 * u])
+                            : 0.f;
             for (int g = 0; g < G; ++g) {
                 float a = 0.f;
 #pragma unroll
@@ -117,7 +130,10 @@ __global__ void __launch_bounds__(kThreads) decode_partial_kernel(DecodeParams p
             const int blk = list_block(p, L, b, h, li);
             const int j0 = blk * p.bs, j1 = min(j0 + p.bs, L.t + 1);
             for (int j = j0; j < j1; ++j, ++jt) {
-                const float vv = to_f32<T>(vc[(long)j * D + e]);
+                const float vv =
+                    SAS_IN_BOUNDS(((long)bh * p.Tmax + j) * D + e, (long)p.B * p.Hkv * p.Tmax * D, p.status)
+                        ? to_f32<T>(vc[(long)j * D + e])
+                        : 0.f;
 #pragma unroll
                 for (int g = 0; g < kMaxG; ++g)
                     if (g < G) acc[g] = fmaf(sc[g * ntok_max + jt], vv, acc[g]);
@@ -139,6 +155,9 @@ __global__ void __launch_bounds__(kThreads) decode_combine_kernel(DecodeParams p
     const int bh = blockIdx.x;
     const int b = bh / p.Hkv, h = bh % p.Hkv;
     const float* part = p.part + (long)bh * p.nsplit * G * (D + 2);
+    if (!SAS_IN_BOUNDS((long)(bh + 1) * p.nsplit * G * (D + 2) - 1, (long)p.B * p.Hkv * p.nsplit * G * (D + 2),
+                       p.status))
+        return;
     for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
         for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, part[(s * G + g) * (D + 2) + D]);
@@ -154,7 +173,8 @@ __global__ void __launch_bounds__(kThreads) decode_combine_kernel(DecodeParams p
                 const float* ps = part + (s * G + g) * (D + 2);
                 if (ps[D + 1] > 0.f) acc += ps[e] * expf(ps[D] - M);
             }
-            static_cast<T*>(p.o)[((long)b * p.Hq + h * G + g) * D + e] = from_f32<T>(acc * inv);
+            const long oi = ((long)b * p.Hq + h * G + g) * D + e;
+            if (SAS_IN_BOUNDS(oi, (long)p.B * p.Hq * D, p.status)) static_cast<T*>(p.o)[oi] = from_f32<T>(acc * inv);
         }
     }
 }

@@ -61,6 +61,7 @@ struct DecArgs {
 // reads as zeros).
 __device__ __forceinline__ int page_of(const DecArgs& a, int b, int blk) {
     if (blk >= a.pages_per_seq) return a.num_pages;
+    if (!SAS_IN_BOUNDS((long)b * a.pages_per_seq + blk, (long)a.B * a.pages_per_seq, a.status)) return a.num_pages;
     const int pg = a.page_table[(long)b * a.pages_per_seq + blk];
     return (pg < 0 || pg >= a.num_pages) ? a.num_pages : pg;
 }
@@ -587,7 +588,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
             const int m = tid + u * kThreads;
-            xs[u] = m < Csel ? srow[m] : 0.f;
+            xs[u] = m < Csel && SAS_IN_BOUNDS((long)bh * a.s_cols + m, (long)a.B * a.Hkv * a.s_cols, a.status)
+                        ? srow[m]
+                        : 0.f;
         }
     }
 
@@ -604,8 +607,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     // q of the group, padded to 16 rows: one 16-byte load per thread
     if (tid < 16 * kD / 8) {
         const int r = tid / (kD / 8), e = (tid % (kD / 8)) * 8;
-        const uint4 val = r < G ? *reinterpret_cast<const uint4*>(a.q + ((long)b * a.Hq + h * G + r) * kD + e)
-                                : make_uint4(0u, 0u, 0u, 0u);
+        const long qi = ((long)b * a.Hq + h * G + r) * kD + e;
+        const uint4 val = r < G && SAS_IN_BOUNDS(qi + 7, (long)a.B * a.Hq * kD, a.status)
+                              ? *reinterpret_cast<const uint4*>(a.q + qi)
+                              : make_uint4(0u, 0u, 0u, 0u);
         *reinterpret_cast<uint4*>(qs + r * kQLd + e) = val;
     }
     // attended list: entry 0 = current (partial) block, entries 1.. = history blocks ascending
@@ -621,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         __syncthreads();
         const int32_t* row = a.idx + (long)bh * a.top_k;
         for (int c = tid; c < a.top_k; c += kThreads) {
-            const int v = row[c];
+            const int v = SAS_IN_BOUNDS((long)bh * a.top_k + c, (long)a.B * a.Hkv * a.top_k, a.status) ? row[c] : -1;
             list[1 + c] = v;
             if (v < 0 || v >= Cb) atomicMin(&misc[3], c);
         }
@@ -643,7 +648,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
                 nsel = cluster_topk<CL>(a, bh, Csel, rank, base, list);
         }
         if (rank == 0 && a.idx_out)
-            for (int i = tid; i < a.top_k; i += kThreads) a.idx_out[(long)bh * a.top_k + i] = i < nsel ? list[1 + i] : -1;
+            for (int i = tid; i < a.top_k; i += kThreads)
+                if (SAS_IN_BOUNDS((long)bh * a.top_k + i, (long)a.B * a.Hkv * a.top_k, a.status))
+                    a.idx_out[(long)bh * a.top_k + i] = i < nsel ? list[1 + i] : -1;
     }
     const int L = nsel + 1;
     // ceil split: CTA 0 always owns entry 0 (the current block, prefetched in mode 1)
@@ -853,7 +860,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
                 n_ += num[r] * f;
                 d_ += den[r] * f;
             }
-            a.o[((long)b * a.Hq + h * G + g) * kD + d] = __float2bfloat16_rn(n_ / d_);
+            const long oi = ((long)b * a.Hq + h * G + g) * kD + d;
+            if (SAS_IN_BOUNDS(oi, (long)a.B * a.Hq * kD, a.status)) a.o[oi] = __float2bfloat16_rn(n_ / d_);
         }
     }
     cluster_sync();  // keep every CTA's shared memory alive until all remote reads are done

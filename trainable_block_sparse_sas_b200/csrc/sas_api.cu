@@ -402,7 +402,9 @@ sas_status sas_get_device_status(int32_t* status, sas_stream_t stream) {
     if (word == 0) return SAS_OK;
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return SAS_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return SAS_ERR_CUDA;
-    return word == SAS_ERR_DEVICE_TIMEOUT ? SAS_ERR_DEVICE_TIMEOUT : SAS_ERR_CUDA;
+    if (word == SAS_ERR_DEVICE_TIMEOUT) return SAS_ERR_DEVICE_TIMEOUT;
+    if ((word & 0xff) == SAS_ERR_DEVICE_BOUNDS) return SAS_ERR_DEVICE_BOUNDS;
+    return SAS_ERR_CUDA;
 }
 
 sas_status sas_selftest_bounded_wait(int32_t limit_ms, int32_t* status, int32_t* trace, sas_stream_t stream) {
@@ -419,6 +421,7 @@ const char* sas_status_string(sas_status status) {
         case SAS_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
         case SAS_ERR_CUDA: return "CUDA error";
         case SAS_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+        case SAS_ERR_DEVICE_BOUNDS: return "a device-side index check failed (debug-bounds build)";
     }
     return "unknown status";
 }

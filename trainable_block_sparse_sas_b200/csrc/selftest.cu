@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(kThreads, 1) selftest_wait_kernel(int* status,
             mma_commit(drain);
             if (mbar_wait_drain(drain, 0, status, limit_ns)) mark(trace, 2);
         }
+        __syncwarp();  // the warp reaches the CTA barrier converged
     } else if (warp == 2) {
         // another role waiting on its own barrier, with a longer limit: it must
         // leave on the abort flag, before its own limit runs out
