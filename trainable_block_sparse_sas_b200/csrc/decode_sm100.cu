@@ -50,6 +50,7 @@ struct DecArgs {
     __nv_bfloat16* o;
     int* status;
     int B, Hq, Hkv, Tmax, top_k, s_cols, mode;  // mode 0: given idx, 1: fused selection, 2: dense
+    int vec_scores;  // the score rows are 16-byte aligned (s_cols % 4 == 0, aligned s): vector loads
     float scale_log2;
     const int32_t* page_table;  // nullptr: contiguous caches
     int pages_per_seq, num_pages;
@@ -113,19 +114,19 @@ __device__ __forceinline__ int block_sum_int(int v, int* scan) {
 
 // Exact Top-K of the row's first Cb block scores, computed by this CTA alone
 // (every CTA of the cluster derives the same list, so no exchange is needed).
-// Each score m becomes the unique 64-bit key (order key << 32) | (2^32 - 1 - m):
-// larger keys are better and equal scores prefer the lower block index.  The
-// K-th largest of the threads' maxima is a lower bound of the K-th largest key
-// (K maxima reach it), so every key at or above it is a candidate; the K
-// best candidates by rank are the selection.  Returns K, or -1 when more than
-// kCandCap keys reach the bound (the caller then runs the radix select).
-// Rows of up to kPer * kThreads blocks (9216: 589,824 tokens at block 64); the
-// caller loads the thread's scores x[u] = s[tid + u * kThreads] at kernel entry,
-// so their latency overlaps the prologue.
+// The row's scores arrive at kernel entry as 16-byte vectors: thread tid holds
+// scores 4 (tid + u kThreads) .. + 3 in x[u], u < nv (nv uniform, the vectors the
+// row needs).  The per-score work uses 32-bit order keys: the K-th largest of the
+// threads' maxima (counted with multiplicity) is a lower bound tau of the K-th
+// largest score, since K maxima reach it; every score whose key is at least tau is
+// a candidate.  Only the 288 maxima and the few candidates carry unique 64-bit
+// keys (order key << 32 | (2^32 - 1 - index)), so that equal scores prefer the
+// lower block index.  Returns K, or -1 when more than kCandCap scores reach tau
+// (the caller then runs the radix select).
 constexpr int kCandCap = 512;
-constexpr int kPer = 32;  // scores per thread held in registers
+constexpr int kVec = 8;  // 16-byte score vectors per thread: rows of up to 4 * kVec * kThreads blocks
 
-__device__ int row_topk_filter(const DecArgs& a, int Cb, const float (&x)[kPer], uint8_t* base, int* list) {
+__device__ int row_topk_filter(const DecArgs& a, int Cb, int nv, const float4 (&x)[kVec], uint8_t* base, int* list) {
     constexpr int kWarps = kThreads / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int K = a.top_k;
@@ -133,23 +134,32 @@ __device__ int row_topk_filter(const DecArgs& a, int Cb, const float (&x)[kPer],
     unsigned long long* sorted = reinterpret_cast<unsigned long long*>(base + Layout::kRing + kStage);
     unsigned long long* cand = sorted + kWarps * 32;
     unsigned long long* chosen = cand + kCandCap;
-    unsigned long long* thr_sh = chosen + 64;
+    uint32_t* thr_sh = reinterpret_cast<uint32_t*>(chosen + 64);
     int* misc = reinterpret_cast<int*>(base + Layout::kMisc);
-    auto key_of = [&](float s, int m) -> unsigned long long {
-        return ((unsigned long long)order_key(s) << 32) | (0xFFFFFFFFu - (uint32_t)m);
-    };
-    unsigned long long v = 0ull;  // 0: no score (every real key is larger)
+    // this thread's maximum: 32-bit key, and the index of a score that has it
+    uint32_t kmax = 0u;  // 0: no score (every real key is larger)
+    int mmax = 0;
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-        const int m = tid + u * kThreads;
-        const unsigned long long k = m < Cb ? key_of(x[u], m) : 0ull;
-        v = k > v ? k : v;
+    for (int u = 0; u < kVec; ++u) {
+        if (u < nv) {
+            const int m0 = 4 * (tid + u * kThreads);
+            const float xe[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t k = m0 + e < Cb ? order_key(xe[e]) : 0u;
+                if (k > kmax) {
+                    kmax = k;
+                    mmax = m0 + e;
+                }
+            }
+        }
     }
     if (tid == 0) {
         misc[5] = 0;
-        *thr_sh = 0ull;
+        *thr_sh = 0u;
     }
-    // each warp's 32 maxima, sorted descending
+    // the maxima as unique keys; each warp's 32 sorted descending
+    unsigned long long v = kmax ? (((unsigned long long)kmax << 32) | (0xFFFFFFFFu - (uint32_t)mmax)) : 0ull;
 #pragma unroll
     for (int k = 2; k <= 32; k <<= 1) {
 #pragma unroll
@@ -183,23 +193,32 @@ __device__ int row_topk_filter(const DecArgs& a, int Cb, const float (&x)[kPer],
             const int c2 = cnt[w2] + (sorted[w2 * 32 + 31] > v ? 1 : 0) * (cnt[w2] == 31 ? 1 : 0);
             rk += w2 == warp ? 0 : c2;
         }
-        if (v != 0ull && rk == K - 1) *thr_sh = v;
+        if (v != 0ull && rk == K - 1) *thr_sh = (uint32_t)(v >> 32);
     }
     __syncthreads();
-    const unsigned long long thr = *thr_sh;
-    // candidates: every key at or above thr, one shared-memory atomic per warp and pass
+    const uint32_t thr = *thr_sh;
+    // candidates: every score whose key reaches tau, one shared-memory atomic per
+    // warp and vector element
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-        const int m = tid + u * kThreads;
-        const unsigned long long k = m < Cb ? key_of(x[u], m) : 0ull;
-        const bool take = m < Cb && k >= thr;
-        const unsigned bal = __ballot_sync(0xffffffffu, take);
-        if (bal) {
-            int base_pos = 0;
-            if (lane == 0) base_pos = atomicAdd(&misc[5], __popc(bal));
-            base_pos = __shfl_sync(0xffffffffu, base_pos, 0);
-            const int pos = base_pos + __popc(bal & ((1u << lane) - 1u));
-            if (take && pos < kCandCap) cand[pos] = k;
+    for (int u = 0; u < kVec; ++u) {
+        if (u < nv) {
+            const int m0 = 4 * (tid + u * kThreads);
+            const float xe[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int m = m0 + e;
+                const uint32_t k = m < Cb ? order_key(xe[e]) : 0u;
+                const bool take = m < Cb && k >= thr;
+                const unsigned bal = __ballot_sync(0xffffffffu, take);
+                if (bal) {
+                    int base_pos = 0;
+                    if (lane == 0) base_pos = atomicAdd(&misc[5], __popc(bal));
+                    base_pos = __shfl_sync(0xffffffffu, base_pos, 0);
+                    const int pos = base_pos + __popc(bal & ((1u << lane) - 1u));
+                    if (take && pos < kCandCap)
+                        cand[pos] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)m);
+                }
+            }
         }
     }
     __syncthreads();
@@ -576,23 +595,30 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     const uint32_t rank = cluster_ctarank();
     const int bh = blockIdx.y;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
+    // fused selection by the per-CTA filter: the row's scores are requested first,
+    // in 16-byte vectors and independently of ctx_len (every one of the row's
+    // s_cols; those past the history are masked later)
+    const int nv = (a.s_cols + 4 * kThreads - 1) / (4 * kThreads);
+    const bool vec_ok = a.mode == 1 && a.vec_scores && nv <= kVec;
+    float4 xv[kVec];
+    if (vec_ok) {
+        const float4* srow4 = reinterpret_cast<const float4*>(a.s + (long)bh * a.s_cols);
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) {
+            if (u < nv) {
+                const int i4 = tid + u * kThreads;
+                xv[u] = 4 * i4 < a.s_cols &&
+                                SAS_IN_BOUNDS((long)bh * a.s_cols + 4 * i4 + 3, (long)a.B * a.Hkv * a.s_cols, a.status)
+                            ? __ldg(srow4 + i4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+    }
     int T = a.ctx_len[b];
     T = max(1, min(T, a.Tmax));
     const int t = T - 1, Cb = t / kBS;
-    // fused selection by the per-CTA filter: this thread's scores, requested first
     const int Csel = min(Cb, a.s_cols);
-    const bool use_filter = a.mode == 1 && a.top_k < Csel && a.top_k <= 64 && Csel <= kPer * kThreads;
-    float xs[kPer];
-    if (use_filter) {
-        const float* srow = a.s + (long)bh * a.s_cols;
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int m = tid + u * kThreads;
-            xs[u] = m < Csel && SAS_IN_BOUNDS((long)bh * a.s_cols + m, (long)a.B * a.Hkv * a.s_cols, a.status)
-                        ? srow[m]
-                        : 0.f;
-        }
-    }
+    const bool use_filter = vec_ok && a.top_k < Csel && a.top_k <= 64;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -640,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
             load_block(a, ring, full(0), b, h, bh, Cb, a.page_table ? page_of(a, b, Cb) : 0);
         }
         const int chunk = (Csel + CL - 1) / CL;
-        nsel = use_filter ? row_topk_filter(a, Csel, xs, base, list) : -1;
+        nsel = use_filter ? row_topk_filter(a, Csel, nv, xv, base, list) : -1;
         if (nsel < 0) {
             if (a.top_k < Csel && chunk <= (int)(kStage / 4) && CL * a.top_k <= (int)(kStage / 8))
                 nsel = cluster_topk_fast<CL>(a, bh, Csel, rank, base, list);
@@ -962,6 +988,7 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_col
     a.top_k = p.top_k;
     a.s_cols = s_cols;
     a.mode = s ? 1 : (p.idx ? 0 : 2);
+    a.vec_scores = s && (s_cols % 4 == 0) && (reinterpret_cast<uintptr_t>(s) & 15u) == 0;
     a.scale_log2 = p.scale * kLog2e;
     const int max_entries = a.mode == 2 ? (p.Tmax + kBS - 1) / kBS : p.top_k + 1;
     const int list_cap = a.mode == 2 ? 1 : p.top_k + 1;
