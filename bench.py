@@ -643,6 +643,25 @@ def extras(api, args, peaks, peak_kind) -> dict:
                    "peak_source": f"{peak_kind} bf16 burst"}
     del r, inp
     torch.cuda.empty_cache()
+    # 8 query heads per KV head (two forward and dq CTAs per query block)
+    w = syn.TRAIN_SPARSE_32K_GQA8
+    inp = syn.train_inputs(w, device="cuda", seed=1700)
+    r = TrainRunner(api, w, inp)
+    for _ in range(2):
+        r.step()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(n):
+        r.step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    fl = train_flops(w)
+    out[w.name] = {"ms_per_step": ms, "tflops": fl["total"] / (ms * 1e-3) / 1e12,
+                   "frac_of_bf16_peak": fl["total"] / (ms * 1e-3) / 1e12 / peak,
+                   "path": list(api.sas_attn_path(r.desc))}
+    del r, inp
+    torch.cuda.empty_cache()
     # the ablated gates on the headline training workload (same FLOP convention;
     # the hard STE gate's dq kernel also walks every dropped block, uncounted)
     w = syn.TRAIN_SPARSE_32K

@@ -166,6 +166,23 @@ sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const vo
                               const float* s, const float* lse_s, const int32_t* idx, void* o, float* lse,
                               int32_t* status, sas_stream_t stream);
 
+/* Kernel family a training call runs. */
+typedef enum { SAS_PATH_SIMT = 0, SAS_PATH_TENSOR_CORE = 1 } sas_path;
+
+/*
+ * sas_attn_path -- which kernels sas_gated_attn_fwd and sas_gated_attn_bwd run for
+ *   this problem, given 16-byte aligned tensors (a misaligned q, k, v, o, dO, dq,
+ *   dk or dv sends a call to the SIMT kernels as well).
+ *   SAS_PATH_TENSOR_CORE: the tcgen05 / TMEM / TMA kernels (bf16, head_dim 128,
+ *   block_size 64, 2, 4 or 8 query heads per kv head, shared memory permitting).
+ *   SAS_PATH_SIMT: the CUDA-core kernels (fp32, and every other shape), tens of
+ *   times slower on the training workloads.
+ * fwd_path, bwd_path  host int32 out (either may be NULL).
+ * Errors: SAS_ERR_INVALID_VALUE (bad desc); SAS_ERR_UNSUPPORTED (a shape neither
+ *   path takes: head_dim not 64 or 128, block_size not 16, 32 or 64).
+ */
+sas_status sas_attn_path(const sas_attn_desc* desc, int32_t* fwd_path, int32_t* bwd_path);
+
 /* Bytes of workspace sas_gated_attn_bwd needs for this problem (0 on bad desc). */
 size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc);
 

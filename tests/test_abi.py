@@ -124,6 +124,29 @@ def test_select_checks(api):
     assert L.sas_topk_select(FAKE, 1, 1, 1, 4, FAKE, 0, 2, FAKE, None, None) == 1   # decode rows need block_size
 
 
+def test_attn_path_names_the_kernels_a_shape_runs(api):
+    """The tensor-core path takes bf16, d 128, block 64 with 2, 4 or 8 query heads
+    per kv head; fp32 and the other shapes run the SIMT kernels."""
+    L = api.lib
+    f, b = ctypes.c_int32(-1), ctypes.c_int32(-1)
+
+    def path(**kw):
+        assert L.sas_attn_path(ctypes.byref(_desc(api, **kw)), ctypes.byref(f), ctypes.byref(b)) == 0
+        return f.value, b.value
+
+    for G in (2, 4, 8):
+        assert path(n_q_heads=2 * G, n_kv_heads=2) == (1, 1), G
+        assert path(n_q_heads=2 * G, n_kv_heads=2, scope=1, top_k=0) == (1, 1), G
+    assert path(n_q_heads=2, n_kv_heads=2) == (0, 0)      # one query head per kv head
+    assert path(n_q_heads=10, n_kv_heads=2) == (0, 0)     # 5
+    assert path(dtype=0) == (0, 0)                        # fp32
+    assert path(head_dim=64) == (0, 0)
+    assert path(block_size=32, seq_len=256) == (0, 0)
+    assert L.sas_attn_path(ctypes.byref(_desc(api, head_dim=96)), None, None) == 2
+    assert L.sas_attn_path(ctypes.byref(_desc(api, batch=0)), None, None) == 1
+    assert api.sas_attn_path(_desc(api)) == ("tensor_core", "tensor_core")
+
+
 def test_status_word_and_selftest_checks(api):
     """The status reader and the failure self-test refuse a missing word or an
     out-of-range limit before touching the device."""

@@ -118,6 +118,8 @@ def test_tiny_fp32_workload(api):
     (1, 512, 4, 2, 128, 64, 0, True),    # full scope
     (1, 256, 4, 2, 64, 64, 0, False),    # K = 0: current block only
     (1, 1024, 4, 1, 128, 64, 40, False), # K >= C: sparse == full
+    (1, 512, 8, 1, 128, 64, 3, False),   # GQA 8: two CTAs per query block (tensor cores)
+    (2, 512, 16, 2, 128, 64, 0, True),   # GQA 8, full scope
 ])
 def test_bf16_shapes(api, B, n, Hq, Hkv, d, bs, K, full):
     Cq = n // bs
@@ -132,6 +134,9 @@ def test_bf16_shapes(api, B, n, Hq, Hkv, d, bs, K, full):
     want = _oracle_train(inp, bs, K, full)
     idx_want = None if (full or K == 0) else oracle.train_select(bits(inp["s"]), K)[0]
     _compare_train(got, want, BF16_TOL, idx_want)
+    tc = d == 128 and bs == 64 and Hq // Hkv in (2, 4, 8)
+    want_path = ("tensor_core",) * 2 if tc else ("simt",) * 2
+    assert api.sas_attn_path(api.attn_desc(inp["q"], inp["k"], bs, K, full)) == want_path
 
 
 def test_unsupported_block_size_is_refused(api):
@@ -151,6 +156,7 @@ def test_unsupported_block_size_is_refused(api):
 @pytest.mark.parametrize("dtype,d,bs,K,full,G", [
     (torch.bfloat16, 128, 64, 3, False, 2),  # tcgen05 kernels, sparse scope
     (torch.bfloat16, 128, 64, 0, True, 2),   # tcgen05 kernels, full scope
+    (torch.bfloat16, 128, 64, 3, False, 8),  # tcgen05 kernels, GQA 8 (head-split dq CTAs add their ds)
     (torch.bfloat16, 64, 32, 4, False, 2),   # SIMT kernels (d = 64)
     (torch.bfloat16, 64, 32, 4, False, 5),   # SIMT kernels, GQA 5
     (torch.bfloat16, 128, 16, 5, False, 4),  # SIMT kernels, 16-token blocks
@@ -164,7 +170,7 @@ def test_gate_variants(api, gate, dtype, d, bs, K, full, G):
     nearly all of a row's mass (raw: weight e^s against the current block's 1);
     its dlogg then sums D_i over all G*b rows of the query block, which is what
     the exact D of both backward paths is tested on here."""
-    B, n, Hkv = 1, 512, 2 if G < 5 else 1
+    B, n, Hkv = 1, 512, 2 if G < 5 or G == 8 else 1
     Hq = G * Hkv
     Cq = n // bs
     qk_std = 1.0 if dtype == torch.bfloat16 else 0.3
@@ -270,6 +276,13 @@ def test_train_sparse_32k_gate_variants_sampled(api, gate, kv_blocks):
     times them; the STE's dq kernel walks up to 511 dropped blocks per row."""
     w = syn.TRAIN_SPARSE_32K
     _sampled_full_size(api, w, q_blocks=(0, 1, 33, 257, 511), kv_blocks=kv_blocks, heads=(3,), gate=gate)
+
+
+def test_train_sparse_32k_gqa8_sampled(api):
+    """The 32K sparse workload with 8 query heads per KV head, on the tensor-core
+    kernels (two dq CTAs per query block adding their ds shares)."""
+    w = syn.TRAIN_SPARSE_32K_GQA8
+    _sampled_full_size(api, w, q_blocks=(0, 1, 33, 257, 511), kv_blocks=(511, 200), heads=(0, 3))
 
 
 def test_train_full_16k_sampled(api):

@@ -59,6 +59,8 @@ lib.sas_topk_select.restype = ctypes.c_int
 lib.sas_topk_select.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _vp, _vp]
 lib.sas_gated_attn_fwd.restype = ctypes.c_int
 lib.sas_gated_attn_fwd.argtypes = [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.sas_attn_path.restype = ctypes.c_int
+lib.sas_attn_path.argtypes = [ctypes.POINTER(AttnDesc), ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]
 lib.sas_gated_attn_bwd_workspace_size.restype = _sz
 lib.sas_gated_attn_bwd_workspace_size.argtypes = [ctypes.POINTER(AttnDesc)]
 lib.sas_gated_attn_bwd.restype = ctypes.c_int
@@ -236,6 +238,15 @@ def sas_gated_attn_fwd(desc, q, k, v, s, lse_s, idx, o, lse, stream=None, status
     _need(lse, desc.batch * desc.n_q_heads * desc.seq_len, _F32, "lse")
     _check(lib.sas_gated_attn_fwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(s), _p(lse_s), _p(idx), _p(o), _p(lse),
                                   _status(status, q), _stream(stream)), "sas_gated_attn_fwd")
+
+
+def sas_attn_path(desc) -> tuple[str, str]:
+    """("tensor_core" | "simt", same) for the forward and the backward of a problem
+    (with 16-byte aligned tensors)."""
+    f, b = ctypes.c_int32(-1), ctypes.c_int32(-1)
+    _check(lib.sas_attn_path(ctypes.byref(desc), ctypes.byref(f), ctypes.byref(b)), "sas_attn_path")
+    name = {0: "simt", 1: "tensor_core"}
+    return name[f.value], name[b.value]
 
 
 def sas_gated_attn_bwd_workspace_size(desc) -> int:

@@ -1,6 +1,8 @@
 // attn_bwd_sm100.cu -- tensor-core (tcgen05 / TMEM / TMA) backward of SAS gated
-// block-sparse attention for bf16, head_dim 128, block size 64, 2 or 4 query
-// heads per KV head.  Two kernels, no atomics (results are deterministic):
+// block-sparse attention for bf16, head_dim 128, block size 64, 2, 4 or 8 query
+// heads per KV head.  Two kernels; results are deterministic (with 8 heads per
+// KV head the dq kernel runs two CTAs of four heads per query block, which add
+// their shares of the ds row -- two addends, so the order does not matter):
 //
 // bwd_dq_sm100: one CTA per (batch, kv head, query block c), the group's query
 //   heads stacked into 128-row M-tiles as in the forward.  For each attended key
@@ -72,6 +74,7 @@ struct BwdArgs {
     float* ds;
     int* status;
     int B, Hq, Hkv, n, Cq, top_k, full_scope, gate;
+    int hsplit;  // dq kernel: CTAs per query block, each taking 2 MT of the group's heads
     float scale, scale_log2;
 };
 
@@ -168,11 +171,14 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     const bool ste = a.gate == kGateSte;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // head-major order (concurrent CTAs share one KV head in L2), long query blocks first
-    const int c = a.Cq - 1 - (int)(blockIdx.x % a.Cq);
-    const int bh = (int)(blockIdx.x / a.Cq);
+    // head-major order (concurrent CTAs share one KV head in L2), long query blocks
+    // first, a query block's head splits adjacent
+    const int hs = (int)(blockIdx.x % a.hsplit);
+    const int c = a.Cq - 1 - (int)((blockIdx.x / a.hsplit) % a.Cq);
+    const int bh = (int)(blockIdx.x / ((long)a.hsplit * a.Cq));
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long unit = (long)bh * a.Cq + c;
+    const int hq0 = (h * a.hsplit + hs) * G;  // first query head of this CTA
     // block masses M_t of the CTA's rows: [list slot][128 * MT rows], bf16
     __nv_bfloat16* mbase = a.Mbuf + (long)blockIdx.x * nl * (128 * MT);
 
@@ -198,8 +204,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
         const int q_row = b * a.n + c * kBS;
         mbar_arrive_expect_tx(q_full, 4 * L::kHalf);
         for (int kh = 0; kh < 2; ++kh) {
-            tma_load_3d(sQ + kh * L::kHalf, &a.tq, q_full, kh * 64, h * G, q_row);
-            tma_load_3d(sDO + kh * L::kHalf, &a.tdo, q_full, kh * 64, h * G, q_row);
+            tma_load_3d(sQ + kh * L::kHalf, &a.tq, q_full, kh * 64, hq0, q_row);
+            tma_load_3d(sDO + kh * L::kHalf, &a.tdo, q_full, kh * 64, hq0, q_row);
         }
     }
     // the score row is read again by the ds epilogue: have it in L2 by then
@@ -343,7 +349,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
             const int row = 32 * quad + lane;
             const int r_unit = 128 * grp + row;
             const int tok = r_unit / G, g = r_unit % G;
-            const int hq = h * G + g;
+            const int hq = hq0 + g;
             const long ri = ((long)b * a.Hq + hq) * a.n + c * kBS + tok;
             const long e0 = (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
             // debug-bounds build: this row's global indices (o, dO, dq rows; lse, D)
@@ -529,6 +535,21 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     // for the softmax gate, 0 otherwise; 0 from c on); then the attended ones are
     // overwritten with their ds, log g_m from the bias kept in smem
     const float lse_c = gate_softmax_family(a.gate) ? a.lse_s[unit] : 0.f;
+    if (a.hsplit > 1) {
+        // the group's heads are split over hsplit CTAs: ds is linear in dlogg, so each
+        // CTA adds its share of every entry m < c to the row (zeroed before the
+        // launch); two addends per entry keep the sum independent of their order
+        float* dlm = reinterpret_cast<float*>(base + L::kQ);  // the freed Q tile: dlogg by block
+        for (int m = threadIdx.x; m < c; m += kDqThreads) dlm[m] = 0.f;
+        __syncthreads();
+        for (int t = threadIdx.x; t < nsel; t += kDqThreads) dlm[list[t]] = part[t * 8];
+        __syncthreads();
+        for (int m = threadIdx.x; m < c; m += kDqThreads) {
+            const float v = gate_ds(dlm[m], gate_log(srow[m], lse_c, a.gate), tot, a.gate);
+            if (v != 0.f) atomicAdd(dsrow + m, v);
+        }
+        return;
+    }
     if (gate_softmax_family(a.gate)) {
         for (int m = threadIdx.x; m < a.Cq; m += kDqThreads) dsrow[m] = m < c ? -expf(srow[m] - lse_c) * tot : 0.f;
     } else {
@@ -885,13 +906,16 @@ static size_t bwd_sm100_mass_bytes(const TrainParams& p) {
     return (b + 255) & ~(size_t)255;
 }
 
-template <int MT>
-cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
-    constexpr int G = 2 * MT;
+// MT: 128-row tiles per CTA of the dq kernel (2 MT query heads, hsplit CTAs per
+// query block); MK: 128-row items per query block of the dk/dv kernel (G = 2 MK).
+template <int MT, int MK>
+cudaError_t launch_mt(const TrainParams& p, int hsplit, cudaStream_t stream) {
+    constexpr int G = 2 * MK;
     BwdArgs a;
     memset(&a, 0, sizeof(a));
     const long rows = (long)p.B * p.n;
     const long grid = (long)p.B * p.Hkv * p.Cq;
+    a.hsplit = hsplit;
     a.s = p.s;
     a.lse_s = p.lse_s;
     a.idx = p.idx;
@@ -916,8 +940,9 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.gate = p.gate;
     a.scale = p.scale;
     a.scale_log2 = p.scale * kLog2e;
-    // query-major kernel: the whole query block (64 tokens x G heads) per box
-    if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, kBS) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, kBS) ||
+    // query-major kernel: the CTA's query heads of the block (64 tokens x 2 MT heads) per box
+    if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, 2 * MT, kBS) ||
+        !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, 2 * MT, kBS) ||
         !encode_tma_rows(&a.tk, p.k, p.Hkv, rows, 1, kBS) || !encode_tma_rows(&a.tv, p.v, p.Hkv, rows, 1, kBS))
         return cudaErrorInvalidValue;
     const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
@@ -926,7 +951,11 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     const size_t smem = st3 ? DqLayout<MT, 3>::bytes(nl) : DqLayout<MT, 2>::bytes(nl);
     auto kern = st3 ? (outer ? bwd_dq_sm100_kernel<MT, 3, true> : bwd_dq_sm100_kernel<MT, 3, false>)
                     : (outer ? bwd_dq_sm100_kernel<MT, 2, true> : bwd_dq_sm100_kernel<MT, 2, false>);
-    cudaError_t err = launch_kernel(kern, grid, kDqThreads, smem, a, stream);
+    cudaError_t err = cudaSuccess;
+    if (hsplit > 1 && (err = cudaMemsetAsync(p.ds, 0, sizeof(float) * (size_t)p.B * p.Hkv * p.Cq * p.Cq, stream)) !=
+                          cudaSuccess)
+        return err;  // the head splits add their shares of ds
+    err = launch_kernel(kern, grid * hsplit, kDqThreads, smem, a, stream);
     if (err != cudaSuccess) return err;
     if (p.phase_event && (err = cudaEventRecord(static_cast<cudaEvent_t>(p.phase_event), stream)) != cudaSuccess)
         return err;
@@ -934,15 +963,15 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, 128 / G) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, 128 / G))
         return cudaErrorInvalidValue;
     return p.gate == kGateOuter
-               ? launch_kernel(bwd_dkdv_sm100_kernel<MT, true>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream)
-               : launch_kernel(bwd_dkdv_sm100_kernel<MT, false>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream);
+               ? launch_kernel(bwd_dkdv_sm100_kernel<MK, true>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream)
+               : launch_kernel(bwd_dkdv_sm100_kernel<MK, false>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream);
 }
 
 }  // namespace
 
 static bool bwd_sm100_shape(const TrainParams& p) {
     const int G = p.Hq / p.Hkv;
-    return p.is_bf16 && p.d == kD && p.bs == kBS && (G == 2 || G == 4);
+    return p.is_bf16 && p.d == kD && p.bs == kBS && (G == 2 || G == 4 || G == 8);
 }
 
 size_t bwd_sm100_workspace(const TrainParams& p) {
@@ -958,14 +987,18 @@ bool bwd_sm100_supported(const TrainParams& p) {
                          reinterpret_cast<uintptr_t>(p.dq) | reinterpret_cast<uintptr_t>(p.dk) |
                          reinterpret_cast<uintptr_t>(p.dv) | reinterpret_cast<uintptr_t>(p.o_in);
     if (al & 15u) return false;
-    if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq > 0x7fffffffL) return false;
+    if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq * (p.Hq / p.Hkv == 8 ? 2 : 1) > 0x7fffffffL)
+        return false;
     const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
     return DqLayout<2, 2>::bytes(nl) <= kSmemLimit && DkvLayout::bytes(p.Cq) <= kSmemLimit;
 }
 
 cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream) {
     const int G = p.Hq / p.Hkv;
-    return G == 4 ? launch_mt<2>(p, stream) : launch_mt<1>(p, stream);
+    // dq: G = 2 one tile per CTA, G = 4 two, G = 8 two CTAs of two tiles; dk/dv: G / 2 items per block
+    if (G == 2) return launch_mt<1, 1>(p, 1, stream);
+    if (G == 4) return launch_mt<2, 2>(p, 1, stream);
+    return launch_mt<2, 4>(p, 2, stream);
 }
 
 }  // namespace sas

@@ -1,6 +1,7 @@
 // attn_fwd_sm100.cu -- tensor-core (tcgen05 / TMEM / TMA) forward of SAS gated
-// block-sparse attention for bf16, head_dim 128, block size 64, and 2 or 4
-// query heads per KV head.
+// block-sparse attention for bf16, head_dim 128, block size 64, and 2, 4 or 8
+// query heads per KV head (8: two CTAs per query block, four heads each, adjacent
+// in the grid so that they share the block's K and V in L2).
 //
 // o = softmax(sigma q K_S^T + log g_S) V_S (jaehun.me review of SAS, Eq. 9 and the
 // Kernel implementation paragraph): for query block c the attended key blocks
@@ -61,6 +62,7 @@ struct FwdArgs {
     float* lse;
     int* status;
     int B, Hq, Hkv, n, Cq, top_k, full_scope, gate;
+    int hsplit;  // CTAs per query block, each taking G = 2 MT of the group's query heads
     float scale_log2;
 };
 
@@ -122,11 +124,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // head-major order: concurrent CTAs share one KV head's K/V in L2; within a
-    // head, long (late) query blocks first
-    const int c = a.Cq - 1 - (int)(blockIdx.x % a.Cq);
-    const int bh = (int)(blockIdx.x / a.Cq);
+    // head, long (late) query blocks first; a query block's head splits adjacent
+    const int hs = (int)(blockIdx.x % a.hsplit);
+    const int c = a.Cq - 1 - (int)((blockIdx.x / a.hsplit) % a.Cq);
+    const int bh = (int)(blockIdx.x / ((long)a.hsplit * a.Cq));
     const int b = bh / a.Hkv, h = bh % a.Hkv;
     const long unit = (long)bh * a.Cq + c;
+    const int hq0 = (h * a.hsplit + hs) * G;  // first query head of this CTA
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -150,8 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
         // Q of the query block does not depend on the selection: request it now
         const int q_row = b * a.n + c * kBS;
         mbar_arrive_expect_tx(q_full, 2 * L::kQHalf);
-        tma_load_3d(sQ, &a.tq, q_full, 0, h * G, q_row);
-        tma_load_3d(sQ + L::kQHalf, &a.tq, q_full, 64, h * G, q_row);
+        tma_load_3d(sQ, &a.tq, q_full, 0, hq0, q_row);
+        tma_load_3d(sQ + L::kQHalf, &a.tq, q_full, 64, hq0, q_row);
         // the current block is the list's first entry: its K and V go out now too
         mbar_arrive_expect_tx(kv_full(0), kStage);
         for (int kh = 0; kh < 2; ++kh) {
@@ -362,14 +366,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
             const int tl = nlist - 1;
             // the row's outputs (the checks of the debug-bounds build skip the stores
             // only: the TMEM loads below are whole-warp instructions)
-            const long orow_i = (((long)b * a.n + c * kBS + tok) * a.Hq + h * G + g) * kD;
-            const long lse_i = ((long)b * a.Hq + h * G + g) * a.n + c * kBS + tok;
+            const long orow_i = (((long)b * a.n + c * kBS + tok) * a.Hq + hq0 + g) * kD;
+            const long lse_i = ((long)b * a.Hq + hq0 + g) * a.n + c * kBS + tok;
             const bool inb = SAS_IN_BOUNDS(orow_i + kD - 1, (long)a.B * a.n * a.Hq * kD, a.status) &&
                              SAS_IN_BOUNDS(lse_i, (long)a.B * a.Hq * a.n, a.status);
             if (ok && warp_wait(pv_done(grp, tl & 1), (tl >> 1) & 1, abort_flag, a.status)) {
                 tc_fence_after();
                 const float inv_l = 1.f / l;
-                const int hq = h * G + g;
+                const int hq = hq0 + g;
                 __nv_bfloat16* orow = a.o + (((long)b * a.n + c * kBS + tok) * a.Hq + hq) * kD;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
@@ -430,7 +434,7 @@ bool encode_tma_rows(CUtensorMap* map, const void* ptr, int heads, long rows, in
 namespace {
 
 template <int MT>
-cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
+cudaError_t launch_mt(const TrainParams& p, int hsplit, cudaStream_t stream) {
     FwdArgs a;
     memset(&a, 0, sizeof(a));
     const long rows = (long)p.B * p.n;
@@ -452,11 +456,12 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
     a.full_scope = p.full_scope;
     a.gate = p.gate;
     a.scale_log2 = p.scale * kLog2e;
+    a.hsplit = hsplit;
     const size_t smem = FwdLayout<MT>::bytes(p.Cq);
     auto kern = p.gate == kGateOuter ? fwd_sm100_kernel<MT, true> : fwd_sm100_kernel<MT, false>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const long grid = (long)p.B * p.Hkv * p.Cq;
+    const long grid = (long)p.B * p.Hkv * p.Cq * hsplit;
     kern<<<(unsigned)grid, kThreads, smem, stream>>>(a);
     err = cudaGetLastError();
     if (err == cudaSuccess) count_launch();
@@ -468,17 +473,19 @@ cudaError_t launch_mt(const TrainParams& p, cudaStream_t stream) {
 bool fwd_sm100_supported(const TrainParams& p) {
     if (!p.is_bf16 || p.d != kD || p.bs != kBS) return false;
     const int G = p.Hq / p.Hkv;
-    if (G != 2 && G != 4) return false;
+    if (G != 2 && G != 4 && G != 8) return false;
     if ((reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) | reinterpret_cast<uintptr_t>(p.v) |
          reinterpret_cast<uintptr_t>(p.o)) & 15u)
         return false;
-    if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq > 0x7fffffffL) return false;
+    if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq * (G == 8 ? 2 : 1) > 0x7fffffffL) return false;
     return FwdLayout<2>::bytes(p.Cq) <= 227 * 1024;
 }
 
 cudaError_t launch_fwd_sm100(const TrainParams& p, cudaStream_t stream) {
     const int G = p.Hq / p.Hkv;
-    return G == 4 ? launch_mt<2>(p, stream) : launch_mt<1>(p, stream);
+    // G = 2: one 128-row tile per CTA; G = 4: two; G = 8: two CTAs of two tiles (4 heads) each
+    if (G == 2) return launch_mt<1>(p, 1, stream);
+    return launch_mt<2>(p, G / 4, stream);
 }
 
 }  // namespace sas

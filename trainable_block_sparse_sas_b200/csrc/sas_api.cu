@@ -177,6 +177,19 @@ sas_status sas_gated_attn_fwd(const sas_attn_desc* desc, const void* q, const vo
     return from_cuda(launch_fwd_simt(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+sas_status sas_attn_path(const sas_attn_desc* desc, int32_t* fwd_path, int32_t* bwd_path) {
+    if (!check_train(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!supported_train(desc)) return SAS_ERR_UNSUPPORTED;
+    TrainParams p = make_train(desc);
+    // aligned stand-ins: the predicates look at shapes and pointer alignment only
+    void* const aligned = reinterpret_cast<void*>(uintptr_t(256));
+    p.q = p.k = p.v = p.o_in = p.dO = aligned;
+    p.o = p.dq = p.dk = p.dv = p.Mbuf = aligned;
+    if (fwd_path) *fwd_path = fwd_sm100_supported(p) ? SAS_PATH_TENSOR_CORE : SAS_PATH_SIMT;
+    if (bwd_path) *bwd_path = bwd_sm100_supported(p) ? SAS_PATH_TENSOR_CORE : SAS_PATH_SIMT;
+    return SAS_OK;
+}
+
 size_t sas_gated_attn_bwd_workspace_size(const sas_attn_desc* desc) {
     if (!check_train(desc)) return 0;
     TrainParams p = make_train(desc);

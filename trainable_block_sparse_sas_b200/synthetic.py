@@ -64,10 +64,14 @@ class DecodeShape:
 TINY_FP32 = TrainShape("tiny_fp32", 1, 2, 1, 64, 512, 16, 4, False, torch.float32, 1.0 / 8.0, 1.0)
 TRAIN_SPARSE_32K = TrainShape("train_sparse_32k", 1, 32, 8, 128, 32768, 64, 32, False, torch.bfloat16, 1.0, 2.0)
 TRAIN_FULL_16K = TrainShape("train_full_16k", 1, 32, 8, 128, 16384, 64, 0, True, torch.bfloat16, 1.0, 2.0)
+# the 32K sparse workload with 8 query heads per KV head (4 KV heads)
+TRAIN_SPARSE_32K_GQA8 = TrainShape("train_sparse_32k_gqa8", 1, 32, 4, 128, 32768, 64, 32, False, torch.bfloat16, 1.0,
+                                   2.0)
 DECODE_128K = DecodeShape("decode_128k", 16, 32, 8, 128, 131073, 64, 16, torch.bfloat16, 1.0)
 DECODE_512K = DecodeShape("decode_512k", 4, 40, 8, 128, 524289, 64, 32, torch.bfloat16, 1.0)
 
-WORKLOADS = {w.name: w for w in (TINY_FP32, TRAIN_SPARSE_32K, TRAIN_FULL_16K, DECODE_128K, DECODE_512K)}
+WORKLOADS = {w.name: w for w in (TINY_FP32, TRAIN_SPARSE_32K, TRAIN_FULL_16K, TRAIN_SPARSE_32K_GQA8, DECODE_128K,
+                                  DECODE_512K)}
 
 
 def _gen(device, seed: int) -> torch.Generator:
