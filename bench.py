@@ -425,6 +425,157 @@ def time_decode(api, w, steps: int, mode: str = "fused"):
     return statistics.median(times)
 
 
+def time_decode_graph(api, w, reps: int = 20, n_steps: int = 16) -> float:
+    """Median device time per fused decode step (sas_sparse_decode_select) when
+    n_steps steps run back to back from one CUDA graph, as a serving loop replays
+    them: events around each replay, time / n_steps.  The steps read n_steps
+    different score tensors, so each attends its own blocks: n_steps x the
+    attended K/V of a step (1.1 GB for decode_128k, 0.56 GB for decode_512k)
+    passes through L2 per replay, and a step's blocks are long evicted when they
+    come round again; q and the current block stay in L2, as they would after the
+    preceding kernels of a decode step."""
+    import torch
+
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    inp = syn.decode_inputs(w, device="cuda", seed=3000)
+    q, kc, vc, ctx, s = (inp[x] for x in ("q", "k_cache", "v_cache", "ctx_len", "s"))
+    desc = api.decode_desc(q, kc, w.bs, w.top_k)
+    idx = torch.empty((w.B, w.Hkv, w.top_k), dtype=torch.int32, device="cuda")
+    o = torch.empty_like(q)
+    gs = torch.Generator(device="cuda")
+    gs.manual_seed(3200)
+    s_rot = [s] + [torch.randn(s.shape, generator=gs, device="cuda") * w.s_std for _ in range(n_steps - 1)]
+    for sc in s_rot[:3]:
+        api.sas_sparse_decode_select(desc, q, kc, vc, ctx, sc, o, idx)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for sc in s_rot:
+                api.sas_sparse_decode_select(desc, q, kc, vc, ctx, sc, o, idx)
+    torch.cuda.current_stream().wait_stream(st)
+    for _ in range(3):
+        g.replay()
+    times = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b) / n_steps)
+    del g, inp, kc, vc, s_rot
+    torch.cuda.empty_cache()
+    return statistics.median(times)
+
+
+PHASES = ("entry", "ctx_len", "cluster_barrier", "scores_landed", "threshold", "candidates", "selected",
+          "first_block", "stream_end", "cta_partial", "slices_received", "exit")
+
+
+def phase_table(rows) -> dict:
+    """Per-phase median and maximum (us after the earliest CTA entry) from the
+    decode kernel's trace rows, each CTA's %clock64 stamps put on the common
+    %globaltimer line by its entry and exit (timer, clock) pairs."""
+    import numpy as np
+
+    raw = np.asarray(rows, dtype=np.int64)
+    n = int(raw[0, 31])
+    raw = raw[:n]
+    # timer values are ns since an epoch (~1e18): offsets first, in integers, so
+    # that float64 keeps ns resolution
+    gt0 = raw[:, 12].min()
+    rows = raw.astype(np.float64)
+    gte = (raw[:, 12] - gt0).astype(np.float64)
+    rate = (raw[:, 14] - raw[:, 12]).astype(np.float64) / (raw[:, 15] - raw[:, 13]).astype(np.float64)  # ns/clock
+    t = gte[:, None] + (raw[:, :12] - raw[:, 13:14]).astype(np.float64) * rate[:, None]
+    t0 = t[:, 0].min()
+    out = {"ctas": n, "sm_clock_ghz": float(np.median(1.0 / rate))}
+    for k, name in enumerate(PHASES):
+        v = (t[:, k] - t0) / 1e3
+        ok = (rows[:, k] >= rows[:, 13] - 1e6) & (rows[:, k] <= rows[:, 15])  # stamped in this launch
+        if ok.all():
+            out[name] = [round(float(np.median(v)), 3), round(float(v.max()), 3)]
+    out["candidates_median"] = float(np.median(rows[:, 17]))
+    out["blocks_per_cta"] = [int(rows[:, 18].min()), int(rows[:, 18].max())]
+    return out
+
+
+def decode_phases(api) -> dict:
+    """Launch floor and phase breakdown of the fused decode step on both decode
+    workloads: events around one launch (L2 flushed before it) and per step of a
+    16-step CUDA graph, for the decode and for an empty kernel on the same grid,
+    cluster, block and shared memory (sas_sparse_decode_launch_floor); with a
+    library built with --phase-trace, the per-phase table of one flushed launch
+    and of the last step of a graph replay."""
+    import torch
+
+    from trainable_block_sparse_sas_b200 import synthetic as syn
+
+    traced = True
+    out = {}
+    for w in (syn.DECODE_128K, syn.DECODE_512K):
+        inp = syn.decode_inputs(w, device="cuda", seed=3000)
+        q, kc, vc, ctx, s = (inp[x] for x in ("q", "k_cache", "v_cache", "ctx_len", "s"))
+        desc = api.decode_desc(q, kc, w.bs, w.top_k)
+        idx = torch.empty((w.B, w.Hkv, w.top_k), dtype=torch.int32, device="cuda")
+        o = torch.empty_like(q)
+        flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")
+        gs = torch.Generator(device="cuda")
+        gs.manual_seed(3200)
+        s_rot = [s] + [torch.randn(s.shape, generator=gs, device="cuda") * w.s_std for _ in range(15)]
+        rec = {}
+        calls = {"decode": lambda sc: api.sas_sparse_decode_select(desc, q, kc, vc, ctx, sc, o, idx),
+                 "floor": lambda sc: api.sas_sparse_decode_launch_floor(desc, q, kc, vc, ctx, sc, o)}
+        for name, call in calls.items():
+            for sc in s_rot[:3]:
+                call(sc)
+            ts = []
+            for i in range(20):
+                flush.sum()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                call(s_rot[i % 16])
+                b.record()
+                b.synchronize()
+                ts.append(a.elapsed_time(b) * 1e3)
+            rec[name + "_single_us"] = statistics.median(ts)
+            if name == "decode" and traced:
+                try:
+                    rec["phases_single"] = phase_table(api.sas_phase_trace_read(1024))
+                except api.SasError:  # a library built without the trace
+                    traced = False
+            g = torch.cuda.CUDAGraph()
+            st = torch.cuda.Stream()
+            st.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(st):
+                with torch.cuda.graph(g, stream=st):
+                    for sc in s_rot:
+                        call(sc)
+            torch.cuda.current_stream().wait_stream(st)
+            g.replay()
+            ts = []
+            for _ in range(20):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                b.synchronize()
+                ts.append(a.elapsed_time(b) * 1e3 / 16)
+            rec[name + "_graph_us"] = statistics.median(ts)
+            if name == "decode" and traced:
+                rec["phases_graph_last_step"] = phase_table(api.sas_phase_trace_read(1024))
+            del g
+        rec["stream_bytes"] = decode_bytes(w)
+        out[w.name] = rec
+        del inp, kc, vc, flush, s_rot
+        torch.cuda.empty_cache()
+    return out
+
+
 def decode_oracle_sample(w) -> dict:
     """The oracle's decode (selection + attention, fp64) timed on the host cores
     on a bounded sample of the workload: sequence 0 and kv head 0 (its G query
@@ -705,13 +856,19 @@ def extras(api, args, peaks, peak_kind) -> dict:
     torch.cuda.empty_cache()
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     for w in (syn.DECODE_128K, syn.DECODE_512K):
-        ms = time_decode(api, w, steps=20, mode="fused")
+        ms = time_decode_graph(api, w)
+        ms1 = time_decode(api, w, steps=20, mode="fused")
         by = decode_bytes(w)
         gbs = by / (ms * 1e-3) / 1e9
         rec = {"ms": ms, "bytes": by, "gbs": gbs, "frac_of_hbm": gbs / hbm, "hbm_peak_gbs": hbm,
                "peak_source": f"{peak_kind} copy", "frac_of_8tbs": gbs / 8000.0,
-               "l2": "flushed (512 MB read) before every repetition",
+               "timing": "per step of 16 back-to-back steps replayed from one CUDA graph, each step with its own "
+                         "score tensor (inputs larger than L2: the steps' attended blocks differ)",
                "includes": "Top-K selection + sparse decode in one launch (sas_sparse_decode_select)",
+               "single_launch_ms": ms1,
+               "single_launch_timing": "events around one launch, L2 flushed (512 MB read) before each; includes "
+                                       "the event and launch floor of a lone kernel (an empty kernel on the same "
+                                       "grid measures ~5-6 us this way)",
                "two_call_ms": time_decode(api, w, steps=10, mode="two_call"),
                "paged_ms": time_decode(api, w, steps=10, mode="paged")}
         rec["decode_scores"] = time_decode_scores(api, w, hbm)
@@ -723,7 +880,7 @@ def extras(api, args, peaks, peak_kind) -> dict:
             rec["dense_gbs"] = byd / (msd * 1e-3) / 1e9
             # the dense stream can exceed the torch-copy figure; the best rate seen is the tighter ceiling
             rec["frac_of_best_stream"] = gbs / max(hbm, rec["dense_gbs"])
-            rec["sparse_over_dense_speedup"] = msd / ms
+            rec["sparse_over_dense_speedup"] = msd / ms1
         out[w.name] = rec
     return out
 
@@ -745,6 +902,12 @@ def main():
     ap.add_argument("--profile-decode", type=int, default=0, metavar="T",
                     help="only run the fused decode of the 128K workload's geometry with a T-token cache "
                          "(a small case for profiler captures) and print its timing")
+    ap.add_argument("--decode-phases", action="store_true",
+                    help="only measure the decode launch floor and (with a --phase-trace build loaded through "
+                         "SAS_LIBRARY) the per-phase breakdown of the fused decode step")
+    ap.add_argument("--profile-scores", type=int, default=0, metavar="N",
+                    help="only run the pooled-key scorer of the 32K workload's geometry at sequence length N (a "
+                         "small case for profiler captures) and print its timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -770,6 +933,33 @@ def main():
         torch.cuda.synchronize()
         ms = {k: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
               for k, (a, b) in {"select": (0, 1), "fwd": (1, 2), "bwd_dq": (2, 3), "bwd_dkdv": (3, 4)}.items()}
+        print(json.dumps({"workload": w.name, "n": w.n, "ms": ms}))
+        return
+    if args.decode_phases:
+        from trainable_block_sparse_sas_b200 import api
+
+        print(json.dumps(decode_phases(api)))
+        return
+    if args.profile_scores:
+        import torch
+
+        from trainable_block_sparse_sas_b200 import api
+        from trainable_block_sparse_sas_b200 import synthetic as syn
+
+        w = dataclasses.replace(syn.TRAIN_SPARSE_32K, name="scores_geometry", n=args.profile_scores)
+        inp = syn.train_inputs(w, device="cuda", seed=2100)
+        desc = api.attn_desc(inp["q"], inp["k"], w.bs, w.top_k)
+        s = torch.empty((w.B, w.Hkv, w.Cq, w.Cq), device="cuda")
+        ws = api.workspace(api.sas_pooled_scores_workspace_size(desc), inp["q"].device)
+        for _ in range(args.warmup):
+            api.sas_pooled_scores(desc, inp["q"], inp["k"], s, ws)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in evs:
+            a.record()
+            api.sas_pooled_scores(desc, inp["q"], inp["k"], s, ws)
+            b.record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
         print(json.dumps({"workload": w.name, "n": w.n, "ms": ms}))
         return
     if args.profile_decode:

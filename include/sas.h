@@ -413,6 +413,30 @@ sas_status sas_get_device_status(int32_t* status, sas_stream_t stream);
  * status word. */
 sas_status sas_selftest_bounded_wait(int32_t limit_ms, int32_t* status, int32_t* trace, sas_stream_t stream);
 
+/* sas_sparse_decode_launch_floor -- launches, on `stream`, an empty kernel with the
+ * grid, cluster, block size and dynamic shared memory that sas_sparse_decode_select
+ * launches for the same arguments.  It reads and writes no buffer; timing it gives
+ * the launch floor under the fused decode step.  Arguments and errors as for
+ * sas_sparse_decode_select (no status word, no idx_out). */
+sas_status sas_sparse_decode_launch_floor(const sas_decode_desc* desc, const void* q, const void* k_cache,
+                                          const void* v_cache, const int32_t* ctx_len, const float* s,
+                                          int32_t s_cols, void* o, sas_stream_t stream);
+
+/* sas_phase_trace_read -- in a library built with SAS_PHASE_TRACE
+ * (`python -m trainable_block_sparse_sas_b200.build --phase-trace`, giving
+ * libsas_trace.so), the decode kernel records per CTA (row = blockIdx.y *
+ * gridDim.x + blockIdx.x, the first 1024 CTAs) 32 uint64 slots: %clock64 at its
+ * phase boundaries (0 entry, 1 ctx_len read, 2 cluster barrier passed, 3 staged
+ * scores landed, 4 threshold known, 5 candidates placed, 6 selection done, 7 first
+ * K/V block landed, 8 last block consumed, 9 partial merged in the CTA, 10 the
+ * cluster's slices received, 11 exit), (%globaltimer, %clock64) pairs at entry
+ * (12, 13) and exit (14, 15), the SM id (16), the candidate count (17), the blocks
+ * this CTA streamed (18) and the grid's CTAs (31).  Slots a launch did not reach
+ * keep older values.  Copies `rows` rows (1..1024) to host memory after a device
+ * synchronisation.  SAS_ERR_UNSUPPORTED in builds without the trace;
+ * SAS_ERR_INVALID_VALUE for a NULL destination or rows out of range. */
+sas_status sas_phase_trace_read(uint64_t* host_dst, int32_t rows);
+
 /* Number of kernels this library has launched in this process (all devices),
  * counted on the host at each successful launch. */
 uint64_t sas_launch_count(void);

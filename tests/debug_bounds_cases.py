@@ -84,8 +84,9 @@ def main():
     assert os.environ.get("SAS_LIBRARY", "").endswith("libsas_debug.so"), "run with SAS_LIBRARY=.../libsas_debug.so"
     assert api._LIB_PATH == os.environ["SAS_LIBRARY"]
     word = api.status_word()
-    # tensor-core training kernels (G 2 and 4; sparse and full scope; the gates)
+    # tensor-core training kernels (G 2, 4 and 8; sparse and full scope; the gates)
     train_case(word, 1, 512, 4, 1, 128, 64, 3, False, torch.bfloat16)
+    train_case(word, 1, 512, 8, 1, 128, 64, 3, False, torch.bfloat16)
     train_case(word, 1, 512, 4, 2, 128, 64, 0, True, torch.bfloat16)
     for gate in ("outer", "ste", "sigmoid"):
         train_case(word, 1, 512, 8, 2, 128, 64, 3, False, torch.bfloat16, gate)

@@ -157,6 +157,16 @@ def test_status_word_and_selftest_checks(api):
         assert L.sas_selftest_bounded_wait(bad, FAKE, None, None) == 1
 
 
+def test_floor_and_trace_checks(api):
+    """The launch-floor and phase-trace diagnostics reject bad arguments before
+    touching the device."""
+    L = api.lib
+    assert L.sas_sparse_decode_launch_floor(None, FAKE, FAKE, FAKE, FAKE, FAKE, 4, FAKE, None) == 1
+    assert L.sas_phase_trace_read(None, 4) == 1
+    for bad in (0, -1, 1025):
+        assert L.sas_phase_trace_read(FAKE, bad) == 1
+
+
 def test_cuda_library_and_oracle_share_nothing(api):
     """The product path never imports, loads or links the oracle, and the oracle
     never includes the library's headers or sources."""

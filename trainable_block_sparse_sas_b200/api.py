@@ -73,6 +73,10 @@ lib.sas_sparse_decode.restype = ctypes.c_int
 lib.sas_sparse_decode.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 7 + [_sz, _vp, _vp]
 lib.sas_sparse_decode_select.restype = ctypes.c_int
 lib.sas_sparse_decode_select.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 5 + [_i32, _vp, _vp, _vp, _vp]
+lib.sas_sparse_decode_launch_floor.restype = ctypes.c_int
+lib.sas_sparse_decode_launch_floor.argtypes = [ctypes.POINTER(DecodeDesc)] + [_vp] * 5 + [_i32, _vp, _vp]
+lib.sas_phase_trace_read.restype = ctypes.c_int
+lib.sas_phase_trace_read.argtypes = [_vp, _i32]
 lib.sas_sparse_decode_paged.restype = ctypes.c_int
 lib.sas_sparse_decode_paged.argtypes = [ctypes.POINTER(DecodeDesc), _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32,
                                         _vp, _vp, _vp, _vp]
@@ -318,6 +322,27 @@ def sas_sparse_decode_select(desc, q, k_cache, v_cache, ctx_len, s, o, idx_out=N
     _check(lib.sas_sparse_decode_select(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(s),
                                         s.shape[-1], _p(o), _p(idx_out), _status(status, q), _stream(stream)),
            "sas_sparse_decode_select")
+
+
+def sas_sparse_decode_launch_floor(desc, q, k_cache, v_cache, ctx_len, s, o, stream=None):
+    """An empty kernel on the grid, cluster, block and shared memory of the fused
+    decode step with these arguments (the launch floor under it)."""
+    _check_decode(desc, q, o, ctx_len)
+    _check_cache(desc, k_cache, v_cache)
+    _need(s, desc.batch * desc.n_kv_heads * s.shape[-1], _F32, "s")
+    _check(lib.sas_sparse_decode_launch_floor(ctypes.byref(desc), _p(q), _p(k_cache), _p(v_cache), _p(ctx_len), _p(s),
+                                              s.shape[-1], _p(o), _stream(stream)),
+           "sas_sparse_decode_launch_floor")
+
+
+def sas_phase_trace_read(rows: int):
+    """The decode kernel's phase trace (a library built with --phase-trace):
+    numpy uint64 [rows, 32], one row per CTA."""
+    import numpy as np
+
+    buf = np.zeros((rows, 32), dtype=np.uint64)
+    _check(lib.sas_phase_trace_read(buf.ctypes.data_as(ctypes.c_void_p), rows), "sas_phase_trace_read")
+    return buf
 
 
 def paged_decode_desc(q, k_pages, block_size: int, top_k: int, max_ctx: int, softmax_scale: float = 0.0) -> DecodeDesc:

@@ -1,13 +1,16 @@
 """Build libsas.so (the CUDA kernels and their C ABI) in-tree for sm_100a.
 
-    python -m trainable_block_sparse_sas_b200.build [--force] [-v] [--debug-bounds]
+    python -m trainable_block_sparse_sas_b200.build [--force] [-v] [--debug-bounds | --phase-trace]
 
 Each csrc/*.cu is compiled to an object under _build/ (in parallel, skipped when
 up to date), then linked into trainable_block_sparse_sas_b200/libsas.so.  With
 --debug-bounds the same sources are built with -DSAS_DEBUG_BOUNDS (every kernel
 checks the global-memory indices it computes against its buffers' extents and
 records a failure in the caller's status word instead of making the access) into
-libsas_debug.so, objects under _build/debug_bounds/.
+libsas_debug.so, objects under _build/debug_bounds/.  With --phase-trace they are
+built with -DSAS_PHASE_TRACE (the decode kernel records %clock64 at its phase
+boundaries, read back by sas_phase_trace_read) into libsas_trace.so, objects
+under _build/phase_trace/.
 """
 from __future__ import annotations
 
@@ -25,6 +28,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsas.so")
 LIB_DEBUG = os.path.join(PKG, "libsas_debug.so")
+LIB_TRACE = os.path.join(PKG, "libsas_trace.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -54,10 +58,15 @@ def _compile(src: str, obj: str, verbose: bool, extra=()) -> str:
     return r.stderr
 
 
-def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False) -> str:
-    out_dir = os.path.join(BUILD, "debug_bounds") if debug_bounds else BUILD
-    lib = LIB_DEBUG if debug_bounds else LIB
-    extra = ("-DSAS_DEBUG_BOUNDS",) if debug_bounds else ()
+def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False, phase_trace: bool = False) -> str:
+    if debug_bounds and phase_trace:
+        raise ValueError("one variant at a time")
+    if debug_bounds:
+        out_dir, lib, extra = os.path.join(BUILD, "debug_bounds"), LIB_DEBUG, ("-DSAS_DEBUG_BOUNDS",)
+    elif phase_trace:
+        out_dir, lib, extra = os.path.join(BUILD, "phase_trace"), LIB_TRACE, ("-DSAS_PHASE_TRACE",)
+    else:
+        out_dir, lib, extra = BUILD, LIB, ()
     os.makedirs(out_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     deps = _deps_mtime()
@@ -83,4 +92,5 @@ def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug_bounds="--debug-bounds" in sys.argv,
+                phase_trace="--phase-trace" in sys.argv))

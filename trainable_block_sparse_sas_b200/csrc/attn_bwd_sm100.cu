@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
     constexpr int kStages = ST;
     constexpr int G = L::G;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = smem_align1024(smem_raw);
     const uint32_t sbase = smem_u32(base);
     const uint32_t sQ = sbase + L::kQ, sDO = sbase + L::kDO, sK = sbase + L::kK, sV = sbase + L::kV;
     const uint32_t bar0 = sbase + L::kBars;
@@ -613,7 +613,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     constexpr int kRowsTok = 128 / G;  // tokens per 128-row item
     constexpr int kPreItems = kStages < MT ? kStages : MT;  // items of query block m, loaded up front
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = smem_align1024(smem_raw);
     const uint32_t sbase = smem_u32(base);
     const uint32_t sK = sbase + L::kK, sV = sbase + L::kV, sQ = sbase + L::kQ, sDO = sbase + L::kDO;
     const uint32_t sP = sbase + L::kP, sDS = sbase + L::kDS;

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_sm100_kernel(const __grid_con
     using L = FwdLayout<MT>;
     constexpr int G = L::G;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = smem_align1024(smem_raw);
     const uint32_t sbase = smem_u32(base);
     const uint32_t sQ = sbase + L::kQ, sKV = sbase + L::kKV;
     const uint32_t bar0 = sbase + L::kBars;

@@ -29,6 +29,35 @@ namespace {
 
 using namespace sm100;
 
+// Phase trace (builds with SAS_PHASE_TRACE only): per CTA of the decode kernel,
+// %clock64 at the phase boundaries named below, plus one (%globaltimer,
+// %clock64) pair at entry and one at exit that put every CTA on one time line
+// (a %globaltimer read costs hundreds of cycles, so it is taken only there, by
+// threads not on the critical path).
+enum TraceSlot {
+    kTrEntry = 0, kTrCtx, kTrClusterSync, kTrScores, kTrTau, kTrCand, kTrSelected, kTrFirstBlock, kTrStreamEnd,
+    kTrPartial, kTrIncoming, kTrExit, kTrGtEntry, kTrClkEntry, kTrGtExit, kTrClkExit, kTrSmid, kTrCandCount,
+    kTrBlocks, kTrGrid = 31
+};
+#ifdef SAS_PHASE_TRACE
+constexpr int kTraceCtas = 1024, kTraceSlots = 32;
+__device__ unsigned long long g_trace[kTraceCtas][kTraceSlots];
+__device__ __forceinline__ unsigned long long clk64() {
+    unsigned long long c;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+    return c;
+}
+__device__ __forceinline__ void trace_put(int slot, unsigned long long v) {
+    const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;
+    if (cta < (unsigned)kTraceCtas) g_trace[cta][slot] = v;
+}
+#define SAS_TRACE(slot) trace_put((slot), clk64())
+#define SAS_TRACE_VALUE(slot, v) trace_put((slot), (unsigned long long)(v))
+#else
+#define SAS_TRACE(slot) ((void)0)
+#define SAS_TRACE_VALUE(slot, v) ((void)0)
+#endif
+
 constexpr int kD = 128;
 constexpr int kBS = 64;
 constexpr int kThreads = 288;  // warp 0: TMA producer; warps 1..8: consumers
@@ -50,7 +79,8 @@ struct DecArgs {
     __nv_bfloat16* o;
     int* status;
     int B, Hq, Hkv, Tmax, top_k, s_cols, mode;  // mode 0: given idx, 1: fused selection, 2: dense
-    int vec_scores;  // the score rows are 16-byte aligned (s_cols % 4 == 0, aligned s): vector loads
+    int vec_scores;  // the score rows are 16-byte aligned (s_cols % 4 == 0, aligned s): one bulk copy
+    int list_cap;    // entries of the attended list (shared-memory layout)
     float scale_log2;
     const int32_t* page_table;  // nullptr: contiguous caches
     int pages_per_seq, num_pages;
@@ -88,14 +118,21 @@ struct Layout {
     static constexpr uint32_t kRing = 0;
     static constexpr uint32_t kQ = kRing + kStages * kStage;  // 16 rows x kQLd bf16
     static constexpr uint32_t kBars = kQ + 16 * kQLd * 2;
-    static constexpr uint32_t kMisc = kBars + 8 * 2 * kStages;  // abort, bin, above, count, scratch
+    static constexpr uint32_t kMisc = kBars + 8 * (2 * kStages + 2);  // abort, bin, above, count, scratch
     static constexpr uint32_t kHist = kMisc + 64;              // 2 x 256 ints
     static constexpr uint32_t kGsum = kHist + 2 * 256 * 4;     // 256 ints
     static constexpr uint32_t kScan = kGsum + 256 * 4;         // 40 ints
     static constexpr uint32_t kCnt = kScan + 40 * 4;           // 2 ints (gt, eq) of this CTA
     static constexpr uint32_t kCpart = kCnt + 16;              // [G][d + 2] floats
     __host__ __device__ static uint32_t list_off(int G) { return kCpart + 4 * (uint32_t)G * (kD + 2); }
-    static size_t bytes(int G, int list_cap) { return 1024 + list_off(G) + 4 * (size_t)list_cap; }
+    // the slices of merged outputs received from the cluster's CTAs: [CL][per + 2 G] floats
+    __host__ __device__ static uint32_t in_off(int G, int list_cap) {
+        return (list_off(G) + 4 * (uint32_t)list_cap + 15) & ~15u;
+    }
+    static size_t bytes(int G, int list_cap, int CL) {
+        const int per = (G * kD + CL - 1) / CL;
+        return 1024 + in_off(G, list_cap) + 4 * (size_t)CL * (per + 2 * G);
+    }
 };
 
 // Histogram increment with one shared-memory atomic per distinct bin in the
@@ -114,136 +151,215 @@ __device__ __forceinline__ int block_sum_int(int v, int* scan) {
 
 // Exact Top-K of the row's first Cb block scores, computed by this CTA alone
 // (every CTA of the cluster derives the same list, so no exchange is needed).
-// The row's scores arrive at kernel entry as 16-byte vectors: thread tid holds
-// scores 4 (tid + u kThreads) .. + 3 in x[u], u < nv (nv uniform, the vectors the
-// row needs).  The per-score work uses 32-bit order keys: the K-th largest of the
-// threads' maxima (counted with multiplicity) is a lower bound tau of the K-th
-// largest score, since K maxima reach it; every score whose key is at least tau is
-// a candidate.  Only the 288 maxima and the few candidates carry unique 64-bit
-// keys (order key << 32 | (2^32 - 1 - index)), so that equal scores prefer the
-// lower block index.  Returns K, or -1 when more than kCandCap scores reach tau
-// (the caller then runs the radix select).
+// The row (s_cols <= kSelMax floats) is staged in ring stage 2 by a bulk copy
+// issued at kernel entry; warps 1..kSelWarps do the work, the other warps wait
+// at the closing CTA barrier.  Keys are 32-bit order keys:
+//   1. every thread keeps the two largest keys of its 16-byte vectors;
+//   2. one warp takes, per lane, the two largest of the values the selection
+//      warps kept for that lane's column, sorts those 64 values (each a distinct
+//      score) and reads off the K-th largest: a lower bound tau of the K-th
+//      largest score, since K scores reach it;
+//   3. every score whose key is at least tau is a candidate (K to a few more on
+//      random rows), placed by a warp-wide scan plus one shared atomic per warp;
+//   4. candidates are ranked exactly on the unique 64-bit key (order key << 32 |
+//      (2^32 - 1 - index)), so equal scores prefer the lower block index, and
+//      the K chosen blocks go to list[1 .. K] in ascending order.
+// Returns K, or -1 when more than kCandCap scores reach tau (the caller then
+// runs the radix select).  Called by every thread of the CTA.
 constexpr int kCandCap = 512;
-constexpr int kVec = 8;  // 16-byte score vectors per thread: rows of up to 4 * kVec * kThreads blocks
+constexpr int kSelWarps = 4;  // warps 1..4
+constexpr int kSelThreads = 32 * kSelWarps;
+constexpr int kSelMax = (int)(kStage / 4);  // scores a staged row may hold (8192)
 
-__device__ int row_topk_filter(const DecArgs& a, int Cb, int nv, const float4 (&x)[kVec], uint8_t* base, int* list) {
-    constexpr int kWarps = kThreads / 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int K = a.top_k;
-    // scratch in ring stage 1 (stage 0 may hold the prefetched current block)
-    unsigned long long* sorted = reinterpret_cast<unsigned long long*>(base + Layout::kRing + kStage);
-    unsigned long long* cand = sorted + kWarps * 32;
-    unsigned long long* chosen = cand + kCandCap;
-    uint32_t* thr_sh = reinterpret_cast<uint32_t*>(chosen + 64);
-    int* misc = reinterpret_cast<int*>(base + Layout::kMisc);
-    // this thread's maximum: 32-bit key, and the index of a score that has it
-    uint32_t kmax = 0u;  // 0: no score (every real key is larger)
-    int mmax = 0;
+__device__ __forceinline__ void sel_bar() { asm volatile("bar.sync 2, %0;" ::"n"(kSelThreads) : "memory"); }
+
+__device__ __forceinline__ void top2_insert(uint32_t k, uint32_t& k1, uint32_t& k2) {
+    const uint32_t lo = min(k, k1);
+    k1 = max(k, k1);
+    k2 = max(k2, lo);
+}
+
+// 64 keys, two per lane (position lane and 32 + lane), sorted descending by a
+// bitonic network; every lane gets the key at sorted position p.
+__device__ __forceinline__ uint32_t warp_kth_of_64(uint32_t x0, uint32_t x1, int p) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-        if (u < nv) {
-            const int m0 = 4 * (tid + u * kThreads);
-            const float xe[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const uint32_t k = m0 + e < Cb ? order_key(xe[e]) : 0u;
-                if (k > kmax) {
-                    kmax = k;
-                    mmax = m0 + e;
-                }
-            }
-        }
-    }
-    if (tid == 0) {
-        misc[5] = 0;
-        *thr_sh = 0u;
-    }
-    // the maxima as unique keys; each warp's 32 sorted descending
-    unsigned long long v = kmax ? (((unsigned long long)kmax << 32) | (0xFFFFFFFFu - (uint32_t)mmax)) : 0ull;
-#pragma unroll
-    for (int k = 2; k <= 32; k <<= 1) {
+    for (int k = 2; k <= 64; k <<= 1) {
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
-            const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, j);
-            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
-            v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
-        }
-    }
-    sorted[warp * 32 + lane] = v;
-    __syncthreads();
-    // rank of this maximum among all: `lane` larger ones in its own list (keys are
-    // unique), plus a branch-free fixed-step search of every other list (the
-    // searches are independent, so their loads overlap)
-    {
-        int cnt[kWarps];
-#pragma unroll
-        for (int w2 = 0; w2 < kWarps; ++w2) cnt[w2] = 0;
-#pragma unroll
-        for (int step = 16; step > 0; step >>= 1) {
-#pragma unroll
-            for (int w2 = 0; w2 < kWarps; ++w2) {
-                const unsigned long long e = sorted[w2 * 32 + cnt[w2] + step - 1];
-                cnt[w2] += e > v ? step : 0;
+            if (j == 32) {  // partners in the same lane (k = 64: the whole sequence descends)
+                const uint32_t hi = max(x0, x1), lo = min(x0, x1);
+                x0 = hi;
+                x1 = lo;
+            } else {
+                const uint32_t y0 = __shfl_xor_sync(0xffffffffu, x0, j);
+                const uint32_t y1 = __shfl_xor_sync(0xffffffffu, x1, j);
+                const bool lower = (lane & j) == 0;
+                const bool desc0 = (lane & k) == 0, desc1 = ((lane + 32) & k) == 0;
+                x0 = (lower == desc0) ? max(x0, y0) : min(x0, y0);
+                x1 = (lower == desc1) ? max(x1, y1) : min(x1, y1);
             }
         }
-        int rk = lane;
-#pragma unroll
-        for (int w2 = 0; w2 < kWarps; ++w2) {
-            // cnt counts up to 31 entries; the last entry is compared apart
-            const int c2 = cnt[w2] + (sorted[w2 * 32 + 31] > v ? 1 : 0) * (cnt[w2] == 31 ? 1 : 0);
-            rk += w2 == warp ? 0 : c2;
-        }
-        if (v != 0ull && rk == K - 1) *thr_sh = (uint32_t)(v >> 32);
     }
-    __syncthreads();
-    const uint32_t thr = *thr_sh;
-    // candidates: every score whose key reaches tau, one shared-memory atomic per
-    // warp and vector element
+    const uint32_t v0 = __shfl_sync(0xffffffffu, x0, p & 31), v1 = __shfl_sync(0xffffffffu, x1, p & 31);
+    return p < 32 ? v0 : v1;
+}
+
+__device__ __forceinline__ float4 lds_f4(uint32_t saddr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(saddr));
+    return v;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t saddr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(saddr));
+    return v;
+}
+
+// rank of k among the first C candidates: how many are larger (four independent sums)
+__device__ __forceinline__ int count_larger(const unsigned long long* cand, int C, unsigned long long k) {
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0, j = 0;
+    for (; j + 4 <= C; j += 4) {
+        r0 += cand[j] > k ? 1 : 0;
+        r1 += cand[j + 1] > k ? 1 : 0;
+        r2 += cand[j + 2] > k ? 1 : 0;
+        r3 += cand[j + 3] > k ? 1 : 0;
+    }
+    for (; j < C; ++j) r0 += cand[j] > k ? 1 : 0;
+    return r0 + r1 + r2 + r3;
+}
+
+constexpr int kSelVecs = kSelMax / 4 / kSelThreads;  // 16-byte vectors per selection thread (16)
+
+__device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* list, uint32_t sbar,
+                               volatile int* abort_flag) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int K = a.top_k;
+    const uint32_t sc = smem_u32(base + Layout::kRing + 2 * kStage);
+    // scratch in ring stage 1 (stage 0 may hold the prefetched current block)
+    uint32_t* tops = reinterpret_cast<uint32_t*>(base + Layout::kRing + kStage);               // [warps][64]
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(tops + kSelWarps * 64);  // [kCandCap]
+    unsigned long long* chosen = cand + kCandCap;                                              // [K]
+    int* misc = reinterpret_cast<int*>(base + Layout::kMisc);  // [5]: candidates, [6]: tau
+    if (warp >= 1 && warp <= kSelWarps) {
+        const int t = tid - 32, w = warp - 1;
+        const int nv = (Cb + 3) / 4;  // vectors holding the first Cb scores; thread t takes t + 128 u
+        const bool ok = warp_wait(sbar, 0, abort_flag, a.status);
+        if (!ok) mbar_wait_drain(sbar, 0, a.status);  // the copy lands before its stage is reused
+        if (t == 0) SAS_TRACE(kTrScores);
+        // the vectors of this thread, four at a time (loads in flight together), as
+        // 32-bit keys; 0 for no score (every real key is larger)
+        auto keys4 = [&](int u0, uint32_t (&k)[16]) {
+            float4 v[4];
 #pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-        if (u < nv) {
-            const int m0 = 4 * (tid + u * kThreads);
-            const float xe[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+            for (int u = 0; u < 4; ++u) {
+                const int i = t + (u0 + u) * kSelThreads;
+                v[u] = i < nv ? lds_f4(sc + 16u * (uint32_t)i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int m = m0 + e;
-                const uint32_t k = m < Cb ? order_key(xe[e]) : 0u;
-                const bool take = m < Cb && k >= thr;
-                const unsigned bal = __ballot_sync(0xffffffffu, take);
-                if (bal) {
-                    int base_pos = 0;
-                    if (lane == 0) base_pos = atomicAdd(&misc[5], __popc(bal));
-                    base_pos = __shfl_sync(0xffffffffu, base_pos, 0);
-                    const int pos = base_pos + __popc(bal & ((1u << lane) - 1u));
-                    if (take && pos < kCandCap)
-                        cand[pos] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)m);
+            for (int u = 0; u < 4; ++u) {
+                const int m0 = 4 * (t + (u0 + u) * kSelThreads);
+                const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) k[4 * u + c] = m0 + c < Cb ? order_key(e[c]) : 0u;
+            }
+        };
+        uint32_t k1 = 0u, k2 = 0u, k1b = 0u, k2b = 0u;
+        if (ok) {
+#pragma unroll
+            for (int u0 = 0; u0 < kSelVecs; u0 += 4) {
+                if (t + u0 * kSelThreads >= nv) break;
+                uint32_t k[16];
+                keys4(u0, k);
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    top2_insert(k[j], k1, k2);
+                    top2_insert(k[j + 1], k1b, k2b);
                 }
             }
         }
+        top2_insert(k1b, k1, k2);
+        top2_insert(k2b, k1, k2);
+        tops[w * 64 + lane] = k1;
+        tops[w * 64 + 32 + lane] = k2;
+        if (t == 0) misc[5] = 0;
+        sel_bar();
+        if (w == 0) {
+            uint32_t c1 = 0u, c2 = 0u;
+#pragma unroll
+            for (int w2 = 0; w2 < kSelWarps; ++w2) {
+                top2_insert(tops[w2 * 64 + lane], c1, c2);
+                top2_insert(tops[w2 * 64 + 32 + lane], c1, c2);
+            }
+            const uint32_t tau = warp_kth_of_64(c1, c2, K - 1);
+            if (lane == 0) misc[6] = (int)tau;
+        }
+        sel_bar();
+        if (t == 0) SAS_TRACE(kTrTau);
+        const uint32_t tau = (uint32_t)misc[6];
+        // candidates of this thread as a bit mask over its (at most 64) scores
+        unsigned long long mask = 0ull;
+        if (ok) {
+#pragma unroll
+            for (int u0 = 0; u0 < kSelVecs; u0 += 4) {
+                if (t + u0 * kSelThreads >= nv) break;
+                uint32_t k[16];
+                keys4(u0, k);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const bool in_row = 4 * (t + (u0 + (j >> 2)) * kSelThreads) + (j & 3) < Cb;
+                    mask |= (in_row && k[j] >= tau) ? (1ull << (4 * u0 + j)) : 0ull;
+                }
+            }
+        }
+        const int cnt = __popcll(mask);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int wbase = 0;
+        if (lane == 31 && incl > 0) wbase = atomicAdd(&misc[5], incl);
+        int pos = __shfl_sync(0xffffffffu, wbase, 31) + incl - cnt;
+        while (mask) {
+            const int bit = __ffsll((long long)mask) - 1;
+            mask &= mask - 1;
+            const int m = 4 * (t + (bit >> 2) * kSelThreads) + (bit & 3);
+            const uint32_t k = order_key(lds_f32(sc + 4u * (uint32_t)m));
+            if (pos < kCandCap) cand[pos] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)m);
+            ++pos;
+        }
+        sel_bar();
+        const int C = misc[5];
+        if (t == 0) {
+            SAS_TRACE(kTrCand);
+            SAS_TRACE_VALUE(kTrCandCount, C);
+        }
+        if (C <= kCandCap) {
+            for (int c = t; c < C; c += kSelThreads) {
+                const unsigned long long k = cand[c];
+                const int rk = count_larger(cand, C, k);
+                if (rk < K) chosen[rk] = k;
+            }
+            sel_bar();
+            for (int j = t; j < K; j += kSelThreads) {
+                const uint32_t m = 0xFFFFFFFFu - (uint32_t)(chosen[j] & 0xFFFFFFFFull);
+                int p0 = 0, p1 = 0, j2 = 0;
+                for (; j2 + 2 <= K; j2 += 2) {
+                    p0 += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m ? 1 : 0;
+                    p1 += (0xFFFFFFFFu - (uint32_t)(chosen[j2 + 1] & 0xFFFFFFFFull)) < m ? 1 : 0;
+                }
+                if (j2 < K) p0 += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m ? 1 : 0;
+                list[1 + p0 + p1] = (int)m;
+            }
+        }
     }
-    __syncthreads();
-    const int C = misc[5];
-    if (C > kCandCap) return -1;
-    for (int c = tid; c < C; c += kThreads) {
-        const unsigned long long k = cand[c];
-        int rk = 0, j = 0;
-        for (; j + 4 <= C; j += 4)
-            rk += (cand[j] > k) + (cand[j + 1] > k) + (cand[j + 2] > k) + (cand[j + 3] > k);
-        for (; j < C; ++j) rk += cand[j] > k;
-        if (rk < K) chosen[rk] = k;
-    }
-    __syncthreads();
-    for (int j = tid; j < K; j += kThreads) {
-        const uint32_t m = 0xFFFFFFFFu - (uint32_t)(chosen[j] & 0xFFFFFFFFull);
-        int pos = 0;
-#pragma unroll 4
-        for (int j2 = 0; j2 < K; ++j2) pos += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m;
-        list[1 + pos] = (int)m;
-    }
-    // generic-proxy writes to ring stage 1 before TMA reuses it
+    // generic-proxy accesses to ring stages 1 and 2 before TMA reuses them
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
-    return K;
+    return misc[5] <= kCandCap ? K : -1;
 }
 
 // Fused Top-K over the row's Cb block scores, split across the cluster.
@@ -579,7 +695,7 @@ __device__ int cluster_topk_fast(const DecArgs& a, int bh, int Cb, uint32_t rank
 template <int CL>
 __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __grid_constant__ DecArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* base = smem_align1024(smem_raw);
     const uint32_t sbase = smem_u32(base);
     const uint32_t ring = sbase + Layout::kRing;
     const uint32_t bar0 = sbase + Layout::kBars;
@@ -595,41 +711,47 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
     const uint32_t rank = cluster_ctarank();
     const int bh = blockIdx.y;
     const int b = bh / a.Hkv, h = bh % a.Hkv;
-    // fused selection by the per-CTA filter: the row's scores are requested first,
-    // in 16-byte vectors and independently of ctx_len (every one of the row's
-    // s_cols; those past the history are masked later)
-    const int nv = (a.s_cols + 4 * kThreads - 1) / (4 * kThreads);
-    const bool vec_ok = a.mode == 1 && a.vec_scores && nv <= kVec;
-    float4 xv[kVec];
-    if (vec_ok) {
-        const float4* srow4 = reinterpret_cast<const float4*>(a.s + (long)bh * a.s_cols);
-#pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-            if (u < nv) {
-                const int i4 = tid + u * kThreads;
-                xv[u] = 4 * i4 < a.s_cols &&
-                                SAS_IN_BOUNDS((long)bh * a.s_cols + 4 * i4 + 3, (long)a.B * a.Hkv * a.s_cols, a.status)
-                            ? __ldg(srow4 + i4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
+    const uint32_t sbar = bar0 + 8u * (2 * kStages), inbar = sbar + 8u;
+    // merged outputs: CTA r finishes outputs [r per, (r + 1) per) of the G*128;
+    // every CTA sends it that slice of its partial plus its (max, sum) per head
+    const int per = (G * kD + CL - 1) / CL, in_len = per + 2 * G;
+    float* incoming = reinterpret_cast<float*>(base + Layout::in_off(G, a.list_cap));  // [CL][in_len]
+    // fused selection: the row's scores (every one of its s_cols; those past the
+    // history are masked later) are requested first, by one bulk copy into ring
+    // stage 2, independently of ctx_len
+    const bool staged = a.mode == 1 && a.vec_scores && a.s_cols > 0 && a.s_cols <= kSelMax;
+    if (tid == 0) SAS_TRACE(kTrEntry);
+    if (tid == kThreads - 1) {
+        SAS_TRACE(kTrClkEntry);
+        SAS_TRACE_VALUE(kTrGtEntry, globaltimer());
     }
-    int T = a.ctx_len[b];
-    T = max(1, min(T, a.Tmax));
-    const int t = T - 1, Cb = t / kBS;
-    const int Csel = min(Cb, a.s_cols);
-    const bool use_filter = vec_ok && a.top_k < Csel && a.top_k <= 64;
-
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), 8);
         }
+        mbar_init(sbar, 1);
+        mbar_init(inbar, 1);
         *abort_flag = 0;
         fence_barrier_init();
+        if (staged) {
+            const uint32_t bytes = 4u * (uint32_t)a.s_cols;
+            const long off = (long)bh * a.s_cols;
+            mbar_arrive_expect_tx(sbar, bytes);
+            if (SAS_IN_BOUNDS(off + a.s_cols - 1, (long)a.B * a.Hkv * a.s_cols, a.status))
+                bulk_load(ring + 2 * kStage, a.s + off, bytes, sbar);
+        }
+        // the pushes of the other CTAs' partials complete this phase
+        mbar_arrive_expect_tx(inbar, 4u * (uint32_t)((CL - 1) * in_len));
         prefetch_tmap(&a.tk);
         prefetch_tmap(&a.tv);
     }
+    int T = a.ctx_len[b];
+    T = max(1, min(T, a.Tmax));
+    if (tid == 0) SAS_TRACE(kTrCtx);
+    const int t = T - 1, Cb = t / kBS;
+    const int Csel = min(Cb, a.s_cols);
+    const bool use_filter = staged && a.top_k < Csel && a.top_k <= 64;
     // q of the group, padded to 16 rows: one 16-byte load per thread
     if (tid < 16 * kD / 8) {
         const int r = tid / (kD / 8), e = (tid % (kD / 8)) * 8;
@@ -639,11 +761,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
                               : make_uint4(0u, 0u, 0u, 0u);
         *reinterpret_cast<uint4*>(qs + r * kQLd + e) = val;
     }
+    // every CTA of the cluster has initialised its barriers and is running before
+    // any shared memory or barrier of it is used remotely (also a CTA barrier)
+    cluster_sync();
+    if (tid == 0) SAS_TRACE(kTrClusterSync);
     // attended list: entry 0 = current (partial) block, entries 1.. = history blocks ascending
     int nsel;
     if (a.mode == 2) {
         nsel = Cb;
-        __syncthreads();
     } else if (a.mode == 0) {
         // the valid prefix of the ascending, -1 padded row: entries before the first
         // one outside [0, Cb)
@@ -659,14 +784,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         __syncthreads();
         nsel = misc[3];
     } else {
-        __syncthreads();
         // the current block (entry 0, on CTA 0) loads while the selection runs
         if (rank == 0 && tid == 0) {
             mbar_arrive_expect_tx(full(0), kStage);
             load_block(a, ring, full(0), b, h, bh, Cb, a.page_table ? page_of(a, b, Cb) : 0);
         }
+        // the staged row must have landed before ring stage 2 is used otherwise
+        if (staged && !use_filter && !warp_wait(sbar, 0, abort_flag, a.status)) mbar_wait_drain(sbar, 0, a.status);
         const int chunk = (Csel + CL - 1) / CL;
-        nsel = use_filter ? row_topk_filter(a, Csel, nv, xv, base, list) : -1;
+        nsel = use_filter ? row_topk_staged(a, Csel, base, list, sbar, abort_flag) : -1;
         if (nsel < 0) {
             if (a.top_k < Csel && chunk <= (int)(kStage / 4) && CL * a.top_k <= (int)(kStage / 8))
                 nsel = cluster_topk_fast<CL>(a, bh, Csel, rank, base, list);
@@ -678,6 +804,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
                 if (SAS_IN_BOUNDS((long)bh * a.top_k + i, (long)a.B * a.Hkv * a.top_k, a.status))
                     a.idx_out[(long)bh * a.top_k + i] = i < nsel ? list[1 + i] : -1;
     }
+    if (tid == 0) SAS_TRACE(kTrSelected);
     const int L = nsel + 1;
     // ceil split: CTA 0 always owns entry 0 (the current block, prefetched in mode 1)
     const int e0 = (int)(((long)rank * L + CL - 1) / CL), e1 = (int)(((long)(rank + 1) * L + CL - 1) / CL);
@@ -723,6 +850,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         for (int i = 0; e0 + i < e1; ++i) {
             const int st = i % kStages;
             if (!warp_wait(full(st), (i / kStages) & 1, abort_flag, a.status)) break;
+            if (i == 0 && tid == 32) SAS_TRACE(kTrFirstBlock);
             const int blk = block_of(e0 + i);
             const uint32_t kb = ring + st * kStage, vb = kb + kTile;
             const int tok0 = blk * kBS + 16 * wg;  // absolute first token of this warp's slice
@@ -809,6 +937,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
             __syncwarp();
             if (lane == 0) mbar_arrive(empty(st));
         }
+        if (tid == 32) SAS_TRACE(kTrStreamEnd);
         // row sums over the 4 lanes sharing a row
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
@@ -858,39 +987,71 @@ __global__ void __launch_bounds__(kThreads, 2) decode_cluster_kernel(const __gri
         }
     }
     __syncwarp();
-    cluster_sync();
-    {
-        // every CTA merges its slice of the G*128 outputs from the cluster's partials
-        const uint32_t cp_local = smem_u32(cpart);
-        const int total = G * kD;
-        const int per = (total + CL - 1) / CL;
-        const int o0 = (int)rank * per, o1 = min(total, o0 + per);
+    // every CTA's partial is complete (CTA barrier); CTA o gets the slice o of the
+    // numerators and the per-head (max, sum) of every CTA, its own by plain stores,
+    // the others' by remote stores that complete the bytes its barrier expects
+    __syncthreads();
+    if (tid == 0) {
+        SAS_TRACE(kTrPartial);
+        SAS_TRACE_VALUE(kTrBlocks, e1 - e0);
+    }
+    for (int j = tid; j < CL * in_len; j += kThreads) {
+        const int o = j / in_len, e = j - o * in_len;
+        float v;
+        if (e < per) {
+            const int i = o * per + e;
+            v = i < G * kD ? cpart[(i / kD) * (kD + 2) + i % kD] : 0.f;
+        } else {
+            const int q2 = e - per;  // maxima of heads 0..G-1, then their sums
+            v = cpart[(q2 % G) * (kD + 2) + kD + (q2 >= G ? 1 : 0)];
+        }
+        float* slot = incoming + (int)rank * in_len + e;
+        if (o == (int)rank) *slot = v;
+        else st_async_b32(mapa(smem_u32(slot), (uint32_t)o), __float_as_uint(v), mapa(inbar, (uint32_t)o));
+    }
+    // wait (ignoring the abort flag: no CTA leaves while others may still write to
+    // its shared memory) for the other CTAs' slices
+    const bool got = mbar_wait_drain(inbar, 0, a.status, 4 * kWaitLimitNs);
+    __syncthreads();
+    if (tid == 0) SAS_TRACE(kTrIncoming);
+    if (got) {
+        const int o0 = (int)rank * per, o1 = min(G * kD, o0 + per);
         for (int i = o0 + tid; i < o1; i += kThreads) {
-            const int g = i / kD, d = i % kD;
-            float mr[CL], num[CL], den[CL];
-#pragma unroll
-            for (int r = 0; r < CL; ++r) {
-                const uint32_t pr = mapa(cp_local, (uint32_t)r) + 4u * (uint32_t)(g * (kD + 2));
-                mr[r] = ld_dsmem_f32(pr + 4u * kD);
-                den[r] = ld_dsmem_f32(pr + 4u * (kD + 1));
-                num[r] = ld_dsmem_f32(pr + 4u * d);
-            }
+            const int e = i - o0, g = i / kD, d = i % kD;
             float M = -INFINITY;
 #pragma unroll
-            for (int r = 0; r < CL; ++r) M = fmaxf(M, mr[r]);
+            for (int r = 0; r < CL; ++r) M = fmaxf(M, incoming[r * in_len + per + g]);
             float n_ = 0.f, d_ = 0.f;
 #pragma unroll
             for (int r = 0; r < CL; ++r) {
-                if (mr[r] == -INFINITY) continue;
-                const float f = ex2(mr[r] - M);
-                n_ += num[r] * f;
-                d_ += den[r] * f;
+                const float mr = incoming[r * in_len + per + g];
+                if (mr == -INFINITY) continue;
+                const float f = ex2(mr - M);
+                n_ += incoming[r * in_len + e] * f;
+                d_ += incoming[r * in_len + per + G + g] * f;
             }
             const long oi = ((long)b * a.Hq + h * G + g) * kD + d;
             if (SAS_IN_BOUNDS(oi, (long)a.B * a.Hq * kD, a.status)) a.o[oi] = __float2bfloat16_rn(n_ / d_);
         }
     }
-    cluster_sync();  // keep every CTA's shared memory alive until all remote reads are done
+    if (tid == 0) {
+        SAS_TRACE(kTrExit);
+        SAS_TRACE(kTrClkExit);
+        SAS_TRACE_VALUE(kTrGtExit, globaltimer());
+        SAS_TRACE_VALUE(kTrGrid, gridDim.x * gridDim.y);
+        unsigned smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        SAS_TRACE_VALUE(kTrSmid, smid);
+    }
+}
+
+// The same grid, cluster, block and shared memory as decode_cluster_kernel<CL>,
+// doing nothing: its launch time is the floor under the decode's.
+template <int CL>
+__global__ void __launch_bounds__(kThreads, 2) decode_floor_kernel(const __grid_constant__ DecArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    (void)a;
+    (void)smem_raw;
 }
 
 bool encode_cache(CUtensorMap* map, const void* ptr, int Tmax, long rows) {
@@ -905,10 +1066,11 @@ bool encode_cache(CUtensorMap* map, const void* ptr, int Tmax, long rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int CL>
+template <int CL, bool kFloor>
 cudaError_t launch_cl(const DecArgs& a, int list_cap, cudaStream_t stream) {
     const int G = a.Hq / a.Hkv;
-    const size_t smem = Layout::bytes(G, list_cap);
+    const size_t smem = Layout::bytes(G, list_cap, CL);
+    auto kernel = kFloor ? decode_floor_kernel<CL> : decode_cluster_kernel<CL>;
     // raise the kernel's shared-memory limit only when a larger size is first needed
     // (no attribute call on the steady path, e.g. inside a CUDA graph capture)
     static size_t smem_set[64] = {};  // per device
@@ -916,7 +1078,7 @@ cudaError_t launch_cl(const DecArgs& a, int list_cap, cudaStream_t stream) {
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 0 || dev >= 64 || smem > smem_set[dev]) {
-        err = cudaFuncSetAttribute(decode_cluster_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
         if (dev >= 0 && dev < 64) smem_set[dev] = smem;
     }
@@ -932,7 +1094,7 @@ cudaError_t launch_cl(const DecArgs& a, int list_cap, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, decode_cluster_kernel<CL>, a);
+    err = cudaLaunchKernelEx(&cfg, kernel, a);
     if (err == cudaSuccess) count_launch();
     return err;
 }
@@ -947,7 +1109,7 @@ bool decode_sm100_supported(const DecodeParams& p) {
         15u)
         return false;
     if ((long)p.B * p.Hkv > 65535) return false;
-    return Layout::bytes(G, p.top_k + 1) <= 227 * 1024;
+    return Layout::bytes(G, p.top_k + 1, 8) <= 227 * 1024;  // the largest cluster needs the most
 }
 
 // Cluster size: about two CTAs per SM over all rows, at most 8, at most the
@@ -959,8 +1121,8 @@ static int pick_cluster(const DecodeParams& p, int max_entries) {
     return cl;
 }
 
-cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,
-                                cudaStream_t stream) {
+static cudaError_t launch_decode_impl(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,
+                                      bool floor, cudaStream_t stream) {
     DecArgs a;
     memset(&a, 0, sizeof(a));
     const long rows = (long)p.B * p.Hkv;
@@ -992,12 +1154,42 @@ cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_col
     a.scale_log2 = p.scale * kLog2e;
     const int max_entries = a.mode == 2 ? (p.Tmax + kBS - 1) / kBS : p.top_k + 1;
     const int list_cap = a.mode == 2 ? 1 : p.top_k + 1;
-    switch (pick_cluster(p, max_entries)) {
-        case 1: return launch_cl<1>(a, list_cap, stream);
-        case 2: return launch_cl<2>(a, list_cap, stream);
-        case 4: return launch_cl<4>(a, list_cap, stream);
-        default: return launch_cl<8>(a, list_cap, stream);
+    a.list_cap = list_cap;
+    const int cl = pick_cluster(p, max_entries);
+    if (floor) {
+        switch (cl) {
+            case 1: return launch_cl<1, true>(a, list_cap, stream);
+            case 2: return launch_cl<2, true>(a, list_cap, stream);
+            case 4: return launch_cl<4, true>(a, list_cap, stream);
+            default: return launch_cl<8, true>(a, list_cap, stream);
+        }
     }
+    switch (cl) {
+        case 1: return launch_cl<1, false>(a, list_cap, stream);
+        case 2: return launch_cl<2, false>(a, list_cap, stream);
+        case 4: return launch_cl<4, false>(a, list_cap, stream);
+        default: return launch_cl<8, false>(a, list_cap, stream);
+    }
+}
+
+cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,
+                                cudaStream_t stream) {
+    return launch_decode_impl(p, s, s_cols, idx_out, false, stream);
+}
+
+cudaError_t launch_decode_floor(const DecodeParams& p, const float* s, int s_cols, cudaStream_t stream) {
+    return launch_decode_impl(p, s, s_cols, nullptr, true, stream);
+}
+
+cudaError_t read_decode_trace(void* dst, size_t bytes) {
+#ifdef SAS_PHASE_TRACE
+    if (bytes > sizeof(g_trace)) bytes = sizeof(g_trace);
+    return cudaMemcpyFromSymbol(dst, g_trace, bytes);
+#else
+    (void)dst;
+    (void)bytes;
+    return cudaErrorNotSupported;
+#endif
 }
 
 }  // namespace sas

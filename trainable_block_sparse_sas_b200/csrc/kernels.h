@@ -107,5 +107,10 @@ bool decode_sm100_supported(const DecodeParams& p);
 // s != nullptr: fused Top-K selection from s [B, Hkv, s_cols] (idx_out nullable)
 cudaError_t launch_decode_sm100(const DecodeParams& p, const float* s, int s_cols, int32_t* idx_out,
                                 cudaStream_t stream);
+// an empty kernel on the grid, cluster, block and shared memory of the fused decode
+// of p (the launch floor under it)
+cudaError_t launch_decode_floor(const DecodeParams& p, const float* s, int s_cols, cudaStream_t stream);
+// the decode kernel's phase trace (builds with SAS_PHASE_TRACE; cudaErrorNotSupported otherwise)
+cudaError_t read_decode_trace(void* dst, size_t bytes);
 
 }  // namespace sas

@@ -379,6 +379,30 @@ sas_status sas_sparse_decode_select(const sas_decode_desc* desc, const void* q, 
     return from_cuda(launch_decode_sm100(p, s, s_cols, idx_out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+sas_status sas_sparse_decode_launch_floor(const sas_decode_desc* desc, const void* q, const void* k_cache,
+                                          const void* v_cache, const int32_t* ctx_len, const float* s,
+                                          int32_t s_cols, void* o, sas_stream_t stream) {
+    if (!check_decode(desc)) return SAS_ERR_INVALID_VALUE;
+    if (!q || !k_cache || !v_cache || !ctx_len || !s || !o || s_cols <= 0) return SAS_ERR_INVALID_VALUE;
+    DecodeParams p = make_decode(desc);
+    p.q = q;
+    p.k = k_cache;
+    p.v = v_cache;
+    p.ctx_len = ctx_len;
+    p.idx = nullptr;
+    p.o = o;
+    if (!supported_decode(desc) || !decode_sm100_supported(p)) return SAS_ERR_UNSUPPORTED;
+    return from_cuda(launch_decode_floor(p, s, s_cols, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_phase_trace_read(uint64_t* host_dst, int32_t rows) {
+    if (!host_dst || rows <= 0 || rows > 1024) return SAS_ERR_INVALID_VALUE;
+    cudaError_t err = cudaDeviceSynchronize();
+    if (err == cudaSuccess) err = read_decode_trace(host_dst, (size_t)rows * 32 * sizeof(uint64_t));
+    if (err == cudaErrorNotSupported) return SAS_ERR_UNSUPPORTED;
+    return from_cuda(err);
+}
+
 sas_status sas_sparse_decode_paged(const sas_decode_desc* desc, const void* q, const void* k_pages,
                                    const void* v_pages, const int32_t* page_table, int32_t pages_per_seq,
                                    int32_t num_pages, const int32_t* ctx_len, const int32_t* idx, const float* s,

@@ -24,6 +24,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared memory rounded up to a 1024-byte boundary (128-byte swizzled
+// tiles need it).  Derived by pointer arithmetic on the shared array, so that the
+// compiler keeps the shared address space and accesses through the result are
+// shared-memory instructions (a pointer rebuilt from an integer is generic).
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* smem_raw) {
+    return smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -119,6 +127,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// one contiguous global -> shared copy (16-byte aligned ends, size a multiple of 16)
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -252,6 +267,14 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t caddr) {
 
 __device__ __forceinline__ void st_dsmem_u32(uint32_t caddr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
+}
+
+// store to another CTA's shared memory that completes 4 bytes of the transaction
+// count of a barrier in that CTA (caddr and cbar: shared::cluster addresses there)
+__device__ __forceinline__ void st_async_b32(uint32_t caddr, uint32_t v, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(caddr), "r"(v),
+                 "r"(cbar)
+                 : "memory");
 }
 
 // ---------------------------------------------------------------- warp MMA (mma.sync)
