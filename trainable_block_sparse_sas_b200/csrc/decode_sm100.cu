@@ -152,8 +152,9 @@ __device__ __forceinline__ int block_sum_int(int v, int* scan) {
 // Exact Top-K of the row's first Cb block scores, computed by this CTA alone
 // (every CTA of the cluster derives the same list, so no exchange is needed).
 // The row (s_cols <= kSelMax floats) is staged in ring stage 2 by a bulk copy
-// issued at kernel entry; warps 1..kSelWarps do the work, the other warps wait
-// at the closing CTA barrier.  Keys are 32-bit order keys:
+// issued at kernel entry; warps 1..4 do the work (warps 1..8 for rows of over
+// 2048 scores), the others wait at the closing CTA barrier.  Keys are 32-bit
+// order keys:
 //   1. every thread keeps the two largest keys of its 16-byte vectors;
 //   2. one warp takes, per lane, the two largest of the values the selection
 //      warps kept for that lane's column, sorts those 64 values (each a distinct
@@ -162,16 +163,16 @@ __device__ __forceinline__ int block_sum_int(int v, int* scan) {
 //   3. every score whose key is at least tau is a candidate (K to a few more on
 //      random rows), placed by a warp-wide scan plus one shared atomic per warp;
 //   4. candidates are ranked exactly on the unique 64-bit key (order key << 32 |
-//      (2^32 - 1 - index)), so equal scores prefer the lower block index, and
-//      the K chosen blocks go to list[1 .. K] in ascending order.
+//      (2^32 - 1 - index)), so equal scores prefer the lower block index (with
+//      exactly K candidates every one is chosen), and the K chosen blocks go to
+//      list[1 .. K] in ascending order.
 // Returns K, or -1 when more than kCandCap scores reach tau (the caller then
 // runs the radix select).  Called by every thread of the CTA.
 constexpr int kCandCap = 512;
-constexpr int kSelWarps = 4;  // warps 1..4
-constexpr int kSelThreads = 32 * kSelWarps;
+constexpr int kSelWarpsMax = 8;  // warps 1..8
 constexpr int kSelMax = (int)(kStage / 4);  // scores a staged row may hold (8192)
 
-__device__ __forceinline__ void sel_bar() { asm volatile("bar.sync 2, %0;" ::"n"(kSelThreads) : "memory"); }
+__device__ __forceinline__ void sel_bar(int nthreads) { asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory"); }
 
 __device__ __forceinline__ void top2_insert(uint32_t k, uint32_t& k1, uint32_t& k2) {
     const uint32_t lo = min(k, k1);
@@ -230,7 +231,7 @@ __device__ __forceinline__ int count_larger(const unsigned long long* cand, int 
     return r0 + r1 + r2 + r3;
 }
 
-constexpr int kSelVecs = kSelMax / 4 / kSelThreads;  // 16-byte vectors per selection thread (16)
+constexpr int kSelVecs = kSelMax / 4 / 128;  // 16-byte vectors per selection thread, at most (16)
 
 __device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* list, uint32_t sbar,
                                volatile int* abort_flag) {
@@ -239,10 +240,12 @@ __device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* lis
     const uint32_t sc = smem_u32(base + Layout::kRing + 2 * kStage);
     // scratch in ring stage 1 (stage 0 may hold the prefetched current block)
     uint32_t* tops = reinterpret_cast<uint32_t*>(base + Layout::kRing + kStage);               // [warps][64]
-    unsigned long long* cand = reinterpret_cast<unsigned long long*>(tops + kSelWarps * 64);  // [kCandCap]
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(tops + kSelWarpsMax * 64);  // [kCandCap]
     unsigned long long* chosen = cand + kCandCap;                                              // [K]
     int* misc = reinterpret_cast<int*>(base + Layout::kMisc);  // [5]: candidates, [6]: tau
-    if (warp >= 1 && warp <= kSelWarps) {
+    const int nsw = Cb > 2048 ? 8 : 4;  // selection warps (uniform over the CTA)
+    const int nst = 32 * nsw;
+    if (warp >= 1 && warp <= nsw) {
         const int t = tid - 32, w = warp - 1;
         const int nv = (Cb + 3) / 4;  // vectors holding the first Cb scores; thread t takes t + 128 u
         const bool ok = warp_wait(sbar, 0, abort_flag, a.status);
@@ -254,12 +257,12 @@ __device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* lis
             float4 v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int i = t + (u0 + u) * kSelThreads;
+                const int i = t + (u0 + u) * nst;
                 v[u] = i < nv ? lds_f4(sc + 16u * (uint32_t)i) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int m0 = 4 * (t + (u0 + u) * kSelThreads);
+                const int m0 = 4 * (t + (u0 + u) * nst);
                 const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) k[4 * u + c] = m0 + c < Cb ? order_key(e[c]) : 0u;
@@ -269,7 +272,7 @@ __device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* lis
         if (ok) {
 #pragma unroll
             for (int u0 = 0; u0 < kSelVecs; u0 += 4) {
-                if (t + u0 * kSelThreads >= nv) break;
+                if (t + u0 * nst >= nv) break;
                 uint32_t k[16];
                 keys4(u0, k);
 #pragma unroll
@@ -284,18 +287,18 @@ __device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* lis
         tops[w * 64 + lane] = k1;
         tops[w * 64 + 32 + lane] = k2;
         if (t == 0) misc[5] = 0;
-        sel_bar();
+        sel_bar(nst);
         if (w == 0) {
             uint32_t c1 = 0u, c2 = 0u;
 #pragma unroll
-            for (int w2 = 0; w2 < kSelWarps; ++w2) {
+            for (int w2 = 0; w2 < nsw; ++w2) {
                 top2_insert(tops[w2 * 64 + lane], c1, c2);
                 top2_insert(tops[w2 * 64 + 32 + lane], c1, c2);
             }
             const uint32_t tau = warp_kth_of_64(c1, c2, K - 1);
             if (lane == 0) misc[6] = (int)tau;
         }
-        sel_bar();
+        sel_bar(nst);
         if (t == 0) SAS_TRACE(kTrTau);
         const uint32_t tau = (uint32_t)misc[6];
         // candidates of this thread as a bit mask over its (at most 64) scores
@@ -303,12 +306,12 @@ __device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* lis
         if (ok) {
 #pragma unroll
             for (int u0 = 0; u0 < kSelVecs; u0 += 4) {
-                if (t + u0 * kSelThreads >= nv) break;
+                if (t + u0 * nst >= nv) break;
                 uint32_t k[16];
                 keys4(u0, k);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const bool in_row = 4 * (t + (u0 + (j >> 2)) * kSelThreads) + (j & 3) < Cb;
+                    const bool in_row = 4 * (t + (u0 + (j >> 2)) * nst) + (j & 3) < Cb;
                     mask |= (in_row && k[j] >= tau) ? (1ull << (4 * u0 + j)) : 0ull;
                 }
             }
@@ -326,32 +329,37 @@ __device__ int row_topk_staged(const DecArgs& a, int Cb, uint8_t* base, int* lis
         while (mask) {
             const int bit = __ffsll((long long)mask) - 1;
             mask &= mask - 1;
-            const int m = 4 * (t + (bit >> 2) * kSelThreads) + (bit & 3);
+            const int m = 4 * (t + (bit >> 2) * nst) + (bit & 3);
             const uint32_t k = order_key(lds_f32(sc + 4u * (uint32_t)m));
             if (pos < kCandCap) cand[pos] = ((unsigned long long)k << 32) | (0xFFFFFFFFu - (uint32_t)m);
             ++pos;
         }
-        sel_bar();
+        sel_bar(nst);
         const int C = misc[5];
         if (t == 0) {
             SAS_TRACE(kTrCand);
             SAS_TRACE_VALUE(kTrCandCount, C);
         }
         if (C <= kCandCap) {
-            for (int c = t; c < C; c += kSelThreads) {
-                const unsigned long long k = cand[c];
-                const int rk = count_larger(cand, C, k);
-                if (rk < K) chosen[rk] = k;
+            // exactly K candidates: all chosen, only their order by index is needed
+            const unsigned long long* pick = cand;
+            if (C > K) {
+                for (int c = t; c < C; c += nst) {
+                    const unsigned long long k = cand[c];
+                    const int rk = count_larger(cand, C, k);
+                    if (rk < K) chosen[rk] = k;
+                }
+                sel_bar(nst);
+                pick = chosen;
             }
-            sel_bar();
-            for (int j = t; j < K; j += kSelThreads) {
-                const uint32_t m = 0xFFFFFFFFu - (uint32_t)(chosen[j] & 0xFFFFFFFFull);
+            for (int j = t; j < K; j += nst) {
+                const uint32_t m = 0xFFFFFFFFu - (uint32_t)(pick[j] & 0xFFFFFFFFull);
                 int p0 = 0, p1 = 0, j2 = 0;
                 for (; j2 + 2 <= K; j2 += 2) {
-                    p0 += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m ? 1 : 0;
-                    p1 += (0xFFFFFFFFu - (uint32_t)(chosen[j2 + 1] & 0xFFFFFFFFull)) < m ? 1 : 0;
+                    p0 += (0xFFFFFFFFu - (uint32_t)(pick[j2] & 0xFFFFFFFFull)) < m ? 1 : 0;
+                    p1 += (0xFFFFFFFFu - (uint32_t)(pick[j2 + 1] & 0xFFFFFFFFull)) < m ? 1 : 0;
                 }
-                if (j2 < K) p0 += (0xFFFFFFFFu - (uint32_t)(chosen[j2] & 0xFFFFFFFFull)) < m ? 1 : 0;
+                if (j2 < K) p0 += (0xFFFFFFFFu - (uint32_t)(pick[j2] & 0xFFFFFFFFull)) < m ? 1 : 0;
                 list[1 + p0 + p1] = (int)m;
             }
         }
