@@ -447,6 +447,38 @@ def test_decode_selection_paths(api):
             compare(f"{name} o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
 
 
+def test_decode_selection_long_rows_and_overflow(api):
+    """Rows of 3000 and 6000 scores over clusters of 8 CTAs, with histories that
+    end early in the row (a few blocks, or far fewer than the row holds), K up to
+    64; and all-equal scores on long and 1500-score rows, where every score is a
+    candidate and the selection falls back to the radix select (ties to the lower
+    index)."""
+    bs = 64
+    B, Hq, Hkv = 2, 8, 2  # 4 rows: clusters of 8 CTAs
+    G = Hq // Hkv
+    rows = [(b, h) for b in range(B) for h in range(Hkv)]
+    for name, nblk, hist, scores, K in (
+            ("long, ragged", 3000, (3000, 2500), "random", 32),
+            ("long, short", 3000, (2100, 9), "random", 5),
+            ("long, K 64", 6000, (6000, 5000), "random", 64),
+            ("long, all equal", 6000, (6000, 4000), "equal", 64),
+            ("whole row, all equal", 1500, (1500, 1200), "equal", 40)):
+        Tmax = bs * nblk + 3
+        C = Tmax // bs
+        ctx = torch.tensor([bs * hist[0] + 1, bs * hist[1] + 2], dtype=torch.int32, device="cuda")
+        s = (_seeded((B, Hkv, C), 1.0, torch.float32, 81) if scores == "random"
+             else torch.full((B, Hkv, C), 0.25, dtype=torch.float32, device="cuda"))
+        inp = {"q": _seeded((B, Hq, 128), 1.0, torch.bfloat16, 82),
+               "k_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 83),
+               "v_cache": _seeded((B, Hkv, Tmax, 128), 1.0, torch.bfloat16, 84),
+               "ctx_len": ctx, "s": s.contiguous()}
+        o, idx = _run_decode(api, inp, bs, K, fused=True)
+        ref = _oracle_decode_rows(inp, rows, bs, K, False)
+        for (b, h), (ro, ridx) in ref.items():
+            np.testing.assert_array_equal(idx[b, h].cpu().numpy(), ridx, err_msg=f"{name} idx[{b},{h}]")
+            compare(f"{name} o[{b},{h}]", host(o[b, h * G:(h + 1) * G]), ro, **BF16_TOL, bf16_out=True)
+
+
 def _paged_from_cache(kc, vc, bs, seed, spare=5):
     """Scatter contiguous caches [B, Hkv, T, d] into shuffled page pools
     [num_pages, bs, Hkv, d] (a few pages left unused) and the page table."""
