@@ -685,7 +685,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # end to end through host buffers: every step copies its inputs in from pinned
     # host memory and its outputs back.  Two device buffer sets let the copies of
     # the neighbouring steps (one copy engine each way) overlap a step's kernels.
-    e2e_steps = max(1, min(args.steps, 8))
+    # At least 16 steps, so that the pipeline's fill (the first step's inputs) and
+    # drain (the last step's outputs) weigh little in the per-step figure.
+    e2e_steps = max(16, min(args.steps, 64))
     host_in = {k: v.cpu().pin_memory() for k, v in inp.items()}
     host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in runner.outputs().items()}
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
