@@ -111,3 +111,36 @@ def test_kernel_breakdown_is_reproducible_from_the_times():
     assert abs(k["executed_tflops"] - k["executed_flops"] / 3.0e-3 / 1e12) < 1e-6
     assert abs(k["frac_executed"] - k["executed_tflops"] / 1595.8) < 1e-12
     assert abs(sum(v["share_of_step"] for v in out.values()) - (1.1 + 5.0) / 6.14) < 1e-9
+
+
+def test_phase_table_puts_ctas_on_one_time_line():
+    """bench.phase_table: each CTA's %clock64 stamps are placed on the common
+    %globaltimer line through its entry and exit (timer, clock) pairs, with the
+    earliest entry as 0, in µs; the timer epoch (~1e18 ns) must not cost
+    precision."""
+    import numpy as np
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    rows = np.zeros((1024, 32), dtype=np.uint64)
+    epoch = 1_700_000_000_000_000_000  # ns, as %globaltimer reads
+    for cta, (gt0, clk0, ghz) in enumerate(((epoch + 1000, 5_000, 2.0), (epoch + 1037, 900_000, 1.0))):
+        # phases 0..11 at 100 ns steps of this CTA's own clock after entry
+        stamps = [clk0 + int(100 * k * ghz) for k in range(12)]
+        rows[cta, :12] = stamps
+        rows[cta, 12], rows[cta, 13] = gt0, clk0  # entry pair
+        rows[cta, 15] = stamps[11]  # exit clock, read with the exit timer
+        rows[cta, 14] = gt0 + 1100
+        rows[cta, 17] = 16 + cta
+        rows[cta, 18] = 8 + cta
+    rows[0, 31] = 2
+    t = bench.phase_table(rows)
+    import pytest
+
+    assert t["ctas"] == 2 and abs(t["sm_clock_ghz"] - 1.5) < 1e-9
+    # [median, latest] in µs; the second CTA entered 37 ns after the first
+    assert t["entry"] == pytest.approx([0.0185, 0.037], abs=1e-3)
+    assert t["threshold"] == pytest.approx([0.4185, 0.437], abs=1e-3)  # phase 4: 400 ns after entry
+    assert t["exit"] == pytest.approx([1.1185, 1.137], abs=1e-3)
+    assert t["candidates_median"] == 16.5 and t["blocks_per_cta"] == [8, 9]
