@@ -67,6 +67,24 @@ def test_select_ties_and_signed_zeros(api):
         _check_select(api, s.contiguous(), k)
 
 
+def test_select_long_rows_filter_and_fallback(api):
+    """Rows of 1024..16384 blocks with K <= 64 take the staged threshold filter:
+    tie-heavy training rows (every history length 0..1099 in one call), signed
+    zeros, Top-K from 1 to 64 and past it (the radix kernel); all-equal decode rows,
+    where every score is a candidate and the filter falls back to the radix
+    select on the staged row."""
+    s = _seeded((1, 2, 1100, 1100), 1.0, torch.float32, 15)
+    s = torch.round(s * 2) / 2
+    s[0, 1, :, ::3] = -0.0
+    s[0, 1, :, 1::3] = 0.0
+    for k in (1, 16, 64, 65):
+        _check_select(api, s.contiguous(), k)
+    for C, T in ((3000, 64 * 3000 + 1), (9000, 64 * 7000 + 5)):
+        s = torch.full((2, 2, 1, C), 0.5, dtype=torch.float32, device="cuda")
+        ctx = torch.tensor([T, 64 * 1500 + 1], dtype=torch.int32, device="cuda")
+        _check_select(api, s, 64, ctx_len=ctx, bs=64)
+
+
 def test_select_decode_rows_bit_exact(api):
     for B, Hkv, C, K, T in ((16, 8, 2048, 16, 131073), (4, 8, 8192, 32, 524289)):
         s = _seeded((B, Hkv, 1, C), 1.0, torch.float32, 13)
