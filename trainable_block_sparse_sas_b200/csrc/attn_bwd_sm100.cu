@@ -581,8 +581,8 @@ struct DkvLayout {
     static constexpr uint32_t kP = kDO + kStages * 2 * kSlab128;  // 128 rows x 64 keys bf16
     static constexpr uint32_t kDS = kP + kSlab128;
     static constexpr uint32_t kBars = kDS + kSlab128;
-    // kv_full, qd_full[S], qd_empty[S], s_full[2], s_free[2], p_ready, item_done, final, drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4;
+    // kv_full, q_full[S], qd_empty[S], s_full[2], s_free[2], p_ready, item_done, final, drain, do_full[S]
+    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4 + kStages;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
     static constexpr uint32_t kList = kMisc + 16;
     static constexpr uint32_t kScan = kList;  // scan scratch precedes the list
@@ -619,7 +619,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     const uint32_t sP = sbase + L::kP, sDS = sbase + L::kDS;
     const uint32_t bar0 = sbase + L::kBars;
     const uint32_t kv_full = bar0;
-    auto qd_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    // Q and dO of a stage land on barriers of their own, so that S starts once Q is in
+    auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto do_full = [&](int s) { return bar0 + 8u * (9 + 2 * kStages + s); };
     auto qd_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
     auto s_full = [&](int i) { return bar0 + 8u * (1 + 2 * kStages + i); };
     auto s_free = [&](int i) { return bar0 + 8u * (3 + 2 * kStages + i); };
@@ -644,7 +646,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         // arrival counts: commits of the chains that must all have completed
         mbar_init(kv_full, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(qd_full(s), 1);
+            mbar_init(q_full(s), 1);
+            mbar_init(do_full(s), 1);
             mbar_init(qd_empty(s), 4);  // dV and dK chains (S/dP of the item completed earlier)
         }
         for (int i = 0; i < 2; ++i) {
@@ -669,11 +672,11 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         // so are the first items: query block m itself, which always attends m
         for (int j = 0; j < kPreItems; ++j) {
             const int qrow = b * a.n + m * kBS + j * kRowsTok;
-            mbar_arrive_expect_tx(qd_full(j), 4 * kSlab128);
-            for (int kh = 0; kh < 2; ++kh) {
-                tma_load_3d(sQ + (j * 2 + kh) * kSlab128, &a.tq, qd_full(j), kh * 64, h * G, qrow);
-                tma_load_3d(sDO + (j * 2 + kh) * kSlab128, &a.tdo, qd_full(j), kh * 64, h * G, qrow);
-            }
+            mbar_arrive_expect_tx(q_full(j), 2 * kSlab128);
+            mbar_arrive_expect_tx(do_full(j), 2 * kSlab128);
+            for (int kh = 0; kh < 2; ++kh) tma_load_3d(sQ + (j * 2 + kh) * kSlab128, &a.tq, q_full(j), kh * 64, h * G, qrow);
+            for (int kh = 0; kh < 2; ++kh)
+                tma_load_3d(sDO + (j * 2 + kh) * kSlab128, &a.tdo, do_full(j), kh * 64, h * G, qrow);
         }
     }
 
@@ -705,11 +708,12 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                 if (j >= kStages && !mbar_wait(qd_empty(st), (j / kStages - 1) & 1, abort_flag, a.status)) break;
                 const int c = list[j / MT], i = j % MT;
                 const int qrow = b * a.n + c * kBS + i * kRowsTok;
-                mbar_arrive_expect_tx(qd_full(st), 4 * kSlab128);
-                for (int kh = 0; kh < 2; ++kh) {
-                    tma_load_3d(sQ + (st * 2 + kh) * kSlab128, &a.tq, qd_full(st), kh * 64, h * G, qrow);
-                    tma_load_3d(sDO + (st * 2 + kh) * kSlab128, &a.tdo, qd_full(st), kh * 64, h * G, qrow);
-                }
+                mbar_arrive_expect_tx(q_full(st), 2 * kSlab128);
+                mbar_arrive_expect_tx(do_full(st), 2 * kSlab128);
+                for (int kh = 0; kh < 2; ++kh)
+                    tma_load_3d(sQ + (st * 2 + kh) * kSlab128, &a.tq, q_full(st), kh * 64, h * G, qrow);
+                for (int kh = 0; kh < 2; ++kh)
+                    tma_load_3d(sDO + (st * 2 + kh) * kSlab128, &a.tdo, do_full(st), kh * 64, h * G, qrow);
             }
         }
         // every warp reaches the CTA barrier below converged: a barrier reached by a
@@ -728,7 +732,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                 for (int j = 0; ok && j < nitems; ++j) {
                     const int st = j % kStages, buf = j & 1;
                     if (j >= 2 && !mbar_wait(s_free(buf), ((j >> 1) - 1) & 1, abort_flag, a.status)) break;
-                    if (!mbar_wait(qd_full(st), (j / kStages) & 1, abort_flag, a.status)) break;
+                    if (!mbar_wait(chain == 0 ? q_full(st) : do_full(st), (j / kStages) & 1, abort_flag, a.status)) break;
                     tc_fence_after();
                     const uint32_t at = a_base + st * 2 * kSlab128;
 #pragma unroll
