@@ -52,7 +52,7 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kBS = 64;
-constexpr int kStages = 2;                   // dk/dv Q/dO ring depth
+constexpr int kDoStages = 2;                 // dk/dv dO ring depth (the Q ring takes 3 where it fits)
 constexpr size_t kSmemLimit = 227 * 1024;     // dynamic shared memory per CTA
 constexpr uint32_t kSlab64 = 64 * 128;    // 64 rows x 128 B: one block, one 64-wide d slab
 constexpr uint32_t kSlab128 = 128 * 128;  // 128 rows x 128 B
@@ -573,20 +573,23 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
 constexpr int kKvThreads = 416;
 constexpr int kKvSoftmaxWarp0 = 5;
 
+template <int QS>
 struct DkvLayout {
+    static constexpr int DS = kDoStages;
     static constexpr uint32_t kK = 0;                     // 2 slabs x 64 rows
     static constexpr uint32_t kV = kK + 2 * kSlab64;
     static constexpr uint32_t kQ = kV + 2 * kSlab64;      // [stage][slab] 128 rows
-    static constexpr uint32_t kDO = kQ + kStages * 2 * kSlab128;
-    static constexpr uint32_t kP = kDO + kStages * 2 * kSlab128;  // 128 rows x 64 keys bf16
+    static constexpr uint32_t kDO = kQ + QS * 2 * kSlab128;
+    static constexpr uint32_t kP = kDO + DS * 2 * kSlab128;  // 128 rows x 64 keys bf16
     static constexpr uint32_t kDS = kP + kSlab128;
     static constexpr uint32_t kBars = kDS + kSlab128;
-    // kv_full, q_full[S], qd_empty[S], s_full[2], s_free[2], p_ready, item_done, final, drain, do_full[S]
-    static constexpr int kNumBars = 1 + 2 * kStages + 4 + 4 + kStages;
+    // kv_full, q_full[QS], q_empty[QS], do_full[DS], do_empty[DS], s_full[2], dp_full[2],
+    // s_free[2], dp_free[2], p_ready, ds_ready, p_done, ds_done, final, drain
+    static constexpr int kNumBars = 1 + 2 * QS + 2 * DS + 14;
     static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
     static constexpr uint32_t kList = kMisc + 16;
-    static constexpr uint32_t kScan = kList;  // scan scratch precedes the list
-    static size_t bytes(int Cq) { return 1024 + kList + 4 * 40 + 4 * (size_t)(Cq + 1); }
+    static constexpr uint32_t kScan = kList;  // 40 ints of scan scratch, then the list as int16
+    static size_t bytes(int Cq) { return 1024 + kList + 4 * 40 + 2 * (size_t)(Cq + 1); }
 };
 
 // is history block m in the ascending selection of query block c (unit uc)?
@@ -605,13 +608,18 @@ __device__ __forceinline__ bool holds(const BwdArgs& a, long uc, int c, int m) {
 }
 
 // kOuter: the outer gate, P and dP scaled by g of the (query block, key block)
-// pair: dV += (g P)^T dO, dS = P (g dP - D)
-template <int MT, bool kOuter>
+// pair: dV += (g P)^T dO, dS = P (g dP - D).
+// QS: depth of the Q ring (dO's is kDoStages).  Q of an item is free once S and dK
+// of the item have completed, dO once dP and dV have; P is published as soon as S
+// lands, so dV and the dO ring do not wait for dP and dS.
+template <int MT, bool kOuter, int QS>
 __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __grid_constant__ BwdArgs a) {
-    using L = DkvLayout;
+    using L = DkvLayout<QS>;
+    constexpr int DS = L::DS;
     constexpr int G = 2 * MT;
     constexpr int kRowsTok = 128 / G;  // tokens per 128-row item
-    constexpr int kPreItems = kStages < MT ? kStages : MT;  // items of query block m, loaded up front
+    // items of query block m, loaded up front
+    constexpr int kPreQ = QS < MT ? QS : MT, kPreDO = DS < MT ? DS : MT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_align1024(smem_raw);
     const uint32_t sbase = smem_u32(base);
@@ -619,20 +627,26 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     const uint32_t sP = sbase + L::kP, sDS = sbase + L::kDS;
     const uint32_t bar0 = sbase + L::kBars;
     const uint32_t kv_full = bar0;
-    // Q and dO of a stage land on barriers of their own, so that S starts once Q is in
     auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto do_full = [&](int s) { return bar0 + 8u * (9 + 2 * kStages + s); };
-    auto qd_empty = [&](int s) { return bar0 + 8u * (1 + kStages + s); };
-    auto s_full = [&](int i) { return bar0 + 8u * (1 + 2 * kStages + i); };
-    auto s_free = [&](int i) { return bar0 + 8u * (3 + 2 * kStages + i); };
-    const uint32_t p_ready = bar0 + 8u * (5 + 2 * kStages);
-    const uint32_t item_done = bar0 + 8u * (6 + 2 * kStages);
-    const uint32_t final_bar = bar0 + 8u * (7 + 2 * kStages);
-    const uint32_t drain = bar0 + 8u * (8 + 2 * kStages);
+    auto q_empty = [&](int s) { return bar0 + 8u * (1 + QS + s); };
+    auto do_full = [&](int s) { return bar0 + 8u * (1 + 2 * QS + s); };
+    auto do_empty = [&](int s) { return bar0 + 8u * (1 + 2 * QS + DS + s); };
+    constexpr int kB = 1 + 2 * QS + 2 * DS;  // first barrier after the rings
+    auto s_full = [&](int i) { return bar0 + 8u * (kB + i); };
+    auto dp_full = [&](int i) { return bar0 + 8u * (kB + 2 + i); };
+    auto s_free = [&](int i) { return bar0 + 8u * (kB + 4 + i); };
+    auto dp_free = [&](int i) { return bar0 + 8u * (kB + 6 + i); };
+    const uint32_t p_ready = bar0 + 8u * (kB + 8);
+    const uint32_t ds_ready = bar0 + 8u * (kB + 9);
+    const uint32_t p_done = bar0 + 8u * (kB + 10);
+    const uint32_t ds_done = bar0 + 8u * (kB + 11);
+    const uint32_t final_bar = bar0 + 8u * (kB + 12);
+    const uint32_t drain = bar0 + 8u * (kB + 13);
+    static_assert(kB + 14 == L::kNumBars, "barrier count");
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L::kMisc + 4);
     int* scan = reinterpret_cast<int*>(base + L::kScan);  // 33 ints
-    int* list = scan + 40;
+    int16_t* list = reinterpret_cast<int16_t*>(scan + 40);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // head-major order (concurrent CTAs share one KV head's Q/dO in L2); within a
@@ -645,17 +659,24 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     if (threadIdx.x == 0) {
         // arrival counts: commits of the chains that must all have completed
         mbar_init(kv_full, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < QS; ++s) {
             mbar_init(q_full(s), 1);
+            mbar_init(q_empty(s), 3);  // S chain and the two dK lanes
+        }
+        for (int s = 0; s < DS; ++s) {
             mbar_init(do_full(s), 1);
-            mbar_init(qd_empty(s), 4);  // dV and dK chains (S/dP of the item completed earlier)
+            mbar_init(do_empty(s), 3);  // dP chain and the two dV lanes
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(s_full(i), 2);    // S and dP chains
+            mbar_init(s_full(i), 1);
+            mbar_init(dp_full(i), 1);
             mbar_init(s_free(i), 256);  // softmax threads have read the buffer
+            mbar_init(dp_free(i), 256);
         }
         mbar_init(p_ready, 256);
-        mbar_init(item_done, 4);
+        mbar_init(ds_ready, 256);
+        mbar_init(p_done, 2);
+        mbar_init(ds_done, 2);
         mbar_init(final_bar, 4);
         mbar_init(drain, 6);
         *abort_flag = 0;
@@ -670,25 +691,28 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             tma_load_3d(sV + kh * kSlab64, &a.tv, kv_full, kh * 64, h, krow);
         }
         // so are the first items: query block m itself, which always attends m
-        for (int j = 0; j < kPreItems; ++j) {
+        for (int j = 0; j < kPreQ; ++j) {
             const int qrow = b * a.n + m * kBS + j * kRowsTok;
             mbar_arrive_expect_tx(q_full(j), 2 * kSlab128);
-            mbar_arrive_expect_tx(do_full(j), 2 * kSlab128);
             for (int kh = 0; kh < 2; ++kh) tma_load_3d(sQ + (j * 2 + kh) * kSlab128, &a.tq, q_full(j), kh * 64, h * G, qrow);
+        }
+        for (int j = 0; j < kPreDO; ++j) {
+            const int qrow = b * a.n + m * kBS + j * kRowsTok;
+            mbar_arrive_expect_tx(do_full(j), 2 * kSlab128);
             for (int kh = 0; kh < 2; ++kh)
                 tma_load_3d(sDO + (j * 2 + kh) * kSlab128, &a.tdo, do_full(j), kh * 64, h * G, qrow);
         }
     }
 
     // query blocks attending key block m: m itself, then every c > m holding m
-    list[0] = m;
+    list[0] = (int16_t)m;
     int nlist = 1;
     for (int c0 = m + 1; c0 < a.Cq; c0 += kKvThreads) {
         const int cc = c0 + (int)threadIdx.x;
         const int att = (cc < a.Cq && (a.full_scope || holds(a, ubase + cc, cc, m))) ? 1 : 0;
         int cnt;
         const int pos = block_exclusive_scan(att, scan, &cnt);
-        if (att) list[nlist + pos] = cc;
+        if (att) list[nlist + pos] = (int16_t)cc;
         nlist += cnt;
     }
     if (warp == 1) {
@@ -702,18 +726,21 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
     // TMEM: S/dP buffers at 0 and 128 (S | dP), dV^T halves at 256 and 320, dK^T halves at 384 and 448
 
     if (warp == 0) {
-        if (lane == 0) {
-            for (int j = kPreItems; j < nitems; ++j) {
-                const int st = j % kStages;
-                if (j >= kStages && !mbar_wait(qd_empty(st), (j / kStages - 1) & 1, abort_flag, a.status)) break;
+        // lane 0 refills the Q ring, lane 1 the dO ring, each in item order
+        if (lane < 2) {
+            const bool is_q = lane == 0;
+            const int ns = is_q ? QS : DS;
+            const uint32_t ring = is_q ? sQ : sDO;
+            const CUtensorMap* tm = is_q ? &a.tq : &a.tdo;
+            int st = is_q ? kPreQ % QS : kPreDO % DS;
+            for (int j = is_q ? kPreQ : kPreDO; j < nitems; ++j) {
+                const uint32_t full = is_q ? q_full(st) : do_full(st), empty = is_q ? q_empty(st) : do_empty(st);
+                if (j >= ns && !mbar_wait(empty, (j / ns - 1) & 1, abort_flag, a.status)) break;
                 const int c = list[j / MT], i = j % MT;
                 const int qrow = b * a.n + c * kBS + i * kRowsTok;
-                mbar_arrive_expect_tx(q_full(st), 2 * kSlab128);
-                mbar_arrive_expect_tx(do_full(st), 2 * kSlab128);
-                for (int kh = 0; kh < 2; ++kh)
-                    tma_load_3d(sQ + (st * 2 + kh) * kSlab128, &a.tq, q_full(st), kh * 64, h * G, qrow);
-                for (int kh = 0; kh < 2; ++kh)
-                    tma_load_3d(sDO + (st * 2 + kh) * kSlab128, &a.tdo, do_full(st), kh * 64, h * G, qrow);
+                mbar_arrive_expect_tx(full, 2 * kSlab128);
+                for (int kh = 0; kh < 2; ++kh) tma_load_3d(ring + (st * 2 + kh) * kSlab128, tm, full, kh * 64, h * G, qrow);
+                st = st + 1 == ns ? 0 : st + 1;
             }
         }
         // every warp reaches the CTA barrier below converged: a barrier reached by a
@@ -723,16 +750,22 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         const int chain = warp - 1;  // 0 S, 1 dP, 2 dV, 3 dK
         if (lane < (chain < 2 ? 1 : 2)) {
             bool ok = true;
+            // Q chains (S, dK) walk the Q ring, dO chains (dP, dV) the dO ring
+            const bool on_q = chain == 0 || chain == 3;
+            const int ns = on_q ? QS : DS;
             if (chain < 2) {
                 // S = Q K^T (chain 0) or dP = dO V^T (chain 1) of item j into TMEM buffer j & 1,
                 // once the softmax threads have read that buffer's previous item
                 constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
                 const uint32_t a_base = chain == 0 ? sQ : sDO, b_base = chain == 0 ? sK : sV;
                 ok = mbar_wait(kv_full, 0, abort_flag, a.status);
+                int st = 0;
                 for (int j = 0; ok && j < nitems; ++j) {
-                    const int st = j % kStages, buf = j & 1;
-                    if (j >= 2 && !mbar_wait(s_free(buf), ((j >> 1) - 1) & 1, abort_flag, a.status)) break;
-                    if (!mbar_wait(chain == 0 ? q_full(st) : do_full(st), (j / kStages) & 1, abort_flag, a.status)) break;
+                    const int buf = j & 1;
+                    if (j >= 2 && !mbar_wait(chain == 0 ? s_free(buf) : dp_free(buf), ((j >> 1) - 1) & 1, abort_flag,
+                                             a.status))
+                        break;
+                    if (!mbar_wait(chain == 0 ? q_full(st) : do_full(st), (j / ns) & 1, abort_flag, a.status)) break;
                     tc_fence_after();
                     const uint32_t at = a_base + st * 2 * kSlab128;
 #pragma unroll
@@ -741,7 +774,9 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                         mma_ss(tmem + buf * 128 + chain * 64, sdesc_sw128(at + kh * kSlab128 + kk * 32, 16, 1024),
                                sdesc_sw128(b_base + kh * kSlab64 + kk * 32, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
                     }
-                    mma_commit(s_full(buf));
+                    mma_commit(chain == 0 ? s_full(buf) : dp_full(buf));
+                    if (j + ns < nitems) mma_commit(chain == 0 ? q_empty(st) : do_empty(st));
+                    st = st + 1 == ns ? 0 : st + 1;
                 }
             } else {
                 // dV^T += dO^T P (chain 2) or dK^T += Q^T dS (chain 3), accumulated over all
@@ -749,21 +784,26 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                 constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, true, true);
                 const uint32_t a_base = chain == 2 ? sDO : sQ, b_base = chain == 2 ? sP : sDS;
                 const uint32_t acc = tmem + 256 + (chain - 2) * 128 + lane * 64;
+                int st = 0;
                 for (int j = 0; j < nitems; ++j) {
-                    if (!mbar_wait(p_ready, j & 1, abort_flag, a.status)) {
+                    // P (dS) of item j is in shared memory, and so is its dO (Q): dV does not
+                    // follow dP, so it waits for dO itself
+                    if (!mbar_wait(chain == 2 ? p_ready : ds_ready, j & 1, abort_flag, a.status) ||
+                        !mbar_wait(chain == 2 ? do_full(st) : q_full(st), (j / ns) & 1, abort_flag, a.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t at = a_base + (j % kStages) * 2 * kSlab128 + lane * 4 * 2048;
+                    const uint32_t at = a_base + st * 2 * kSlab128 + lane * 4 * 2048;
                     const uint32_t bt = b_base + lane * 4 * 2048;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         mma_ss(acc, sdesc_sw128(at + ks * 2048, kSlab128, 1024), sdesc_sw128(bt + ks * 2048, kSlab128, 1024),
                                idesc_g, (j > 0 || ks > 0) ? 1u : 0u);
                     }
-                    mma_commit(item_done);
-                    if (j + kStages < nitems) mma_commit(qd_empty(j % kStages));
+                    mma_commit(chain == 2 ? p_done : ds_done);
+                    if (j + ns < nitems) mma_commit(chain == 2 ? do_empty(st) : q_empty(st));
+                    st = st + 1 == ns ? 0 : st + 1;
                 }
                 if (ok) mma_commit(final_bar);
             }
@@ -801,24 +841,25 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
         int tok = 0;
         bool diag = false;
         if (nitems > 0) fetch(0, off, dneg, w, tok, diag);
+        const uint32_t rbase = (uint32_t)row * 128u;
         for (int j = 0; j < nitems; ++j) {
             const int buf = j & 1;
             float n_off = 0.f, n_dneg = 0.f, n_w = 1.f;
             int n_tok = 0;
             bool n_diag = false;
             if (j + 1 < nitems) fetch(j + 1, n_off, n_dneg, n_w, n_tok, n_diag);
+            // P from S alone, published before dP is read
             if (!warp_wait(s_full(buf), (j >> 1) & 1, abort_flag, a.status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
-            const uint64_t dn2 = f2_pack(dneg, dneg), w2 = f2_pack(w, w);
-            uint32_t pp[16], dd[16];
+            float p[32];
+            uint32_t pk[16];
             {
-                uint32_t sr[32], dr[32];
-                tmem_ld32x2_sync(tmem + lane_off + buf * 128 + 32 * kw, tmem + lane_off + buf * 128 + 64 + 32 * kw,
-                                 sr, dr);
+                const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), off2 = f2_pack(off, off);
+                uint32_t sr[32];
+                tmem_ld32_sync(tmem + lane_off + buf * 128 + 32 * kw, sr);
                 tc_fence_before();
                 mbar_arrive(s_free(buf));
 #pragma unroll
@@ -832,12 +873,43 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
                         if (key > tok) p0 = 0.f;
                         if (key + 1 > tok) p1 = 0.f;
                     }
+                    p[2 * jj] = p0;
+                    p[2 * jj + 1] = p1;
+                    pk[jj] = kOuter ? pack_bf16x2(p0 * w, p1 * w) : pack_bf16x2(p0, p1);
+                }
+            }
+            // the P buffer is free once the dV MMAs of item j-1 completed
+            if (j > 0 && !warp_wait(p_done, (j - 1) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+            }
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                const int chunk = 4 * kw + ch;  // 16-byte chunk = 8 keys
+                const uint32_t sw = (uint32_t)((chunk ^ (row & 7)) * 16);
+                st_shared_v4(sP + rbase + sw, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(p_ready);
+            // dS = P (w dP - D)
+            if (!warp_wait(dp_full(buf), (j >> 1) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            {
+                const uint64_t dn2 = f2_pack(dneg, dneg), w2 = f2_pack(w, w);
+                uint32_t dr[32];
+                tmem_ld32_sync(tmem + lane_off + buf * 128 + 64 + 32 * kw, dr);
+                tc_fence_before();
+                mbar_arrive(dp_free(buf));
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
                     float d0, d1;
-                    f2_unpack(f2_mul(f2_pack(p0, p1),
+                    f2_unpack(f2_mul(f2_pack(p[2 * jj], p[2 * jj + 1]),
                                      f2_fma(f2_pack(__uint_as_float(dr[2 * jj]), __uint_as_float(dr[2 * jj + 1])), w2, dn2)),
                               d0, d1);
-                    pp[jj] = kOuter ? pack_bf16x2(p0 * w, p1 * w) : pack_bf16x2(p0, p1);
-                    dd[jj] = pack_bf16x2(d0, d1);
+                    pk[jj] = pack_bf16x2(d0, d1);
                 }
             }
             off = n_off;
@@ -845,22 +917,19 @@ __global__ void __launch_bounds__(kKvThreads, 1) bwd_dkdv_sm100_kernel(const __g
             w = n_w;
             tok = n_tok;
             diag = n_diag;
-            tc_fence_before();
-            // P / dS smem buffers are free once the MMAs of item j-1 completed
-            if (j > 0 && !warp_wait(item_done, (j - 1) & 1, abort_flag, a.status)) {
+            // the dS buffer is free once the dK MMAs of item j-1 completed
+            if (j > 0 && !warp_wait(ds_done, (j - 1) & 1, abort_flag, a.status)) {
                 ok = false;
                 break;
             }
-            const uint32_t rbase = (uint32_t)row * 128u;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
-                const int chunk = 4 * kw + ch;  // 16-byte chunk = 8 keys
+                const int chunk = 4 * kw + ch;
                 const uint32_t sw = (uint32_t)((chunk ^ (row & 7)) * 16);
-                st_shared_v4(sP + rbase + sw, pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
-                st_shared_v4(sDS + rbase + sw, dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
+                st_shared_v4(sDS + rbase + sw, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             }
             fence_proxy_async_smem();
-            mbar_arrive(p_ready);
+            mbar_arrive(ds_ready);
         }
         if (ok && warp_wait(final_bar, 0, abort_flag, a.status)) {
             tc_fence_after();
@@ -966,9 +1035,14 @@ cudaError_t launch_mt(const TrainParams& p, int hsplit, cudaStream_t stream) {
     // key-major kernel: 128-row items (128/G tokens x G heads) per box
     if (!encode_tma_rows(&a.tq, p.q, p.Hq, rows, G, 128 / G) || !encode_tma_rows(&a.tdo, p.dO, p.Hq, rows, G, 128 / G))
         return cudaErrorInvalidValue;
+    // a third Q stage where the list of attending query blocks leaves room for it
+    if (DkvLayout<3>::bytes(p.Cq) <= kSmemLimit)
+        return p.gate == kGateOuter
+                   ? launch_kernel(bwd_dkdv_sm100_kernel<MK, true, 3>, grid, kKvThreads, DkvLayout<3>::bytes(p.Cq), a, stream)
+                   : launch_kernel(bwd_dkdv_sm100_kernel<MK, false, 3>, grid, kKvThreads, DkvLayout<3>::bytes(p.Cq), a, stream);
     return p.gate == kGateOuter
-               ? launch_kernel(bwd_dkdv_sm100_kernel<MK, true>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream)
-               : launch_kernel(bwd_dkdv_sm100_kernel<MK, false>, grid, kKvThreads, DkvLayout::bytes(p.Cq), a, stream);
+               ? launch_kernel(bwd_dkdv_sm100_kernel<MK, true, 2>, grid, kKvThreads, DkvLayout<2>::bytes(p.Cq), a, stream)
+               : launch_kernel(bwd_dkdv_sm100_kernel<MK, false, 2>, grid, kKvThreads, DkvLayout<2>::bytes(p.Cq), a, stream);
 }
 
 }  // namespace
@@ -994,7 +1068,7 @@ bool bwd_sm100_supported(const TrainParams& p) {
     if ((long)p.B * p.n > 0x7fffffffL || (long)p.B * p.Hkv * p.Cq * (p.Hq / p.Hkv == 8 ? 2 : 1) > 0x7fffffffL)
         return false;
     const int nl = dq_list_max(p.Cq, p.top_k, p.full_scope, p.gate);
-    return DqLayout<2, 2>::bytes(nl) <= kSmemLimit && DkvLayout::bytes(p.Cq) <= kSmemLimit;
+    return DqLayout<2, 2>::bytes(nl) <= kSmemLimit && DkvLayout<2>::bytes(p.Cq) <= kSmemLimit;
 }
 
 cudaError_t launch_bwd_sm100(const TrainParams& p, cudaStream_t stream) {
