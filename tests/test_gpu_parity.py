@@ -157,6 +157,27 @@ def test_bf16_shapes(api, B, n, Hq, Hkv, d, bs, K, full):
     assert api.sas_attn_path(api.attn_desc(inp["q"], inp["k"], bs, K, full)) == want_path
 
 
+def test_fwd_lse_tight(api):
+    """The forward's row log-sum-exp against the oracle at 3e-4 (natural-log units),
+    far inside the bf16 tolerance of o: S is an fp32 accumulation of exact bf16
+    products and the row sum is fp32, so an approximate exponential, a lost
+    rescale of the running sum or a wrong log-gate bias shows here first."""
+    B, n, Hq, Hkv, d, bs, K = 2, 1024, 8, 2, 128, 64, 6
+    Cq = n // bs
+    inp = {
+        "q": _seeded((B, n, Hq, d), 1.0, torch.bfloat16, 31),
+        "k": _seeded((B, n, Hkv, d), 1.0, torch.bfloat16, 32),
+        "v": _seeded((B, n, Hkv, d), 1.0, torch.bfloat16, 33),
+        "s": _seeded((B, Hkv, Cq, Cq), 2.0, torch.float32, 34),
+        "dO": _seeded((B, n, Hq, d), 1.0, torch.bfloat16, 35),
+    }
+    got = run_train(api, inp, bs, K, False)
+    want = _oracle_train(inp, bs, K, False)
+    assert api.sas_attn_path(api.attn_desc(inp["q"], inp["k"], bs, K, False))[0] == "tensor_core"
+    err = np.abs(host(got["lse"]) - want["lse"])
+    assert err.max() <= 3e-4, err.max()
+
+
 def test_unsupported_block_size_is_refused(api):
     q = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
     k = torch.zeros((1, 256, 1, 128), dtype=torch.bfloat16, device="cuda")
