@@ -324,6 +324,16 @@ def test_train_sparse_32k_gqa8_sampled(api):
     _sampled_full_size(api, w, q_blocks=(0, 1, 33, 257, 511), kv_blocks=(511, 200), heads=(0, 3))
 
 
+def test_train_sparse_64k_two_q_stages_sampled(api):
+    """64K tokens (1024 query blocks): the list of query blocks attending a key
+    block no longer leaves room for a third Q stage, so the dk/dv kernel runs its
+    two-stage Q ring; sampled key blocks with short and long lists."""
+    import dataclasses
+
+    w = dataclasses.replace(syn.TRAIN_SPARSE_32K, name="train_sparse_64k_small", Hq=8, Hkv=2, n=65536)
+    _sampled_full_size(api, w, q_blocks=(0, 1, 33, 700, 1023), kv_blocks=(1022, 400), heads=(1,))
+
+
 def test_train_full_16k_sampled(api):
     w = syn.TRAIN_FULL_16K
     _sampled_full_size(api, w, q_blocks=(0, 1, 100, 255), kv_blocks=(255, 250), heads=(3,))
