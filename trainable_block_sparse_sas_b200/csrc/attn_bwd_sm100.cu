@@ -102,8 +102,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // dq / ds kernel
 // ============================================================================
 // warp 0 TMA; per M-tile i, warp 1 + 2i issues the S chain and warp 2 + 2i the
-// dQ and dP chain (a single thread's chain of small MMAs is latency-bound, so
-// each tile has two); warps 5..12 softmax, one group per M-tile.  The two tiles
+// dQ and dP chain (separate threads, so that a chain waiting for its operands
+// does not hold up the other); warps 5..12 softmax, one group per M-tile.  The two tiles
 // take turns: tile 1 issues block t once tile 0 has issued it, tile 0 issues
 // block t+1 once tile 1 has issued block t, so one tile's MMAs run while the
 // other tile's softmax does.
@@ -567,8 +567,8 @@ __global__ void __launch_bounds__(kDqThreads, 1) bwd_dq_sm100_kernel(const __gri
 // ============================================================================
 // warp 0 TMA; warps 1 and 2 issue the S and dP MMA chains, warps 3 and 4 the dV
 // and dK chains with lanes 0 and 1 taking the two 64-row halves of each item
-// into separate accumulators (a single thread's chain of small MMAs is
-// latency-bound; several chains run concurrently); warps 5..12 two softmax
+// into separate accumulators (separate threads, so that a chain waiting for its
+// operands or its P / dS does not hold up another); warps 5..12 two softmax
 // groups (key halves)
 constexpr int kKvThreads = 416;
 constexpr int kKvSoftmaxWarp0 = 5;

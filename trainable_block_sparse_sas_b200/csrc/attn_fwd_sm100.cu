@@ -16,8 +16,8 @@
 // time (N = 64 keys) through a 4-stage shared-memory ring of K and V.
 //   warp 0      TMA producer: K and V blocks of the list after the first (Q and the
 //               current block's K and V are requested at the start)
-//   warps 1..4  MMA issuers, two per M-tile (a single thread's chain of small
-//               MMAs is latency-bound; the chains run concurrently):
+//   warps 1..4  MMA issuers, two per M-tile (separate threads, so that the PV
+//               chain waiting for P does not hold up the next S):
 //                 S_i = Q_i K^T   (SS MMA into TMEM buffer t mod 2 of tile i)
 //                 O_i += P_i V    (TS MMA, P read from the buffer it was written to)
 //               With two S buffers per tile, S of block t+1 is computed while the
