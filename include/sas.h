@@ -72,7 +72,7 @@ typedef enum {
 typedef enum { SAS_F32 = 0, SAS_BF16 = 1 } sas_dtype;
 typedef enum { SAS_SCOPE_SPARSE = 0, SAS_SCOPE_FULL = 1 } sas_scope;
 /* Gate.  SOFTMAX is the method: log g = s - LSE(s) added to the logits inside the
- * attention softmax.  The others are the ablations of the pages' design choices
+ * attention softmax.  The others are the ablations of SAS's design choices
  * (jaehun.me review, "Why the Four Design Choices Matter"; shibing624 review,
  * Fig. 2):
  *   SIGMOID  log g = log sigmoid(s), inside the softmax   (gate activation)
@@ -93,7 +93,7 @@ typedef enum {
 
 /* Training-shape problem.  Sparse scope attends the Top-K history blocks of each
  * query block plus the current block; full scope attends every history block,
- * all gated (the "training scope" design choice of the pages, shibing624 review
+ * all gated (the "training scope" design choice of SAS, shibing624 review
  * Fig. 2(d); jaehun.me review, "Why the Four Design Choices Matter"). */
 typedef struct {
     int32_t batch, n_q_heads, n_kv_heads, head_dim;
@@ -229,7 +229,7 @@ sas_status sas_gated_attn_bwd_timed(const sas_attn_desc* desc, const void* q, co
 /*
  * Parameter-free pooled-key scorer (jaehun.me review, walkthrough Step 1: scores
  * from the query and per-block key summaries; Limitations: pooling-based block
- * summaries).  The pages' trained selector is not given; this is its weight-free
+ * summaries).  SAS's trained selector is not given; this is its weight-free
  * form, mean pooling on both sides, producing the score array s the selection
  * and the gate read.
  *
@@ -314,7 +314,7 @@ sas_status sas_sparse_decode(const sas_decode_desc* desc, const void* q, const v
  *   Top-K of the block scores (as sas_topk_select in decode mode: ties to the
  *   lower index) and the gate-free attention of sas_sparse_decode, in one launch
  *   and without workspace (one thread-block cluster per (sequence, kv head)).
- *   The selection stage is the decode bottleneck the pages report at long
+ *   The selection stage is the decode bottleneck the SAS reviews report at long
  *   context (shibing624 review, Fig. 7c; jaehun.me review, Decoding Efficiency).
  * s        [B, Hkv, s_cols] fp32 block scores; row (b, h) scores blocks
  *          0 .. floor((ctx_len[b]-1)/block_size) - 1, which must be <= s_cols.

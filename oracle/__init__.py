@@ -5,7 +5,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 shares no code with the CUDA library: the arithmetic lives in ``sas_oracle.c``
 (plain loops in double precision), this module only marshals numpy arrays.
 
-Every function follows a definition on the pages about SAS ("SAS: Simple
+Every function follows a definition in the reviews of SAS ("SAS: Simple
 Attention Sparsification via End-to-End Optimization of Context Ranking"); the
 C file cites each one.  Parity status: every function here (selection, the
 gated forward and backward with every gate variant and the bf16-stored-output

@@ -5,7 +5,7 @@
  * this file: only the tests, the smoke check and the benchmark's CPU-baseline leg
  * use it.  It shares no code, header, table or helper with the CUDA library.
  *
- * Every function below writes out a definition from the pages on SAS ("SAS: Simple
+ * Every function below writes out a definition from the reviews of SAS ("SAS: Simple
  * Attention Sparsification via End-to-End Optimization of Context Ranking"):
  *   - block partition, C = n/b blocks (jaehun.me review, Background, Eq. 3 text);
  *   - gate g = softmax(s) over the history blocks, log g_m = s_m - LSE(s)
@@ -28,7 +28,7 @@
  *   - a weight-free pooled-key scorer: mean-pooled query and key block summaries
  *     and their scaled dot product (jaehun.me review, walkthrough Step 1 and
  *     Limitations: pooling-based block summaries).
- * Readings where the pages are silent (all listed in the design notes):
+ * Readings where the reviews are silent:
  *   softmax scale sigma (default 1/sqrt(d)); one score row per (kv head, query
  *   block) shared by the query heads of a GQA group; 0-based blocks, history of
  *   query block c is m < c, current block causally masked token by token; ties in
@@ -191,7 +191,7 @@ typedef struct {
     int gate;       /* 0: plain block-sparse attention (no bias);
                        1: log g = s - LSE(s) (softmax gate, the method);
                        2: log g = log sigmoid(s); 3: log g = s (raw logit) -- the
-                       gate-activation variants the pages ablate (jaehun.me review,
+                       gate-activation variants SAS ablates (jaehun.me review,
                        "Why the Four Design Choices Matter", gate activation);
                        4: outer gate, o = sum_j g_{m(j)} p_j v_j with p the gate-free
                        softmax (gate placement, section 4.2.2 Eq. 5);

@@ -1,10 +1,11 @@
-"""Pins of the fp64 CPU oracle against facts fixed by the pages and by mathematics.
+"""Pins of the fp64 CPU oracle against facts fixed by the SAS reviews and by mathematics.
 
 None of these tests touches a GPU.  Each pin is independent of the oracle's own
-code: printed values of the pages' worked example, brute-force selection, dense
+code: printed values of the jaehun.me review's worked example, brute-force selection, dense
 attention and its autograd gradients from torch (fp64), an explicit dense-mask
 formulation of the gated attention differentiated by torch autograd, central
-finite differences, the inner-gate gradient identity (Eq. 5 of the pages),
+finite differences, the inner-gate gradient identity (jaehun.me review, "Why the Four
+Design Choices Matter", quoting the paper's Eq. 5),
 and invariants (shift invariance of s, ds summing to zero, sparse == full scope
 when the budget covers the history).
 """
@@ -289,7 +290,8 @@ def test_central_finite_differences():
 
 
 def test_inner_gate_gradient_identity_eq5():
-    """Eq. 5 of the pages (inner gate): dg_m = sum_{i in B_m} (p_i/g_m) do.(v_i - o),
+    """The inner-gate gradient (jaehun.me review, "Why the Four Design Choices Matter", the
+    paper's Eq. 5): dg_m = sum_{i in B_m} (p_i/g_m) do.(v_i - o),
     i.e. d(log g)_m = sum_{i in B_m} p_i do.(v_i - o), summed over the query rows
     sharing the score row.  Evaluated here from the forward outputs only."""
     rng = np.random.default_rng(9)

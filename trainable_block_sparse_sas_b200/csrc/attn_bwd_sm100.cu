@@ -34,7 +34,7 @@
 // then corrected by delta_i; the corrected value is written to the workspace for
 // the dk/dv kernel, which runs after it.
 //
-// Gate variants (the pages' ablations): sigmoid and raw logit change log g; the
+// Gate variants (SAS's ablations of its design choices): sigmoid and raw logit change log g; the
 // outer gate scales P by g (dS = P (g dP - D), dV from g P, dlogg = g sum P dP);
 // the hard STE gate has bias 0 and its dq kernel also walks the dropped history
 // blocks, whose dS feeds dlogg but not dQ.

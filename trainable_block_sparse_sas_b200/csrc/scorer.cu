@@ -1,6 +1,6 @@
 // scorer.cu -- the parameter-free pooled-key selector scorer.
 //
-// The pages' selector scores a query against per-block key summaries built by
+// SAS's selector scores a query against per-block key summaries built by
 // pooling (jaehun.me review, walkthrough Step 1; Limitations: pooling-based block
 // summaries); its trained weights are not given, so this is the weight-free form:
 // mean pooling on both sides.

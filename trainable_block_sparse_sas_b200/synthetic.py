@@ -4,7 +4,7 @@ This module only draws random tensors of the workloads' shapes and value
 distributions; it holds none of the method's arithmetic.  Both the CUDA path
 (bench, GPU tests) and the CPU oracle (tests) consume what it produces.
 
-Workloads (shapes and distributions of the pages' Qwen3 settings: block size 64,
+Workloads (shapes and distributions of the Qwen3 settings the SAS reviews report: block size 64,
 training length 32768, budgets of 1024 / 2048 tokens):
   tiny_fp32          B=1, 1 KV head, 2 query heads, d=64, n=512, b=16, Top-K 4, fp32,
                      q,k,v ~ N(0,1)/8, s ~ N(0,1), dO ~ N(0,1)
