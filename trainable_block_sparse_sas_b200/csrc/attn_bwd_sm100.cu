@@ -25,10 +25,14 @@
 //   blocks that attend m (m itself with the causal mask, and every later block
 //   whose selection holds m), one 128-row M-tile at a time:
 //     S = Q K_m^T and dP = dO V_m^T                   (SS MMAs, double-buffered TMEM)
-//     softmax warps: P and dS as above, written as bf16 rows into swizzled smem
+//     softmax warps: P (from S alone) and then dS as above, each written as bf16
+//       rows into swizzled smem and published on its own barrier
 //     dV^T += dO^T P and dK^T += Q^T dS               (SS MMAs, M = head_dim = 128)
-//   Epilogue: dk = sigma dK, dv = dV.  The first items (query block m itself) are
-//   requested together with K and V, before the list of attending blocks is built.
+//   Q and dO come through rings of their own (three Q stages where the list of
+//   attending blocks leaves room, two dO stages), each stage freed by the MMAs
+//   that read it.  Epilogue: dk = sigma dK, dv = dV.  The first items (query
+//   block m itself) are requested together with K and V, before the list of
+//   attending blocks is built.
 //
 // D_i is computed by the dq kernel's softmax threads (one row each): dO_i . o_i,
 // then corrected by delta_i; the corrected value is written to the workspace for
